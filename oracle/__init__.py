@@ -1,0 +1,178 @@
+"""CPU oracle for the BLASST attention forward -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library
+(``dynamic_block_sparse_fa_b200``) neither imports nor links it.
+
+The arithmetic lives in ``blasst_oracle.c`` (plain float64 loops, one query
+tile at a time, blocks in ascending order); this module only marshals numpy
+arrays into that library.  Every function takes bfloat16 tensors as raw
+``uint16`` bit patterns, so the oracle reads exactly the bytes the GPU reads.
+
+Parity pins (see ``tests/test_oracle_pins.py``): dense limit against a
+float64 brute-force softmax, an independent closed-form skip mask, the
+skipped-mass bound, mask monotonicity in lambda and the split/merge identity.
+"""
+import ctypes
+import math
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+NOT_VISITED, KEPT, SKIPPED = 0, 1, 2
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        lib.oracle_prefill.restype = ctypes.c_int
+        lib.oracle_prefill.argtypes = [
+            _u16p, _u16p, _u16p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+            ctypes.c_double, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, _i32p, _dp, _dp, _u8p, _dp, _i64p, ctypes.c_int]
+        lib.oracle_decode.restype = ctypes.c_int
+        lib.oracle_decode.argtypes = [
+            _u16p, _u16p, _u16p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_double, ctypes.c_double, ctypes.c_int,
+            ctypes.c_int, _dp, _dp, _dp, _dp, _u8p, _dp, _i64p, ctypes.c_int]
+        lib.oracle_combine.restype = None
+        lib.oracle_combine.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, _dp, _dp]
+        lib.oracle_split_begin.restype = ctypes.c_int
+        lib.oracle_split_begin.argtypes = [ctypes.c_int] * 3
+        _lib = lib
+    return _lib
+
+
+def _ptr(a, t):
+    return a.ctypes.data_as(t)
+
+
+def _bits(x):
+    """bf16 tensor/array -> contiguous uint16 numpy array of its bit patterns."""
+    if hasattr(x, "detach"):  # torch tensor
+        import torch
+        assert x.dtype == torch.bfloat16, x.dtype
+        x = x.detach().cpu().contiguous().view(torch.int16).numpy()
+    x = np.ascontiguousarray(x)
+    assert x.dtype in (np.uint16, np.int16), x.dtype
+    return x.view(np.uint16)
+
+
+def n_threads_default():
+    return os.cpu_count() or 1
+
+
+def prefill(q, k, v, scale, causal, ln_lambda, Br, Bc, units=None,
+            n_threads=0):
+    """BLASST prefill forward for query tiles ``units`` (list of (b, hq, i)).
+
+    q [B,Hq,Lq,d], k/v [B,Hkv,Lkv,d] bf16.  Returns a dict with
+    ``o`` [n_units,Br,d] f64, ``lse`` [n_units,Br], ``mask`` [n_units,nk] u8,
+    ``margin`` [n_units,nk], ``visited``, ``skipped``, ``units`` and
+    ``threads``.  ``units=None`` means every tile of every head.
+    """
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, Hq, Lq, d = qb.shape
+    _, Hkv, Lkv, _ = kb.shape
+    nq = -(-Lq // Br)
+    nk = -(-Lkv // Bc)
+    if units is None:
+        units = [(b, h, i) for b in range(B) for h in range(Hq)
+                 for i in range(nq)]
+    ua = np.ascontiguousarray(np.asarray(units, dtype=np.int32).reshape(-1, 3))
+    n = ua.shape[0]
+    o = np.zeros((n, Br, d), np.float64)
+    lse = np.zeros((n, Br), np.float64)
+    mask = np.zeros((n, nk), np.uint8)
+    margin = np.zeros((n, nk), np.float64)
+    counts = np.zeros(2, np.int64)
+    rc = lib.oracle_prefill(
+        _ptr(qb, _u16p), _ptr(kb, _u16p), _ptr(vb, _u16p),
+        B, Hq, Hkv, Lq, Lkv, d, float(scale), int(bool(causal)),
+        float(ln_lambda), Br, Bc, n, _ptr(ua, _i32p),
+        _ptr(o, _dp), _ptr(lse, _dp), _ptr(mask, _u8p), _ptr(margin, _dp),
+        _ptr(counts, _i64p), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_prefill rejected its arguments")
+    threads = n_threads if n_threads > 0 else n_threads_default()
+    return dict(o=o, lse=lse, mask=mask, margin=margin,
+                visited=int(counts[0]), skipped=int(counts[1]),
+                units=ua, threads=threads)
+
+
+def decode(q, k, v, scale, ln_lambda, Bc, num_splits, n_threads=0):
+    """BLASST decode forward with split-KV and log-sum-exp merge.
+
+    q [B,Hq,d], k/v [B,Hkv,Lkv,d] bf16.  Returns ``o`` [B,Hq,d], ``lse``
+    [B,Hq], ``o_part`` [B,Hq,S,d], ``lse_part`` [B,Hq,S], ``mask``
+    [B,Hkv,nk], ``margin`` [B,Hkv,nk], ``visited``, ``skipped``.
+    """
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, Hq, d = qb.shape
+    _, Hkv, Lkv, _ = kb.shape
+    nk = -(-Lkv // Bc)
+    S = int(num_splits)
+    o = np.zeros((B, Hq, d), np.float64)
+    lse = np.zeros((B, Hq), np.float64)
+    op = np.zeros((B, Hq, S, d), np.float64)
+    lp = np.zeros((B, Hq, S), np.float64)
+    mask = np.zeros((B, Hkv, nk), np.uint8)
+    margin = np.zeros((B, Hkv, nk), np.float64)
+    counts = np.zeros(2, np.int64)
+    rc = lib.oracle_decode(
+        _ptr(qb, _u16p), _ptr(kb, _u16p), _ptr(vb, _u16p),
+        B, Hq, Hkv, Lkv, d, float(scale), float(ln_lambda), Bc, S,
+        _ptr(o, _dp), _ptr(lse, _dp), _ptr(op, _dp), _ptr(lp, _dp),
+        _ptr(mask, _u8p), _ptr(margin, _dp), _ptr(counts, _i64p),
+        int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_decode rejected its arguments")
+    threads = n_threads if n_threads > 0 else n_threads_default()
+    return dict(o=o, lse=lse, o_part=op, lse_part=lp, mask=mask,
+                margin=margin, visited=int(counts[0]),
+                skipped=int(counts[1]), threads=threads)
+
+
+def combine(o_part, lse_part):
+    """Log-sum-exp merge of split partials: o_part [n,S,d], lse_part [n,S]."""
+    lib = _load()
+    op = np.ascontiguousarray(o_part, dtype=np.float64)
+    lp = np.ascontiguousarray(lse_part, dtype=np.float64)
+    n, S, d = op.shape
+    o = np.zeros((n, d), np.float64)
+    lse = np.zeros(n, np.float64)
+    lib.oracle_combine(_ptr(op, _dp), _ptr(lp, _dp), n, S, d, _ptr(o, _dp),
+                       _ptr(lse, _dp))
+    return o, lse
+
+
+def split_begin(nk, S, s):
+    return _load().oracle_split_begin(nk, S, s)
+
+
+def sparsity(res):
+    return res["skipped"] / res["visited"] if res["visited"] else 0.0
+
+
+def lambda_fit(lambdas, lengths):
+    """Least-squares fit of lambda = a / L in log space: a = exp(mean ln(lambda*L))."""
+    vals = [math.log(lam * L) for lam, L in zip(lambdas, lengths)]
+    return math.exp(sum(vals) / len(vals))

@@ -1,0 +1,331 @@
+/*
+ * CPU oracle for the BLASST attention forward -- TEST INFRASTRUCTURE ONLY.
+ * See blasst_oracle.h for what is computed, the passages followed and the
+ * readings taken where the pages are silent.
+ *
+ * Plain loops in float64: no blocking, fusion or reordering beyond the
+ * blockwise order the algorithm itself prescribes.  OpenMP only distributes
+ * independent query tiles (prefill) or (sequence, KV head) pairs (decode)
+ * over threads; it does not change any arithmetic.
+ */
+#include "blasst_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+double oracle_bf16_to_double(uint16_t h) {
+    /* A bfloat16 is the upper half of an IEEE binary32 value. */
+    uint32_t bits = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+int oracle_split_begin(int nk, int S, int s) {
+    return (int)(((int64_t)s * nk) / S);
+}
+
+/*
+ * One query tile against KV blocks [j0, j1) of one KV head.
+ *
+ * The tile's rows are the query vectors qrows[r] (already converted to
+ * float64); row r may attend to keys 0..limit[r] (inclusive).  State m, l,
+ * acc is the blockwise online-softmax state, initialised here.
+ *
+ * Block j (keys c in [j*Bc, min((j+1)*Bc, Lkv))):
+ *   S[r][c]  = scale * q_r . k_c, or -inf when c > limit[r]
+ *   visited  = some S[r][c] is finite
+ *   mt[r]    = max_c S[r][c]                         (block-local row max)
+ *   skip     = ln_lambda > -inf and for every row:  mt[r] == -inf  or
+ *              mt[r] - m[r] < ln_lambda              (criterion, per tile)
+ *   kept     : m_new = max(m, mt); alpha = exp(m - m_new);
+ *              p = exp(S - m_new); l = alpha*l + sum p;
+ *              acc = alpha*acc + sum_c p_c v_c;  m = m_new
+ *   skipped  : no exp, no V, no P.V; m, l, acc unchanged
+ */
+static void run_tile(int nrows, const double *qrows, const int *limit,
+                     const uint16_t *kh, const uint16_t *vh, int Lkv, int d,
+                     double scale, double ln_lambda, int Bc, int j0, int j1,
+                     double *m, double *l, double *acc, uint8_t *mask,
+                     double *margin, int64_t *n_visited, int64_t *n_skipped) {
+    double *S = (double *)malloc(sizeof(double) * (size_t)nrows * Bc);
+    double *mt = (double *)malloc(sizeof(double) * (size_t)nrows);
+    double *kd = (double *)malloc(sizeof(double) * (size_t)Bc * d);
+    double *vd = (double *)malloc(sizeof(double) * (size_t)Bc * d);
+
+    for (int r = 0; r < nrows; ++r) {
+        m[r] = -INFINITY;
+        l[r] = 0.0;
+        for (int x = 0; x < d; ++x) acc[(size_t)r * d + x] = 0.0;
+    }
+
+    for (int j = j0; j < j1; ++j) {
+        int c0 = j * Bc;
+        int c1 = c0 + Bc < Lkv ? c0 + Bc : Lkv;
+        int nc = c1 - c0;
+
+        /* Is any entry of this (tile, block) pair unmasked? */
+        int visited = 0;
+        for (int r = 0; r < nrows; ++r)
+            if (limit[r] >= c0) visited = 1;
+        if (!visited) {
+            if (mask) mask[j] = ORACLE_NOT_VISITED;
+            if (margin) margin[j] = NAN;
+            continue;
+        }
+        *n_visited += 1;
+
+        /* K block, then scores and block-local row max. */
+        for (int c = 0; c < nc; ++c)
+            for (int x = 0; x < d; ++x)
+                kd[(size_t)c * d + x] =
+                    oracle_bf16_to_double(kh[(size_t)(c0 + c) * d + x]);
+        for (int r = 0; r < nrows; ++r) {
+            mt[r] = -INFINITY;
+            for (int c = 0; c < nc; ++c) {
+                double s;
+                if (c0 + c > limit[r]) {
+                    s = -INFINITY;
+                } else {
+                    double dot = 0.0;
+                    for (int x = 0; x < d; ++x)
+                        dot += qrows[(size_t)r * d + x] * kd[(size_t)c * d + x];
+                    s = scale * dot;
+                }
+                S[(size_t)r * Bc + c] = s;
+                if (s > mt[r]) mt[r] = s;
+            }
+        }
+
+        /* Skip criterion: every row's block max lies more than |ln lambda|
+         * below its running max. */
+        int skip = ln_lambda > -INFINITY;
+        double mu = -INFINITY;
+        for (int r = 0; r < nrows; ++r) {
+            if (mt[r] == -INFINITY) continue; /* fully masked row: no vote */
+            double diff = mt[r] - m[r];       /* +inf while m = -inf */
+            if (!(diff < ln_lambda)) skip = 0;
+            if (diff > mu) mu = diff;
+        }
+        if (margin) margin[j] = mu - ln_lambda;
+        if (skip) {
+            *n_skipped += 1;
+            if (mask) mask[j] = ORACLE_SKIPPED;
+            continue;
+        }
+        if (mask) mask[j] = ORACLE_KEPT;
+
+        /* Kept block: exp, V load and P.V product. */
+        for (int c = 0; c < nc; ++c)
+            for (int x = 0; x < d; ++x)
+                vd[(size_t)c * d + x] =
+                    oracle_bf16_to_double(vh[(size_t)(c0 + c) * d + x]);
+        for (int r = 0; r < nrows; ++r) {
+            if (mt[r] == -INFINITY) continue; /* p = 0, alpha = 1 */
+            double m_new = m[r] > mt[r] ? m[r] : mt[r];
+            double alpha = (m[r] == -INFINITY) ? 0.0 : exp(m[r] - m_new);
+            double psum = 0.0;
+            double *a = acc + (size_t)r * d;
+            for (int x = 0; x < d; ++x) a[x] *= alpha;
+            for (int c = 0; c < nc; ++c) {
+                double s = S[(size_t)r * Bc + c];
+                if (s == -INFINITY) continue;
+                double p = exp(s - m_new);
+                psum += p;
+                for (int x = 0; x < d; ++x) a[x] += p * vd[(size_t)c * d + x];
+            }
+            l[r] = alpha * l[r] + psum;
+            m[r] = m_new;
+        }
+    }
+    free(S);
+    free(mt);
+    free(kd);
+    free(vd);
+}
+
+static int set_threads(int n_threads) {
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+    return omp_get_max_threads();
+#else
+    (void)n_threads;
+    return 1;
+#endif
+}
+
+int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                   int B, int Hq, int Hkv, int Lq, int Lkv, int d,
+                   double scale, int causal, double ln_lambda, int Br, int Bc,
+                   int n_units, const int32_t *units,
+                   double *o, double *lse, uint8_t *mask, double *margin,
+                   int64_t *counts, int n_threads) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || Lq < 1 || Lkv < 1 ||
+        d < 1 || Br < 1 || Bc < 1 || n_units < 0 || !(ln_lambda <= 0.0))
+        return -1;
+    int nq = (Lq + Br - 1) / Br;
+    int nk = (Lkv + Bc - 1) / Bc;
+    int G = Hq / Hkv;
+    for (int u = 0; u < n_units; ++u) {
+        int b = units[3 * u], hq = units[3 * u + 1], i = units[3 * u + 2];
+        if (b < 0 || b >= B || hq < 0 || hq >= Hq || i < 0 || i >= nq)
+            return -1;
+    }
+    set_threads(n_threads);
+    int64_t vis = 0, skp = 0;
+
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : vis, skp)
+    for (int u = 0; u < n_units; ++u) {
+        int b = units[3 * u], hq = units[3 * u + 1], i = units[3 * u + 2];
+        int hkv = hq / G;
+        int r0 = i * Br;
+        int r1 = r0 + Br < Lq ? r0 + Br : Lq;
+        int nrows = r1 - r0;
+        double *qrows = (double *)malloc(sizeof(double) * (size_t)nrows * d);
+        int *limit = (int *)malloc(sizeof(int) * (size_t)nrows);
+        double *m = (double *)malloc(sizeof(double) * (size_t)nrows);
+        double *l = (double *)malloc(sizeof(double) * (size_t)nrows);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)nrows * d);
+        const uint16_t *qh = q + ((size_t)b * Hq + hq) * (size_t)Lq * d;
+        const uint16_t *kh = k + ((size_t)b * Hkv + hkv) * (size_t)Lkv * d;
+        const uint16_t *vh = v + ((size_t)b * Hkv + hkv) * (size_t)Lkv * d;
+        for (int r = 0; r < nrows; ++r) {
+            for (int x = 0; x < d; ++x)
+                qrows[(size_t)r * d + x] =
+                    oracle_bf16_to_double(qh[(size_t)(r0 + r) * d + x]);
+            int lim = Lkv - 1;
+            if (causal) {
+                int diag = r0 + r + (Lkv - Lq); /* bottom-right alignment */
+                if (diag < lim) lim = diag;
+            }
+            limit[r] = lim;
+        }
+        int64_t uv = 0, us = 0;
+        run_tile(nrows, qrows, limit, kh, vh, Lkv, d, scale, ln_lambda, Bc, 0,
+                 nk, m, l, acc, mask ? mask + (size_t)u * nk : NULL,
+                 margin ? margin + (size_t)u * nk : NULL, &uv, &us);
+        vis += uv;
+        skp += us;
+        double *ou = o + (size_t)u * Br * d;
+        double *lu = lse + (size_t)u * Br;
+        for (int r = 0; r < Br; ++r) {
+            if (r < nrows && l[r] > 0.0) {
+                for (int x = 0; x < d; ++x)
+                    ou[(size_t)r * d + x] = acc[(size_t)r * d + x] / l[r];
+                lu[r] = m[r] + log(l[r]);
+            } else {
+                for (int x = 0; x < d; ++x) ou[(size_t)r * d + x] = 0.0;
+                lu[r] = -INFINITY;
+            }
+        }
+        free(qrows);
+        free(limit);
+        free(m);
+        free(l);
+        free(acc);
+    }
+    counts[0] = vis;
+    counts[1] = skp;
+    return 0;
+}
+
+void oracle_combine(const double *o_part, const double *lse_part, int n,
+                    int S, int d, double *o, double *lse) {
+    for (int i = 0; i < n; ++i) {
+        const double *ls = lse_part + (size_t)i * S;
+        const double *os = o_part + (size_t)i * S * d;
+        double mx = -INFINITY;
+        for (int s = 0; s < S; ++s)
+            if (ls[s] > mx) mx = ls[s];
+        double *oi = o + (size_t)i * d;
+        for (int x = 0; x < d; ++x) oi[x] = 0.0;
+        if (mx == -INFINITY) {
+            lse[i] = -INFINITY;
+            continue;
+        }
+        double sum = 0.0;
+        for (int s = 0; s < S; ++s) sum += exp(ls[s] - mx);
+        double L = mx + log(sum);
+        lse[i] = L;
+        for (int s = 0; s < S; ++s) {
+            if (ls[s] == -INFINITY) continue;
+            double w = exp(ls[s] - L);
+            for (int x = 0; x < d; ++x) oi[x] += w * os[(size_t)s * d + x];
+        }
+    }
+}
+
+int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                  int B, int Hq, int Hkv, int Lkv, int d, double scale,
+                  double ln_lambda, int Bc, int num_splits,
+                  double *o, double *lse, double *o_part, double *lse_part,
+                  uint8_t *mask, double *margin, int64_t *counts,
+                  int n_threads) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || Lkv < 1 || d < 1 ||
+        Bc < 1 || num_splits < 1 || !(ln_lambda <= 0.0))
+        return -1;
+    int nk = (Lkv + Bc - 1) / Bc;
+    int G = Hq / Hkv;
+    int S = num_splits;
+    double *op = (double *)malloc(sizeof(double) * (size_t)B * Hq * S * d);
+    double *lp = (double *)malloc(sizeof(double) * (size_t)B * Hq * S);
+    set_threads(n_threads);
+    int64_t vis = 0, skp = 0;
+
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : vis, skp)
+    for (int bh = 0; bh < B * Hkv; ++bh) {
+        int b = bh / Hkv, hkv = bh % Hkv;
+        double *qrows = (double *)malloc(sizeof(double) * (size_t)G * d);
+        int *limit = (int *)malloc(sizeof(int) * (size_t)G);
+        double *m = (double *)malloc(sizeof(double) * (size_t)G);
+        double *l = (double *)malloc(sizeof(double) * (size_t)G);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)G * d);
+        for (int g = 0; g < G; ++g) {
+            const uint16_t *qg = q + ((size_t)b * Hq + hkv * G + g) * d;
+            for (int x = 0; x < d; ++x)
+                qrows[(size_t)g * d + x] = oracle_bf16_to_double(qg[x]);
+            limit[g] = Lkv - 1; /* the decode token sees the whole cache */
+        }
+        const uint16_t *kh = k + (size_t)bh * Lkv * d;
+        const uint16_t *vh = v + (size_t)bh * Lkv * d;
+        uint8_t *mk = mask ? mask + (size_t)bh * nk : NULL;
+        double *mg = margin ? margin + (size_t)bh * nk : NULL;
+        for (int s = 0; s < S; ++s) {
+            int j0 = oracle_split_begin(nk, S, s);
+            int j1 = oracle_split_begin(nk, S, s + 1);
+            int64_t uv = 0, us = 0;
+            run_tile(G, qrows, limit, kh, vh, Lkv, d, scale, ln_lambda, Bc,
+                     j0, j1, m, l, acc, mk, mg, &uv, &us);
+            vis += uv;
+            skp += us;
+            for (int g = 0; g < G; ++g) {
+                size_t row = ((size_t)b * Hq + hkv * G + g) * S + s;
+                if (l[g] > 0.0) {
+                    for (int x = 0; x < d; ++x)
+                        op[row * d + x] = acc[(size_t)g * d + x] / l[g];
+                    lp[row] = m[g] + log(l[g]);
+                } else { /* empty split */
+                    for (int x = 0; x < d; ++x) op[row * d + x] = 0.0;
+                    lp[row] = -INFINITY;
+                }
+            }
+        }
+        free(qrows);
+        free(limit);
+        free(m);
+        free(l);
+        free(acc);
+    }
+    oracle_combine(op, lp, B * Hq, S, d, o, lse);
+    if (o_part) memcpy(o_part, op, sizeof(double) * (size_t)B * Hq * S * d);
+    if (lse_part) memcpy(lse_part, lp, sizeof(double) * (size_t)B * Hq * S);
+    free(op);
+    free(lp);
+    counts[0] = vis;
+    counts[1] = skp;
+    return 0;
+}

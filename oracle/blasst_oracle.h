@@ -1,0 +1,116 @@
+/*
+ * CPU oracle for the BLASST attention forward -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Only the test suite, the smoke check and the benchmark's CPU-baseline leg
+ * may load or call this code.  The product library never links it and shares
+ * no code with it.
+ *
+ * What it computes: the blockwise online-softmax attention forward with the
+ * BLASST skip rule, written out step by step in float64 so that a reader can
+ * check each step against the method's description:
+ *
+ *   - running row max m and normaliser l, rescaled when m grows
+ *     ("BLASST: Dynamic BLocked Attention Sparsity via Softmax Thresholding",
+ *      gist.science summary, section 2 "Estatisticas Online");
+ *   - block j is negligible for row i when  m~_i(j) - m_i(j) < ln(lambda)
+ *     (same page, section 2 "Criterio de Pulo"; Hindi summary, section 2
+ *      "Core Insight");
+ *   - a negligible block costs no exp, no V load and no P.V product
+ *     (same pages, section 2 "Acoes de Otimizacao");
+ *   - the decision is taken per block for the whole query tile
+ *     (MLSys'26 reading notes, "design trade-offs": block skip vs token skip).
+ *
+ * Readings of points the pages leave open (documented in the design notes):
+ *   - m is the running max over blocks before j (identical decisions to the
+ *     after-update reading whenever ln(lambda) <= 0);
+ *   - strict '<';
+ *   - a tile skips block j only if EVERY row satisfies the criterion; a row
+ *     whose entries in block j are all masked satisfies it trivially;
+ *   - the first visited block (m = -inf) is never skipped;
+ *   - a (tile, block) pair whose entries are all masked is not visited;
+ *   - causal masking is bottom-right aligned: key c is visible to query r
+ *     iff c <= r + (Lkv - Lq);
+ *   - GQA: query head hq reads KV head hq / (Hq / Hkv);
+ *   - decode split-KV: each split runs the algorithm independently
+ *     (m restarts at -inf) over blocks [floor(s*nk/S), floor((s+1)*nk/S)),
+ *     then the partials are merged by log-sum-exp;
+ *   - lse is the natural-log normaliser of the kept entries, m + ln l.
+ *
+ * Tensors are row-major, innermost dimension last:
+ *   prefill q [B,Hq,Lq,d], k/v [B,Hkv,Lkv,d]; decode q [B,Hq,d],
+ *   k/v [B,Hkv,Lkv,d].  Inputs are raw bfloat16 bit patterns (uint16).
+ */
+#ifndef BLASST_ORACLE_H
+#define BLASST_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Decision codes written to the per-(tile, block) mask. */
+#define ORACLE_NOT_VISITED 0
+#define ORACLE_KEPT 1
+#define ORACLE_SKIPPED 2
+
+/* bfloat16 bit pattern -> value (exact). */
+double oracle_bf16_to_double(uint16_t h);
+
+/*
+ * Prefill forward for a list of query tiles.
+ *
+ * units:  n_units triples (b, hq, i); tile i covers query rows
+ *         [i*Br, min((i+1)*Br, Lq)).
+ * o:      [n_units][Br][d]   normalised output (rows past Lq are left 0)
+ * lse:    [n_units][Br]      m + ln l (natural log); -inf for rows past Lq
+ * mask:   [n_units][nk]      ORACLE_* decision per KV block (may be NULL)
+ * margin: [n_units][nk]      max_r(m~_r - m_r) - ln_lambda for visited
+ *                            pairs (+inf for the first visited block, NaN
+ *                            for pairs not visited) (may be NULL)
+ * counts: [2]                visited and skipped pairs, summed over units
+ * ln_lambda = -INFINITY gives the dense forward.
+ * Returns 0, or -1 on invalid arguments.
+ */
+int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                   int B, int Hq, int Hkv, int Lq, int Lkv, int d,
+                   double scale, int causal, double ln_lambda, int Br, int Bc,
+                   int n_units, const int32_t *units,
+                   double *o, double *lse, uint8_t *mask, double *margin,
+                   int64_t *counts, int n_threads);
+
+/*
+ * Decode forward: one query token per sequence, the G = Hq/Hkv query heads
+ * of a KV head form the rows of one tile.
+ *
+ * o:        [B,Hq,d]     merged output
+ * lse:      [B,Hq]       merged log-sum-exp
+ * o_part:   [B,Hq,S,d]   per-split normalised output (may be NULL)
+ * lse_part: [B,Hq,S]     per-split lse, -inf for an empty split (may be NULL)
+ * mask:     [B,Hkv,nk]   ORACLE_* decision per block (may be NULL)
+ * margin:   [B,Hkv,nk]   as for prefill (may be NULL)
+ * counts:   [2]          visited and skipped (b, hkv, block) triples
+ */
+int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                  int B, int Hq, int Hkv, int Lkv, int d, double scale,
+                  double ln_lambda, int Bc, int num_splits,
+                  double *o, double *lse, double *o_part, double *lse_part,
+                  uint8_t *mask, double *margin, int64_t *counts,
+                  int n_threads);
+
+/*
+ * Log-sum-exp merge of S partial results for n rows:
+ *   lse = ln sum_s exp(lse_s),  o = sum_s exp(lse_s - lse) * o_s.
+ * o_part [n][S][d], lse_part [n][S]; o [n][d], lse [n].
+ */
+void oracle_combine(const double *o_part, const double *lse_part, int n,
+                    int S, int d, double *o, double *lse);
+
+/* First block of split s when nk blocks are divided into S splits. */
+int oracle_split_begin(int nk, int S, int s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif
