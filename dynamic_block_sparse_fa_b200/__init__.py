@@ -1,0 +1,17 @@
+"""BLASST attention forward for NVIDIA B200 (sm_100a).
+
+The kernels live in libblasst.so (C ABI: include/blasst.h); this package is
+its Python binding.  Importing it loads the library and fails if it has not
+been built (``python -m dynamic_block_sparse_fa_b200.build``).
+"""
+from .blasst import (BlasstError, Stats, blasst_calibrate,
+                     blasst_check_device_error, blasst_decode,
+                     blasst_decode_splits, blasst_decode_workspace_size,
+                     blasst_fit_a, blasst_last_error, blasst_prefill,
+                     blasst_skip_stats_reset, blasst_strerror, blasst_version)
+
+__all__ = ["BlasstError", "Stats", "blasst_calibrate",
+           "blasst_check_device_error", "blasst_decode", "blasst_decode_splits",
+           "blasst_decode_workspace_size", "blasst_fit_a", "blasst_last_error",
+           "blasst_prefill", "blasst_skip_stats_reset", "blasst_strerror",
+           "blasst_version"]

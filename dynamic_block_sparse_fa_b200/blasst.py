@@ -1,0 +1,277 @@
+"""Thin ctypes binding of libblasst.so (include/blasst.h).
+
+Argument marshalling only: every function forwards to the C entry point of
+the same name, passing torch tensors as device pointers and the current
+CUDA stream.  Outputs the caller does not provide are allocated with torch
+(device memory plumbing); all computation runs in the library's kernels.
+There is no fallback: if the library is missing, importing this module
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libblasst.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with "
+        "`python -m dynamic_block_sparse_fa_b200.build` (needs nvcc)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+BLASST_OK = 0
+_STATUS = {
+    0: "BLASST_OK", 1: "BLASST_ERR_INVALID_ARG",
+    2: "BLASST_ERR_UNSUPPORTED_SHAPE", 3: "BLASST_ERR_MISALIGNED",
+    4: "BLASST_ERR_CUDA", 5: "BLASST_ERR_TIMEOUT",
+    6: "BLASST_ERR_NO_CONVERGE", 7: "BLASST_ERR_WORKSPACE",
+}
+
+
+class BlasstError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.blasst_strerror(status).decode()
+        detail = _lib.blasst_last_error().decode()
+        super().__init__(f"{where}: {_STATUS.get(status, status)} ({msg})"
+                         + (f": {detail}" if detail and status == 4 else ""))
+
+
+class SkipStats(ctypes.Structure):
+    """Host struct of device pointers (blasst_skip_stats_t)."""
+    _fields_ = [("counters", ctypes.c_void_p), ("mask", ctypes.c_void_p)]
+
+
+class CalibSample(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int), ("q", ctypes.c_void_p),
+                ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("Hq", ctypes.c_int),
+                ("Hkv", ctypes.c_int), ("Lq", ctypes.c_int),
+                ("Lkv", ctypes.c_int), ("d", ctypes.c_int),
+                ("scale", ctypes.c_float), ("causal", ctypes.c_int),
+                ("Br", ctypes.c_int), ("Bc", ctypes.c_int),
+                ("num_splits", ctypes.c_int)]
+
+
+class CalibResult(ctypes.Structure):
+    _fields_ = [("ln_lambda", ctypes.c_double), ("lambda_", ctypes.c_double),
+                ("a", ctypes.c_double), ("achieved", ctypes.c_double),
+                ("L", ctypes.c_int), ("iterations", ctypes.c_int),
+                ("visited", ctypes.c_ulonglong),
+                ("skipped", ctypes.c_ulonglong)]
+
+
+_vp, _i, _f, _d, _sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float,
+                        ctypes.c_double, ctypes.c_size_t)
+_lib.blasst_prefill.restype = _i
+_lib.blasst_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                _i, _f, _i, _f, _i, _i,
+                                ctypes.POINTER(SkipStats), _vp]
+_lib.blasst_decode.restype = _i
+_lib.blasst_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                               _f, _f, _i, _i, _vp, _sz,
+                               ctypes.POINTER(SkipStats), _vp]
+_lib.blasst_decode_workspace_size.restype = _sz
+_lib.blasst_decode_workspace_size.argtypes = [_i, _i, _i, _i]
+_lib.blasst_decode_splits.restype = _i
+_lib.blasst_decode_splits.argtypes = [_i, _i, _i, _i]
+_lib.blasst_calibrate.restype = _i
+_lib.blasst_calibrate.argtypes = [_d, ctypes.POINTER(CalibSample), _d, _vp,
+                                  ctypes.POINTER(CalibResult), _vp]
+_lib.blasst_fit_a.restype = _d
+_lib.blasst_fit_a.argtypes = [_i, ctypes.POINTER(_d), ctypes.POINTER(_i)]
+_lib.blasst_skip_stats_reset.restype = _i
+_lib.blasst_skip_stats_reset.argtypes = [_vp, _vp]
+_lib.blasst_check_device_error.restype = _i
+_lib.blasst_check_device_error.argtypes = [ctypes.POINTER(_i)]
+_lib.blasst_strerror.restype = ctypes.c_char_p
+_lib.blasst_strerror.argtypes = [_i]
+_lib.blasst_last_error.restype = ctypes.c_char_p
+_lib.blasst_last_error.argtypes = []
+_lib.blasst_version.restype = ctypes.c_char_p
+_lib.blasst_version.argtypes = []
+
+EXPORTED = ["blasst_prefill", "blasst_decode", "blasst_decode_workspace_size",
+            "blasst_decode_splits", "blasst_calibrate", "blasst_fit_a",
+            "blasst_skip_stats_reset", "blasst_check_device_error",
+            "blasst_strerror", "blasst_last_error", "blasst_version"]
+
+
+def _check(status, where):
+    if status != BLASST_OK:
+        raise BlasstError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class Stats:
+    """Device skip counters (uint64[2]: visited, skipped) and an optional
+    per-(tile, block) decision mask, allocated with torch."""
+
+    def __init__(self, device="cuda", mask_numel: int = 0):
+        self.counters = torch.zeros(2, dtype=torch.int64, device=device)
+        self.mask = (torch.zeros(mask_numel, dtype=torch.uint8, device=device)
+                     if mask_numel else None)
+        self._c = SkipStats(self.counters.data_ptr(),
+                            self.mask.data_ptr() if self.mask is not None else None)
+
+    @property
+    def c_struct(self):
+        return ctypes.byref(self._c)
+
+    def reset(self, stream=None):
+        blasst_skip_stats_reset(self.counters, stream)
+        if self.mask is not None:
+            self.mask.zero_()
+
+    def read(self):
+        v, s = (int(x) for x in self.counters.tolist())
+        return v, s
+
+    def sparsity(self):
+        v, s = self.read()
+        return s / v if v else 0.0
+
+
+def blasst_version() -> str:
+    return _lib.blasst_version().decode()
+
+
+def blasst_strerror(status: int) -> str:
+    return _lib.blasst_strerror(status).decode()
+
+
+def blasst_last_error() -> str:
+    return _lib.blasst_last_error().decode()
+
+
+def blasst_skip_stats_reset(counters: torch.Tensor, stream=None):
+    _check(_lib.blasst_skip_stats_reset(_ptr(counters), _stream(stream)),
+           "blasst_skip_stats_reset")
+
+
+def blasst_check_device_error():
+    """Returns (status, where): status 0 or BLASST_ERR_TIMEOUT (5)."""
+    where = ctypes.c_int(0)
+    st = _lib.blasst_check_device_error(ctypes.byref(where))
+    if st not in (0, 5):
+        _check(st, "blasst_check_device_error")
+    return st, where.value
+
+
+def blasst_prefill(q, k, v, *, scale=None, causal=True, ln_lambda=-math.inf,
+                   Br=128, Bc=128, o=None, lse=None, want_lse=True,
+                   stats: Stats | None = None, stats_only=False, stream=None):
+    """BLASST prefill forward.  q [B,Hq,Lq,d], k/v [B,Hkv,Lkv,d] bf16 CUDA.
+
+    Returns (o, lse); both None when stats_only (decisions and counters
+    only)."""
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if not stats_only:
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and want_lse:
+            lse = torch.empty(B, Hq, Lq, dtype=torch.float32, device=q.device)
+    else:
+        o, lse = None, None
+    st = _lib.blasst_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lkv, d,
+        float(scale), int(bool(causal)), float(ln_lambda), Br, Bc,
+        stats.c_struct if stats is not None else None, _stream(stream))
+    _check(st, "blasst_prefill")
+    return o, lse
+
+
+def blasst_decode_workspace_size(B, Hq, d, num_splits) -> int:
+    return int(_lib.blasst_decode_workspace_size(B, Hq, d, num_splits))
+
+
+def blasst_decode_splits(B, Hkv, Lkv, Bc=64) -> int:
+    return int(_lib.blasst_decode_splits(B, Hkv, Lkv, Bc))
+
+
+def blasst_decode(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
+                  num_splits=0, o=None, lse=None, want_lse=True,
+                  workspace=None, stats: Stats | None = None,
+                  stats_only=False, stream=None):
+    """BLASST decode forward.  q [B,Hq,d], k/v [B,Hkv,Lkv,d] bf16 CUDA.
+
+    Returns (o, lse); both None when stats_only."""
+    B, Hq, d = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    S = num_splits if num_splits > 0 else blasst_decode_splits(B, Hkv, Lkv, Bc)
+    ws_bytes = 0
+    if not stats_only:
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and want_lse:
+            lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+        need = blasst_decode_workspace_size(B, Hq, d, S)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    else:
+        o, lse, workspace = None, None, None
+    st = _lib.blasst_decode(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lkv, d,
+        float(scale), float(ln_lambda), Bc, S, _ptr(workspace), ws_bytes,
+        stats.c_struct if stats is not None else None, _stream(stream))
+    _check(st, "blasst_decode")
+    return o, lse
+
+
+def blasst_calibrate(target, *, mode, q, k, v, scale=None, causal=True,
+                     Br=128, Bc=128, num_splits=0, tol=0.002,
+                     counters=None, stream=None, raise_on_no_converge=True):
+    """Bisection of ln(lambda) until the sample's sparsity reaches `target`.
+
+    mode 'prefill' (q [B,Hq,Lq,d]) or 'decode' (q [B,Hq,d]).  Returns a dict
+    with ln_lambda, lambda, a (= lambda * Lkv), achieved, L, iterations,
+    visited, skipped, status."""
+    m = {"prefill": 0, "decode": 1}[mode]
+    d = q.shape[-1]
+    B, Hq = q.shape[0], q.shape[1]
+    Lq = q.shape[2] if m == 0 else 1
+    _, Hkv, Lkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if counters is None:
+        counters = torch.zeros(2, dtype=torch.int64, device=q.device)
+    smp = CalibSample(m, q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv,
+                      Lq, Lkv, d, float(scale), int(bool(causal)), Br, Bc,
+                      num_splits)
+    res = CalibResult()
+    st = _lib.blasst_calibrate(float(target), ctypes.byref(smp), float(tol),
+                               _ptr(counters), ctypes.byref(res),
+                               _stream(stream))
+    if st != BLASST_OK and (st != 6 or raise_on_no_converge):
+        _check(st, "blasst_calibrate")
+    return dict(ln_lambda=res.ln_lambda, lambda_=res.lambda_, a=res.a,
+                achieved=res.achieved, L=res.L, iterations=res.iterations,
+                visited=res.visited, skipped=res.skipped, status=st)
+
+
+def blasst_fit_a(lambdas, lengths) -> float:
+    n = len(lambdas)
+    la = (ctypes.c_double * n)(*lambdas)
+    le = (ctypes.c_int * n)(*lengths)
+    return float(_lib.blasst_fit_a(n, la, le))

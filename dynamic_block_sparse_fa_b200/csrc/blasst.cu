@@ -1,0 +1,337 @@
+// blasst.cu -- the C ABI declared in include/blasst.h: argument validation,
+// launch configuration, the calibration search and the error plumbing.
+// Kernels live in decode.cuh / prefill.cuh; this is one translation unit so
+// that the device error word is a single symbol.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "blasst.h"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+blasst_status_t cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return BLASST_OK;
+  snprintf(g_last_error, sizeof g_last_error, "%s: %s", what,
+           cudaGetErrorString(e));
+  return BLASST_ERR_CUDA;
+}
+
+bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+bool valid_ln_lambda(float x) { return x <= 0.0f; }  // false for NaN, > 0
+
+constexpr int kNumSmB200 = 148;
+
+}  // namespace
+
+extern "C" {
+
+const char* blasst_version(void) { return "0.1.0"; }
+
+const char* blasst_last_error(void) { return g_last_error; }
+
+const char* blasst_strerror(blasst_status_t s) {
+  switch (s) {
+    case BLASST_OK: return "ok";
+    case BLASST_ERR_INVALID_ARG: return "invalid argument";
+    case BLASST_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case BLASST_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case BLASST_ERR_CUDA: return "CUDA error";
+    case BLASST_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    case BLASST_ERR_NO_CONVERGE: return "calibration did not reach the target";
+    case BLASST_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+blasst_status_t blasst_skip_stats_reset(unsigned long long* counters,
+                                        void* stream) {
+  if (!counters) return BLASST_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(counters, 0, 2 * sizeof(unsigned long long),
+                                     (cudaStream_t)stream),
+                     "cudaMemsetAsync(counters)");
+}
+
+blasst_status_t blasst_check_device_error(int* where_out) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_status(e, "cudaDeviceSynchronize");
+  unsigned int code = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&code, blasst::g_error_code, sizeof code);
+  if (e != cudaSuccess) return cuda_status(e, "read error word");
+  if (where_out) *where_out = (int)code;
+  if (code == 0) return BLASST_OK;
+  cudaMemcpyToSymbol(blasst::g_error_code, &zero, sizeof zero);
+  cudaMemcpyToSymbol(blasst::g_error_count, &zero, sizeof zero);
+  return BLASST_ERR_TIMEOUT;
+}
+
+// ---------------------------------------------------------------------------
+// Decode
+// ---------------------------------------------------------------------------
+int blasst_decode_splits(int B, int Hkv, int Lkv, int Bc) {
+  if (B < 1 || Hkv < 1 || Lkv < 1 || Bc < 1) return 1;
+  const long long nk = (Lkv + (long long)Bc - 1) / Bc;
+  const long long units = (long long)B * Hkv;
+  // About four waves of two resident CTAs per SM on a 148-SM B200, with at
+  // least 8 blocks per split.
+  const long long target = (long long)kNumSmB200 * 2 * 4;
+  long long s = (target + units - 1) / units;
+  if (s > nk / 8) s = nk / 8;
+  if (s < 1) s = 1;
+  return (int)s;
+}
+
+size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits) {
+  if (B < 1 || Hq < 1 || d < 1 || num_splits < 1) return 0;
+  const size_t rows = (size_t)B * Hq * num_splits;
+  const size_t o_bytes = (rows * d * sizeof(float) + 255) & ~(size_t)255;
+  const size_t l_bytes = (rows * sizeof(float) + 255) & ~(size_t)255;
+  return o_bytes + l_bytes;
+}
+
+blasst_status_t blasst_decode(const void* q, const void* k_cache,
+                              const void* v_cache, void* o, float* lse, int B,
+                              int Hq, int Hkv, int Lkv, int d, float scale,
+                              float ln_lambda, int Bc, int num_splits,
+                              void* workspace, size_t workspace_bytes,
+                              const blasst_skip_stats_t* skip_stats,
+                              void* stream) {
+  if (!q || !k_cache || !v_cache) return BLASST_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lkv < 1 || Hq % Hkv != 0)
+    return BLASST_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !valid_ln_lambda(ln_lambda))
+    return BLASST_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (d != blasst::kDecD || Bc != blasst::kDecBc ||
+      !(G == 1 || G == 2 || G == 4 || G == 8))
+    return BLASST_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (o && !aligned16(o)))
+    return BLASST_ERR_MISALIGNED;
+  const int nk = (Lkv + Bc - 1) / Bc;
+  const int S = num_splits == 0 ? blasst_decode_splits(B, Hkv, Lkv, Bc)
+                                : num_splits;
+  if (S < 1 || S > nk) return BLASST_ERR_INVALID_ARG;
+  const long long grid = (long long)B * Hkv * S;
+  if (grid > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED_SHAPE;
+  const bool stats_only = (o == nullptr);
+  float* o_part = nullptr;
+  float* lse_part = nullptr;
+  if (!stats_only) {
+    const size_t need = blasst_decode_workspace_size(B, Hq, d, S);
+    if (!workspace || workspace_bytes < need) return BLASST_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return BLASST_ERR_MISALIGNED;
+    const size_t rows = (size_t)B * Hq * S;
+    o_part = static_cast<float*>(workspace);
+    lse_part = reinterpret_cast<float*>(
+        static_cast<char*>(workspace) +
+        ((rows * d * sizeof(float) + 255) & ~(size_t)255));
+  }
+  blasst::DecodeArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k_cache);
+  a.v = static_cast<const __nv_bfloat16*>(v_cache);
+  a.o_part = o_part;
+  a.lse_part = lse_part;
+  a.counters = skip_stats ? skip_stats->counters : nullptr;
+  a.mask = skip_stats ? skip_stats->mask : nullptr;
+  a.Hkv = Hkv;
+  a.Lkv = Lkv;
+  a.nk = nk;
+  a.S = S;
+  a.scale = scale;
+  a.ln_lambda = ln_lambda;
+  a.stats_only = stats_only ? 1 : 0;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  switch (G) {
+#define BLASST_LAUNCH_DECODE(GG)                                               \
+  case GG: {                                                                   \
+    const int smem = blasst::DecodeSmem<GG>::kTotal;                           \
+    e = cudaFuncSetAttribute(blasst::decode_split_kernel<GG>,                  \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,      \
+                             smem);                                            \
+    if (e == cudaSuccess)                                                      \
+      blasst::decode_split_kernel<GG>                                          \
+          <<<(unsigned)grid, blasst::kDecThreads, smem, st>>>(a);              \
+    break;                                                                     \
+  }
+    BLASST_LAUNCH_DECODE(1)
+    BLASST_LAUNCH_DECODE(2)
+    BLASST_LAUNCH_DECODE(4)
+    BLASST_LAUNCH_DECODE(8)
+#undef BLASST_LAUNCH_DECODE
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "decode split launch");
+  if (stats_only) return BLASST_OK;
+
+  // Merge, launched as a programmatic dependent of the split kernel so its
+  // launch overlaps the split kernel's tail (it waits on griddepcontrol).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(B * Hq));
+  cfg.blockDim = dim3(blasst::kDecD);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, blasst::decode_combine_kernel,
+                         (const float*)o_part, (const float*)lse_part,
+                         static_cast<__nv_bfloat16*>(o), lse, S);
+  return cuda_status(e, "decode merge launch");
+}
+
+// ---------------------------------------------------------------------------
+// Prefill
+// ---------------------------------------------------------------------------
+blasst_status_t blasst_prefill(const void* q, const void* k, const void* v,
+                               void* o, float* lse, int B, int Hq, int Hkv,
+                               int Lq, int Lkv, int d, float scale, int causal,
+                               float ln_lambda, int Br, int Bc,
+                               const blasst_skip_stats_t* skip_stats,
+                               void* stream) {
+  if (!q || !k || !v) return BLASST_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lkv < 1 || Hq % Hkv != 0)
+    return BLASST_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !valid_ln_lambda(ln_lambda))
+    return BLASST_ERR_INVALID_ARG;
+  if (causal && Lq > Lkv) return BLASST_ERR_INVALID_ARG;
+  if (!((d == 64 || d == 128) &&
+        ((Br == 64 && Bc == 64) || (Br == 128 && Bc == 128))))
+    return BLASST_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (o && !aligned16(o)))
+    return BLASST_ERR_MISALIGNED;
+  blasst::PrefillProblem p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Lq = Lq;
+  p.Lkv = Lkv;
+  p.d = d;
+  p.scale = scale;
+  p.causal = causal ? 1 : 0;
+  p.ln_lambda = ln_lambda;
+  p.Br = Br;
+  p.Bc = Bc;
+  p.counters = skip_stats ? skip_stats->counters : nullptr;
+  p.mask = skip_stats ? skip_stats->mask : nullptr;
+  cudaError_t e = blasst::launch_prefill(p, static_cast<cudaStream_t>(stream));
+  return cuda_status(e, "prefill launch");
+}
+
+// ---------------------------------------------------------------------------
+// Calibration
+// ---------------------------------------------------------------------------
+namespace {
+
+blasst_status_t sparsity_at(const blasst_calib_sample_t* s, double ln_lambda,
+                            unsigned long long* counters, cudaStream_t st,
+                            unsigned long long* vis, unsigned long long* skp) {
+  blasst_status_t rc = blasst_skip_stats_reset(counters, st);
+  if (rc != BLASST_OK) return rc;
+  blasst_skip_stats_t stats = {counters, nullptr};
+  const float lnl = (float)ln_lambda;
+  if (s->mode == 0) {
+    rc = blasst_prefill(s->q, s->k, s->v, nullptr, nullptr, s->B, s->Hq,
+                        s->Hkv, s->Lq, s->Lkv, s->d, s->scale, s->causal, lnl,
+                        s->Br, s->Bc, &stats, st);
+  } else {
+    rc = blasst_decode(s->q, s->k, s->v, nullptr, nullptr, s->B, s->Hq, s->Hkv,
+                       s->Lkv, s->d, s->scale, lnl, s->Bc, s->num_splits,
+                       nullptr, 0, &stats, st);
+  }
+  if (rc != BLASST_OK) return rc;
+  unsigned long long h[2] = {0, 0};
+  cudaError_t e = cudaMemcpyAsync(h, counters, sizeof h, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_status(e, "calibration counters");
+  *vis = h[0];
+  *skp = h[1];
+  return BLASST_OK;
+}
+
+}  // namespace
+
+blasst_status_t blasst_calibrate(double target, const blasst_calib_sample_t* s,
+                                 double tol, unsigned long long* counters_dev,
+                                 blasst_calib_result_t* out, void* stream) {
+  if (!s || !out || !counters_dev || !(target >= 0.0 && target < 1.0) ||
+      !(tol >= 0.0) || (s->mode != 0 && s->mode != 1))
+    return BLASST_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  memset(out, 0, sizeof *out);
+  out->L = s->Lkv;
+  // s(ln_lambda) is a non-decreasing step function.  Keep lo with s < target
+  // and hi with s >= target; return hi.
+  double lo = -64.0, hi = 0.0;
+  unsigned long long v_hi = 0, k_hi = 0, v_lo = 0, k_lo = 0;
+  blasst_status_t rc = sparsity_at(s, hi, counters_dev, st, &v_hi, &k_hi);
+  int it = 1;
+  if (rc != BLASST_OK) return rc;
+  double s_hi = v_hi ? (double)k_hi / (double)v_hi : 0.0;
+  auto fill = [&](double lnl, unsigned long long vv, unsigned long long kk) {
+    out->ln_lambda = lnl;
+    out->lambda = std::exp(lnl);
+    out->a = out->lambda * (double)s->Lkv;
+    out->visited = vv;
+    out->skipped = kk;
+    out->achieved = vv ? (double)kk / (double)vv : 0.0;
+    out->iterations = it;
+  };
+  if (s_hi < target) {  // even ln(lambda) = 0 does not reach the target
+    fill(hi, v_hi, k_hi);
+    return BLASST_ERR_NO_CONVERGE;
+  }
+  rc = sparsity_at(s, lo, counters_dev, st, &v_lo, &k_lo);
+  ++it;
+  if (rc != BLASST_OK) return rc;
+  const double s_lo = v_lo ? (double)k_lo / (double)v_lo : 0.0;
+  if (s_lo >= target) {  // target reached everywhere (e.g. target 0)
+    fill(lo, v_lo, k_lo);
+    return BLASST_OK;
+  }
+  while (hi - lo > 1e-6 && s_hi - target > tol && it < 100) {
+    const double mid = 0.5 * (lo + hi);
+    unsigned long long vv = 0, kk = 0;
+    rc = sparsity_at(s, mid, counters_dev, st, &vv, &kk);
+    ++it;
+    if (rc != BLASST_OK) return rc;
+    const double sm = vv ? (double)kk / (double)vv : 0.0;
+    if (sm >= target) {
+      hi = mid;
+      s_hi = sm;
+      v_hi = vv;
+      k_hi = kk;
+    } else {
+      lo = mid;
+    }
+  }
+  fill(hi, v_hi, k_hi);
+  return BLASST_OK;
+}
+
+double blasst_fit_a(int n, const double* lambdas, const int* lengths) {
+  if (n < 1 || !lambdas || !lengths) return NAN;
+  double acc = 0.0;
+  for (int i = 0; i < n; ++i) acc += std::log(lambdas[i] * (double)lengths[i]);
+  return std::exp(acc / n);
+}
+
+}  // extern "C"

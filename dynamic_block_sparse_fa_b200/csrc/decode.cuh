@@ -1,0 +1,455 @@
+// decode.cuh -- BLASST decode forward: one query token per sequence against a
+// contiguous bf16 KV cache, split-KV, GQA head packing, V read only for kept
+// blocks, then a log-sum-exp merge of the splits.
+//
+// Method: "BLASST: Dynamic BLocked Attention Sparsity via Softmax
+// Thresholding" (gist.science summary, section 2 "Criterio de Pulo" and
+// "Acoes de Otimizacao"; section 3: in the memory-bound decode the saving is
+// the V blocks never loaded from HBM).  The Hindi summary (section 2, kernel
+// optimisation) notes that conditional V loads cause pipeline bubbles unless
+// several Q.K products are scored before deciding which V blocks to fetch;
+// here K runs a fixed number of blocks ahead of the decisions and the P.V
+// product of a kept block runs a fixed number of kept blocks behind its V
+// load, so the loads of the decided blocks are in flight while later blocks
+// are scored.  The decision for block j still uses the running max over the
+// blocks before j (the order of the blockwise algorithm is unchanged).
+//
+// One CTA of 128 threads per (sequence b, KV head, split).  The G query
+// heads of the KV head are the rows of the tile: every K and V byte fetched
+// serves G heads.  K and V blocks (Bc = 64 keys x d = 128 = 16 KB, contiguous
+// in the cache) arrive through bulk asynchronous copies into shared memory
+// and are read back with 128-bit shared loads.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace blasst {
+
+struct DecodeArgs {
+  const __nv_bfloat16* q;  // [B, Hq, D]
+  const __nv_bfloat16* k;  // [B, Hkv, Lkv, D]
+  const __nv_bfloat16* v;  // [B, Hkv, Lkv, D]
+  float* o_part;           // [B*Hq, S, D]  normalised split outputs
+  float* lse_part;         // [B*Hq, S]
+  unsigned long long* counters;  // [2] visited, skipped (may be null)
+  unsigned char* mask;           // [B*Hkv, nk] (may be null)
+  int Hkv, Lkv, nk, S;
+  float scale, ln_lambda;
+  int stats_only;
+};
+
+constexpr int kDecD = 128;       // head dimension
+constexpr int kDecBc = 64;       // keys per block
+constexpr int kDecThreads = 128;
+constexpr int kDecNK = 3;        // K blocks in flight ahead of the scoring
+constexpr int kDecNV = 3;        // V block slots
+constexpr int kDecLag = 2;       // P.V of kept block n runs when n+Lag+1 are issued
+static_assert(kDecNV >= kDecLag + 1, "V ring must cover the lag");
+constexpr int kDecBlockBytes = kDecBc * kDecD * 2;  // 16 KB
+constexpr int kDecRowBytes = kDecD * 2;             // 256 B per key
+
+template <int G>
+struct DecodeSmem {
+  static constexpr int kK = 0;                                    // [NK][Bc][D] bf16
+  static constexpr int kV = kK + kDecNK * kDecBlockBytes;          // [NV][Bc][D] bf16
+  static constexpr int kP = kV + kDecNV * kDecBlockBytes;          // [NV][Bc][G] f32
+  static constexpr int kS = kP + kDecNV * kDecBc * G * 4;          // [2][G][Bc] f32
+  static constexpr int kM = kS + 2 * G * kDecBc * 4;               // [8] f32
+  static constexpr int kA = kM + 8 * 4;                            // [NV][8] f32
+  static constexpr int kL = kA + kDecNV * 8 * 4;                   // [8] f32
+  static constexpr int kNV = kL + 8 * 4;                           // [NV] int
+  static constexpr int kBar = (kNV + kDecNV * 4 + 15) & ~15;       // [NK+NV] u64
+  static constexpr int kTotal = kBar + (kDecNK + kDecNV) * 8;
+  // The end-of-split reduction [8 key groups][G][D] f32 reuses the K ring.
+  static_assert(8 * G * kDecD * 4 <= kDecNK * kDecBlockBytes, "reduction fits");
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Sum over the 8 lanes that share a key (lane bits 0..2) of G partial dot
+// products.  While more than one value is held, each exchange step keeps half
+// of the values and sends the other half, so the lane ends up holding the
+// full sum of head  head_of_lane<G>(lane).
+template <int G>
+__device__ __forceinline__ float reduce8_transpose(float (&v)[G], int lane) {
+  float x[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) x[g] = v[g];
+  int n = G;
+#pragma unroll
+  for (int msk = 4; msk >= 1; msk >>= 1) {
+    if (n > 1) {
+      const int h = n / 2;
+      const bool upper = (lane & msk) != 0;
+#pragma unroll
+      for (int i = 0; i < G / 2; ++i) {
+        if (i < h) {
+          float send = upper ? x[i] : x[i + h];
+          float keep = upper ? x[i + h] : x[i];
+          x[i] = keep + __shfl_xor_sync(0xffffffffu, send, msk);
+        }
+      }
+      n = h;
+    } else {
+      x[0] += __shfl_xor_sync(0xffffffffu, x[0], msk);
+    }
+  }
+  return x[0];
+}
+
+template <int G>
+__device__ __forceinline__ int head_of_lane(int lane) {
+  int h = 0, n = G;
+#pragma unroll
+  for (int msk = 4; msk >= 1; msk >>= 1) {
+    if (n > 1) {
+      n /= 2;
+      if (lane & msk) h += n;
+    }
+  }
+  return h;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kDecThreads, 2)
+    decode_split_kernel(const DecodeArgs a) {
+  using L = DecodeSmem<G>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+
+  const int s = blockIdx.x % a.S;
+  const int bh = blockIdx.x / a.S;  // b * Hkv + hkv
+  const int j0 = (int)(((long long)s * a.nk) / a.S);
+  const int j1 = (int)(((long long)(s + 1) * a.nk) / a.S);
+  const int nblk = j1 - j0;
+  const int Hq = a.Hkv * G;
+  const int b = bh / a.Hkv;
+  const int hkv = bh - b * a.Hkv;
+
+  uint8_t* sK = smem + L::kK;
+  uint8_t* sV = smem + L::kV;
+  float* sP = reinterpret_cast<float*>(smem + L::kP);
+  float* sS = reinterpret_cast<float*>(smem + L::kS);
+  float* sM = reinterpret_cast<float*>(smem + L::kM);
+  float* sA = reinterpret_cast<float*>(smem + L::kA);
+  float* sL = reinterpret_cast<float*>(smem + L::kL);
+  int* sNV = reinterpret_cast<int*>(smem + L::kNV);
+  uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* vfull = kfull + kDecNK;
+
+  const __nv_bfloat16* kbase = a.k + (size_t)bh * a.Lkv * kDecD;
+  const __nv_bfloat16* vbase = a.v + (size_t)bh * a.Lkv * kDecD;
+  const uint64_t pol = policy_evict_first();
+
+  if (tid == 0) {
+    for (int i = 0; i < kDecNK; ++i) mbar_init(&kfull[i], 1);
+    for (int i = 0; i < kDecNV; ++i) mbar_init(&vfull[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  auto rows_of = [&](int j) { return min(kDecBc, a.Lkv - j * kDecBc); };
+  auto issue_k = [&](int r) {
+    const int j = j0 + r;
+    const uint32_t bytes = (uint32_t)rows_of(j) * kDecRowBytes;
+    uint64_t* bar = &kfull[r % kDecNK];
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(sK + (r % kDecNK) * kDecBlockBytes,
+              kbase + (size_t)j * kDecBc * kDecD, bytes, bar, pol);
+  };
+  if (tid == 0) {
+    const int n0 = nblk < kDecNK ? nblk : kDecNK;
+    for (int r = 0; r < n0; ++r) issue_k(r);
+  }
+
+  // Scoring layout: 8 lanes per key (kl = lane-in-key), 16 keys per pass.
+  // Lane kl holds dims [8kl, 8kl+8) and [64+8kl, 64+8kl+8) so that the 8
+  // lanes of a key read 128 contiguous bytes per shared load.
+  const int kl = tid & 7;
+  const int ks = tid >> 3;
+  float qf[G][16];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const __nv_bfloat16* qg = a.q + ((size_t)b * Hq + hkv * G + g) * kDecD;
+    const uint4 w0 = *reinterpret_cast<const uint4*>(qg + 8 * kl);
+    const uint4 w1 = *reinterpret_cast<const uint4*>(qg + 64 + 8 * kl);
+    const uint32_t ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      qf[g][2 * i] = bf16lo(ww[i]);
+      qf[g][2 * i + 1] = bf16hi(ww[i]);
+    }
+  }
+  const int my_head = head_of_lane<G>(lane);
+  // For G <= 4 the lowest lane bits below the last split duplicate sums.
+  constexpr int kDupMask = G >= 8 ? 0 : (G == 4 ? 1 : (G == 2 ? 3 : 7));
+  const bool writer = (lane & kDupMask) == 0;
+
+  // P.V layout: 16 lanes cover the 128 dims of a key (8 dims each), 8 key
+  // groups, keys c = kg + 8 i.
+  const int dc = tid & 15;
+  const int kg = tid >> 4;
+  float acc[G][8];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int x = 0; x < 8; ++x) acc[g][x] = 0.f;
+
+  float m_run[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) m_run[g] = -INFINITY;
+  float l_part[G];  // per-lane partial normaliser of the heads of this warp
+#pragma unroll
+  for (int g = 0; g < G; ++g) l_part[g] = 0.f;
+
+  int kept_issued = 0, kept_done = 0;
+  unsigned long long n_vis = 0, n_skp = 0;
+  const float ln_lambda = a.ln_lambda;
+
+  auto pv = [&](int kidx) -> bool {
+    const int slot = kidx % kDecNV;
+    if (!mbar_wait(&vfull[slot], (uint32_t)(kidx / kDecNV) & 1u, kWaitDecodeV))
+      return false;
+    const float* al = sA + slot * 8;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float f = al[g];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) acc[g][x] *= f;
+    }
+    const int nvalid = sNV[slot];
+    const uint8_t* vst = sV + slot * kDecBlockBytes;
+    const float* ps = sP + slot * kDecBc * G;
+#pragma unroll 4
+    for (int i = 0; i < 8; ++i) {
+      const int c = kg + 8 * i;
+      if (c < nvalid) {
+        const uint4 vw =
+            *reinterpret_cast<const uint4*>(vst + c * kDecRowBytes + dc * 16);
+        const uint32_t w[4] = {vw.x, vw.y, vw.z, vw.w};
+        float vf[8];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          vf[2 * t] = bf16lo(w[t]);
+          vf[2 * t + 1] = bf16hi(w[t]);
+        }
+        float pg[G];
+        if constexpr (G % 4 == 0) {
+#pragma unroll
+          for (int g4 = 0; g4 < G; g4 += 4) {
+            const float4 p4 = *reinterpret_cast<const float4*>(ps + c * G + g4);
+            pg[g4] = p4.x;
+            pg[g4 + 1] = p4.y;
+            pg[g4 + 2] = p4.z;
+            pg[g4 + 3] = p4.w;
+          }
+        } else {
+#pragma unroll
+          for (int g = 0; g < G; ++g) pg[g] = ps[c * G + g];
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+#pragma unroll
+          for (int x = 0; x < 8; x += 2) {
+            float2 r = __ffma2_rn(make_float2(pg[g], pg[g]),
+                                  make_float2(vf[x], vf[x + 1]),
+                                  make_float2(acc[g][x], acc[g][x + 1]));
+            acc[g][x] = r.x;
+            acc[g][x + 1] = r.y;
+          }
+        }
+      }
+    }
+    return true;
+  };
+
+  bool ok = true;
+  for (int r = 0; r < nblk; ++r) {
+    const int j = j0 + r;
+    const int stage = r % kDecNK;
+    const int nvalid = rows_of(j);
+    float* sSr = sS + (r & 1) * G * kDecBc;
+
+    if (ok) ok = mbar_wait(&kfull[stage], (uint32_t)(r / kDecNK) & 1u, kWaitDecodeK);
+    if (ok) {
+      const uint8_t* kst = sK + stage * kDecBlockBytes;
+#pragma unroll
+      for (int i = 0; i < kDecBc / 16; ++i) {
+        const int c = ks + 16 * i;
+        float part[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) part[g] = 0.f;
+        if (c < nvalid) {
+          const uint4 w0 =
+              *reinterpret_cast<const uint4*>(kst + c * kDecRowBytes + kl * 16);
+          const uint4 w1 = *reinterpret_cast<const uint4*>(
+              kst + c * kDecRowBytes + 128 + kl * 16);
+          const uint32_t ww[8] = {w0.x, w0.y, w0.z, w0.w,
+                                  w1.x, w1.y, w1.z, w1.w};
+          float kf[16];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            kf[2 * t] = bf16lo(ww[t]);
+            kf[2 * t + 1] = bf16hi(ww[t]);
+          }
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int x = 0; x < 16; x += 2)
+              s2 = __ffma2_rn(make_float2(qf[g][x], qf[g][x + 1]),
+                              make_float2(kf[x], kf[x + 1]), s2);
+            part[g] = s2.x + s2.y;
+          }
+        }
+        const float tot = reduce8_transpose<G>(part, lane);
+        if (writer)
+          sSr[my_head * kDecBc + c] = (c < nvalid) ? tot * a.scale : -INFINITY;
+      }
+    }
+    if (__syncthreads_or(!ok)) { ok = false; break; }  // (1)
+    if (tid == 0 && r + kDecNK < nblk) issue_k(r + kDecNK);
+
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      if ((g & 3) != warp) continue;  // warp w owns heads w, w+4
+      float x = fmaxf(sSr[g * kDecBc + lane], sSr[g * kDecBc + lane + 32]);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1)
+        x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+      if (lane == 0) sM[g] = x;
+    }
+    __syncthreads();  // (2)
+
+    // Criterion, decided for the whole tile: skip block j iff every head's
+    // block max lies more than |ln lambda| below its running max.
+    float mt[G];
+    bool skip = ln_lambda > -INFINITY;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      mt[g] = sM[g];
+      if (!(mt[g] - m_run[g] < ln_lambda)) skip = false;
+    }
+    if (tid == 0) {
+      ++n_vis;
+      if (skip) ++n_skp;
+      if (a.mask) a.mask[(size_t)bh * a.nk + j] = skip ? 2 : 1;
+    }
+    if (!skip && !a.stats_only) {
+      const int slot = kept_issued % kDecNV;
+      if (tid == 0) {
+        const uint32_t bytes = (uint32_t)nvalid * kDecRowBytes;
+        sNV[slot] = nvalid;
+        mbar_arrive_expect_tx(&vfull[slot], bytes);
+        bulk_load(sV + slot * kDecBlockBytes,
+                  vbase + (size_t)j * kDecBc * kDecD, bytes, &vfull[slot], pol);
+      }
+      float* ps = sP + slot * kDecBc * G;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        if ((g & 3) != warp) continue;
+        const float mn = fmaxf(m_run[g], mt[g]);
+        const float alpha =
+            (m_run[g] == -INFINITY) ? 0.f : ex2_approx((m_run[g] - mn) * kLog2e);
+        const float p0 = ex2_approx((sSr[g * kDecBc + lane] - mn) * kLog2e);
+        const float p1 = ex2_approx((sSr[g * kDecBc + lane + 32] - mn) * kLog2e);
+        ps[lane * G + g] = p0;
+        ps[(lane + 32) * G + g] = p1;
+        l_part[g] = alpha * l_part[g] + p0 + p1;
+        if (lane == 0) sA[slot * 8 + g] = alpha;
+      }
+      ++kept_issued;
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) m_run[g] = fmaxf(m_run[g], mt[g]);
+
+    while (ok && kept_issued - kept_done > kDecLag) {
+      ok = pv(kept_done);
+      ++kept_done;
+    }
+  }
+  if (__syncthreads_or(!ok)) ok = false;
+  while (ok && kept_done < kept_issued) {
+    ok = pv(kept_done);
+    ++kept_done;
+  }
+  if (__syncthreads_or(!ok)) ok = false;
+
+  if (!ok) {
+    // Give outstanding copies a bounded chance to land before the CTA's
+    // shared memory is released.
+    if (tid == 0) {
+      for (int i = 0; i < kDecNK; ++i)
+        mbar_wait(&kfull[i], 0, kWaitDecodeDrain, 1000000);
+      for (int i = 0; i < kDecNV; ++i)
+        mbar_wait(&vfull[i], 0, kWaitDecodeDrain, 1000000);
+    }
+    return;
+  }
+
+  if (tid == 0 && a.counters) {
+    atomicAdd(&a.counters[0], n_vis);
+    atomicAdd(&a.counters[1], n_skp);
+  }
+  if (a.stats_only) return;
+
+  // Normaliser of each head: sum of the lane partials of its warp.
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    if ((g & 3) != warp) continue;
+    float x = l_part[g];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if (lane == 0) sL[g] = x;
+  }
+  // Partial outputs of the 8 key groups -> shared (reusing the K ring).
+  float* red = reinterpret_cast<float*>(sK);
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float4* dst = reinterpret_cast<float4*>(red + ((kg * G + g) * kDecD + dc * 8));
+    dst[0] = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
+    dst[1] = make_float4(acc[g][4], acc[g][5], acc[g][6], acc[g][7]);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int dd = tid;  // 128 threads = 128 dims
+    float sum = 0.f;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) sum += red[(t * G + g) * kDecD + dd];
+    const float l = sL[g];
+    const size_t row = (size_t)b * Hq + hkv * G + g;
+    a.o_part[(row * a.S + s) * kDecD + dd] = sum / l;
+    if (dd == 0) a.lse_part[row * a.S + s] = m_run[g] + __logf(l);
+  }
+}
+
+// Log-sum-exp merge of the S split partials of one (sequence, query head):
+//   lse = ln sum_s exp(lse_s),  o = sum_s exp(lse_s - lse) o_s.
+__global__ void __launch_bounds__(kDecD)
+    decode_combine_kernel(const float* __restrict__ o_part,
+                          const float* __restrict__ lse_part,
+                          __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
+                          int S) {
+#if defined(__CUDA_ARCH__)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+  const size_t row = blockIdx.x;
+  const int dd = threadIdx.x;
+  const float* lp = lse_part + row * S;
+  float mx = -INFINITY;
+  for (int s = 0; s < S; ++s) mx = fmaxf(mx, lp[s]);
+  float sum = 0.f;
+  for (int s = 0; s < S; ++s) sum += ex2_approx((lp[s] - mx) * kLog2e);
+  const float L = mx + __logf(sum);
+  float acc = 0.f;
+  const float* op = o_part + row * S * kDecD + dd;
+  for (int s = 0; s < S; ++s)
+    acc += ex2_approx((lp[s] - L) * kLog2e) * op[(size_t)s * kDecD];
+  o[row * kDecD + dd] = __float2bfloat16_rn(acc);
+  if (dd == 0 && lse) lse[row] = L;
+}
+
+}  // namespace blasst

@@ -1,0 +1,219 @@
+/*
+ * blasst.h -- C ABI of the BLASST attention forward for NVIDIA B200 (sm_100a).
+ *
+ * BLASST ("BLASST: Dynamic BLocked Attention Sparsity via Softmax
+ * Thresholding"; gist.science summary, section 2 "Metodologia") is the
+ * FlashAttention blockwise online-softmax forward in which KV block j is
+ * skipped for a query tile when, for every row i of the tile,
+ *
+ *        m~_i(j) - m_i(j) < ln(lambda)                      (criterion)
+ *
+ * where m~_i(j) is the row's maximum scaled score inside block j and m_i(j)
+ * the running row maximum over the blocks before j (section 2 "Criterio de
+ * Pulo"; Hindi summary, section 2 "Core Insight").  A skipped block costs no
+ * exp, no V load from HBM and no P.V product (section 2 "Acoes de
+ * Otimizacao"); the decision is made per block for the whole tile (MLSys'26
+ * reading notes, "design trade-offs": block skip vs token skip).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are dense row-major with the head dimension innermost:
+ *      prefill  q [B,Hq,Lq,d]   k, v [B,Hkv,Lkv,d]   o [B,Hq,Lq,d]
+ *               lse [B,Hq,Lq]
+ *      decode   q [B,Hq,d]      k, v [B,Hkv,Lkv,d]   o [B,Hq,d]  lse [B,Hq]
+ *    q, k, v, o are bfloat16; lse is float32 (natural log of the kept
+ *    entries' normaliser, m + ln l).  Query head hq reads KV head
+ *    hq / (Hq / Hkv) (GQA; MQA is Hkv = 1, MHA is Hkv = Hq).
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates device memory in these calls and never keeps a pointer
+ *    after a call returns.  q, k, v, o must be 16-byte aligned.
+ *  - scale multiplies q.k (usually 1/sqrt(d)); ln_lambda is in the same
+ *    natural-log units as the scaled scores.  ln_lambda must be <= 0, or
+ *    -INFINITY for the dense path (nothing is skipped).
+ *  - Causal masking is bottom-right aligned: key c is visible to query r iff
+ *    c <= r + (Lkv - Lq).  Causal calls need Lq <= Lkv.
+ *  - stream is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *    enqueue work and return; results are ready when the stream is.
+ *  - Errors are returned by value and never thrown.  Validation errors are
+ *    detected before any work is enqueued; BLASST_ERR_CUDA reports a failed
+ *    launch (the message of the last CUDA error is in blasst_last_error()).
+ */
+#ifndef BLASST_H
+#define BLASST_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BLASST_OK = 0,
+    BLASST_ERR_INVALID_ARG = 1,       /* null pointer, bad size, ln_lambda > 0 */
+    BLASST_ERR_UNSUPPORTED_SHAPE = 2, /* d, Br/Bc or head ratio not built */
+    BLASST_ERR_MISALIGNED = 3,        /* a tensor pointer not 16-byte aligned */
+    BLASST_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed */
+    BLASST_ERR_TIMEOUT = 5,           /* a kernel gave up a bounded wait */
+    BLASST_ERR_NO_CONVERGE = 6,       /* calibration bracket exhausted */
+    BLASST_ERR_WORKSPACE = 7          /* workspace missing or too small */
+} blasst_status_t;
+
+/*
+ * Skip statistics ("sparsity" = skipped / visited (tile, block) pairs).
+ * The struct itself lives in HOST memory; its fields are DEVICE pointers.
+ *
+ *  counters  device uint64[2]: [0] += visited pairs, [1] += skipped pairs.
+ *            Kernels ADD to them (atomics), so one pair of counters can sum
+ *            several calls; clear with blasst_skip_stats_reset().
+ *  mask      optional device uint8 buffer (NULL = not written) receiving one
+ *            decision per (tile, block): 0 not visited, 1 kept, 2 skipped.
+ *            Prefill layout [B, Hq, ceil(Lq/Br), ceil(Lkv/Bc)];
+ *            decode layout  [B, Hkv, ceil(Lkv/Bc)] (a block belongs to
+ *            exactly one split).  Entries of pairs that are not visited are
+ *            written as 0 by prefill only for tiles it runs; callers that
+ *            need them zeroed clear the buffer first.
+ * A NULL blasst_skip_stats_t* disables both.
+ */
+typedef struct {
+    unsigned long long *counters;
+    unsigned char *mask;
+} blasst_skip_stats_t;
+
+/*
+ * blasst_prefill -- prefill (many query tokens) forward with block skipping.
+ *
+ * The query rows are cut into tiles of Br rows and the keys into blocks of
+ * Bc keys; each (tile, block) pair follows the online-softmax update and the
+ * criterion above, blocks in ascending order.  The kernel issues the V
+ * block's TMA load and the P.V tensor-core product only for kept pairs.
+ *
+ *  q, k, v     device bf16 inputs (layouts above)
+ *  o           device bf16 output [B,Hq,Lq,d], or NULL for a statistics-only
+ *              pass: decisions and counters are produced exactly as in a
+ *              full call (the running max never depends on them) but no
+ *              exp, V load or P.V product is executed and nothing is written
+ *              to o/lse.
+ *  lse         device float32 [B,Hq,Lq] or NULL
+ *  d           64 or 128
+ *  Br, Bc      (64, 64) or (128, 128)
+ *  skip_stats  host pointer to the statistics struct, or NULL
+ */
+blasst_status_t blasst_prefill(const void *q, const void *k, const void *v,
+                               void *o, float *lse, int B, int Hq, int Hkv,
+                               int Lq, int Lkv, int d, float scale, int causal,
+                               float ln_lambda, int Br, int Bc,
+                               const blasst_skip_stats_t *skip_stats,
+                               void *stream);
+
+/*
+ * blasst_decode -- one query token per sequence against a contiguous bf16
+ * KV cache, split-KV with a log-sum-exp merge.
+ *
+ * The G = Hq/Hkv query heads sharing a KV head form the rows of one tile, so
+ * every K and V byte read serves all G heads.  The Lkv keys are cut into
+ * nk = ceil(Lkv/Bc) blocks and the blocks into num_splits contiguous splits
+ * (split s covers blocks [floor(s*nk/S), floor((s+1)*nk/S))).  Each split
+ * runs the blockwise forward independently (its running max starts at
+ * -inf), reading V only for kept blocks; a second kernel merges the splits:
+ * lse = ln sum_s exp(lse_s), o = sum_s exp(lse_s - lse) o_s.
+ *
+ *  o           device bf16 [B,Hq,d], or NULL for a statistics-only pass
+ *              (K is read and scored, V is never read)
+ *  lse         device float32 [B,Hq] or NULL
+ *  d           128;  Hq/Hkv in {1, 2, 4, 8};  Bc = 64
+ *  num_splits  >= 1, or 0 for the automatic choice blasst_decode_splits()
+ *  workspace   device buffer of at least blasst_decode_workspace_size()
+ *              bytes (16-byte aligned) holding the per-split partials;
+ *              caller-owned, contents need not be initialised.  May be NULL
+ *              in a statistics-only pass.
+ */
+blasst_status_t blasst_decode(const void *q, const void *k_cache,
+                              const void *v_cache, void *o, float *lse, int B,
+                              int Hq, int Hkv, int Lkv, int d, float scale,
+                              float ln_lambda, int Bc, int num_splits,
+                              void *workspace, size_t workspace_bytes,
+                              const blasst_skip_stats_t *skip_stats,
+                              void *stream);
+
+/* Bytes of decode workspace: B*Hq*S*(d+1) float32 values, rounded up to 256.
+ * num_splits must be the resolved value (>= 1). */
+size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits);
+
+/* The automatic split count used when num_splits == 0: enough
+ * (sequence, KV head, split) work items to give every SM several, never more
+ * splits than blocks.  Pure function of its arguments. */
+int blasst_decode_splits(int B, int Hkv, int Lkv, int Bc);
+
+/*
+ * Calibration of the threshold lambda = a / L for a target sparsity
+ * (gist.science summary, section 2 "Calibracao Automatica"; MLSys'26 reading
+ * notes, observation 2: a is fitted on calibration data, not universal).
+ *
+ * The sparsity s(ln_lambda) of a fixed input is a non-decreasing step
+ * function.  The routine bisects ln_lambda over [-64, 0] with
+ * statistics-only passes of the chosen operation on the caller's sample and
+ * returns the smallest ln_lambda found whose sparsity reaches the target
+ * (within tol), together with a = lambda * L where L = Lkv of the sample.
+ * It synchronises the stream once per bisection step.
+ */
+typedef struct {
+    int mode;                   /* 0 = prefill, 1 = decode */
+    const void *q, *k, *v;      /* device bf16 sample (layouts as above) */
+    int B, Hq, Hkv, Lq, Lkv, d; /* Lq is ignored for decode */
+    float scale;
+    int causal;                 /* prefill only */
+    int Br, Bc;                 /* Br ignored for decode */
+    int num_splits;             /* decode only; 0 = automatic */
+} blasst_calib_sample_t;
+
+typedef struct {
+    double ln_lambda;           /* calibrated threshold (natural log) */
+    double lambda;              /* exp(ln_lambda) */
+    double a;                   /* lambda * L */
+    double achieved;            /* sparsity at ln_lambda */
+    int L;                      /* the sample's Lkv */
+    int iterations;             /* statistics-only passes run */
+    unsigned long long visited, skipped; /* counts at ln_lambda */
+} blasst_calib_result_t;
+
+/*
+ *  target        sparsity in [0, 1)
+ *  tol           accepted |achieved - target| (e.g. 0.005); the search also
+ *                stops when the ln_lambda bracket is narrower than 1e-6
+ *  counters_dev  device uint64[2] scratch for the counters (caller-owned)
+ *  out           host pointer receiving the result
+ * Returns BLASST_ERR_NO_CONVERGE (with out filled with the closest value
+ * reached from above) when no ln_lambda <= 0 reaches the target.
+ */
+blasst_status_t blasst_calibrate(double target, const blasst_calib_sample_t *sample,
+                                 double tol, unsigned long long *counters_dev,
+                                 blasst_calib_result_t *out, void *stream);
+
+/* a of lambda = a / L fitted over n calibrations in log space:
+ * a = exp(mean_i ln(lambda_i * L_i)). */
+double blasst_fit_a(int n, const double *lambdas, const int *lengths);
+
+/* cudaMemsetAsync of the two counters. */
+blasst_status_t blasst_skip_stats_reset(unsigned long long *counters,
+                                        void *stream);
+
+/* Reads and clears the library's device error word for the current device
+ * (set by a kernel that abandoned a bounded wait).  Synchronises the device.
+ * Returns BLASST_OK or BLASST_ERR_TIMEOUT; *where_out (may be NULL) receives
+ * the code of the wait that gave up. */
+blasst_status_t blasst_check_device_error(int *where_out);
+
+const char *blasst_strerror(blasst_status_t status);
+
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char *blasst_last_error(void);
+
+/* Library version, e.g. "0.1.0". */
+const char *blasst_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BLASST_H */

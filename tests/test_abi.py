@@ -1,0 +1,135 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry
+point include/blasst.h declares, and its host-side logic (argument
+validation, split policy, workspace sizing, the lambda = a/L fit) behaves.
+No call here reaches a CUDA runtime function: every compute entry point is
+given arguments that validation rejects first."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "blasst.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from dynamic_block_sparse_fa_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(blasst_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("blasst_prefill", "blasst_decode", "blasst_calibrate",
+                 "blasst_decode_splits", "blasst_decode_workspace_size",
+                 "blasst_skip_stats_reset", "blasst_strerror"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared but not exported"
+
+
+def test_binding_uses_the_same_names():
+    import dynamic_block_sparse_fa_b200 as m
+    for name in declared_functions():
+        if name == "blasst_last_error":
+            continue
+        assert hasattr(m, name), f"binding lacks {name}"
+
+
+def _prefill(lib, q=0x1000, k=0x1000, v=0x1000, o=0x2000, B=1, Hq=2, Hkv=2,
+             Lq=128, Lkv=128, d=128, scale=0.088, causal=1, lnl=-1.0, Br=128,
+             Bc=128):
+    f = lib.blasst_prefill
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 + [
+        ctypes.c_float, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+        ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    return f(q, k, v, o, None, B, Hq, Hkv, Lq, Lkv, d, scale, causal, lnl, Br,
+             Bc, None, None)
+
+
+def test_prefill_validation(lib):
+    assert _prefill(lib, q=None) == 1                  # null input
+    assert _prefill(lib, lnl=0.5) == 1                 # ln lambda > 0
+    assert _prefill(lib, lnl=float("nan")) == 1
+    assert _prefill(lib, Lq=256, Lkv=128) == 1         # causal, Lq > Lkv
+    assert _prefill(lib, Hq=3, Hkv=2) == 1             # Hq % Hkv
+    assert _prefill(lib, d=96) == 2                    # head dim not built
+    assert _prefill(lib, Br=64, Bc=128) == 2           # tile pair not built
+    assert _prefill(lib, q=0x1001) == 3                # misaligned
+    assert _prefill(lib, B=0) == 1
+    assert _prefill(lib, scale=float("inf")) == 1
+
+
+def _decode(lib, q=0x1000, k=0x1000, v=0x1000, o=0x2000, B=1, Hq=4, Hkv=1,
+            Lkv=256, d=128, lnl=-1.0, Bc=64, S=1, ws=None, ws_bytes=0):
+    f = lib.blasst_decode
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5 + [
+        ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+    return f(q, k, v, o, None, B, Hq, Hkv, Lkv, d, 0.088, lnl, Bc, S, ws,
+             ws_bytes, None, None)
+
+
+def test_decode_validation(lib):
+    assert _decode(lib, k=None) == 1
+    assert _decode(lib, lnl=1.0) == 1
+    assert _decode(lib, S=5) == 1                      # more splits than blocks
+    assert _decode(lib, d=64) == 2                     # decode built for d=128
+    assert _decode(lib, Bc=128) == 2
+    assert _decode(lib, Hq=12, Hkv=4) == 2             # G = 3 not built
+    assert _decode(lib, v=0x1008) == 3
+    assert _decode(lib) == 7                           # no workspace
+    assert _decode(lib, ws=0x4000, ws_bytes=64) == 7   # too small
+
+
+def test_split_policy_and_workspace(lib):
+    import dynamic_block_sparse_fa_b200 as m
+    # batch 32 x 8 KV heads at 32K: 5 splits; batch 148: 1 split
+    assert m.blasst_decode_splits(32, 8, 32768, 64) == 5
+    assert m.blasst_decode_splits(148, 8, 32768, 64) == 1
+    assert m.blasst_decode_splits(1, 1, 64, 64) == 1
+    for B, Hkv, L in [(1, 1, 10 ** 6), (7, 3, 1000), (2, 8, 640)]:
+        s = m.blasst_decode_splits(B, Hkv, L, 64)
+        nk = -(-L // 64)
+        assert 1 <= s <= max(1, nk // 8)
+    ws = m.blasst_decode_workspace_size(32, 32, 128, 5)
+    rows = 32 * 32 * 5
+    assert ws >= rows * 129 * 4 and ws % 256 == 0
+
+
+def test_fit_a_and_strings(lib):
+    import dynamic_block_sparse_fa_b200 as m
+    assert m.blasst_fit_a([50 / 4096, 50 / 65536], [4096, 65536]) == \
+        pytest.approx(50.0)
+    assert m.blasst_fit_a([1e-3, 4e-3], [1000, 1000]) == pytest.approx(2.0)
+    assert m.blasst_strerror(0) == "ok"
+    assert "aligned" in m.blasst_strerror(3)
+    assert m.blasst_version().count(".") == 2
+
+
+def test_calibrate_validation(lib):
+    import dynamic_block_sparse_fa_b200.blasst as b
+    smp = b.CalibSample(0, 0x1000, 0x1000, 0x1000, 1, 2, 2, 128, 128, 128,
+                        0.088, 1, 128, 128, 0)
+    res = b.CalibResult()
+    f = b._lib.blasst_calibrate
+    assert f(1.5, ctypes.byref(smp), 0.01, ctypes.c_void_p(0x3000),
+             ctypes.byref(res), None) == 1
+    assert f(0.5, ctypes.byref(smp), 0.01, None, ctypes.byref(res), None) == 1
+    smp.mode = 7
+    assert f(0.5, ctypes.byref(smp), 0.01, ctypes.c_void_p(0x3000),
+             ctypes.byref(res), None) == 1
