@@ -165,11 +165,14 @@ def blasst_skip_stats_reset(counters: torch.Tensor, stream=None):
 
 
 def blasst_check_device_error():
-    """Returns (status, where): status 0 or BLASST_ERR_TIMEOUT (5)."""
+    """Returns (status, where): status 0 or BLASST_ERR_TIMEOUT (5); for a
+    timeout `where` is a string naming the first failed wait."""
     where = ctypes.c_int(0)
     st = _lib.blasst_check_device_error(ctypes.byref(where))
     if st not in (0, 5):
         _check(st, "blasst_check_device_error")
+    if st == 5:
+        return st, f"{where.value}: {blasst_last_error()}"
     return st, where.value
 
 

@@ -67,6 +67,13 @@ blasst_status_t blasst_check_device_error(int* where_out) {
   if (e != cudaSuccess) return cuda_status(e, "read error word");
   if (where_out) *where_out = (int)code;
   if (code == 0) return BLASST_OK;
+  unsigned int info[4] = {0, 0, 0, 0}, count = 0;
+  cudaMemcpyFromSymbol(info, blasst::g_error_info, sizeof info);
+  cudaMemcpyFromSymbol(&count, blasst::g_error_count, sizeof count);
+  snprintf(g_last_error, sizeof g_last_error,
+           "wait %u gave up first (block %u, step %u, parity %u, slot %u); "
+           "%u waits gave up in total",
+           code, info[0], info[1], info[2], info[3], count);
   cudaMemcpyToSymbol(blasst::g_error_code, &zero, sizeof zero);
   cudaMemcpyToSymbol(blasst::g_error_count, &zero, sizeof zero);
   return BLASST_ERR_TIMEOUT;

@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 
   auto pv = [&](int kidx) -> bool {
     const int slot = kidx % kDecNV;
-    if (!mbar_wait(&vfull[slot], (uint32_t)(kidx / kDecNV) & 1u, kWaitDecodeV))
+    if (!mbar_wait(&vfull[slot], (uint32_t)(kidx / kDecNV) & 1u, kWaitDecodeV, kidx, slot))
       return false;
     const float* al = sA + slot * 8;
 #pragma unroll
@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     const int nvalid = rows_of(j);
     float* sSr = sS + (r & 1) * G * kDecBc;
 
-    if (ok) ok = mbar_wait(&kfull[stage], (uint32_t)(r / kDecNK) & 1u, kWaitDecodeK);
+    if (ok) ok = mbar_wait(&kfull[stage], (uint32_t)(r / kDecNK) & 1u, kWaitDecodeK, r, stage);
     if (ok) {
       const uint8_t* kst = sK + stage * kDecBlockBytes;
 #pragma unroll
@@ -382,9 +382,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     // shared memory is released.
     if (tid == 0) {
       for (int i = 0; i < kDecNK; ++i)
-        mbar_wait(&kfull[i], 0, kWaitDecodeDrain, 1000000);
+        mbar_wait(&kfull[i], 0, kWaitDecodeDrain, i, 0, 1000000);
       for (int i = 0; i < kDecNV; ++i)
-        mbar_wait(&vfull[i], 0, kWaitDecodeDrain, 1000000);
+        mbar_wait(&vfull[i], 0, kWaitDecodeDrain, i, 1, 1000000);
     }
     return;
   }

@@ -88,7 +88,6 @@ struct PrefillCfg {
   static constexpr int NBAR = B_OD + 1;
   static constexpr int OFF_DEC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_TMEM = OFF_DEC + R * 4;
-  static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int SMEM = OFF_TMEM + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;  // slack for 1024 alignment
   static constexpr int TMEM_COLS = (2 * BN + D <= 256) ? 256 : 512;
@@ -132,7 +131,6 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   volatile int* dec_flag = reinterpret_cast<volatile int*>(smem + C::OFF_DEC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
-  volatile int* sm_abort = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
 
   if (threadIdx.x == 0) {
     mbar_init(&bar[C::B_Q], 1);
@@ -150,7 +148,6 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int i = 0; i < C::R; ++i) mbar_init(&bar[C::B_DEC + i], 1);
     mbar_init(&bar[C::B_OD], 1);
-    *sm_abort = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -163,60 +160,70 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   const bool stats_only = p.stats_only != 0;
 
+  // Every role loop below is run by whole warps with warp-uniform control
+  // flow; a single elected lane issues TMA / MMA instructions.
+  constexpr unsigned FULL = 0xffffffffu;
+  const bool leader = (lane == 0);
+
   if (warp == 0) {
     // ------------------------------------------------------------------
     // TMA producer
     // ------------------------------------------------------------------
-    if (lane == 0) {
+    const uint64_t pol_q = policy_evict_first();
+    const uint64_t pol_kv = policy_evict_last();
+    const int zq = b * p.Hq + hq;
+    const int zk = b * p.Hkv + hkv;
+    auto issue_k = [&](int j) {
+      const int st = j % C::NKS;
+      mbar_arrive_expect_tx(&bar[C::B_KF + st], C::KBYTES);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_3d(sK + st * C::KBYTES + c * C::BOX_K, &p.tk,
+                    &bar[C::B_KF + st], c * 64, j * BN, zk, pol_kv);
+    };
+    if (leader) {
       prefetch_tmap(&p.tq);
       prefetch_tmap(&p.tk);
       prefetch_tmap(&p.tv);
-      const uint64_t pol_q = policy_evict_first();
-      const uint64_t pol_kv = policy_evict_last();
-      const int zq = b * p.Hq + hq;
-      const int zk = b * p.Hkv + hkv;
       mbar_arrive_expect_tx(&bar[C::B_Q], C::QBYTES);
 #pragma unroll
       for (int c = 0; c < D / 64; ++c)
         tma_load_3d(sQ + c * C::BOX_Q, &p.tq, &bar[C::B_Q], c * 64, row0, zq,
                     pol_q);
-      auto issue_k = [&](int j) {
-        const int st = j % C::NKS;
-        mbar_arrive_expect_tx(&bar[C::B_KF + st], C::KBYTES);
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sK + st * C::KBYTES + c * C::BOX_K, &p.tk,
-                      &bar[C::B_KF + st], c * 64, j * BN, zk, pol_kv);
-      };
       const int n0 = nblk < C::NKS ? nblk : C::NKS;
       for (int j = 0; j < n0; ++j) issue_k(j);
-      int kept = 0;
-      bool ok = true;
-      for (int j = 0; j < nblk && ok; ++j) {
-        if (j + C::NKS < nblk) {
-          ok = mbar_wait(&bar[C::B_KE + j % C::NKS], (j / C::NKS) & 1,
-                         kWaitPrefillLoad);
-          if (!ok) break;
-          issue_k(j + C::NKS);
-        }
-        if (!stats_only) {
-          ok = mbar_wait(&bar[C::B_DEC + j % C::R], (j / C::R) & 1,
-                         kWaitPrefillLoad);
-          if (!ok) break;
-          if (dec_flag[j % C::R]) {
-            const int n = kept++;
-            const int slot = n % C::NVS;
-            if (n >= C::NVS) {
-              ok = mbar_wait(&bar[C::B_VE + slot], ((n / C::NVS) - 1) & 1,
-                             kWaitPrefillLoad);
-              if (!ok) break;
-            }
+    }
+    __syncwarp();
+    int kept = 0;
+    for (int j = 0; j < nblk; ++j) {
+      if (j + C::NKS < nblk) {
+        const bool w = mbar_wait(&bar[C::B_KE + j % C::NKS], (j / C::NKS) & 1,
+                                 kWaitPrefillLoad, j, j % C::NKS);
+        if (!__all_sync(FULL, w)) break;
+        if (leader) issue_k(j + C::NKS);
+        __syncwarp();
+      }
+      if (!stats_only) {
+        const bool w = mbar_wait(&bar[C::B_DEC + j % C::R], (j / C::R) & 1,
+                                 kWaitPrefillLoad, j, 100 + j % C::R);
+        if (!__all_sync(FULL, w)) break;
+        if (dec_flag[j % C::R]) {
+          const int n = kept++;
+          const int slot = n % C::NVS;
+          if (n >= C::NVS) {
+            const bool w2 = mbar_wait(&bar[C::B_VE + slot],
+                                      ((n / C::NVS) - 1) & 1, kWaitPrefillLoad,
+                                      j, 200 + slot);
+            if (!__all_sync(FULL, w2)) break;
+          }
+          if (leader) {
             mbar_arrive_expect_tx(&bar[C::B_VF + slot], C::KBYTES);
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
               tma_load_3d(sV + slot * C::KBYTES + c * C::BOX_K, &p.tv,
                           &bar[C::B_VF + slot], c * 64, j * BN, zk, pol_kv);
           }
+          __syncwarp();
         }
       }
     }
@@ -224,21 +231,22 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------------------
     // MMA issuer
     // ------------------------------------------------------------------
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16(128, BN, 0, 0);
-      constexpr uint32_t idesc_o = idesc_bf16(128, D, 0, 1);
-      const uint32_t aQ = smem_u32(sQ);
-      const uint32_t aK = smem_u32(sK);
-      const uint32_t aV = smem_u32(sV);
-      bool ok = mbar_wait(&bar[C::B_Q], 0, kWaitPrefillMma);
-      tc_fence_after();
-      int kept = 0;
-      for (int j = 0; j <= nblk && ok; ++j) {
-        if (j < nblk) {
-          const int st = j % C::NKS;
-          ok = mbar_wait(&bar[C::B_KF + st], (j / C::NKS) & 1, kWaitPrefillMma);
-          if (!ok) break;
-          tc_fence_after();
+    constexpr uint32_t idesc_s = idesc_bf16(128, BN, 0, 0);
+    constexpr uint32_t idesc_o = idesc_bf16(128, D, 0, 1);
+    const uint32_t aQ = smem_u32(sQ);
+    const uint32_t aK = smem_u32(sK);
+    const uint32_t aV = smem_u32(sV);
+    bool ok = __all_sync(FULL, mbar_wait(&bar[C::B_Q], 0, kWaitPrefillMma, 0, 0));
+    tc_fence_after();
+    int kept = 0;
+    for (int j = 0; j <= nblk && ok; ++j) {
+      if (j < nblk) {
+        const int st = j % C::NKS;
+        ok = __all_sync(FULL, mbar_wait(&bar[C::B_KF + st], (j / C::NKS) & 1,
+                                        kWaitPrefillMma, j, st));
+        if (!ok) break;
+        tc_fence_after();
+        if (leader) {
           const uint32_t d_s = tmem + C::COL_S + (j & 1) * BN;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
@@ -252,32 +260,39 @@ __global__ void __launch_bounds__(192, 1)
           mma_commit(&bar[C::B_SF + (j & 1)]);
           mma_commit(&bar[C::B_KE + st]);
         }
-        if (j >= 1) {
-          const int jj = j - 1;
-          ok = mbar_wait(&bar[C::B_DEC + jj % C::R], (jj / C::R) & 1,
-                         kWaitPrefillMma);
+        __syncwarp();
+      }
+      if (j >= 1) {
+        const int jj = j - 1;
+        ok = __all_sync(FULL, mbar_wait(&bar[C::B_DEC + jj % C::R],
+                                        (jj / C::R) & 1, kWaitPrefillMma, jj,
+                                        100 + jj % C::R));
+        if (!ok) break;
+        if (!stats_only && dec_flag[jj % C::R]) {
+          ok = __all_sync(FULL, mbar_wait(&bar[C::B_PF + (jj & 1)],
+                                          (jj >> 1) & 1, kWaitPrefillMma, jj,
+                                          300 + (jj & 1)));
           if (!ok) break;
-          if (!stats_only && dec_flag[jj % C::R]) {
-            ok = mbar_wait(&bar[C::B_PF + (jj & 1)], (jj >> 1) & 1,
-                           kWaitPrefillMma);
-            if (!ok) break;
-            const int n = kept++;
-            const int slot = n % C::NVS;
-            ok = mbar_wait(&bar[C::B_VF + slot], (n / C::NVS) & 1,
-                           kWaitPrefillMma);
-            if (!ok) break;
-            tc_fence_after();
+          const int n = kept++;
+          const int slot = n % C::NVS;
+          ok = __all_sync(FULL, mbar_wait(&bar[C::B_VF + slot],
+                                          (n / C::NVS) & 1, kWaitPrefillMma,
+                                          jj, 200 + slot));
+          if (!ok) break;
+          tc_fence_after();
+          if (leader) {
             const uint32_t a_p = tmem + C::COL_S + (jj & 1) * BN;
 #pragma unroll
             for (int k = 0; k < BN / 16; ++k) {
-              const uint64_t db =
-                  smem_desc(aV + slot * C::KBYTES + k * 2048, C::BOX_K, 1024, 2);
+              const uint64_t db = smem_desc(aV + slot * C::KBYTES + k * 2048,
+                                            C::BOX_K, 1024, 2);
               mma_ts(tmem + C::COL_O, a_p + k * 8, db, idesc_o,
                      (n > 0 || k > 0) ? 1u : 0u);
             }
             mma_commit(&bar[C::B_VE + slot]);
             mma_commit(&bar[C::B_OD]);
           }
+          __syncwarp();
         }
       }
     }
@@ -306,13 +321,15 @@ __global__ void __launch_bounds__(192, 1)
     unsigned long long n_vis = 0, n_skp = 0;
     bool ok = true;
 
-    // A thread whose bounded wait fails flags sm_abort and keeps meeting the
-    // warpgroup's named barrier, so the whole warpgroup leaves together.
+    // A failed bounded wait is voted on (OR over the warpgroup) at the top of
+    // the next block, so the warpgroup always leaves the loop together.
     for (int j = 0; j < nblk; ++j) {
       const int buf = j & 1;
-      if (ok) ok = mbar_wait(&bar[C::B_SF + buf], (j >> 1) & 1, kWaitPrefillSoftmax);
-      if (!ok) *sm_abort = 1;
+      if (ok)
+        ok = mbar_wait(&bar[C::B_SF + buf], (j >> 1) & 1, kWaitPrefillSoftmax,
+                       j, 400 + buf);
       tc_fence_after();
+      if (named_sync_or(1, 128, !ok)) { ok = false; break; }
       uint32_t sr[BN / 32][32];
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c)
@@ -320,7 +337,6 @@ __global__ void __launch_bounds__(192, 1)
       tc_wait_ld();
 
       const int col0 = j * BN;
-      float mt = -INFINITY;
       if (col0 + BN - 1 > lim) {  // diagonal or ragged block: mask per entry
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c)
@@ -329,6 +345,7 @@ __global__ void __launch_bounds__(192, 1)
             if (col0 + c * 32 + x > lim) sr[c][x] = __float_as_uint(-INFINITY);
           }
       }
+      float mt;
       {
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -344,7 +361,6 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       const bool skip =
           named_sync_and(1, 128, pred) && (ln_lambda > -INFINITY);
-      if (*sm_abort) { ok = false; break; }
       if (elected) {
         ++n_vis;
         if (skip) ++n_skp;
@@ -398,12 +414,17 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_wait_st();
       // Observe the completion of the previous kept block's P.V (the O
-      // accumulator may only be touched once it is done).
+      // accumulator may only be touched once it is done).  The rescale is
+      // done by whole warps (tcgen05.ld/st are warp-collective); rows that
+      // do not rescale multiply by 1.
       if (kept > 0) {
-        ok = mbar_wait(&bar[C::B_OD], (kept - 1) & 1, kWaitPrefillSoftmax);
-        if (!ok) *sm_abort = 1;
+        if (ok)
+          ok = mbar_wait(&bar[C::B_OD], (kept - 1) & 1, kWaitPrefillSoftmax, j,
+                         500);
         tc_fence_after();
-        if (ok && rescale) {
+        const bool warp_ok = __all_sync(FULL, ok);
+        if (warp_ok && __any_sync(FULL, rescale)) {
+          const float f = rescale ? alpha : 1.f;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t orow[32];
@@ -411,7 +432,7 @@ __global__ void __launch_bounds__(192, 1)
             tc_wait_ld();
 #pragma unroll
             for (int x = 0; x < 32; ++x)
-              orow[x] = __float_as_uint(__uint_as_float(orow[x]) * alpha);
+              orow[x] = __float_as_uint(__uint_as_float(orow[x]) * f);
             tmem_st32(lane_base + C::COL_O + c * 32, orow);
           }
           tc_wait_st();
@@ -423,8 +444,7 @@ __global__ void __launch_bounds__(192, 1)
       ++kept;
       if (active) m_crit = fmaxf(m_crit, mt_s);
     }
-    named_sync(1, 128);
-    if (*sm_abort) ok = false;
+    if (named_sync_or(1, 128, !ok)) ok = false;
 
     if (ok && elected) {
       if (p.counters) {
@@ -435,11 +455,12 @@ __global__ void __launch_bounds__(192, 1)
         for (int j = nblk; j < p.nk; ++j) p.mask[mask_row + j] = 0;
     }
     if (ok && !stats_only) {
-      if (kept > 0) {
-        ok = mbar_wait(&bar[C::B_OD], (kept - 1) & 1, kWaitPrefillEpilogue);
-      }
+      bool w = true;
+      if (kept > 0)
+        w = mbar_wait(&bar[C::B_OD], (kept - 1) & 1, kWaitPrefillEpilogue,
+                      nblk, 600);
       tc_fence_after();
-      if (ok) {
+      if (__all_sync(FULL, w)) {
         const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
         __nv_bfloat16* orow_g =
             p.o + ((size_t)(b * p.Hq + hq) * p.Lq + row_g) * D;
@@ -452,16 +473,16 @@ __global__ void __launch_bounds__(192, 1)
             uint4* dst = reinterpret_cast<uint4*>(orow_g + c * 32);
 #pragma unroll
             for (int x = 0; x < 32; x += 8) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(orow[x]) * inv_l,
-                                __uint_as_float(orow[x + 1]) * inv_l);
-              w.y = pack_bf16x2(__uint_as_float(orow[x + 2]) * inv_l,
-                                __uint_as_float(orow[x + 3]) * inv_l);
-              w.z = pack_bf16x2(__uint_as_float(orow[x + 4]) * inv_l,
-                                __uint_as_float(orow[x + 5]) * inv_l);
-              w.w = pack_bf16x2(__uint_as_float(orow[x + 6]) * inv_l,
-                                __uint_as_float(orow[x + 7]) * inv_l);
-              dst[x / 8] = w;
+              uint4 w4;
+              w4.x = pack_bf16x2(__uint_as_float(orow[x]) * inv_l,
+                                 __uint_as_float(orow[x + 1]) * inv_l);
+              w4.y = pack_bf16x2(__uint_as_float(orow[x + 2]) * inv_l,
+                                 __uint_as_float(orow[x + 3]) * inv_l);
+              w4.z = pack_bf16x2(__uint_as_float(orow[x + 4]) * inv_l,
+                                 __uint_as_float(orow[x + 5]) * inv_l);
+              w4.w = pack_bf16x2(__uint_as_float(orow[x + 6]) * inv_l,
+                                 __uint_as_float(orow[x + 7]) * inv_l);
+              dst[x / 8] = w4;
             }
           }
         }

@@ -16,6 +16,7 @@ namespace blasst {
 // ---------------------------------------------------------------------------
 __device__ unsigned int g_error_code;   // 0 = none, else a kWait* code
 __device__ unsigned int g_error_count;  // number of waits that gave up
+__device__ unsigned int g_error_info[4];  // first failure: block, step, parity, slot
 
 enum : unsigned int {
   kWaitDecodeK = 1,
@@ -32,8 +33,16 @@ enum : unsigned int {
 // kernels, short enough that a lost arrival returns control to the host.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
-__device__ __forceinline__ void record_error(unsigned int where) {
-  atomicCAS(&g_error_code, 0u, where);
+__device__ __forceinline__ void record_error(unsigned int where,
+                                             unsigned int step = 0xffffffffu,
+                                             unsigned int parity = 0,
+                                             unsigned int slot = 0) {
+  if (atomicCAS(&g_error_code, 0u, where) == 0u) {
+    g_error_info[0] = blockIdx.x;
+    g_error_info[1] = step;
+    g_error_info[2] = parity;
+    g_error_info[3] = slot;
+  }
   atomicAdd(&g_error_count, 1u);
 }
 
@@ -85,12 +94,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // (after recording `where`) if it has not completed within `limit` cycles.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           unsigned int where,
+                                          unsigned int step = 0xffffffffu,
+                                          unsigned int slot = 0,
                                           long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (clock64() - t0 > limit) {
-      record_error(where);
+      record_error(where, step, parity, slot);
       return false;
     }
   }
@@ -149,6 +160,21 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// OR-reduction of a predicate over the `nthreads` threads of barrier `id`.
+__device__ __forceinline__ bool named_sync_or(uint32_t id, uint32_t nthreads,
+                                              bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %3, 0;\n\t"
+      "barrier.cta.red.or.pred q, %1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(id), "r"(nthreads), "r"((uint32_t)pred)
+      : "memory");
+  return out != 0;
 }
 
 // AND-reduction of a predicate over the `nthreads` threads of barrier `id`.

@@ -201,7 +201,8 @@ blasst_status_t blasst_skip_stats_reset(unsigned long long *counters,
 /* Reads and clears the library's device error word for the current device
  * (set by a kernel that abandoned a bounded wait).  Synchronises the device.
  * Returns BLASST_OK or BLASST_ERR_TIMEOUT; *where_out (may be NULL) receives
- * the code of the wait that gave up. */
+ * the code of the wait that gave up, and blasst_last_error() then describes
+ * the first failed wait (block, step, parity, slot). */
 blasst_status_t blasst_check_device_error(int *where_out);
 
 const char *blasst_strerror(blasst_status_t status);
