@@ -123,6 +123,10 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # algorithmic work
 # ---------------------------------------------------------------------------
+def _r(x, nd):
+    return None if (x is None or x != x) else round(x, nd)
+
+
 def decode_bytes(B, Hq, Hkv, Lkv, d, Bc, S, kept_rows):
     """Bytes one decode call must move: all of K, V rows of kept blocks, q,
     split partials (written then read), o and lse."""
@@ -178,24 +182,32 @@ def time_calls(fn, steps, warmup, stream, barrier=None):
     return start.elapsed_time(end)
 
 
-def cpu_oracle_decode_sample(q, k, v, ln_lambda, S, n_seq=1):
-    """Times the CPU oracle (as it stands) on n_seq sequences of the decode
-    workload; returns (GB/s of algorithmic bytes, seconds, threads, sample)."""
+def cpu_oracle_decode_sample(q, k, v, ln_lambda, S, budget_s=10.0):
+    """Times the CPU oracle (as it stands, all host cores) on the decode
+    workload's own bytes, one sequence at a time, until about `budget_s`
+    seconds of CPU work; returns (GB/s of algorithmic bytes, seconds,
+    threads, description of the sample)."""
     import oracle
     d = q.shape[-1]
-    qs, ks, vs = q[:n_seq].cpu(), k[:n_seq].cpu(), v[:n_seq].cpu()
     threads = os.cpu_count() or 1
-    t0 = time.perf_counter()
-    res = oracle.decode(qs, ks, vs, 1.0 / math.sqrt(d), ln_lambda, DEC["Bc"], S,
-                        n_threads=threads)
-    dt = time.perf_counter() - t0
-    kept_rows = kept_rows_from_mask(torch.from_numpy(res["mask"]), k.shape[2],
-                                    DEC["Bc"])
-    by = decode_bytes(n_seq, q.shape[1], k.shape[1], k.shape[2], d, DEC["Bc"],
-                      S, kept_rows)
-    return by / dt / 1e9, dt, threads, (
-        f"{n_seq} of {q.shape[0]} sequences (all {k.shape[1]} KV heads x "
-        f"{k.shape[2]} keys), same splits and lambda")
+    total_bytes, total_t, n = 0, 0.0, 0
+    B = q.shape[0]
+    while total_t < budget_s and n < 16 * B:
+        b = n % B
+        qs, ks, vs = q[b:b + 1].cpu(), k[b:b + 1].cpu(), v[b:b + 1].cpu()
+        t0 = time.perf_counter()
+        res = oracle.decode(qs, ks, vs, 1.0 / math.sqrt(d), ln_lambda,
+                            DEC["Bc"], S, n_threads=threads)
+        total_t += time.perf_counter() - t0
+        kept_rows = kept_rows_from_mask(torch.from_numpy(res["mask"]),
+                                        k.shape[2], DEC["Bc"])
+        total_bytes += decode_bytes(1, q.shape[1], k.shape[1], k.shape[2], d,
+                                    DEC["Bc"], S, kept_rows)
+        n += 1
+    return total_bytes / total_t / 1e9, total_t, threads, (
+        f"{n} sequence passes over the batch of {B} (each: all {k.shape[1]} "
+        f"KV heads x {k.shape[2]} keys), same splits and lambda, "
+        f"~{budget_s:.0f} s budget")
 
 
 # ---------------------------------------------------------------------------
@@ -223,15 +235,41 @@ def run_blasst(args):
     hbm_peak, tf_burst, tf_sust, peak_kind = _peaks()
     stream = torch.cuda.current_stream()
 
-    # ---------------- decode workload ----------------
+    line = None
+    if not args.no_decode:
+        line = run_decode(args, bl, dev, stream, world, rank, local, dist,
+                          barrier, hbm_peak, peak_kind)
+    else:
+        line = {"metric": METRIC, "value": None, "unit": "GB/s",
+                "n_gpus": world, "note": "decode leg skipped"}
+
+    # ---------------- prefill workload (rank 0) ----------------
+    if rank == 0 and not args.no_prefill:
+        line["prefill"], line["roofline_prefill"] = run_prefill(
+            args, bl, dev, stream, tf_burst, peak_kind)
+    barrier()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
+               hbm_peak, peak_kind):
+    from synth import config_seed, planted_gap_kv_inplace
     B, Hq, Hkv, Lkv, d, Bc = (DEC[x] for x in ("B", "Hq", "Hkv", "Lkv", "d", "Bc"))
+    B = args.decode_batch
     q = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev)
     k = torch.empty(B, Hkv, Lkv, d, dtype=torch.bfloat16, device=dev)
     v = torch.empty_like(k)
     planted_gap_kv_inplace(k, v, q, block=Bc, gap=8.0, heavy_frac=0.03,
                            seed=config_seed(1, 1000 * rank))
-    cal = bl.blasst_calibrate(DEC["target"], mode="decode", q=q, k=k, v=v,
-                              Bc=Bc, tol=0.002)
+    if args.decode_lnl is None:
+        cal = bl.blasst_calibrate(DEC["target"], mode="decode", q=q, k=k, v=v,
+                                  Bc=Bc, tol=0.002)
+    else:
+        cal = {"ln_lambda": args.decode_lnl, "iterations": 0,
+               "a": math.exp(args.decode_lnl) * Lkv}
     lnl = cal["ln_lambda"]
     S = bl.blasst_decode_splits(B, Hkv, Lkv, Bc)
     nk = -(-Lkv // Bc)
@@ -260,7 +298,8 @@ def run_blasst(args):
     if dist is not None:
         dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
     ms_max = float(ms_t.item())
-    ms_dense = time_calls(dense_call, K, W, stream, barrier)
+    ms_dense = (time_calls(dense_call, K, W, stream, barrier)
+                if not args.no_dense else float("nan"))
     t_call = ms_max / K / 1e3
     value = by_call * world / t_call / 1e9  # GB/s over all ranks
     achieved = by_call / t_call / 1e9       # per GPU, per call
@@ -282,7 +321,8 @@ def run_blasst(args):
         l_h.copy_(lse, non_blocking=True)
         stream.synchronize()  # the host reads the step's result
 
-    ms_e2e = time_calls(e2e_step, K, W, stream, barrier)
+    ms_e2e = (time_calls(e2e_step, K, W, stream, barrier)
+              if not args.no_e2e else float("nan"))
     e2e_t = torch.tensor([ms_e2e], device=dev)
     if dist is not None:
         dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
@@ -314,10 +354,10 @@ def run_blasst(args):
         },
         "decode": {
             "us": round(ms_max / K * 1e3, 2),
-            "dense_us": round(ms_dense / K * 1e3, 2),
-            "speedup_vs_dense": round(ms_dense / ms_max, 4),
+            "dense_us": _r(ms_dense / K * 1e3, 2),
+            "speedup_vs_dense": _r(ms_dense / ms_max, 4),
             "GBps": round(achieved, 1),
-            "dense_GBps": round(by_dense / (ms_dense / K / 1e3) / 1e9, 1),
+            "dense_GBps": _r(by_dense / (ms_dense / K / 1e3) / 1e9, 1),
             "bytes_per_call": by_call,
             "sparsity": skp / vis,
             "calibration_iterations": cal["iterations"],
@@ -328,37 +368,29 @@ def run_blasst(args):
             "peak_kind": peak_kind + " copy bandwidth", "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4), "traffic": None,
         },
-        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
+        "e2e": {"value": _r(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(float(e2e_t.item()) / K, 4),
+                "ms_per_step": _r(float(e2e_t.item()) / K, 4),
                 "what": "h2d of q and the new token's K/V rows, decode, "
                         "d2h of o and lse, host sync, per step"},
         "gpu_launches": 2 * K,
         "clocks": clk.summary(),
     }
 
-    # ---------------- prefill workload (rank 0) ----------------
-    if rank == 0 and not args.no_prefill:
-        line["prefill"], line["roofline_prefill"] = run_prefill(
-            args, bl, dev, stream, tf_burst, peak_kind)
-    barrier()
-
     # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
     if rank == 0 and world == 1 and not args.no_cpu:
-        gbs, secs, threads, sample = cpu_oracle_decode_sample(q, k, v, lnl, S,
-                                                              n_seq=1)
+        gbs, secs, threads, sample = cpu_oracle_decode_sample(
+            q, k, v, lnl, S, budget_s=args.cpu_seconds)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s",
                                 "cores": threads, "kind": "oracle",
                                 "sample": sample, "seconds": round(secs, 2)}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if dist is not None:
-        dist.destroy_process_group()
+    return line
 
 
 def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
     from synth import config_seed, planted_gap
     B, Hq, Hkv, L, d, Br, Bc = (PRE[x] for x in ("B", "Hq", "Hkv", "L", "d", "Br", "Bc"))
+    L = args.prefill_L
     x = planted_gap(B, Hq, Hkv, L, L, d, block=Br, gap=8.0, heavy_frac=0.02,
                     window=512, seed=config_seed(2), device=dev)
     q, k, v = x.q, x.k, x.v
@@ -383,6 +415,13 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
                 "executed_tflops": round(ex / (ms / 1e3) / 1e12, 1),
                 "tensor_frac": round(ex / (ms / 1e3) / 1e12 / tf_peak, 4)}
 
+    if args.prefill_lnl is not None:
+        out["fixed"] = measure(args.prefill_lnl)
+        r = out["fixed"]
+        return out, {"bound": "tensor", "kernel": "prefill_kernel<128,128,128>",
+                     "achieved": r["executed_tflops"], "peak": tf_peak,
+                     "peak_kind": peak_kind + " bf16 burst", "unit": "TFLOP/s",
+                     "frac": r["tensor_frac"], "traffic": None}
     dense = measure(-math.inf)
     out["dense"] = dense
     for tgt, key in ((0.5, "s50"), (0.7, "s70")):
@@ -413,9 +452,11 @@ def run_reference(args):
     from synth import config_seed, planted_gap
 
     B, Hq, Hkv, Lkv, d, Bc = (DEC[x] for x in ("B", "Hq", "Hkv", "Lkv", "d", "Bc"))
-    n_seq = 1  # bounded sample: one sequence of the batch per step
+    n_seq = 4  # bounded sample: four sequences of the batch per step
     x = planted_gap(n_seq, Hq, Hkv, 1, Lkv, d, decode=True, block=Bc, gap=8.0,
                     heavy_frac=0.03, seed=config_seed(1), device="cpu")
+    # the library's automatic split count for this workload (batch 32 x 8 KV
+    # heads at 32K keys -> 5 splits), restated so this arm loads no GPU code
     S = max(1, min(-(-Lkv // Bc) // 8, -(-(148 * 2 * 4) // (B * Hkv))))
     scale = 1.0 / math.sqrt(d)
     threads = os.cpu_count() or 1
@@ -463,7 +504,20 @@ def main():
     ap.add_argument("--prefill-steps", type=int, default=10)
     ap.add_argument("--impl", choices=["blasst", "reference"], default="blasst")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode workload (profiling runs only)")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--decode-batch", type=int, default=DEC["B"],
+                    help="sequences per GPU (profiling runs use fewer)")
+    ap.add_argument("--decode-lnl", type=float, default=None,
+                    help="fixed ln(lambda) instead of calibrating")
+    ap.add_argument("--prefill-L", type=int, default=PRE["L"])
+    ap.add_argument("--prefill-lnl", type=float, default=None,
+                    help="measure prefill only at this ln(lambda)")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="approximate CPU time budget of the oracle baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -2,7 +2,7 @@
 
 The kernels live in libblasst.so (C ABI: include/blasst.h); this package is
 its Python binding.  Importing it loads the library and fails if it has not
-been built (``python -m dynamic_block_sparse_fa_b200.build``).
+been built (``python dynamic_block_sparse_fa_b200/build.py``).
 """
 from .blasst import (BlasstError, Stats, blasst_calibrate,
                      blasst_check_device_error, blasst_decode,
@@ -11,7 +11,8 @@ from .blasst import (BlasstError, Stats, blasst_calibrate,
                      blasst_skip_stats_reset, blasst_strerror, blasst_version)
 
 __all__ = ["BlasstError", "Stats", "blasst_calibrate",
-           "blasst_check_device_error", "blasst_decode", "blasst_decode_splits",
+           "blasst_check_device_error", "blasst_decode",
+           "blasst_decode_splits",
            "blasst_decode_workspace_size", "blasst_fit_a", "blasst_last_error",
            "blasst_prefill", "blasst_skip_stats_reset", "blasst_strerror",
            "blasst_version"]

@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libblasst.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"{LIB_PATH} is missing: build it with "
-        "`python -m dynamic_block_sparse_fa_b200.build` (needs nvcc)")
+        "`python dynamic_block_sparse_fa_b200/build.py` (needs nvcc)")
 
 _lib = ctypes.CDLL(LIB_PATH)
 

@@ -1,6 +1,6 @@
 """Builds libblasst.so (the C-ABI library of include/blasst.h) for sm_100a.
 
-    python -m dynamic_block_sparse_fa_b200.build [--force] [--verbose]
+    python dynamic_block_sparse_fa_b200/build.py [--force] [--verbose]
 
 The library is one nvcc translation unit (csrc/blasst.cu) compiled for
 sm_100a with the CUDA runtime linked statically; it lands next to this file

@@ -16,7 +16,12 @@ HEADER = os.path.join(ROOT, "include", "blasst.h")
 
 @pytest.fixture(scope="module")
 def lib():
-    from dynamic_block_sparse_fa_b200 import build
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_blasst_build", os.path.join(ROOT, "dynamic_block_sparse_fa_b200",
+                                      "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
     path = build.build()
     return ctypes.CDLL(path)
 
