@@ -77,6 +77,10 @@ _lib.blasst_decode.restype = _i
 _lib.blasst_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                _f, _f, _i, _i, _vp, _sz,
                                ctypes.POINTER(SkipStats), _vp]
+_lib.blasst_decode_noalloc.restype = _i
+_lib.blasst_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                       _i, _f, _f, _i, _i,
+                                       ctypes.POINTER(SkipStats), _vp]
 _lib.blasst_decode_workspace_size.restype = _sz
 _lib.blasst_decode_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.blasst_decode_splits.restype = _i
@@ -97,7 +101,8 @@ _lib.blasst_last_error.argtypes = []
 _lib.blasst_version.restype = ctypes.c_char_p
 _lib.blasst_version.argtypes = []
 
-EXPORTED = ["blasst_prefill", "blasst_decode", "blasst_decode_workspace_size",
+EXPORTED = ["blasst_prefill", "blasst_decode", "blasst_decode_noalloc",
+            "blasst_decode_workspace_size",
             "blasst_decode_splits", "blasst_calibrate", "blasst_fit_a",
             "blasst_skip_stats_reset", "blasst_check_device_error",
             "blasst_strerror", "blasst_last_error", "blasst_version"]
@@ -239,6 +244,35 @@ def blasst_decode(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
         float(scale), float(ln_lambda), Bc, S, _ptr(workspace), ws_bytes,
         stats.c_struct if stats is not None else None, _stream(stream))
     _check(st, "blasst_decode")
+    return o, lse
+
+
+def blasst_decode_noalloc(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
+                          num_splits=0, o=None, lse=None, want_lse=True,
+                          stats: Stats | None = None, stats_only=False,
+                          stream=None):
+    """blasst_decode with the split partials in the library's own fixed
+    device array (8 MiB per device) instead of a caller workspace; for
+    callers that may not allocate device memory at call time.  Calls that
+    could overlap on the GPU share that array and must be serialised."""
+    B, Hq, d = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if not stats_only:
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and want_lse:
+            lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    else:
+        o, lse = None, None
+    st = _lib.blasst_decode_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lkv, d,
+        float(scale), float(ln_lambda), Bc, num_splits,
+        stats.c_struct if stats is not None else None, _stream(stream))
+    if st == 7:
+        raise BlasstError(st, "blasst_decode_noalloc: " + blasst_last_error())
+    _check(st, "blasst_decode_noalloc")
     return o, lse
 
 

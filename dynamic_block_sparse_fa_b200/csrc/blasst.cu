@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "blasst.h"
 #include "decode.cuh"
@@ -198,6 +199,75 @@ blasst_status_t blasst_decode(const void* q, const void* k_cache,
                          (const float*)o_part, (const float*)lse_part,
                          static_cast<__nv_bfloat16*>(o), lse, S);
   return cuda_status(e, "decode merge launch");
+}
+
+// ---------------------------------------------------------------------------
+// Decode with library-owned scratch (no allocation by anyone at call time)
+// ---------------------------------------------------------------------------
+// Some callers may not allocate device memory when they run the decode: an
+// inference-engine plugin whose enqueue step is forbidden to allocate, or a
+// latency-critical decode loop that cannot afford cudaMalloc's implicit
+// device-wide synchronisation and has no workspace of its own to lend.  For
+// them the split partials live in this fixed array, which the CUDA runtime
+// places in device memory when the library is loaded: every GPU that loads
+// the library keeps these bytes until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name only stands in for the symbol; its device address must be
+// asked of the runtime, once per device, with that device current.
+blasst_status_t noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return BLASST_ERR_UNSUPPORTED_SHAPE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return BLASST_OK;
+}
+}  // namespace
+
+blasst_status_t blasst_decode_noalloc(const void* q, const void* k_cache,
+                                      const void* v_cache, void* o, float* lse,
+                                      int B, int Hq, int Hkv, int Lkv, int d,
+                                      float scale, float ln_lambda, int Bc,
+                                      int num_splits,
+                                      const blasst_skip_stats_t* skip_stats,
+                                      void* stream) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lkv < 1 || Bc < 1 || num_splits < 0)
+    return BLASST_ERR_INVALID_ARG;
+  const int S = num_splits == 0 ? blasst_decode_splits(B, Hkv, Lkv, Bc)
+                                : num_splits;
+  const size_t need = blasst_decode_workspace_size(B, Hq, d, S);
+  if (o && need > kNoAllocScratchBytes) {
+    snprintf(g_last_error, sizeof g_last_error,
+             "blasst_decode_noalloc: these shapes need %zu bytes of split "
+             "partials, the built-in scratch holds %zu (use blasst_decode with "
+             "a caller workspace, or fewer splits)",
+             need, kNoAllocScratchBytes);
+    return BLASST_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  blasst_status_t rc = noalloc_scratch(&scratch);
+  if (rc != BLASST_OK) return rc;
+  // Nothing in the scratch needs clearing: the split kernel writes every
+  // partial it later merges.
+  return blasst_decode(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Lkv, d, scale,
+                       ln_lambda, Bc, S, scratch, kNoAllocScratchBytes,
+                       skip_stats, stream);
 }
 
 // ---------------------------------------------------------------------------

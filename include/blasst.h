@@ -136,6 +136,37 @@ blasst_status_t blasst_decode(const void *q, const void *k_cache,
                               const blasst_skip_stats_t *skip_stats,
                               void *stream);
 
+/*
+ * blasst_decode_noalloc -- blasst_decode for callers that may not allocate
+ * device memory at call time and have no workspace to pass: for example an
+ * inference-engine plugin whose enqueue step must not allocate, or a
+ * latency-critical decode loop that cannot take cudaMalloc's implicit
+ * device-wide synchronisation.  (No counterpart in the BLASST papers: this
+ * is a deployment convenience of this library.)
+ *
+ * Same arguments and results as blasst_decode minus the workspace.  The
+ * split partials go to an 8 MiB array that the library holds in device
+ * memory on every GPU that loads it, until the process exits.
+ *  - The first call on a device looks up that array's device address for
+ *    the current device (once per device); make that first call before any
+ *    stream capture.
+ *  - Shapes whose partials exceed 8 MiB (B*Hq*S*(d+1) float32 values plus
+ *    alignment, see blasst_decode_workspace_size) are rejected with
+ *    BLASST_ERR_WORKSPACE and a message in blasst_last_error().
+ *  - All calls on a device share the one array and it keeps the previous
+ *    call's contents (nothing in it needs to start at zero).  Calls whose
+ *    kernels may overlap on the GPU (different streams without ordering)
+ *    race on it: serialise them, or use blasst_decode with one workspace per
+ *    stream.
+ */
+blasst_status_t blasst_decode_noalloc(const void *q, const void *k_cache,
+                                      const void *v_cache, void *o, float *lse,
+                                      int B, int Hq, int Hkv, int Lkv, int d,
+                                      float scale, float ln_lambda, int Bc,
+                                      int num_splits,
+                                      const blasst_skip_stats_t *skip_stats,
+                                      void *stream);
+
 /* Bytes of decode workspace: B*Hq*S*(d+1) float32 values, rounded up to 256.
  * num_splits must be the resolved value (>= 1). */
 size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits);
