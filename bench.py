@@ -442,6 +442,26 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
 # ---------------------------------------------------------------------------
 # the reference arm: the CPU oracle, as it stands, on the host cores
 # ---------------------------------------------------------------------------
+def auto_splits(B, Hkv, Lkv, Bc, n_sm=148, ctas_per_sm=3):
+    """The library's automatic split count (blasst_decode_splits), restated
+    so that the reference arm loads no GPU code: >= 2 waves, >= 8 blocks per
+    split, best-filled last wave among up to twice the minimum."""
+    nk = -(-Lkv // Bc)
+    units = B * Hkv
+    slots = n_sm * ctas_per_sm
+    s_max = max(1, nk // 8)
+    s_min = max(1, -(-2 * slots // units))
+    if s_min > s_max:
+        return s_max
+    best, best_eff = s_min, -1.0
+    for s in range(s_min, min(2 * s_min, s_max) + 1):
+        waves = units * s / slots
+        eff = waves / math.ceil(waves)
+        if eff > best_eff + 1e-9:
+            best, best_eff = s, eff
+    return best
+
+
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -455,9 +475,7 @@ def run_reference(args):
     n_seq = 4  # bounded sample: four sequences of the batch per step
     x = planted_gap(n_seq, Hq, Hkv, 1, Lkv, d, decode=True, block=Bc, gap=8.0,
                     heavy_frac=0.03, seed=config_seed(1), device="cpu")
-    # the library's automatic split count for this workload (batch 32 x 8 KV
-    # heads at 32K keys -> 5 splits), restated so this arm loads no GPU code
-    S = max(1, min(-(-Lkv // Bc) // 8, -(-(148 * 2 * 4) // (B * Hkv))))
+    S = auto_splits(B, Hkv, Lkv, Bc)
     scale = 1.0 / math.sqrt(d)
     threads = os.cpu_count() or 1
     # lambda for 70% sparsity from the oracle's own margins (exact quantile)

@@ -87,13 +87,27 @@ int blasst_decode_splits(int B, int Hkv, int Lkv, int Bc) {
   if (B < 1 || Hkv < 1 || Lkv < 1 || Bc < 1) return 1;
   const long long nk = (Lkv + (long long)Bc - 1) / Bc;
   const long long units = (long long)B * Hkv;
-  // About four waves of two resident CTAs per SM on a 148-SM B200, with at
-  // least 8 blocks per split.
-  const long long target = (long long)kNumSmB200 * 2 * 4;
-  long long s = (target + units - 1) / units;
-  if (s > nk / 8) s = nk / 8;
-  if (s < 1) s = 1;
-  return (int)s;
+  // At least two waves of the split kernel on a 148-SM B200 with 3 resident
+  // CTAs per SM, at least 8 blocks per split, and among the split counts up
+  // to twice that minimum the one whose last wave is fullest (fewer splits
+  // on ties: every split restarts the running max).
+  const long long slots = (long long)kNumSmB200 * 3;
+  const long long s_max = nk / 8 > 1 ? nk / 8 : 1;
+  long long s_min = (2 * slots + units - 1) / units;
+  if (s_min > s_max) return (int)s_max;
+  if (s_min < 1) s_min = 1;
+  const long long s_hi = 2 * s_min < s_max ? 2 * s_min : s_max;
+  long long best = s_min;
+  double best_eff = -1.0;
+  for (long long s = s_min; s <= s_hi; ++s) {
+    const double waves = (double)(units * s) / (double)slots;
+    const double eff = waves / std::ceil(waves);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return (int)best;
 }
 
 size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits) {

@@ -41,27 +41,32 @@ struct DecodeArgs {
 constexpr int kDecD = 128;       // head dimension
 constexpr int kDecBc = 64;       // keys per block
 constexpr int kDecThreads = 128;
-constexpr int kDecNK = 3;        // K blocks in flight ahead of the scoring
-constexpr int kDecNV = 3;        // V block slots
-constexpr int kDecLag = 2;       // P.V of kept block n runs when n+Lag+1 are issued
+// Resident CTAs per SM the kernel is sized for (registers and shared memory).
+template <int G>
+constexpr int dec_ctas_per_sm() { return G >= 8 ? 2 : 3; }
+constexpr int kDecNK = 2;        // K blocks staged (one ahead of the scoring)
+constexpr int kDecNV = 2;        // V block slots
+constexpr int kDecLag = 1;       // P.V of kept block n runs once n+Lag+1 are issued
 static_assert(kDecNV >= kDecLag + 1, "V ring must cover the lag");
 constexpr int kDecBlockBytes = kDecBc * kDecD * 2;  // 16 KB
 constexpr int kDecRowBytes = kDecD * 2;             // 256 B per key
 
 template <int G>
 struct DecodeSmem {
-  static constexpr int kK = 0;                                    // [NK][Bc][D] bf16
-  static constexpr int kV = kK + kDecNK * kDecBlockBytes;          // [NV][Bc][D] bf16
-  static constexpr int kP = kV + kDecNV * kDecBlockBytes;          // [NV][Bc][G] f32
-  static constexpr int kS = kP + kDecNV * kDecBc * G * 4;          // [2][G][Bc] f32
-  static constexpr int kM = kS + 2 * G * kDecBc * 4;               // [8] f32
-  static constexpr int kA = kM + 8 * 4;                            // [NV][8] f32
-  static constexpr int kL = kA + kDecNV * 8 * 4;                   // [8] f32
-  static constexpr int kNV = kL + 8 * 4;                           // [NV] int
-  static constexpr int kBar = (kNV + kDecNV * 4 + 15) & ~15;       // [NK+NV] u64
+  static constexpr int kK = 0;                                  // [NK][Bc][D] bf16
+  static constexpr int kV = kK + kDecNK * kDecBlockBytes;        // [NV][Bc][D] bf16
+  static constexpr int kP = kV + kDecNV * kDecBlockBytes;        // [NV][Bc][G] f32
+  static constexpr int kM = kP + kDecNV * kDecBc * G * 4;        // [2][4 warps][8] f32
+  static constexpr int kA = kM + 2 * 4 * 8 * 4;                  // [NV][8] f32
+  static constexpr int kL = kA + kDecNV * 8 * 4;                 // [4 warps][8] f32
+  static constexpr int kNV = kL + 4 * 8 * 4;                     // [NV] int
+  static constexpr int kBar = (kNV + kDecNV * 4 + 15) & ~15;     // [NK+NV] u64
   static constexpr int kTotal = kBar + (kDecNK + kDecNV) * 8;
-  // The end-of-split reduction [8 key groups][G][D] f32 reuses the K ring.
-  static_assert(8 * G * kDecD * 4 <= kDecNK * kDecBlockBytes, "reduction fits");
+  // The end-of-split reduction [8 key groups][G][D] f32 reuses the K and V
+  // rings (all copies into them have been consumed by then).
+  static_assert(8 * G * kDecD * 4 <= kP, "reduction fits in the rings");
+  static_assert(dec_ctas_per_sm<G>() * (kTotal + 1024) <= 228 * 1024,
+                "shared memory for the intended residency");
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -111,7 +116,7 @@ __device__ __forceinline__ int head_of_lane(int lane) {
 }
 
 template <int G>
-__global__ void __launch_bounds__(kDecThreads, 2)
+__global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
     decode_split_kernel(const DecodeArgs a) {
   using L = DecodeSmem<G>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -131,7 +136,6 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   uint8_t* sK = smem + L::kK;
   uint8_t* sV = smem + L::kV;
   float* sP = reinterpret_cast<float*>(smem + L::kP);
-  float* sS = reinterpret_cast<float*>(smem + L::kS);
   float* sM = reinterpret_cast<float*>(smem + L::kM);
   float* sA = reinterpret_cast<float*>(smem + L::kA);
   float* sL = reinterpret_cast<float*>(smem + L::kL);
@@ -164,7 +168,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     for (int r = 0; r < n0; ++r) issue_k(r);
   }
 
-  // Scoring layout: 8 lanes per key (kl = lane-in-key), 16 keys per pass.
+  // Scoring layout: 8 lanes per key (kl = lane-in-key), 16 keys per pass,
+  // 4 passes per block; warp w scores keys 4w..4w+3 (+16 per pass).
   // Lane kl holds dims [8kl, 8kl+8) and [64+8kl, 64+8kl+8) so that the 8
   // lanes of a key read 128 contiguous bytes per shared load.
   const int kl = tid & 7;
@@ -182,8 +187,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       qf[g][2 * i + 1] = bf16hi(ww[i]);
     }
   }
+  // After the 8-lane reduction a lane holds the score of one head for one
+  // key; lanes that differ only in kDupMask bits hold the same value.
   const int my_head = head_of_lane<G>(lane);
-  // For G <= 4 the lowest lane bits below the last split duplicate sums.
   constexpr int kDupMask = G >= 8 ? 0 : (G == 4 ? 1 : (G == 2 ? 3 : 7));
   const bool writer = (lane & kDupMask) == 0;
 
@@ -197,12 +203,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 #pragma unroll
     for (int x = 0; x < 8; ++x) acc[g][x] = 0.f;
 
-  float m_run[G];
+  float m_run[G];  // running max per head (replicated in every thread)
 #pragma unroll
   for (int g = 0; g < G; ++g) m_run[g] = -INFINITY;
-  float l_part[G];  // per-lane partial normaliser of the heads of this warp
-#pragma unroll
-  for (int g = 0; g < G; ++g) l_part[g] = 0.f;
+  float l_part = 0.f;  // writer lanes: partial normaliser of my_head
 
   int kept_issued = 0, kept_done = 0;
   unsigned long long n_vis = 0, n_skp = 0;
@@ -210,7 +214,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 
   auto pv = [&](int kidx) -> bool {
     const int slot = kidx % kDecNV;
-    if (!mbar_wait(&vfull[slot], (uint32_t)(kidx / kDecNV) & 1u, kWaitDecodeV, kidx, slot))
+    if (!mbar_wait(&vfull[slot], (uint32_t)(kidx / kDecNV) & 1u, kWaitDecodeV,
+                   kidx, slot))
       return false;
     const float* al = sA + slot * 8;
 #pragma unroll
@@ -270,9 +275,12 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     const int j = j0 + r;
     const int stage = r % kDecNK;
     const int nvalid = rows_of(j);
-    float* sSr = sS + (r & 1) * G * kDecBc;
 
-    if (ok) ok = mbar_wait(&kfull[stage], (uint32_t)(r / kDecNK) & 1u, kWaitDecodeK, r, stage);
+    // ---- scores of block j (kept in registers) and per-warp head maxima
+    float sc[kDecBc / 16];
+    if (ok)
+      ok = mbar_wait(&kfull[stage], (uint32_t)(r / kDecNK) & 1u, kWaitDecodeK,
+                     r, stage);
     if (ok) {
       const uint8_t* kst = sK + stage * kDecBlockBytes;
 #pragma unroll
@@ -305,31 +313,26 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           }
         }
         const float tot = reduce8_transpose<G>(part, lane);
-        if (writer)
-          sSr[my_head * kDecBc + c] = (c < nvalid) ? tot * a.scale : -INFINITY;
+        sc[i] = (c < nvalid) ? tot * a.scale : -INFINITY;
       }
+      float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      // per-warp maxima, double-buffered by block parity: a fast warp may
+      // write block j+1's while a slow one still reads block j's
+      if ((lane & (kDupMask | 24)) == 0) sM[(r & 1) * 32 + warp * 8 + my_head] = mx;
     }
-    if (__syncthreads_or(!ok)) { ok = false; break; }  // (1)
+    if (__syncthreads_or(!ok)) { ok = false; break; }
     if (tid == 0 && r + kDecNK < nblk) issue_k(r + kDecNK);
 
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      if ((g & 3) != warp) continue;  // warp w owns heads w, w+4
-      float x = fmaxf(sSr[g * kDecBc + lane], sSr[g * kDecBc + lane + 32]);
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1)
-        x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-      if (lane == 0) sM[g] = x;
-    }
-    __syncthreads();  // (2)
-
-    // Criterion, decided for the whole tile: skip block j iff every head's
-    // block max lies more than |ln lambda| below its running max.
+    // ---- decision, identical in every thread: skip block j iff every
+    // head's block max lies more than |ln lambda| below its running max.
     float mt[G];
     bool skip = ln_lambda > -INFINITY;
+    const float* sMr = sM + (r & 1) * 32;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      mt[g] = sM[g];
+      mt[g] = fmaxf(fmaxf(sMr[g], sMr[8 + g]), fmaxf(sMr[16 + g], sMr[24 + g]));
       if (!(mt[g] - m_run[g] < ln_lambda)) skip = false;
     }
     if (tid == 0) {
@@ -346,19 +349,29 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         bulk_load(sV + slot * kDecBlockBytes,
                   vbase + (size_t)j * kDecBc * kDecD, bytes, &vfull[slot], pol);
       }
-      float* ps = sP + slot * kDecBc * G;
+      // new running max, rescale factor and P, per head
+      float mn_mine = 0.f, al_mine = 1.f;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        if ((g & 3) != warp) continue;
         const float mn = fmaxf(m_run[g], mt[g]);
-        const float alpha =
+        const float al =
             (m_run[g] == -INFINITY) ? 0.f : ex2_approx((m_run[g] - mn) * kLog2e);
-        const float p0 = ex2_approx((sSr[g * kDecBc + lane] - mn) * kLog2e);
-        const float p1 = ex2_approx((sSr[g * kDecBc + lane + 32] - mn) * kLog2e);
-        ps[lane * G + g] = p0;
-        ps[(lane + 32) * G + g] = p1;
-        l_part[g] = alpha * l_part[g] + p0 + p1;
-        if (lane == 0) sA[slot * 8 + g] = alpha;
+        if (tid == 0) sA[slot * 8 + g] = al;
+        if (g == my_head) {
+          mn_mine = mn;
+          al_mine = al;
+        }
+      }
+      if (writer) {
+        float* ps = sP + slot * kDecBc * G;
+        float psum = 0.f;
+#pragma unroll
+        for (int i = 0; i < kDecBc / 16; ++i) {
+          const float pv_ = ex2_approx((sc[i] - mn_mine) * kLog2e);
+          ps[(ks + 16 * i) * G + my_head] = pv_;
+          psum += pv_;
+        }
+        l_part = al_mine * l_part + psum;
       }
       ++kept_issued;
     }
@@ -395,16 +408,18 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   }
   if (a.stats_only) return;
 
-  // Normaliser of each head: sum of the lane partials of its warp.
+  // Normaliser of each head: writer lanes hold partials of their head; sum
+  // over the lanes of the warp that share it, then over the 4 warps.
+  {
+    float x = writer ? l_part : 0.f;
+    x += __shfl_xor_sync(0xffffffffu, x, 8);
+    x += __shfl_xor_sync(0xffffffffu, x, 16);
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    if ((g & 3) != warp) continue;
-    float x = l_part[g];
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    if (lane == 0) sL[g] = x;
+    for (int msk = 1; msk <= 4; msk <<= 1)
+      if (kDupMask & msk) x += __shfl_xor_sync(0xffffffffu, x, msk);
+    if ((lane & (kDupMask | 24)) == 0) sL[warp * 8 + my_head] = x;
   }
-  // Partial outputs of the 8 key groups -> shared (reusing the K ring).
+  // Partial outputs of the 8 key groups -> shared (reusing the rings).
   float* red = reinterpret_cast<float*>(sK);
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -419,7 +434,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     float sum = 0.f;
 #pragma unroll
     for (int t = 0; t < 8; ++t) sum += red[(t * G + g) * kDecD + dd];
-    const float l = sL[g];
+    const float l = sL[g] + sL[8 + g] + sL[16 + g] + sL[24 + g];
     const size_t row = (size_t)b * Hq + hkv * G + g;
     a.o_part[(row * a.S + s) * kDecD + dd] = sum / l;
     if (dd == 0) a.lse_part[row * a.S + s] = m_run[g] + __logf(l);

@@ -171,9 +171,12 @@ blasst_status_t blasst_decode_noalloc(const void *q, const void *k_cache,
  * num_splits must be the resolved value (>= 1). */
 size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits);
 
-/* The automatic split count used when num_splits == 0: enough
- * (sequence, KV head, split) work items to give every SM several, never more
- * splits than blocks.  Pure function of its arguments. */
+/* The automatic split count used when num_splits == 0.  Pure function of
+ * its arguments (so a reference can reproduce the masks): at least two waves
+ * of (sequence, KV head, split) work items on a 148-SM B200 with 3 resident
+ * CTAs per SM, at least 8 blocks per split, and among the counts up to twice
+ * that minimum the one that fills the last wave best (fewest splits on
+ * ties).  Batch 32 x 8 KV heads at 32K keys gives 5; batch 148 gives 1. */
 int blasst_decode_splits(int B, int Hkv, int Lkv, int Bc);
 
 /*

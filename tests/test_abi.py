@@ -138,3 +138,15 @@ def test_calibrate_validation(lib):
     smp.mode = 7
     assert f(0.5, ctypes.byref(smp), 0.01, ctypes.c_void_p(0x3000),
              ctypes.byref(res), None) == 1
+
+
+def test_reference_arm_split_policy_matches_library(lib):
+    """bench.py's reference arm restates the automatic split count so that it
+    loads no GPU code; both must agree or the arms would run different
+    masks."""
+    import itertools
+    import bench
+    import dynamic_block_sparse_fa_b200 as m
+    for B, H, L in itertools.product([1, 2, 3, 8, 32, 148], [1, 8],
+                                     [64, 1000, 32768, 131072]):
+        assert bench.auto_splits(B, H, L, 64) == m.blasst_decode_splits(B, H, L, 64)
