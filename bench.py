@@ -182,6 +182,15 @@ def time_calls(fn, steps, warmup, stream, barrier=None):
     return start.elapsed_time(end)
 
 
+def reduce_max(value, dist, device):
+    """Maximum of a per-rank float over all ranks (the value itself when
+    not distributed)."""
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def cpu_oracle_decode_sample(q, k, v, ln_lambda, S, budget_s=10.0):
     """Times the CPU oracle (as it stands, all host cores) on the decode
     workload's own bytes, one sequence at a time, until about `budget_s`
@@ -294,10 +303,7 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
     K, W = args.steps, args.warmup
     with ClockSampler(local) as clk:
         ms = time_calls(sparse_call, K, W, stream, barrier)
-    ms_t = torch.tensor([ms], device=dev)
-    if dist is not None:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = reduce_max(ms, dist, dev)
     ms_dense = (time_calls(dense_call, K, W, stream, barrier)
                 if not args.no_dense else float("nan"))
     t_call = ms_max / K / 1e3
@@ -323,10 +329,8 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
 
     ms_e2e = (time_calls(e2e_step, K, W, stream, barrier)
               if not args.no_e2e else float("nan"))
-    e2e_t = torch.tensor([ms_e2e], device=dev)
-    if dist is not None:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_value = by_call * world / (float(e2e_t.item()) / K / 1e3) / 1e9
+    e2e_max = reduce_max(ms_e2e, dist, dev)
+    e2e_value = by_call * world / (e2e_max / K / 1e3) / 1e9
     h2d = q_h.numel() * 2 + kv_new_h.numel() * 2
     d2h = o_h.numel() * 2 + l_h.numel() * 4
 
@@ -370,7 +374,7 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
         },
         "e2e": {"value": _r(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": _r(float(e2e_t.item()) / K, 4),
+                "ms_per_step": _r(e2e_max / K, 4),
                 "what": "h2d of q and the new token's K/V rows, decode, "
                         "d2h of o and lse, host sync, per step"},
         "gpu_launches": 2 * K,

@@ -9,11 +9,13 @@ from .blasst import (BlasstError, Stats, blasst_calibrate,
                      blasst_decode_noalloc,
                      blasst_decode_splits, blasst_decode_workspace_size,
                      blasst_fit_a, blasst_last_error, blasst_prefill,
-                     blasst_skip_stats_reset, blasst_strerror, blasst_version)
+                     blasst_selftest_wait_timeout, blasst_skip_stats_reset,
+                     blasst_strerror, blasst_version)
 
 __all__ = ["BlasstError", "Stats", "blasst_calibrate",
            "blasst_check_device_error", "blasst_decode",
            "blasst_decode_noalloc", "blasst_decode_splits",
            "blasst_decode_workspace_size", "blasst_fit_a", "blasst_last_error",
-           "blasst_prefill", "blasst_skip_stats_reset", "blasst_strerror",
+           "blasst_prefill", "blasst_selftest_wait_timeout",
+           "blasst_skip_stats_reset", "blasst_strerror",
            "blasst_version"]

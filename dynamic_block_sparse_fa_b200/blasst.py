@@ -94,6 +94,8 @@ _lib.blasst_skip_stats_reset.restype = _i
 _lib.blasst_skip_stats_reset.argtypes = [_vp, _vp]
 _lib.blasst_check_device_error.restype = _i
 _lib.blasst_check_device_error.argtypes = [ctypes.POINTER(_i)]
+_lib.blasst_selftest_wait_timeout.restype = _i
+_lib.blasst_selftest_wait_timeout.argtypes = [ctypes.c_longlong, _vp]
 _lib.blasst_strerror.restype = ctypes.c_char_p
 _lib.blasst_strerror.argtypes = [_i]
 _lib.blasst_last_error.restype = ctypes.c_char_p
@@ -105,6 +107,7 @@ EXPORTED = ["blasst_prefill", "blasst_decode", "blasst_decode_noalloc",
             "blasst_decode_workspace_size",
             "blasst_decode_splits", "blasst_calibrate", "blasst_fit_a",
             "blasst_skip_stats_reset", "blasst_check_device_error",
+            "blasst_selftest_wait_timeout",
             "blasst_strerror", "blasst_last_error", "blasst_version"]
 
 
@@ -179,6 +182,12 @@ def blasst_check_device_error():
     if st == 5:
         return st, f"{where.value}: {blasst_last_error()}"
     return st, where.value
+
+
+def blasst_selftest_wait_timeout(limit_cycles=1_000_000, stream=None):
+    """Launch the diagnostic kernel whose bounded wait is bound to give up."""
+    _check(_lib.blasst_selftest_wait_timeout(int(limit_cycles), _stream(stream)),
+           "blasst_selftest_wait_timeout")
 
 
 def blasst_prefill(q, k, v, *, scale=None, causal=True, ln_lambda=-math.inf,

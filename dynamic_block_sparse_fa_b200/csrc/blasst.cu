@@ -10,6 +10,7 @@
 #include "blasst.h"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "prefill2.cuh"
 
 namespace {
 
@@ -58,6 +59,31 @@ blasst_status_t blasst_skip_stats_reset(unsigned long long* counters,
   return cuda_status(cudaMemsetAsync(counters, 0, 2 * sizeof(unsigned long long),
                                      (cudaStream_t)stream),
                      "cudaMemsetAsync(counters)");
+}
+
+namespace {
+// Waits on an mbarrier that nothing arrives at, with the given limit: the
+// wait gives up, records kWaitSelfTest in the device error word and the
+// kernel returns.  Exercises the failure path of every bounded wait of the
+// library without faulting the GPU.
+__global__ void selftest_wait_kernel(long long limit_cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    blasst::mbar_init(&bar, 1);
+    blasst::fence_mbar_init();
+  }
+  __syncthreads();
+  blasst::mbar_wait(&bar, 0, blasst::kWaitSelfTest, 0, 0, limit_cycles);
+}
+}  // namespace
+
+blasst_status_t blasst_selftest_wait_timeout(long long limit_cycles,
+                                             void* stream) {
+  if (limit_cycles < 1 || limit_cycles > 4000000000LL)
+    return BLASST_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      limit_cycles);
+  return cuda_status(cudaGetLastError(), "selftest launch");
 }
 
 blasst_status_t blasst_check_device_error(int* where_out) {

@@ -575,10 +575,15 @@ cudaError_t launch_prefill_t(const PrefillProblem& pr, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// 128x128 tiles run prefill2_kernel (prefill2.cuh); 64x64 tiles run the
+// single-tile kernel above.
+template <int D>
+cudaError_t launch_prefill2(const PrefillProblem& pr, cudaStream_t st);
+
 inline cudaError_t launch_prefill(const PrefillProblem& pr, cudaStream_t st) {
-  if (pr.d == 128 && pr.Br == 128) return launch_prefill_t<128, 128, 128>(pr, st);
+  if (pr.d == 128 && pr.Br == 128) return launch_prefill2<128>(pr, st);
+  if (pr.d == 64 && pr.Br == 128) return launch_prefill2<64>(pr, st);
   if (pr.d == 128 && pr.Br == 64) return launch_prefill_t<128, 64, 64>(pr, st);
-  if (pr.d == 64 && pr.Br == 128) return launch_prefill_t<64, 128, 128>(pr, st);
   return launch_prefill_t<64, 64, 64>(pr, st);
 }
 

@@ -1,0 +1,603 @@
+// prefill2.cuh -- BLASST prefill forward on sm_100a for 128x128 tiles with
+// two query tiles per CTA that take turns on the tensor core.
+//
+// Same method and decisions as prefill.cuh ("BLASST: Dynamic BLocked
+// Attention Sparsity via Softmax Thresholding", gist.science summary,
+// section 2; MLSys'26 reading notes, core method and design trade-offs): per
+// (tile, block) pair the row maxima of S = Q K^T are voted on, and a skipped
+// pair computes no exp, issues no P.V MMA, and (unless the other tile of the
+// CTA keeps the block) issues no V TMA load.
+//
+// CTA = 10 warps, query tiles t0 = 2p and t1 = 2p+1 of one head:
+//   warp 0        TMA producer: Q0, Q1 once; K ring (2 blocks); V per block
+//                 that at least one of the two tiles keeps, issued as soon as
+//                 the first keeping decision is known
+//   warp 1        MMA issuer; per block j: [tile 0] P0.V_j then QK0(j+1),
+//                 [tile 1] P1.V_j then QK1(j+1), so that while one tile's
+//                 softmax runs the tensor core works on the other tile
+//   warps 2..5    softmax of tile 0 (thread = row; TMEM lane quadrants
+//                 2, 3, 0, 1)
+//   warps 6..9    softmax of tile 1
+// Tensor memory (512 columns): S0 | S1 | O0 | O1, each 128 columns; P_t
+// aliases the first 64 columns of S_t (two bf16 per column).  Because the
+// MMA warp issues QK_t(j+1) after P_t.V_j, the arrival of S_t(j+1) also
+// certifies that O_t is no longer being written, so the softmax may rescale
+// O_t without a further wait.
+#pragma once
+
+#include "prefill.cuh"
+
+// 1: score rows are read from tensor memory twice (max pass, exp pass) so
+// that only 32 of them are live in registers; 0: the whole row stays live.
+#ifndef BLASST_PREFILL2_TWO_PASS
+#define BLASST_PREFILL2_TWO_PASS 0
+#endif
+// 1: exponentials of a kept block are evaluated two per instruction in
+// bf16x2 (P feeds the bf16 MMA in any case; the row sum is accumulated in
+// fp32 from the same bf16 values); 0: one fp32 exp2 per element.
+#ifndef BLASST_PREFILL2_EX2_BF16X2
+#define BLASST_PREFILL2_EX2_BF16X2 0
+#endif
+#ifndef BLASST_PREFILL2_NKS
+#define BLASST_PREFILL2_NKS 2
+#endif
+// Number of the four 32-column chunks of a kept score row whose exponentials
+// run on the FMA pipe (exp2_poly) instead of the MUFU pipe.
+#ifndef BLASST_PREFILL2_EXP_EMU
+#define BLASST_PREFILL2_EXP_EMU 0
+#endif
+
+namespace blasst {
+
+template <int D>
+struct Prefill2Cfg {
+  static constexpr int BM = 128;
+  static constexpr int BN = 128;
+  static constexpr int NKS = BLASST_PREFILL2_NKS;  // K ring depth
+  static constexpr int NVS = 2;
+  static constexpr int R = 8;  // decision ring per tile (> NKS)
+  static constexpr int BOX_Q = BM * 128;
+  static constexpr int BOX_K = BN * 128;
+  static constexpr int QBYTES = BM * D * 2;
+  static constexpr int KBYTES = BN * D * 2;
+  static constexpr int OFF_Q = 0;  // Q0 then Q1
+  static constexpr int OFF_K = OFF_Q + 2 * QBYTES;
+  static constexpr int OFF_V = OFF_K + NKS * KBYTES;
+  static constexpr int OFF_BAR = OFF_V + NVS * KBYTES;
+  static constexpr int B_Q = 0;
+  static constexpr int B_KF = 1;
+  static constexpr int B_KE = B_KF + NKS;
+  static constexpr int B_VF = B_KE + NKS;
+  static constexpr int B_VE = B_VF + NVS;
+  static constexpr int B_SF = B_VE + NVS;  // [2]
+  static constexpr int B_PF = B_SF + 2;    // [2]
+  static constexpr int B_OD = B_PF + 2;    // [2]
+  static constexpr int B_DEC = B_OD + 2;   // [2][R]
+  static constexpr int NBAR = B_DEC + 2 * R;
+  static constexpr int OFF_DEC = OFF_BAR + NBAR * 8;  // int [2][R]
+  static constexpr int OFF_TMEM = OFF_DEC + 2 * R * 4;
+  static constexpr int SMEM = OFF_TMEM + 16;
+  static constexpr int SMEM_ALLOC = SMEM + 1024;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int COL_S = 0;    // tile t at COL_S + t * 128
+  static constexpr int COL_O = 256;  // tile t at COL_O + t * 128
+  static constexpr int THREADS = 320;
+  static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    prefill2_kernel(const __grid_constant__ PrefillParams p) {
+  using C = Prefill2Cfg<D>;
+  constexpr int BN = C::BN;
+  constexpr unsigned FULL = 0xffffffffu;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const bool leader = (lane == 0);
+
+  // Work item: KV-head-major (the CTAs resident at any time share one KV
+  // head's K and V, which then stay in L2), and within a KV head the
+  // longest tile pairs first; the G query heads of a pair are adjacent.
+  const int nq2 = (p.nq + 1) >> 1;
+  const int per_kv = nq2 * p.G;
+  const int lin = blockIdx.x;
+  const int kvi = lin / per_kv;  // b * Hkv + hkv
+  const int rem = lin - kvi * per_kv;
+  const int pair = nq2 - 1 - rem / p.G;
+  const int b = kvi / p.Hkv;
+  const int hkv = kvi - b * p.Hkv;
+  const int hq = hkv * p.G + (rem - (rem / p.G) * p.G);
+  int nblk_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int tile = 2 * pair + t;
+    if (tile >= p.nq) {
+      nblk_t[t] = 0;
+    } else {
+      const int last_row = min((tile + 1) * 128, p.Lq) - 1;
+      const int kmax = p.causal ? min(p.Lkv - 1, last_row + (p.Lkv - p.Lq))
+                                : p.Lkv - 1;
+      nblk_t[t] = kmax / BN + 1;
+    }
+  }
+  const int nblk = max(nblk_t[0], nblk_t[1]);
+
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  volatile int* dec_flag = reinterpret_cast<volatile int*>(smem + C::OFF_DEC);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[C::B_Q], 1);
+    for (int i = 0; i < C::NKS; ++i) {
+      mbar_init(&bar[C::B_KF + i], 1);
+      mbar_init(&bar[C::B_KE + i], 1);
+    }
+    for (int i = 0; i < C::NVS; ++i) {
+      mbar_init(&bar[C::B_VF + i], 1);
+      mbar_init(&bar[C::B_VE + i], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar[C::B_SF + t], 1);
+      mbar_init(&bar[C::B_PF + t], 4);
+      mbar_init(&bar[C::B_OD + t], 1);
+      for (int i = 0; i < C::R; ++i) mbar_init(&bar[C::B_DEC + t * C::R + i], 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool stats_only = p.stats_only != 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------
+    // TMA producer
+    // ------------------------------------------------------------------
+    const uint64_t pol_q = policy_evict_first();
+    const uint64_t pol_kv = policy_evict_last();
+    const int zq = b * p.Hq + hq;
+    const int zk = b * p.Hkv + hkv;
+    auto issue_k = [&](int j) {
+      const int st = j % C::NKS;
+      mbar_arrive_expect_tx(&bar[C::B_KF + st], C::KBYTES);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_3d(sK + st * C::KBYTES + c * C::BOX_K, &p.tk,
+                    &bar[C::B_KF + st], c * 64, j * BN, zk, pol_kv);
+    };
+    if (leader) {
+      prefetch_tmap(&p.tq);
+      prefetch_tmap(&p.tk);
+      prefetch_tmap(&p.tv);
+      const int nt = nblk_t[1] > 0 ? 2 : 1;
+      mbar_arrive_expect_tx(&bar[C::B_Q], C::QBYTES * nt);
+      for (int t = 0; t < nt; ++t)
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sQ + t * C::QBYTES + c * C::BOX_Q, &p.tq, &bar[C::B_Q],
+                      c * 64, (2 * pair + t) * 128, zq, pol_q);
+      const int n0 = nblk < C::NKS ? nblk : C::NKS;
+      for (int j = 0; j < n0; ++j) issue_k(j);
+    }
+    __syncwarp();
+    int vcount = 0;
+    for (int j = 0; j < nblk; ++j) {
+      if (j + C::NKS < nblk) {
+        const bool w = mbar_wait(&bar[C::B_KE + j % C::NKS], (j / C::NKS) & 1,
+                                 kWaitPrefillLoad, j, j % C::NKS);
+        if (!__all_sync(FULL, w)) break;
+        if (leader) issue_k(j + C::NKS);
+        __syncwarp();
+      }
+      if (stats_only) continue;
+      bool need = false, ok = true;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (need || j >= nblk_t[t]) continue;
+        const bool w = mbar_wait(&bar[C::B_DEC + t * C::R + j % C::R],
+                                 (j / C::R) & 1, kWaitPrefillLoad, j,
+                                 100 + t * C::R + j % C::R);
+        if (!__all_sync(FULL, w)) { ok = false; break; }
+        need = dec_flag[t * C::R + j % C::R] != 0;
+      }
+      if (!ok) break;
+      if (need) {
+        const int n = vcount++;
+        const int slot = n % C::NVS;
+        if (n >= C::NVS) {
+          const bool w = mbar_wait(&bar[C::B_VE + slot], ((n / C::NVS) - 1) & 1,
+                                   kWaitPrefillLoad, j, 200 + slot);
+          if (!__all_sync(FULL, w)) break;
+        }
+        if (leader) {
+          mbar_arrive_expect_tx(&bar[C::B_VF + slot], C::KBYTES);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sV + slot * C::KBYTES + c * C::BOX_K, &p.tv,
+                        &bar[C::B_VF + slot], c * 64, j * BN, zk, pol_kv);
+        }
+        __syncwarp();
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------
+    // MMA issuer
+    // ------------------------------------------------------------------
+    constexpr uint32_t idesc_s = idesc_bf16(128, BN, 0, 0);
+    constexpr uint32_t idesc_o = idesc_bf16(128, D, 0, 1);
+    const uint32_t aQ = smem_u32(sQ);
+    const uint32_t aK = smem_u32(sK);
+    const uint32_t aV = smem_u32(sV);
+    auto qk = [&](int t, int j) {
+      const int st = j % C::NKS;
+      const uint32_t d_s = tmem + C::COL_S + t * 128;
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (uint32_t)(k & 3) * 32;  // 16 columns = 32 B
+        const uint64_t da = smem_desc(
+            aQ + t * C::QBYTES + (k >> 2) * C::BOX_Q + off, 16, 1024, 2);
+        const uint64_t db = smem_desc(
+            aK + st * C::KBYTES + (k >> 2) * C::BOX_K + off, 16, 1024, 2);
+        mma_ss(d_s, da, db, idesc_s, k > 0 ? 1u : 0u);
+      }
+      mma_commit(&bar[C::B_SF + t]);
+    };
+    bool ok = __all_sync(FULL, mbar_wait(&bar[C::B_Q], 0, kWaitPrefillMma, 0, 0));
+    if (ok)
+      ok = __all_sync(FULL, mbar_wait(&bar[C::B_KF], 0, kWaitPrefillMma, 0, 0));
+    tc_fence_after();
+    if (ok) {
+      if (leader) {
+        for (int t = 0; t < 2; ++t)
+          if (nblk_t[t] > 0) qk(t, 0);
+        mma_commit(&bar[C::B_KE]);
+      }
+      __syncwarp();
+    }
+    int vcount = 0;
+    int npv[2] = {0, 0};
+    for (int j = 0; j < nblk && ok; ++j) {
+      int vslot = -1;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (!ok || j >= nblk_t[t]) continue;
+        ok = __all_sync(FULL, mbar_wait(&bar[C::B_PF + t], j & 1,
+                                        kWaitPrefillMma, j, 300 + t));
+        if (!ok) break;
+        const bool kept = dec_flag[t * C::R + j % C::R] != 0;
+        if (kept && !stats_only) {
+          if (vslot < 0) {
+            vslot = vcount % C::NVS;
+            ok = __all_sync(FULL, mbar_wait(&bar[C::B_VF + vslot],
+                                            (vcount / C::NVS) & 1,
+                                            kWaitPrefillMma, j, 200 + vslot));
+            ++vcount;
+            if (!ok) break;
+          }
+          tc_fence_after();
+          if (leader) {
+            const uint32_t a_p = tmem + C::COL_S + t * 128;
+#pragma unroll
+            for (int k = 0; k < BN / 16; ++k) {
+              const uint64_t db = smem_desc(aV + vslot * C::KBYTES + k * 2048,
+                                            C::BOX_K, 1024, 2);
+              mma_ts(tmem + C::COL_O + t * 128, a_p + k * 8, db, idesc_o,
+                     (npv[t] > 0 || k > 0) ? 1u : 0u);
+            }
+          }
+          ++npv[t];
+        }
+        if (j + 1 < nblk_t[t]) {
+          ok = __all_sync(FULL, mbar_wait(&bar[C::B_KF + (j + 1) % C::NKS],
+                                          ((j + 1) / C::NKS) & 1,
+                                          kWaitPrefillMma, j + 1,
+                                          (j + 1) % C::NKS));
+          if (!ok) break;
+          tc_fence_after();
+          if (leader) qk(t, j + 1);
+        } else if (leader) {
+          mma_commit(&bar[C::B_OD + t]);  // tile t has issued its last MMA
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (leader) {
+        if (vslot >= 0) mma_commit(&bar[C::B_VE + vslot]);
+        if (j + 1 < nblk) mma_commit(&bar[C::B_KE + (j + 1) % C::NKS]);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------------
+    // Softmax warpgroups: warps 2..5 tile 0, warps 6..9 tile 1
+    // ------------------------------------------------------------------
+    const int t = (warp - 2) >> 2;
+    const uint32_t bar_id = 1 + t;
+    const int nb = nblk_t[t];
+    const int quad = warp & 3;
+    const int rr = quad * 32 + lane;
+    const int tile = 2 * pair + t;
+    const int row_g = tile * 128 + rr;
+    const bool active = nb > 0 && row_g < p.Lq;
+    const int lim = p.causal ? min(row_g + (p.Lkv - p.Lq), p.Lkv - 1)
+                             : p.Lkv - 1;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t col_s = C::COL_S + t * 128;
+    const uint32_t col_o = C::COL_O + t * 128;
+    const float scale = p.scale;
+    const float ln_lambda = p.ln_lambda;
+    const float sl2 = scale * kPrefLog2e;
+    const bool elected = (((warp - 2) & 3) == 0 && lane == 0);
+    const size_t mask_row =
+        ((size_t)(b * p.Hq + hq) * p.nq + tile) * (size_t)p.nk;
+
+    float m_crit = -INFINITY;
+    float m_ref = -INFINITY;
+    float l = 0.f;
+    unsigned long long n_vis = 0, n_skp = 0;
+    bool ok = true;
+
+    for (int j = 0; j < nb; ++j) {
+      if (ok)
+        ok = mbar_wait(&bar[C::B_SF + t], j & 1, kWaitPrefillSoftmax, j, 400 + t);
+      tc_fence_after();
+      if (named_sync_or(bar_id, 128, !ok)) { ok = false; break; }
+      const int col0 = j * BN;
+      const bool need_mask = col0 + BN - 1 > lim;
+#if BLASST_PREFILL2_TWO_PASS
+      // Pass 1: row max over the score row, 32 columns at a time.
+      float mt;
+      {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        const int lim_rel = lim - col0;  // last visible column of the block
+#pragma unroll
+        for (int h = 0; h < BN / 32; ++h) {
+          uint32_t sr[32];
+          tmem_ld32(lane_base + col_s + h * 32, sr);
+          tc_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            float v = __uint_as_float(sr[x]);
+            if (need_mask && h * 32 + x > lim_rel) v = -INFINITY;
+            m4[x & 3] = fmaxf(m4[x & 3], v);
+          }
+        }
+        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      }
+#else
+      uint32_t sr[BN / 32][32];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c)
+        tmem_ld32(lane_base + col_s + c * 32, sr[c]);
+      tc_wait_ld();
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            if (col0 + c * 32 + x > lim) sr[c][x] = __float_as_uint(-INFINITY);
+      }
+      float mt;
+      {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            m4[x & 3] = fmaxf(m4[x & 3], __uint_as_float(sr[c][x]));
+        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      }
+#endif
+      const float mt_s = mt * scale;
+      const bool pred = !active || mt_s == -INFINITY ||
+                        (mt_s - m_crit < ln_lambda);
+      tc_fence_before();
+      const bool skip =
+          named_sync_and(bar_id, 128, pred) && (ln_lambda > -INFINITY);
+      if (elected) {
+        ++n_vis;
+        if (skip) ++n_skp;
+        if (p.mask) p.mask[mask_row + j] = skip ? 2 : 1;
+        dec_flag[t * C::R + j % C::R] = skip ? 0 : 1;
+        mbar_arrive(&bar[C::B_DEC + t * C::R + j % C::R]);
+      }
+      if (skip || stats_only) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[C::B_PF + t]);
+        if (active) m_crit = fmaxf(m_crit, mt_s);
+        continue;
+      }
+
+      float alpha = 1.f;
+      bool rescale = false;
+      if (active && mt_s != -INFINITY) {
+        const float m_new = fmaxf(m_crit, mt_s);
+        if (m_ref == -INFINITY || m_new > m_ref + kRescaleNats) {
+          alpha = (m_ref == -INFINITY) ? 0.f
+                                       : ex2_approx((m_ref - m_new) * kPrefLog2e);
+          m_ref = m_new;
+          rescale = true;
+        }
+      }
+      const float mb = (active && m_ref != -INFINITY) ? m_ref * kPrefLog2e
+                                                      : INFINITY;
+      float rowsum = 0.f;
+#if BLASST_PREFILL2_TWO_PASS
+      // Pass 2: reload 32 columns at a time, exp, P over the first half.
+      const int lim_rel = lim - col0;
+#pragma unroll
+      for (int h = 0; h < BN / 32; ++h) {
+        uint32_t sr[32];
+        tmem_ld32(lane_base + col_s + h * 32, sr);
+        tc_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          float v0 = __uint_as_float(sr[x]);
+          float v1 = __uint_as_float(sr[x + 1]);
+          if (need_mask) {
+            if (h * 32 + x > lim_rel) v0 = -INFINITY;
+            if (h * 32 + x + 1 > lim_rel) v1 = -INFINITY;
+          }
+          const float p0 = ex2_approx(fmaf(v0, sl2, -mb));
+          const float p1 = ex2_approx(fmaf(v1, sl2, -mb));
+          rowsum += p0 + p1;
+          pk[x / 2] = pack_bf16x2(p0, p1);
+        }
+        // P of chunk h (16 columns) lands in columns [16h, 16h+16), below
+        // the scores of every chunk not yet reloaded (chunk h' starts at 32h').
+        tmem_st16(lane_base + col_s + h * 16, pk);
+      }
+#else
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t pk[16];
+#if BLASST_PREFILL2_EX2_BF16X2
+        float2 rs2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const float2 a2 = __ffma2_rn(
+              make_float2(__uint_as_float(sr[c][x]), __uint_as_float(sr[c][x + 1])),
+              make_float2(sl2, sl2), make_float2(-mb, -mb));
+          const uint32_t e = ex2_bf16x2(pack_bf16x2(a2.x, a2.y));
+          pk[x / 2] = e;
+          rs2 = __fadd2_rn(rs2, make_float2(bf16lo(e), bf16hi(e)));
+        }
+        rowsum += rs2.x + rs2.y;
+#else
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const float a0 = fmaf(__uint_as_float(sr[c][x]), sl2, -mb);
+          const float a1 = fmaf(__uint_as_float(sr[c][x + 1]), sl2, -mb);
+          const float p0 = c < BLASST_PREFILL2_EXP_EMU ? exp2_poly(a0) : ex2_approx(a0);
+          const float p1 = c < BLASST_PREFILL2_EXP_EMU ? exp2_poly(a1) : ex2_approx(a1);
+          rowsum += p0 + p1;
+          pk[x / 2] = pack_bf16x2(p0, p1);
+        }
+#endif
+        tmem_st16(lane_base + col_s + c * 16, pk);
+      }
+#endif
+      l = alpha * l + rowsum;
+      tc_wait_st();
+      // O_t is idle here (see the header comment); rescale whole warps.
+      if (__any_sync(FULL, rescale)) {
+        const float f = rescale ? alpha : 1.f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orow[32];
+          tmem_ld32(lane_base + col_o + c * 32, orow);
+          tc_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            orow[x] = __float_as_uint(__uint_as_float(orow[x]) * f);
+          tmem_st32(lane_base + col_o + c * 32, orow);
+        }
+        tc_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[C::B_PF + t]);
+      if (active) m_crit = fmaxf(m_crit, mt_s);
+    }
+    if (named_sync_or(bar_id, 128, !ok)) ok = false;
+
+    if (ok && elected && nb > 0) {
+      if (p.counters) {
+        atomicAdd(&p.counters[0], n_vis);
+        atomicAdd(&p.counters[1], n_skp);
+      }
+      if (p.mask)
+        for (int j = nb; j < p.nk; ++j) p.mask[mask_row + j] = 0;
+    }
+    if (ok && !stats_only && nb > 0) {
+      const bool w = mbar_wait(&bar[C::B_OD + t], 0, kWaitPrefillEpilogue, nb,
+                               600 + t);
+      tc_fence_after();
+      if (__all_sync(FULL, w)) {
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        __nv_bfloat16* orow_g =
+            p.o + ((size_t)(b * p.Hq + hq) * p.Lq + row_g) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orow[32];
+          tmem_ld32(lane_base + col_o + c * 32, orow);
+          tc_wait_ld();
+          if (active) {
+            uint4* dst = reinterpret_cast<uint4*>(orow_g + c * 32);
+#pragma unroll
+            for (int x = 0; x < 32; x += 8) {
+              uint4 w4;
+              w4.x = pack_bf16x2(__uint_as_float(orow[x]) * inv_l,
+                                 __uint_as_float(orow[x + 1]) * inv_l);
+              w4.y = pack_bf16x2(__uint_as_float(orow[x + 2]) * inv_l,
+                                 __uint_as_float(orow[x + 3]) * inv_l);
+              w4.z = pack_bf16x2(__uint_as_float(orow[x + 4]) * inv_l,
+                                 __uint_as_float(orow[x + 5]) * inv_l);
+              w4.w = pack_bf16x2(__uint_as_float(orow[x + 6]) * inv_l,
+                                 __uint_as_float(orow[x + 7]) * inv_l);
+              dst[x / 8] = w4;
+            }
+          }
+        }
+        if (active && p.lse)
+          p.lse[(size_t)(b * p.Hq + hq) * p.Lq + row_g] = m_ref + __logf(l);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+cudaError_t launch_prefill2(const PrefillProblem& pr, cudaStream_t st) {
+  using C = Prefill2Cfg<D>;
+  PrefillParams p;
+  memset(&p, 0, sizeof p);
+  if (!encode_map(&p.tq, pr.q, D, pr.Lq, (long long)pr.B * pr.Hq, 128) ||
+      !encode_map(&p.tk, pr.k, D, pr.Lkv, (long long)pr.B * pr.Hkv, 128) ||
+      !encode_map(&p.tv, pr.v, D, pr.Lkv, (long long)pr.B * pr.Hkv, 128))
+    return cudaErrorInvalidValue;
+  p.o = static_cast<__nv_bfloat16*>(pr.o);
+  p.lse = pr.lse;
+  p.counters = pr.counters;
+  p.mask = pr.mask;
+  p.B = pr.B;
+  p.Hq = pr.Hq;
+  p.Hkv = pr.Hkv;
+  p.Lq = pr.Lq;
+  p.Lkv = pr.Lkv;
+  p.nq = (pr.Lq + 127) / 128;
+  p.nk = (pr.Lkv + 127) / 128;
+  p.G = pr.Hq / pr.Hkv;
+  p.scale = pr.scale;
+  p.ln_lambda = pr.ln_lambda;
+  p.causal = pr.causal;
+  p.stats_only = pr.o == nullptr ? 1 : 0;
+  const long long grid = (long long)((p.nq + 1) / 2) * pr.B * pr.Hq;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(prefill2_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  prefill2_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM_ALLOC, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace blasst

@@ -239,6 +239,15 @@ blasst_status_t blasst_skip_stats_reset(unsigned long long *counters,
  * the first failed wait (block, step, parity, slot). */
 blasst_status_t blasst_check_device_error(int *where_out);
 
+/* Diagnostic: launches one CTA that waits on an mbarrier nothing arrives
+ * at, giving up after limit_cycles (1 .. 4e9) SM clock cycles the way every
+ * bounded wait of the library does.  The next blasst_check_device_error()
+ * then returns BLASST_ERR_TIMEOUT with where = 99.  Nothing faults: the
+ * context stays usable.  (Test support for the failure path; the BLASST
+ * pages have no counterpart.) */
+blasst_status_t blasst_selftest_wait_timeout(long long limit_cycles,
+                                             void *stream);
+
 const char *blasst_strerror(blasst_status_t status);
 
 /* Text of the last CUDA error seen by this thread's calls ("" if none). */
