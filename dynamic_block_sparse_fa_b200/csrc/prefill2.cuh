@@ -27,17 +27,6 @@
 
 #include "prefill.cuh"
 
-// 1: score rows are read from tensor memory twice (max pass, exp pass) so
-// that only 32 of them are live in registers; 0: the whole row stays live.
-#ifndef BLASST_PREFILL2_TWO_PASS
-#define BLASST_PREFILL2_TWO_PASS 0
-#endif
-// 1: exponentials of a kept block are evaluated two per instruction in
-// bf16x2 (P feeds the bf16 MMA in any case; the row sum is accumulated in
-// fp32 from the same bf16 values); 0: one fp32 exp2 per element.
-#ifndef BLASST_PREFILL2_EX2_BF16X2
-#define BLASST_PREFILL2_EX2_BF16X2 0
-#endif
 #ifndef BLASST_PREFILL2_NKS
 #define BLASST_PREFILL2_NKS 2
 #endif
@@ -45,6 +34,11 @@
 // run on the FMA pipe (exp2_poly) instead of the MUFU pipe.
 #ifndef BLASST_PREFILL2_EXP_EMU
 #define BLASST_PREFILL2_EXP_EMU 0
+#endif
+// Threads per score row (1 or 2): with 2, each tile's softmax runs on 8
+// warps, each thread owning half of the row's score and output columns.
+#ifndef BLASST_PREFILL2_COL_SPLIT
+#define BLASST_PREFILL2_COL_SPLIT 1
 #endif
 
 namespace blasst {
@@ -76,17 +70,22 @@ struct Prefill2Cfg {
   static constexpr int NBAR = B_DEC + 2 * R;
   static constexpr int OFF_DEC = OFF_BAR + NBAR * 8;  // int [2][R]
   static constexpr int OFF_TMEM = OFF_DEC + 2 * R * 4;
-  static constexpr int SMEM = OFF_TMEM + 16;
+  static constexpr int OFF_ABORT = OFF_TMEM + 4;      // int [2]
+  static constexpr int NH = BLASST_PREFILL2_COL_SPLIT;  // threads per row
+  static constexpr int WPT = 4 * NH;                  // softmax warps per tile
+  static constexpr int OFF_XMAX = (OFF_ABORT + 8 + 15) & ~15;  // f32 [2][2][NH][128]
+  static constexpr int OFF_XSUM = OFF_XMAX + 2 * 2 * NH * 128 * 4;  // f32 [2][NH][128]
+  static constexpr int SMEM = OFF_XSUM + 2 * NH * 128 * 4;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
   static constexpr int TMEM_COLS = 512;
   static constexpr int COL_S = 0;    // tile t at COL_S + t * 128
   static constexpr int COL_O = 256;  // tile t at COL_O + t * 128
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 64 + 2 * WPT * 32;
   static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1)
     prefill2_kernel(const __grid_constant__ PrefillParams p) {
   using C = Prefill2Cfg<D>;
   constexpr int BN = C::BN;
@@ -144,10 +143,12 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar[C::B_SF + t], 1);
-      mbar_init(&bar[C::B_PF + t], 4);
+      mbar_init(&bar[C::B_PF + t], C::WPT);  // one arrival per softmax warp
       mbar_init(&bar[C::B_OD + t], 1);
       for (int i = 0; i < C::R; ++i) mbar_init(&bar[C::B_DEC + t * C::R + i], 1);
     }
+    reinterpret_cast<volatile int*>(smem + C::OFF_ABORT)[0] = 0;
+    reinterpret_cast<volatile int*>(smem + C::OFF_ABORT)[1] = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -191,42 +192,46 @@ __global__ void __launch_bounds__(320, 1)
       for (int j = 0; j < n0; ++j) issue_k(j);
     }
     __syncwarp();
+    // Per block: first the V load (needed by the P.V right after the exp of
+    // this block), then the K prefetch two blocks ahead (needed only by the
+    // next block's QK, and blocked until this block's QKs release a slot).
     int vcount = 0;
     for (int j = 0; j < nblk; ++j) {
+      if (!stats_only) {
+        bool need = false, ok = true;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (need || j >= nblk_t[t]) continue;
+          const bool w = mbar_wait(&bar[C::B_DEC + t * C::R + j % C::R],
+                                   (j / C::R) & 1, kWaitPrefillLoad, j,
+                                   100 + t * C::R + j % C::R);
+          if (!__all_sync(FULL, w)) { ok = false; break; }
+          need = dec_flag[t * C::R + j % C::R] != 0;
+        }
+        if (!ok) break;
+        if (need) {
+          const int n = vcount++;
+          const int slot = n % C::NVS;
+          if (n >= C::NVS) {
+            const bool w = mbar_wait(&bar[C::B_VE + slot], ((n / C::NVS) - 1) & 1,
+                                     kWaitPrefillLoad, j, 200 + slot);
+            if (!__all_sync(FULL, w)) break;
+          }
+          if (leader) {
+            mbar_arrive_expect_tx(&bar[C::B_VF + slot], C::KBYTES);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(sV + slot * C::KBYTES + c * C::BOX_K, &p.tv,
+                          &bar[C::B_VF + slot], c * 64, j * BN, zk, pol_kv);
+          }
+          __syncwarp();
+        }
+      }
       if (j + C::NKS < nblk) {
         const bool w = mbar_wait(&bar[C::B_KE + j % C::NKS], (j / C::NKS) & 1,
                                  kWaitPrefillLoad, j, j % C::NKS);
         if (!__all_sync(FULL, w)) break;
         if (leader) issue_k(j + C::NKS);
-        __syncwarp();
-      }
-      if (stats_only) continue;
-      bool need = false, ok = true;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (need || j >= nblk_t[t]) continue;
-        const bool w = mbar_wait(&bar[C::B_DEC + t * C::R + j % C::R],
-                                 (j / C::R) & 1, kWaitPrefillLoad, j,
-                                 100 + t * C::R + j % C::R);
-        if (!__all_sync(FULL, w)) { ok = false; break; }
-        need = dec_flag[t * C::R + j % C::R] != 0;
-      }
-      if (!ok) break;
-      if (need) {
-        const int n = vcount++;
-        const int slot = n % C::NVS;
-        if (n >= C::NVS) {
-          const bool w = mbar_wait(&bar[C::B_VE + slot], ((n / C::NVS) - 1) & 1,
-                                   kWaitPrefillLoad, j, 200 + slot);
-          if (!__all_sync(FULL, w)) break;
-        }
-        if (leader) {
-          mbar_arrive_expect_tx(&bar[C::B_VF + slot], C::KBYTES);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sV + slot * C::KBYTES + c * C::BOX_K, &p.tv,
-                        &bar[C::B_VF + slot], c * 64, j * BN, zk, pol_kv);
-        }
         __syncwarp();
       }
     }
@@ -320,10 +325,19 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     // ------------------------------------------------------------------
-    // Softmax warpgroups: warps 2..5 tile 0, warps 6..9 tile 1
+    // Softmax: warps 2 .. 2+WPT-1 tile 0, the next WPT warps tile 1.  A row
+    // is shared by NH threads (warps with the same TMEM lane quadrant), each
+    // owning BN/NH score columns and D/NH output columns.
     // ------------------------------------------------------------------
-    const int t = (warp - 2) >> 2;
+    constexpr int NH = C::NH;
+    constexpr int CPT = BN / NH;      // score columns per thread
+    constexpr int OPT = D / NH;       // output columns per thread
+    const int gw = warp - 2;
+    const int t = gw / C::WPT;
+    const int wi = gw - t * C::WPT;
+    const int half = wi >> 2;
     const uint32_t bar_id = 1 + t;
+    constexpr uint32_t kBarThreads = 32 * C::WPT;
     const int nb = nblk_t[t];
     const int quad = warp & 3;
     const int rr = quad * 32 + lane;
@@ -333,57 +347,39 @@ __global__ void __launch_bounds__(320, 1)
     const int lim = p.causal ? min(row_g + (p.Lkv - p.Lq), p.Lkv - 1)
                              : p.Lkv - 1;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t col_s = C::COL_S + t * 128;
-    const uint32_t col_o = C::COL_O + t * 128;
+    const uint32_t col_s = C::COL_S + t * 128 + half * CPT;      // my scores
+    const uint32_t col_p = C::COL_S + t * 128 + half * (CPT / 2);  // my P
+    const uint32_t col_o = C::COL_O + t * 128 + half * OPT;      // my O
     const float scale = p.scale;
     const float ln_lambda = p.ln_lambda;
     const float sl2 = scale * kPrefLog2e;
-    const bool elected = (((warp - 2) & 3) == 0 && lane == 0);
+    const bool elected = (wi == 0 && lane == 0);
     const size_t mask_row =
         ((size_t)(b * p.Hq + hq) * p.nq + tile) * (size_t)p.nk;
+    float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);  // [2][2][NH][128]
+    float* xsum = reinterpret_cast<float*>(smem + C::OFF_XSUM);  // [2][NH][128]
+    volatile int* abort_t = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
 
     float m_crit = -INFINITY;
     float m_ref = -INFINITY;
-    float l = 0.f;
+    float l = 0.f;  // this thread's part of the row normaliser
     unsigned long long n_vis = 0, n_skp = 0;
     bool ok = true;
 
     for (int j = 0; j < nb; ++j) {
-      if (ok)
-        ok = mbar_wait(&bar[C::B_SF + t], j & 1, kWaitPrefillSoftmax, j, 400 + t);
+      if (!mbar_wait(&bar[C::B_SF + t], j & 1, kWaitPrefillSoftmax, j, 400 + t))
+        abort_t[t] = 1;  // read by every thread of the tile after the vote
       tc_fence_after();
-      if (named_sync_or(bar_id, 128, !ok)) { ok = false; break; }
-      const int col0 = j * BN;
-      const bool need_mask = col0 + BN - 1 > lim;
-#if BLASST_PREFILL2_TWO_PASS
-      // Pass 1: row max over the score row, 32 columns at a time.
-      float mt;
-      {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        const int lim_rel = lim - col0;  // last visible column of the block
+      uint32_t sr[CPT / 32][32];
 #pragma unroll
-        for (int h = 0; h < BN / 32; ++h) {
-          uint32_t sr[32];
-          tmem_ld32(lane_base + col_s + h * 32, sr);
-          tc_wait_ld();
-#pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            float v = __uint_as_float(sr[x]);
-            if (need_mask && h * 32 + x > lim_rel) v = -INFINITY;
-            m4[x & 3] = fmaxf(m4[x & 3], v);
-          }
-        }
-        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      }
-#else
-      uint32_t sr[BN / 32][32];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c)
+      for (int c = 0; c < CPT / 32; ++c)
         tmem_ld32(lane_base + col_s + c * 32, sr[c]);
       tc_wait_ld();
-      if (need_mask) {
+
+      const int col0 = j * BN + half * CPT;  // first score column of mine
+      if (col0 + CPT - 1 > lim) {
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
+        for (int c = 0; c < CPT / 32; ++c)
 #pragma unroll
           for (int x = 0; x < 32; ++x)
             if (col0 + c * 32 + x > lim) sr[c][x] = __float_as_uint(-INFINITY);
@@ -392,19 +388,27 @@ __global__ void __launch_bounds__(320, 1)
       {
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
+        for (int c = 0; c < CPT / 32; ++c)
 #pragma unroll
           for (int x = 0; x < 32; ++x)
             m4[x & 3] = fmaxf(m4[x & 3], __uint_as_float(sr[c][x]));
         mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
-#endif
-      const float mt_s = mt * scale;
-      const bool pred = !active || mt_s == -INFINITY ||
-                        (mt_s - m_crit < ln_lambda);
+      float* xm = xmax + (((j & 1) * 2 + t) * NH) * 128;
+      if (NH > 1) xm[half * 128 + rr] = mt;
+      // A row passes the criterion iff each of its parts does, so the vote
+      // needs no exchange; the barrier also publishes the part maxima.
+      const float mt_part = mt * scale;
+      const bool pred = !active || mt_part == -INFINITY ||
+                        (mt_part - m_crit < ln_lambda);
       tc_fence_before();
       const bool skip =
-          named_sync_and(bar_id, 128, pred) && (ln_lambda > -INFINITY);
+          named_sync_and(bar_id, kBarThreads, pred) && (ln_lambda > -INFINITY);
+      if (abort_t[t]) { ok = false; break; }
+#pragma unroll
+      for (int h = 0; h < NH; ++h)
+        if (h != half) mt = fmaxf(mt, xm[h * 128 + rr]);
+      const float mt_s = mt * scale;  // whole-row block max
       if (elected) {
         ++n_vis;
         if (skip) ++n_skp;
@@ -432,70 +436,28 @@ __global__ void __launch_bounds__(320, 1)
       }
       const float mb = (active && m_ref != -INFINITY) ? m_ref * kPrefLog2e
                                                       : INFINITY;
-      float rowsum = 0.f;
-#if BLASST_PREFILL2_TWO_PASS
-      // Pass 2: reload 32 columns at a time, exp, P over the first half.
-      const int lim_rel = lim - col0;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int h = 0; h < BN / 32; ++h) {
-        uint32_t sr[32];
-        tmem_ld32(lane_base + col_s + h * 32, sr);
-        tc_wait_ld();
+      for (int c = 0; c < CPT / 32; ++c) {
         uint32_t pk[16];
-#pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          float v0 = __uint_as_float(sr[x]);
-          float v1 = __uint_as_float(sr[x + 1]);
-          if (need_mask) {
-            if (h * 32 + x > lim_rel) v0 = -INFINITY;
-            if (h * 32 + x + 1 > lim_rel) v1 = -INFINITY;
-          }
-          const float p0 = ex2_approx(fmaf(v0, sl2, -mb));
-          const float p1 = ex2_approx(fmaf(v1, sl2, -mb));
-          rowsum += p0 + p1;
-          pk[x / 2] = pack_bf16x2(p0, p1);
-        }
-        // P of chunk h (16 columns) lands in columns [16h, 16h+16), below
-        // the scores of every chunk not yet reloaded (chunk h' starts at 32h').
-        tmem_st16(lane_base + col_s + h * 16, pk);
-      }
-#else
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t pk[16];
-#if BLASST_PREFILL2_EX2_BF16X2
-        float2 rs2 = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          const float2 a2 = __ffma2_rn(
-              make_float2(__uint_as_float(sr[c][x]), __uint_as_float(sr[c][x + 1])),
-              make_float2(sl2, sl2), make_float2(-mb, -mb));
-          const uint32_t e = ex2_bf16x2(pack_bf16x2(a2.x, a2.y));
-          pk[x / 2] = e;
-          rs2 = __fadd2_rn(rs2, make_float2(bf16lo(e), bf16hi(e)));
-        }
-        rowsum += rs2.x + rs2.y;
-#else
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
           const float a0 = fmaf(__uint_as_float(sr[c][x]), sl2, -mb);
           const float a1 = fmaf(__uint_as_float(sr[c][x + 1]), sl2, -mb);
           const float p0 = c < BLASST_PREFILL2_EXP_EMU ? exp2_poly(a0) : ex2_approx(a0);
           const float p1 = c < BLASST_PREFILL2_EXP_EMU ? exp2_poly(a1) : ex2_approx(a1);
-          rowsum += p0 + p1;
+          rs[(x >> 1) & 3] += p0 + p1;
           pk[x / 2] = pack_bf16x2(p0, p1);
         }
-#endif
-        tmem_st16(lane_base + col_s + c * 16, pk);
+        tmem_st16(lane_base + col_p + c * 16, pk);
       }
-#endif
-      l = alpha * l + rowsum;
+      l = alpha * l + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
       tc_wait_st();
       // O_t is idle here (see the header comment); rescale whole warps.
       if (__any_sync(FULL, rescale)) {
         const float f = rescale ? alpha : 1.f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < OPT / 32; ++c) {
           uint32_t orow[32];
           tmem_ld32(lane_base + col_o + c * 32, orow);
           tc_wait_ld();
@@ -511,7 +473,6 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) mbar_arrive(&bar[C::B_PF + t]);
       if (active) m_crit = fmaxf(m_crit, mt_s);
     }
-    if (named_sync_or(bar_id, 128, !ok)) ok = false;
 
     if (ok && elected && nb > 0) {
       if (p.counters) {
@@ -525,12 +486,20 @@ __global__ void __launch_bounds__(320, 1)
       const bool w = mbar_wait(&bar[C::B_OD + t], 0, kWaitPrefillEpilogue, nb,
                                600 + t);
       tc_fence_after();
-      if (__all_sync(FULL, w)) {
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-        __nv_bfloat16* orow_g =
-            p.o + ((size_t)(b * p.Hq + hq) * p.Lq + row_g) * D;
+      float lrow = l;
+      if (NH > 1) {
+        xsum[(t * NH + half) * 128 + rr] = l;
+        named_sync(bar_id, kBarThreads);
+        lrow = 0.f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int h = 0; h < NH; ++h) lrow += xsum[(t * NH + h) * 128 + rr];
+      }
+      if (__all_sync(FULL, w)) {
+        const float inv_l = (lrow > 0.f) ? 1.f / lrow : 0.f;
+        __nv_bfloat16* orow_g =
+            p.o + ((size_t)(b * p.Hq + hq) * p.Lq + row_g) * D + half * OPT;
+#pragma unroll
+        for (int c = 0; c < OPT / 32; ++c) {
           uint32_t orow[32];
           tmem_ld32(lane_base + col_o + c * 32, orow);
           tc_wait_ld();
@@ -551,8 +520,8 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
         }
-        if (active && p.lse)
-          p.lse[(size_t)(b * p.Hq + hq) * p.Lq + row_g] = m_ref + __logf(l);
+        if (active && half == 0 && p.lse)
+          p.lse[(size_t)(b * p.Hq + hq) * p.Lq + row_g] = m_ref + __logf(lrow);
       }
     }
   }

@@ -220,13 +220,6 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return x < -126.0f ? 0.0f : r;
 }
 
-// Two base-2 exponentials of a packed bf16 pair in one instruction.
-__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
-  uint32_t y;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
 // bf16x2 word -> two floats (exact: a bf16 is the top half of an f32).
 __device__ __forceinline__ float bf16lo(uint32_t w) {
   return __uint_as_float(w << 16);
