@@ -73,9 +73,11 @@ struct Prefill2Cfg {
   static constexpr int OFF_ABORT = OFF_TMEM + 4;      // int [2]
   static constexpr int NH = BLASST_PREFILL2_COL_SPLIT;  // threads per row
   static constexpr int WPT = 4 * NH;                  // softmax warps per tile
+  // row-part exchange buffers, needed only when a row is split (NH > 1)
+  static constexpr int XN = NH > 1 ? NH : 0;
   static constexpr int OFF_XMAX = (OFF_ABORT + 8 + 15) & ~15;  // f32 [2][2][NH][128]
-  static constexpr int OFF_XSUM = OFF_XMAX + 2 * 2 * NH * 128 * 4;  // f32 [2][NH][128]
-  static constexpr int SMEM = OFF_XSUM + 2 * NH * 128 * 4;
+  static constexpr int OFF_XSUM = OFF_XMAX + 2 * 2 * XN * 128 * 4;  // f32 [2][NH][128]
+  static constexpr int SMEM = OFF_XSUM + 2 * XN * 128 * 4;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
   static constexpr int TMEM_COLS = 512;
   static constexpr int COL_S = 0;    // tile t at COL_S + t * 128
