@@ -50,6 +50,14 @@ def _load():
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_double, ctypes.c_double, ctypes.c_int,
             ctypes.c_int, _dp, _dp, _dp, _dp, _u8p, _dp, _i64p, ctypes.c_int]
+        lib.oracle_decode_paged.restype = ctypes.c_int
+        lib.oracle_decode_paged.argtypes = [
+            _u16p, _u16p, _u16p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+            _i32p, ctypes.c_int, _i32p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_double, ctypes.c_double, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int,
+            _dp, _dp, _dp, _dp, _u8p, _dp, _i64p, ctypes.c_int]
         lib.oracle_combine.restype = None
         lib.oracle_combine.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_int, _dp, _dp]
@@ -145,6 +153,67 @@ def decode(q, k, v, scale, ln_lambda, Bc, num_splits, n_threads=0):
         int(n_threads))
     if rc != 0:
         raise ValueError("oracle_decode rejected its arguments")
+    threads = n_threads if n_threads > 0 else n_threads_default()
+    return dict(o=o, lse=lse, o_part=op, lse_part=lp, mask=mask,
+                margin=margin, visited=int(counts[0]),
+                skipped=int(counts[1]), threads=threads)
+
+
+def _i32(x):
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(x), dtype=np.int32)
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale, ln_lambda,
+                 num_splits, Bc=64, per_length=False, nk_max=None,
+                 page_stride=None, n_threads=0):
+    """Paged, variable-length decode: gather, then the decode above.
+
+    q [B,Hq,d] bf16.  k_pages / v_pages: either [num_pages,Hkv,page_size,d]
+    bf16 (made contiguous), or flat 1-D pools with ``page_stride`` given
+    (then pass ``(pool, num_pages, Hkv, page_size, d)`` tuples).
+    block_table [B,max_pages] int32, seq_lens [B] int32.  ``per_length``:
+    ln_lambda is ln a and sequence b uses min(0, ln a - ln L_b).
+    Returns the keys of ``decode`` with mask/margin [B,Hkv,nk_max].
+    """
+    lib = _load()
+    qb = _bits(q)
+    B, Hq, d = qb.shape
+    if isinstance(k_pages, tuple):
+        kp, num_pages, Hkv, ps, d2 = k_pages
+        vp = v_pages[0]
+        kb, vb = _bits(kp).reshape(-1), _bits(vp).reshape(-1)
+        stride = int(page_stride)
+    else:
+        kb, vb = _bits(k_pages), _bits(v_pages)
+        num_pages, Hkv, ps, d2 = kb.shape
+        stride = Hkv * ps * d2 if page_stride is None else int(page_stride)
+    assert d2 == d
+    bt = _i32(block_table)
+    sl = _i32(seq_lens).reshape(-1)
+    assert sl.shape[0] == B and bt.shape[0] == B
+    max_pages = bt.shape[1] if bt.ndim == 2 else 0
+    if nk_max is None:
+        nk_max = -(-int(max_pages * ps) // Bc)
+    S = int(num_splits)
+    o = np.zeros((B, Hq, d), np.float64)
+    lse = np.zeros((B, Hq), np.float64)
+    op = np.zeros((B, Hq, S, d), np.float64)
+    lp = np.zeros((B, Hq, S), np.float64)
+    mask = np.zeros((B, Hkv, nk_max), np.uint8)
+    margin = np.zeros((B, Hkv, nk_max), np.float64)
+    counts = np.zeros(2, np.int64)
+    rc = lib.oracle_decode_paged(
+        _ptr(qb, _u16p), _ptr(kb, _u16p), _ptr(vb, _u16p), stride,
+        int(num_pages), int(ps), _ptr(bt, _i32p), int(max_pages),
+        _ptr(sl, _i32p), B, Hq, Hkv, d, float(scale), float(ln_lambda),
+        int(bool(per_length)), Bc, S, int(nk_max),
+        _ptr(o, _dp), _ptr(lse, _dp), _ptr(op, _dp), _ptr(lp, _dp),
+        _ptr(mask, _u8p), _ptr(margin, _dp), _ptr(counts, _i64p),
+        int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_decode_paged rejected its arguments")
     threads = n_threads if n_threads > 0 else n_threads_default()
     return dict(o=o, lse=lse, o_part=op, lse_part=lp, mask=mask,
                 margin=margin, visited=int(counts[0]),

@@ -329,3 +329,118 @@ int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     counts[1] = skp;
     return 0;
 }
+
+/*
+ * Paged, variable-length decode.  The logical cache of (sequence b, KV head
+ * h) is gathered from the page pool token by token -- token t of sequence b
+ * is row (h * page_size + t % page_size) of page
+ * block_table[b * max_pages + t / page_size] -- and then decoded exactly as
+ * oracle_decode decodes a contiguous cache of length seq_lens[b].
+ */
+int oracle_decode_paged(const uint16_t *q, const uint16_t *k_pool,
+                        const uint16_t *v_pool, int64_t page_stride,
+                        int num_pages, int page_size,
+                        const int32_t *block_table, int max_pages,
+                        const int32_t *seq_lens, int B, int Hq, int Hkv, int d,
+                        double scale, double ln_lambda, int per_length, int Bc,
+                        int num_splits, int nk_max, double *o, double *lse,
+                        double *o_part, double *lse_part, uint8_t *mask,
+                        double *margin, int64_t *counts, int n_threads) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || d < 1 || Bc < 1 ||
+        num_splits < 1 || page_size < 1 || num_pages < 0 || max_pages < 0 ||
+        nk_max < 0 || isnan(ln_lambda) || ln_lambda == INFINITY ||
+        (!per_length && ln_lambda > 0.0) ||
+        page_stride < (int64_t)Hkv * page_size * d)
+        return -1;
+    /* Every length and every page id the lengths reach must be valid. */
+    for (int b = 0; b < B; ++b) {
+        int L = seq_lens[b];
+        if (L < 0 || (int64_t)L > (int64_t)max_pages * page_size ||
+            (L + Bc - 1) / Bc > nk_max)
+            return -1;
+        for (int p = 0; p < (L + page_size - 1) / page_size; ++p) {
+            int id = block_table[(size_t)b * max_pages + p];
+            if (id < 0 || id >= num_pages) return -1;
+        }
+    }
+    int G = Hq / Hkv;
+    int S = num_splits;
+    double *op = (double *)malloc(sizeof(double) * (size_t)B * Hq * S * d);
+    double *lp = (double *)malloc(sizeof(double) * (size_t)B * Hq * S);
+    if (mask) memset(mask, ORACLE_NOT_VISITED, (size_t)B * Hkv * nk_max);
+    if (margin)
+        for (size_t i = 0; i < (size_t)B * Hkv * nk_max; ++i) margin[i] = NAN;
+    set_threads(n_threads);
+    int64_t vis = 0, skp = 0;
+
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : vis, skp)
+    for (int bh = 0; bh < B * Hkv; ++bh) {
+        int b = bh / Hkv, hkv = bh % Hkv;
+        int L = seq_lens[b];
+        int nk = (L + Bc - 1) / Bc;
+        /* lambda = a / L with L this sequence's own context length */
+        double lnl = ln_lambda;
+        if (per_length && L > 0 && ln_lambda > -INFINITY) {
+            lnl = ln_lambda - log((double)L);
+            if (lnl > 0.0) lnl = 0.0;
+        }
+        /* gather the logical K and V rows of (b, hkv) */
+        uint16_t *kh = (uint16_t *)malloc(sizeof(uint16_t) * ((size_t)L * d + 1));
+        uint16_t *vh = (uint16_t *)malloc(sizeof(uint16_t) * ((size_t)L * d + 1));
+        for (int t = 0; t < L; ++t) {
+            int id = block_table[(size_t)b * max_pages + t / page_size];
+            size_t src = (size_t)id * page_stride +
+                         ((size_t)hkv * page_size + t % page_size) * d;
+            memcpy(kh + (size_t)t * d, k_pool + src, sizeof(uint16_t) * d);
+            memcpy(vh + (size_t)t * d, v_pool + src, sizeof(uint16_t) * d);
+        }
+        double *qrows = (double *)malloc(sizeof(double) * (size_t)G * d);
+        int *limit = (int *)malloc(sizeof(int) * (size_t)G);
+        double *m = (double *)malloc(sizeof(double) * (size_t)G);
+        double *l = (double *)malloc(sizeof(double) * (size_t)G);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)G * d);
+        for (int g = 0; g < G; ++g) {
+            const uint16_t *qg = q + ((size_t)b * Hq + hkv * G + g) * d;
+            for (int x = 0; x < d; ++x)
+                qrows[(size_t)g * d + x] = oracle_bf16_to_double(qg[x]);
+            limit[g] = L - 1;
+        }
+        uint8_t *mk = mask ? mask + (size_t)bh * nk_max : NULL;
+        double *mg = margin ? margin + (size_t)bh * nk_max : NULL;
+        for (int s = 0; s < S; ++s) {
+            int j0 = oracle_split_begin(nk, S, s);
+            int j1 = oracle_split_begin(nk, S, s + 1);
+            int64_t uv = 0, us = 0;
+            run_tile(G, qrows, limit, kh, vh, L, d, scale, lnl, Bc, j0, j1, m,
+                     l, acc, mk, mg, &uv, &us);
+            vis += uv;
+            skp += us;
+            for (int g = 0; g < G; ++g) {
+                size_t row = ((size_t)b * Hq + hkv * G + g) * S + s;
+                if (l[g] > 0.0) {
+                    for (int x = 0; x < d; ++x)
+                        op[row * d + x] = acc[(size_t)g * d + x] / l[g];
+                    lp[row] = m[g] + log(l[g]);
+                } else { /* empty split */
+                    for (int x = 0; x < d; ++x) op[row * d + x] = 0.0;
+                    lp[row] = -INFINITY;
+                }
+            }
+        }
+        free(kh);
+        free(vh);
+        free(qrows);
+        free(limit);
+        free(m);
+        free(l);
+        free(acc);
+    }
+    oracle_combine(op, lp, B * Hq, S, d, o, lse);
+    if (o_part) memcpy(o_part, op, sizeof(double) * (size_t)B * Hq * S * d);
+    if (lse_part) memcpy(lse_part, lp, sizeof(double) * (size_t)B * Hq * S);
+    free(op);
+    free(lp);
+    counts[0] = vis;
+    counts[1] = skp;
+    return 0;
+}

@@ -99,6 +99,37 @@ int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                   int n_threads);
 
 /*
+ * Paged, variable-length decode (block-table indirection).
+ *
+ * Sequence b holds seq_lens[b] tokens.  Its token t lives in page
+ * block_table[b * max_pages + t / page_size]; inside a page, KV head h holds
+ * rows [h * page_size, (h + 1) * page_size) of d elements, and page p starts
+ * p * page_stride elements into k_pool / v_pool.  The logical cache of each
+ * (b, h) is gathered from the pool and decoded as oracle_decode decodes a
+ * contiguous cache of length seq_lens[b]: S splits over the sequence's own
+ * ceil(L_b / Bc) blocks, empty splits contribute nothing, and an empty
+ * sequence gives o = 0 and lse = -inf.
+ *
+ * per_length != 0: ln_lambda holds ln a (any finite value, or -inf) and
+ * sequence b uses
+ *   ln lambda_b = min(0, ln a - ln L_b)       (lambda = a / L, L its length)
+ * per_length == 0: ln_lambda <= 0 (or -inf) for every sequence.
+ * mask / margin: [B,Hkv,nk_max]; blocks past a sequence's end stay
+ * ORACLE_NOT_VISITED / NaN.
+ * Returns -1 on invalid arguments, including a length outside
+ * [0, max_pages * page_size] or a page id outside [0, num_pages).
+ */
+int oracle_decode_paged(const uint16_t *q, const uint16_t *k_pool,
+                        const uint16_t *v_pool, int64_t page_stride,
+                        int num_pages, int page_size,
+                        const int32_t *block_table, int max_pages,
+                        const int32_t *seq_lens, int B, int Hq, int Hkv, int d,
+                        double scale, double ln_lambda, int per_length, int Bc,
+                        int num_splits, int nk_max, double *o, double *lse,
+                        double *o_part, double *lse_part, uint8_t *mask,
+                        double *margin, int64_t *counts, int n_threads);
+
+/*
  * Log-sum-exp merge of S partial results for n rows:
  *   lse = ln sum_s exp(lse_s),  o = sum_s exp(lse_s - lse) * o_s.
  * o_part [n][S][d], lse_part [n][S]; o [n][d], lse [n].
