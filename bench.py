@@ -381,6 +381,11 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
         "clocks": clk.summary(),
     }
 
+    if not args.no_paged:
+        line["decode_paged"] = run_decode_paged(args, bl, dev, stream, q, k, v,
+                                                lnl, cal["a"], S, ms_max / K,
+                                                by_call)
+
     # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
     if rank == 0 and world == 1 and not args.no_cpu:
         gbs, secs, threads, sample = cpu_oracle_decode_sample(
@@ -389,6 +394,98 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
                                 "cores": threads, "kind": "oracle",
                                 "sample": sample, "seconds": round(secs, 2)}
     return line
+
+
+def paged_kept_rows(mask, lens, Bc):
+    """Rows of V a paged call reads: Bc per kept block, fewer for each
+    sequence's ragged last block.  mask [B, Hkv, nk_max]."""
+    kept = (mask == 1)
+    rows = kept.sum().item() * Bc
+    for b, L in enumerate(lens):
+        nk = -(-L // Bc)
+        last = L - (nk - 1) * Bc
+        if nk and last != Bc:
+            rows -= int(kept[b, :, nk - 1].sum().item()) * (Bc - last)
+    return rows
+
+
+def run_decode_paged(args, bl, dev, stream, q, k, v, lnl, a, S, ms_contig,
+                     by_contig):
+    """Paged-cache decode on the same workload: the contiguous cache's tokens
+    in a shuffled pool (64- and 16-token pages), then a variable-length
+    batch (lengths uniform in [1K, 64K]) with the per-sequence threshold
+    lambda = a / L_b."""
+    from synth import config_seed, paginate, planted_gap_kv_inplace
+    B, Hq, d = q.shape
+    Hkv, Lkv = k.shape[1], k.shape[2]
+    Bc = DEC["Bc"]
+    K, W = args.steps, args.warmup
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    out = {}
+    for ps in (64, 16):
+        pk = paginate(k, v, [Lkv] * B, ps, seed=config_seed(7, ps))
+        ws = torch.empty(bl.blasst_decode_workspace_size(B, Hq, d, S),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: bl.blasst_decode_paged(
+            q, pk.k_pages, pk.v_pages, pk.block_table, pk.seq_lens,
+            max_seq_len=Lkv, ln_lambda=lnl, num_splits=S, o=o, lse=lse,
+            workspace=ws)
+        ms = time_calls(fn, K, W, stream) / K
+        out[f"uniform_page{ps}"] = {
+            "workload": f"same tokens as the contiguous run, shuffled pool of "
+                        f"{ps}-token pages",
+            "us": round(ms * 1e3, 2), "GBps": round(by_contig / (ms / 1e3) / 1e9, 1),
+            "vs_contiguous": round(ms_contig / ms, 4)}
+        del pk, ws
+        torch.cuda.empty_cache()
+
+    # variable lengths
+    g = torch.Generator().manual_seed(config_seed(8))
+    lens = torch.randint(1024, 65536 + 1, (B,), generator=g).tolist()
+    Lmax = max(lens)
+    kk = torch.empty(B, Hkv, Lmax, d, dtype=torch.bfloat16, device=dev)
+    vv = torch.empty_like(kk)
+    qq = torch.empty_like(q)
+    planted_gap_kv_inplace(kk, vv, qq, block=Bc, gap=8.0, heavy_frac=0.03,
+                           seed=config_seed(8, 1))
+    pk = paginate(kk, vv, lens, 16, seed=config_seed(8, 2))
+    del kk, vv
+    torch.cuda.empty_cache()
+    Sv = bl.blasst_decode_splits(B, Hkv, Lmax, Bc)
+    nk_max = -(-Lmax // Bc)
+    ws = torch.empty(bl.blasst_decode_workspace_size(B, Hq, d, Sv),
+                     dtype=torch.uint8, device=dev)
+    st = bl.Stats(device=dev, mask_numel=B * Hkv * nk_max)
+    ln_a = math.log(a)
+    kw = dict(max_seq_len=Lmax, ln_lambda=ln_a, per_length=True,
+              num_splits=Sv, o=o, lse=lse, workspace=ws)
+    bl.blasst_decode_paged(qq, pk.k_pages, pk.v_pages, pk.block_table,
+                           pk.seq_lens, stats=st, **kw)
+    torch.cuda.synchronize()
+    vis, skp = st.read()
+    rows = paged_kept_rows(st.mask.view(B, Hkv, nk_max), lens, Bc)
+    by = (2 * d * Hkv * sum(lens) + 2 * d * rows + 2 * B * Hq * d
+          + B * Hq * Sv * (d + 1) * 4 * 2 + B * Hq * d * 2 + B * Hq * 4)
+    fn = lambda: bl.blasst_decode_paged(qq, pk.k_pages, pk.v_pages,
+                                        pk.block_table, pk.seq_lens, **kw)
+    ms = time_calls(fn, K, W, stream) / K
+    kw_dense = dict(kw, ln_lambda=-math.inf, per_length=False)
+    fn_d = lambda: bl.blasst_decode_paged(qq, pk.k_pages, pk.v_pages,
+                                          pk.block_table, pk.seq_lens,
+                                          **kw_dense)
+    ms_d = time_calls(fn_d, K, W, stream) / K
+    out["varlen_page16"] = {
+        "workload": f"B{B} lengths uniform in [1K, 64K] (sum {sum(lens)}), "
+                    f"shuffled pool of 16-token pages, lambda = a / L_b "
+                    f"with a = {a:.4g}",
+        "splits": Sv, "sparsity": skp / vis, "us": round(ms * 1e3, 2),
+        "GBps": round(by / (ms / 1e3) / 1e9, 1), "bytes_per_call": by,
+        "dense_us": round(ms_d * 1e3, 2),
+        "speedup_vs_dense": round(ms_d / ms, 4)}
+    del pk, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
@@ -531,6 +628,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-paged", action="store_true",
+                    help="skip the paged-cache decode measurements")
     ap.add_argument("--decode-batch", type=int, default=DEC["B"],
                     help="sequences per GPU (profiling runs use fewer)")
     ap.add_argument("--decode-lnl", type=float, default=None,

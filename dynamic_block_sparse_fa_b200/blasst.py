@@ -77,6 +77,11 @@ _lib.blasst_decode.restype = _i
 _lib.blasst_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                _f, _f, _i, _i, _vp, _sz,
                                ctypes.POINTER(SkipStats), _vp]
+_lib.blasst_decode_paged.restype = _i
+_lib.blasst_decode_paged.argtypes = [_vp, _vp, _vp, ctypes.c_longlong, _i, _i,
+                                     _vp, _i, _vp, _i, _vp, _vp, _i, _i, _i,
+                                     _i, _f, _f, _i, _i, _vp, _sz,
+                                     ctypes.POINTER(SkipStats), _vp]
 _lib.blasst_decode_noalloc.restype = _i
 _lib.blasst_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                        _i, _f, _f, _i, _i,
@@ -104,6 +109,7 @@ _lib.blasst_version.restype = ctypes.c_char_p
 _lib.blasst_version.argtypes = []
 
 EXPORTED = ["blasst_prefill", "blasst_decode", "blasst_decode_noalloc",
+            "blasst_decode_paged",
             "blasst_decode_workspace_size",
             "blasst_decode_splits", "blasst_calibrate", "blasst_fit_a",
             "blasst_skip_stats_reset", "blasst_check_device_error",
@@ -173,13 +179,14 @@ def blasst_skip_stats_reset(counters: torch.Tensor, stream=None):
 
 
 def blasst_check_device_error():
-    """Returns (status, where): status 0 or BLASST_ERR_TIMEOUT (5); for a
-    timeout `where` is a string naming the first failed wait."""
+    """Returns (status, where): status 0, BLASST_ERR_TIMEOUT (5, a wait gave
+    up) or BLASST_ERR_INVALID_ARG (1, a paged-decode length or page id out of
+    range); for either error `where` is a string naming the first one."""
     where = ctypes.c_int(0)
     st = _lib.blasst_check_device_error(ctypes.byref(where))
-    if st not in (0, 5):
+    if st not in (0, 1, 5):
         _check(st, "blasst_check_device_error")
-    if st == 5:
+    if st in (1, 5):
         return st, f"{where.value}: {blasst_last_error()}"
     return st, where.value
 
@@ -253,6 +260,66 @@ def blasst_decode(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
         float(scale), float(ln_lambda), Bc, S, _ptr(workspace), ws_bytes,
         stats.c_struct if stats is not None else None, _stream(stream))
     _check(st, "blasst_decode")
+    return o, lse
+
+
+def blasst_decode_paged(q, k_pages, v_pages, block_table, seq_lens, *,
+                        max_seq_len=None, scale=None, ln_lambda=-math.inf,
+                        per_length=False, num_splits=0, o=None, lse=None,
+                        want_lse=True, workspace=None,
+                        stats: Stats | None = None, stats_only=False,
+                        stream=None):
+    """BLASST decode over a paged KV cache.
+
+    q [B,Hq,d] bf16.  k_pages / v_pages: [num_pages, Hkv, page_size, d] bf16
+    views whose last three dimensions are contiguous (dimension 0 may have
+    any stride, e.g. the K and V halves of one interleaved pool
+    [num_pages, 2, Hkv, page_size, d]); both must have the same page stride.
+    block_table [B, max_pages] int32, seq_lens [B] int32, on the device.
+    max_seq_len: host upper bound on seq_lens (default: what the table
+    holds, max_pages * page_size; it sizes the split policy and the mask).
+    per_length: ln_lambda is ln a and sequence b uses min(0, ln a - ln L_b).
+    Returns (o, lse); both None when stats_only.  Bad lengths or page ids
+    are caught on the device: see blasst_check_device_error()."""
+    B, Hq, d = q.shape
+    P, Hkv, ps, d2 = k_pages.shape
+    if d2 != d or tuple(v_pages.shape) != tuple(k_pages.shape):
+        raise ValueError("k_pages / v_pages shapes")
+    for t in (k_pages, v_pages):
+        if t.stride()[1:] != (ps * d, d, 1):
+            raise ValueError("pages must be contiguous inside a page")
+    if k_pages.stride(0) != v_pages.stride(0):
+        raise ValueError("k_pages and v_pages must share the page stride")
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_table and seq_lens must be int32")
+    block_table = block_table.contiguous()
+    seq_lens = seq_lens.contiguous()
+    max_pages = block_table.shape[1]
+    if max_seq_len is None:
+        max_seq_len = max_pages * ps
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    S = num_splits if num_splits > 0 else blasst_decode_splits(
+        B, Hkv, max_seq_len, 64)
+    ws_bytes = 0
+    if not stats_only:
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and want_lse:
+            lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+        need = blasst_decode_workspace_size(B, Hq, d, S)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    else:
+        o, lse, workspace = None, None, None
+    st = _lib.blasst_decode_paged(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), int(k_pages.stride(0)), P, ps,
+        _ptr(block_table), max_pages, _ptr(seq_lens), int(max_seq_len),
+        _ptr(o), _ptr(lse), B, Hq, Hkv, d, float(scale), float(ln_lambda),
+        int(bool(per_length)), S, _ptr(workspace), ws_bytes,
+        stats.c_struct if stats is not None else None, _stream(stream))
+    _check(st, "blasst_decode_paged")
     return o, lse
 
 

@@ -97,12 +97,26 @@ blasst_status_t blasst_check_device_error(int* where_out) {
   unsigned int info[4] = {0, 0, 0, 0}, count = 0;
   cudaMemcpyFromSymbol(info, blasst::g_error_info, sizeof info);
   cudaMemcpyFromSymbol(&count, blasst::g_error_count, sizeof count);
+  cudaMemcpyToSymbol(blasst::g_error_code, &zero, sizeof zero);
+  cudaMemcpyToSymbol(blasst::g_error_count, &zero, sizeof zero);
+  if (code == blasst::kBadSeqLen) {
+    snprintf(g_last_error, sizeof g_last_error,
+             "paged decode: sequence %u has length %d, outside [0, "
+             "max_seq_len]",
+             info[1], (int)info[2]);
+    return BLASST_ERR_INVALID_ARG;
+  }
+  if (code == blasst::kBadPageId) {
+    snprintf(g_last_error, sizeof g_last_error,
+             "paged decode: sequence %u, block-table entry %u holds page id "
+             "%d, outside [0, num_pages)",
+             info[1], info[2], (int)info[3]);
+    return BLASST_ERR_INVALID_ARG;
+  }
   snprintf(g_last_error, sizeof g_last_error,
            "wait %u gave up first (block %u, step %u, parity %u, slot %u); "
            "%u waits gave up in total",
            code, info[0], info[1], info[2], info[3], count);
-  cudaMemcpyToSymbol(blasst::g_error_code, &zero, sizeof zero);
-  cudaMemcpyToSymbol(blasst::g_error_count, &zero, sizeof zero);
   return BLASST_ERR_TIMEOUT;
 }
 
@@ -144,6 +158,79 @@ size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits) {
   return o_bytes + l_bytes;
 }
 
+}  // extern "C"
+
+namespace {
+// Split kernel, then (unless statistics only) the merge, launched as a
+// programmatic dependent of the split kernel so its launch overlaps the
+// split kernel's tail (it waits on griddepcontrol).
+template <int G, bool PAGED>
+cudaError_t launch_split(const blasst::DecodeArgs& a, long long grid,
+                         cudaStream_t st) {
+  const int smem = blasst::DecodeSmem<G>::kTotal;
+  cudaError_t e = cudaFuncSetAttribute(
+      blasst::decode_split_kernel<G, PAGED>,
+      cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  blasst::decode_split_kernel<G, PAGED>
+      <<<(unsigned)grid, blasst::kDecThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+blasst_status_t launch_decode(const blasst::DecodeArgs& a, int G, bool paged,
+                              long long grid, bool stats_only, void* o,
+                              float* lse, int rows, int S, cudaStream_t st) {
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (G) {
+#define BLASST_LAUNCH_DECODE(GG)                                             \
+  case GG:                                                                   \
+    e = paged ? launch_split<GG, true>(a, grid, st)                          \
+              : launch_split<GG, false>(a, grid, st);                        \
+    break;
+    BLASST_LAUNCH_DECODE(1)
+    BLASST_LAUNCH_DECODE(2)
+    BLASST_LAUNCH_DECODE(4)
+    BLASST_LAUNCH_DECODE(8)
+#undef BLASST_LAUNCH_DECODE
+  }
+  if (e != cudaSuccess) return cuda_status(e, "decode split launch");
+  if (stats_only) return BLASST_OK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)rows);
+  cfg.blockDim = dim3(blasst::kDecD);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, blasst::decode_combine_kernel,
+                         (const float*)a.o_part, (const float*)a.lse_part,
+                         static_cast<__nv_bfloat16*>(o), lse, a.S);
+  return cuda_status(e, "decode merge launch");
+}
+
+// Split partials inside a caller workspace (layout of
+// blasst_decode_workspace_size).
+blasst_status_t carve_workspace(void* workspace, size_t workspace_bytes,
+                                int B, int Hq, int d, int S, float** o_part,
+                                float** lse_part) {
+  const size_t need = blasst_decode_workspace_size(B, Hq, d, S);
+  if (!workspace || workspace_bytes < need) return BLASST_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return BLASST_ERR_MISALIGNED;
+  const size_t rows = (size_t)B * Hq * S;
+  *o_part = static_cast<float*>(workspace);
+  *lse_part = reinterpret_cast<float*>(
+      static_cast<char*>(workspace) +
+      ((rows * d * sizeof(float) + 255) & ~(size_t)255));
+  return BLASST_OK;
+}
+}  // namespace
+
+extern "C" {
+
 blasst_status_t blasst_decode(const void* q, const void* k_cache,
                               const void* v_cache, void* o, float* lse, int B,
                               int Hq, int Hkv, int Lkv, int d, float scale,
@@ -173,17 +260,11 @@ blasst_status_t blasst_decode(const void* q, const void* k_cache,
   float* o_part = nullptr;
   float* lse_part = nullptr;
   if (!stats_only) {
-    const size_t need = blasst_decode_workspace_size(B, Hq, d, S);
-    if (!workspace || workspace_bytes < need) return BLASST_ERR_WORKSPACE;
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-      return BLASST_ERR_MISALIGNED;
-    const size_t rows = (size_t)B * Hq * S;
-    o_part = static_cast<float*>(workspace);
-    lse_part = reinterpret_cast<float*>(
-        static_cast<char*>(workspace) +
-        ((rows * d * sizeof(float) + 255) & ~(size_t)255));
+    const blasst_status_t ws = carve_workspace(workspace, workspace_bytes, B,
+                                               Hq, d, S, &o_part, &lse_part);
+    if (ws != BLASST_OK) return ws;
   }
-  blasst::DecodeArgs a;
+  blasst::DecodeArgs a = {};
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k = static_cast<const __nv_bfloat16*>(k_cache);
   a.v = static_cast<const __nv_bfloat16*>(v_cache);
@@ -199,46 +280,87 @@ blasst_status_t blasst_decode(const void* q, const void* k_cache,
   a.ln_lambda = ln_lambda;
   a.stats_only = stats_only ? 1 : 0;
 
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaSuccess;
-  switch (G) {
-#define BLASST_LAUNCH_DECODE(GG)                                               \
-  case GG: {                                                                   \
-    const int smem = blasst::DecodeSmem<GG>::kTotal;                           \
-    e = cudaFuncSetAttribute(blasst::decode_split_kernel<GG>,                  \
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,      \
-                             smem);                                            \
-    if (e == cudaSuccess)                                                      \
-      blasst::decode_split_kernel<GG>                                          \
-          <<<(unsigned)grid, blasst::kDecThreads, smem, st>>>(a);              \
-    break;                                                                     \
-  }
-    BLASST_LAUNCH_DECODE(1)
-    BLASST_LAUNCH_DECODE(2)
-    BLASST_LAUNCH_DECODE(4)
-    BLASST_LAUNCH_DECODE(8)
-#undef BLASST_LAUNCH_DECODE
-  }
-  if (e == cudaSuccess) e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_status(e, "decode split launch");
-  if (stats_only) return BLASST_OK;
+  return launch_decode(a, G, false, grid, stats_only, o, lse, B * Hq, S,
+                       static_cast<cudaStream_t>(stream));
+}
 
-  // Merge, launched as a programmatic dependent of the split kernel so its
-  // launch overlaps the split kernel's tail (it waits on griddepcontrol).
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(B * Hq));
-  cfg.blockDim = dim3(blasst::kDecD);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, blasst::decode_combine_kernel,
-                         (const float*)o_part, (const float*)lse_part,
-                         static_cast<__nv_bfloat16*>(o), lse, S);
-  return cuda_status(e, "decode merge launch");
+// ---------------------------------------------------------------------------
+// Decode over a paged cache (block table + per-sequence lengths)
+// ---------------------------------------------------------------------------
+blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
+                                    const void* v_pages, long long page_stride,
+                                    int num_pages, int page_size,
+                                    const int* block_table, int max_pages,
+                                    const int* seq_lens, int max_seq_len,
+                                    void* o, float* lse, int B, int Hq,
+                                    int Hkv, int d, float scale,
+                                    float ln_lambda, int per_length,
+                                    int num_splits, void* workspace,
+                                    size_t workspace_bytes,
+                                    const blasst_skip_stats_t* skip_stats,
+                                    void* stream) {
+  if (!q || !k_pages || !v_pages || !block_table || !seq_lens)
+    return BLASST_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || num_pages < 1 ||
+      max_pages < 1 || max_seq_len < 1 || num_splits < 0)
+    return BLASST_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return BLASST_ERR_INVALID_ARG;
+  if (per_length ? (std::isnan(ln_lambda) || ln_lambda == INFINITY)
+                 : !valid_ln_lambda(ln_lambda))
+    return BLASST_ERR_INVALID_ARG;
+  int log2_page = -1;
+  for (int l2 = 4; l2 <= 8; ++l2)
+    if (page_size == (1 << l2)) log2_page = l2;
+  if (log2_page < 0) return BLASST_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)max_seq_len > (long long)max_pages * page_size)
+    return BLASST_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (d != blasst::kDecD || !(G == 1 || G == 2 || G == 4 || G == 8))
+    return BLASST_ERR_UNSUPPORTED_SHAPE;
+  if (page_stride < (long long)Hkv * page_size * d || page_stride % 8 != 0)
+    return BLASST_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) ||
+      (o && !aligned16(o)))
+    return BLASST_ERR_MISALIGNED;
+  const int Bc = blasst::kDecBc;
+  const int nk = (max_seq_len + Bc - 1) / Bc;
+  const int S = num_splits == 0 ? blasst_decode_splits(B, Hkv, max_seq_len, Bc)
+                                : num_splits;
+  if (S < 1 || S > nk) return BLASST_ERR_INVALID_ARG;
+  const long long grid = (long long)B * Hkv * S;
+  if (grid > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED_SHAPE;
+  const bool stats_only = (o == nullptr);
+  float* o_part = nullptr;
+  float* lse_part = nullptr;
+  if (!stats_only) {
+    const blasst_status_t ws = carve_workspace(workspace, workspace_bytes, B,
+                                               Hq, d, S, &o_part, &lse_part);
+    if (ws != BLASST_OK) return ws;
+  }
+  blasst::DecodeArgs a = {};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k_pages);
+  a.v = static_cast<const __nv_bfloat16*>(v_pages);
+  a.o_part = o_part;
+  a.lse_part = lse_part;
+  a.counters = skip_stats ? skip_stats->counters : nullptr;
+  a.mask = skip_stats ? skip_stats->mask : nullptr;
+  a.Hkv = Hkv;
+  a.Lkv = max_seq_len;
+  a.nk = nk;
+  a.S = S;
+  a.scale = scale;
+  a.ln_lambda = ln_lambda;
+  a.stats_only = stats_only ? 1 : 0;
+  a.block_table = block_table;
+  a.seq_lens = seq_lens;
+  a.page_stride = page_stride;
+  a.log2_page = log2_page;
+  a.max_pages = max_pages;
+  a.num_pages = num_pages;
+  a.per_length = per_length ? 1 : 0;
+  return launch_decode(a, G, true, grid, stats_only, o, lse, B * Hq, S,
+                       static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------

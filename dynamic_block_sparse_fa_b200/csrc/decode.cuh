@@ -16,9 +16,15 @@
 //
 // One CTA of 128 threads per (sequence b, KV head, split).  The G query
 // heads of the KV head are the rows of the tile: every K and V byte fetched
-// serves G heads.  K and V blocks (Bc = 64 keys x d = 128 = 16 KB, contiguous
-// in the cache) arrive through bulk asynchronous copies into shared memory
-// and are read back with 128-bit shared loads.
+// serves G heads.  K and V blocks (Bc = 64 keys x d = 128 = 16 KB) arrive
+// through bulk asynchronous copies into shared memory and are read back with
+// 128-bit shared loads.
+//
+// Two cache forms share the kernel.  Contiguous: [B, Hkv, Lkv, d], one copy
+// per block.  Paged: a pool of pages of page_size tokens, page p of KV head
+// h at p * page_stride + h * page_size * d, a block table per sequence and a
+// length per sequence (device-resident); a block is one copy when pages hold
+// 64 tokens or more, else one copy per page.
 #pragma once
 
 #include "ptx.cuh"
@@ -33,9 +39,15 @@ struct DecodeArgs {
   float* lse_part;         // [B*Hq, S]
   unsigned long long* counters;  // [2] visited, skipped (may be null)
   unsigned char* mask;           // [B*Hkv, nk] (may be null)
-  int Hkv, Lkv, nk, S;
+  int Hkv, Lkv, nk, S;  // paged: Lkv = upper bound on the lengths
   float scale, ln_lambda;
   int stats_only;
+  // paged cache only
+  const int* block_table;  // [B, max_pages]
+  const int* seq_lens;     // [B]
+  long long page_stride;   // elements
+  int log2_page, max_pages, num_pages;
+  int per_length;  // ln_lambda is ln a; sequence b uses min(0, ln a - ln L_b)
 };
 
 constexpr int kDecD = 128;       // head dimension
@@ -115,7 +127,7 @@ __device__ __forceinline__ int head_of_lane(int lane) {
   return h;
 }
 
-template <int G>
+template <int G, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
     decode_split_kernel(const DecodeArgs a) {
   using L = DecodeSmem<G>;
@@ -126,12 +138,43 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
 
   const int s = blockIdx.x % a.S;
   const int bh = blockIdx.x / a.S;  // b * Hkv + hkv
-  const int j0 = (int)(((long long)s * a.nk) / a.S);
-  const int j1 = (int)(((long long)(s + 1) * a.nk) / a.S);
-  const int nblk = j1 - j0;
   const int Hq = a.Hkv * G;
   const int b = bh / a.Hkv;
   const int hkv = bh - b * a.Hkv;
+  int Lb = a.Lkv;  // keys of this sequence
+  float ln_lambda = a.ln_lambda;
+  if constexpr (PAGED) {
+    Lb = __ldg(a.seq_lens + b);
+    if (Lb < 0 || Lb > a.Lkv) {  // uniform across the CTA
+      if (tid == 0) record_error(kBadSeqLen, (unsigned)b, (unsigned)Lb, 0);
+      return;
+    }
+    // lambda = a / L with L this sequence's own context length
+    if (a.per_length && ln_lambda > -INFINITY && Lb > 0)
+      ln_lambda = fminf(0.f, ln_lambda - logf((float)Lb));
+  }
+  const int nk_b = (Lb + kDecBc - 1) / kDecBc;
+  const int j0 = (int)(((long long)s * nk_b) / a.S);
+  const int j1 = (int)(((long long)(s + 1) * nk_b) / a.S);
+  const int nblk = j1 - j0;
+  const int* bt_row = nullptr;
+  if constexpr (PAGED) {
+    // Every page id this split will read is checked before its first copy.
+    bt_row = a.block_table + (size_t)b * a.max_pages;
+    const int t0 = j0 * kDecBc;
+    const int t1 = min(j1 * kDecBc, Lb);
+    const int p0 = t0 >> a.log2_page;
+    const int p1 = t1 > t0 ? ((t1 - 1) >> a.log2_page) + 1 : p0;
+    bool bad = false;
+    for (int p = p0 + tid; p < p1; p += kDecThreads) {
+      const int id = __ldg(bt_row + p);
+      if (id < 0 || id >= a.num_pages) {
+        bad = true;
+        record_error(kBadPageId, (unsigned)b, (unsigned)p, (unsigned)id);
+      }
+    }
+    if (__syncthreads_or(bad)) return;
+  }
 
   uint8_t* sK = smem + L::kK;
   uint8_t* sV = smem + L::kV;
@@ -143,8 +186,17 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
   uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* vfull = kfull + kDecNK;
 
-  const __nv_bfloat16* kbase = a.k + (size_t)bh * a.Lkv * kDecD;
-  const __nv_bfloat16* vbase = a.v + (size_t)bh * a.Lkv * kDecD;
+  // contiguous: the (b, hkv) cache; paged: the pool, offset to head hkv
+  const __nv_bfloat16* kbase;
+  const __nv_bfloat16* vbase;
+  if constexpr (PAGED) {
+    const size_t hoff = (size_t)hkv * ((size_t)kDecD << a.log2_page);
+    kbase = a.k + hoff;
+    vbase = a.v + hoff;
+  } else {
+    kbase = a.k + (size_t)bh * a.Lkv * kDecD;
+    vbase = a.v + (size_t)bh * a.Lkv * kDecD;
+  }
   const uint64_t pol = policy_evict_first();
 
   if (tid == 0) {
@@ -154,14 +206,33 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
   }
   __syncthreads();
 
-  auto rows_of = [&](int j) { return min(kDecBc, a.Lkv - j * kDecBc); };
+  auto rows_of = [&](int j) { return min(kDecBc, Lb - j * kDecBc); };
+  // Copy the rows of block j from base (K or V) into dst; the barrier
+  // expects every byte.  Issued by one thread.
+  auto copy_block = [&](uint8_t* dst, const __nv_bfloat16* base, int j,
+                        uint64_t* bar) {
+    const int n = rows_of(j);
+    mbar_arrive_expect_tx(bar, (uint32_t)n * kDecRowBytes);
+    if constexpr (!PAGED) {
+      bulk_load(dst, base + (size_t)j * kDecBc * kDecD,
+                (uint32_t)n * kDecRowBytes, bar, pol);
+    } else {
+      const int ps = 1 << a.log2_page;
+      const int seg = ps < kDecBc ? ps : kDecBc;  // rows per copy
+      for (int t = 0; t < n; t += seg) {
+        const int tok = j * kDecBc + t;
+        const int id = __ldg(bt_row + (tok >> a.log2_page));
+        const __nv_bfloat16* src = base + (size_t)id * a.page_stride +
+                                   (size_t)(tok & (ps - 1)) * kDecD;
+        const int c = min(seg, n - t);
+        bulk_load(dst + t * kDecRowBytes, src, (uint32_t)c * kDecRowBytes,
+                  bar, pol);
+      }
+    }
+  };
   auto issue_k = [&](int r) {
-    const int j = j0 + r;
-    const uint32_t bytes = (uint32_t)rows_of(j) * kDecRowBytes;
-    uint64_t* bar = &kfull[r % kDecNK];
-    mbar_arrive_expect_tx(bar, bytes);
-    bulk_load(sK + (r % kDecNK) * kDecBlockBytes,
-              kbase + (size_t)j * kDecBc * kDecD, bytes, bar, pol);
+    copy_block(sK + (r % kDecNK) * kDecBlockBytes, kbase, j0 + r,
+               &kfull[r % kDecNK]);
   };
   if (tid == 0) {
     const int n0 = nblk < kDecNK ? nblk : kDecNK;
@@ -210,7 +281,6 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
 
   int kept_issued = 0, kept_done = 0;
   unsigned long long n_vis = 0, n_skp = 0;
-  const float ln_lambda = a.ln_lambda;
 
   auto pv = [&](int kidx) -> bool {
     const int slot = kidx % kDecNV;
@@ -343,11 +413,8 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
     if (!skip && !a.stats_only) {
       const int slot = kept_issued % kDecNV;
       if (tid == 0) {
-        const uint32_t bytes = (uint32_t)nvalid * kDecRowBytes;
         sNV[slot] = nvalid;
-        mbar_arrive_expect_tx(&vfull[slot], bytes);
-        bulk_load(sV + slot * kDecBlockBytes,
-                  vbase + (size_t)j * kDecBc * kDecD, bytes, &vfull[slot], pol);
+        copy_block(sV + slot * kDecBlockBytes, vbase, j, &vfull[slot]);
       }
       // new running max, rescale factor and P, per head
       float mn_mine = 0.f, al_mine = 1.f;
@@ -436,13 +503,17 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
     for (int t = 0; t < 8; ++t) sum += red[(t * G + g) * kDecD + dd];
     const float l = sL[g] + sL[8 + g] + sL[16 + g] + sL[24 + g];
     const size_t row = (size_t)b * Hq + hkv * G + g;
-    a.o_part[(row * a.S + s) * kDecD + dd] = sum / l;
-    if (dd == 0) a.lse_part[row * a.S + s] = m_run[g] + __logf(l);
+    // a split with no blocks (only a short paged sequence has one)
+    // contributes o = 0, lse = -inf
+    a.o_part[(row * a.S + s) * kDecD + dd] = l > 0.f ? sum / l : 0.f;
+    if (dd == 0)
+      a.lse_part[row * a.S + s] = l > 0.f ? m_run[g] + __logf(l) : -INFINITY;
   }
 }
 
 // Log-sum-exp merge of the S split partials of one (sequence, query head):
 //   lse = ln sum_s exp(lse_s),  o = sum_s exp(lse_s - lse) o_s.
+// An empty split (lse_s = -inf, o_s = 0) gets weight 0.
 __global__ void __launch_bounds__(kDecD)
     decode_combine_kernel(const float* __restrict__ o_part,
                           const float* __restrict__ lse_part,
@@ -456,6 +527,11 @@ __global__ void __launch_bounds__(kDecD)
   const float* lp = lse_part + row * S;
   float mx = -INFINITY;
   for (int s = 0; s < S; ++s) mx = fmaxf(mx, lp[s]);
+  if (mx == -INFINITY) {  // no keys at all (a paged sequence of length 0)
+    o[row * kDecD + dd] = __float2bfloat16_rn(0.f);
+    if (dd == 0 && lse) lse[row] = -INFINITY;
+    return;
+  }
   float sum = 0.f;
   for (int s = 0; s < S; ++s) sum += ex2_approx((lp[s] - mx) * kLog2e);
   const float L = mx + __logf(sum);

@@ -27,6 +27,10 @@ enum : unsigned int {
   kWaitPrefillSoftmax = 12,
   kWaitPrefillEpilogue = 13,
   kWaitSelfTest = 99,
+  // Device-resident arguments found out of range (paged decode); these are
+  // reported as invalid arguments, not as waits that gave up.
+  kBadSeqLen = 100,
+  kBadPageId = 101,
 };
 
 // About one second at B200 clocks: far beyond any legitimate wait of these

@@ -167,6 +167,74 @@ blasst_status_t blasst_decode_noalloc(const void *q, const void *k_cache,
                                       const blasst_skip_stats_t *skip_stats,
                                       void *stream);
 
+/*
+ * blasst_decode_paged -- blasst_decode over a paged KV cache with a block
+ * table and per-sequence lengths: the cache form of serving engines.  The
+ * MLSys'26 reading notes ("limitations and follow-up work") name end-to-end
+ * runs on PagedAttention serving stacks as future work, and the
+ * gist.science summary (section 3, "Integracao") the integration into
+ * TensorRT-LLM and FlashInfer, whose decode kernels read such caches.
+ *
+ * Sequence b holds seq_lens[b] tokens; its token t lives in page
+ * block_table[b * max_pages + t / page_size] at row t % page_size.  Pool
+ * layout: page p of KV head h starts at element
+ *     p * page_stride + h * page_size * d
+ * of k_pages (and of v_pages), its page_size rows of d bf16 elements
+ * contiguous -- [num_pages, Hkv, page_size, d] when page_stride =
+ * Hkv * page_size * d; an interleaved pool [num_pages, 2, Hkv, page_size, d]
+ * is v_pages = k_pages + Hkv * page_size * d with page_stride twice that.
+ * Each sequence is decoded exactly as blasst_decode decodes a contiguous
+ * cache of length seq_lens[b]: its ceil(L_b / 64) blocks of 64 keys (the
+ * last one ragged) cut into the call's num_splits splits by the same
+ * formula; a split with no blocks contributes nothing, and a sequence of
+ * length 0 gives o = 0 and lse = -inf.
+ *
+ *  q, o, lse       as blasst_decode ([B,Hq,d] bf16, [B,Hq,d] bf16 or NULL
+ *                  for statistics only, [B,Hq] float32 or NULL)
+ *  k_pages,v_pages device bf16 pools, 16-byte aligned
+ *  page_stride     elements between consecutive pages, >= Hkv*page_size*d,
+ *                  a multiple of 8 (16 bytes)
+ *  num_pages       pages in the pool (page ids must lie in [0, num_pages))
+ *  page_size       tokens per page: 16, 32, 64, 128 or 256
+ *  block_table     device int32 [B, max_pages]; entries past a sequence's
+ *                  last page are never read
+ *  seq_lens        device int32 [B], each in [0, max_seq_len]
+ *  max_seq_len     host upper bound on seq_lens (1 .. max_pages*page_size):
+ *                  sizes the split policy (blasst_decode_splits(B, Hkv,
+ *                  max_seq_len, 64) when num_splits == 0) and the mask
+ *  ln_lambda       per_length == 0: ln lambda (<= 0 or -INFINITY) for every
+ *                  sequence.  per_length != 0: ln a of the law lambda = a/L
+ *                  (finite or -INFINITY), and sequence b uses
+ *                  ln lambda_b = min(0, ln a - ln L_b), L_b its own length
+ *                  (gist.science summary, section 2 "Calibracao Automatica")
+ *  d = 128, Hq/Hkv in {1, 2, 4, 8}
+ *  num_splits      >= 1 (at most ceil(max_seq_len / 64)), or 0 = automatic
+ *  workspace       as blasst_decode: blasst_decode_workspace_size(B, Hq, d,
+ *                  resolved num_splits) bytes
+ *  skip_stats      as blasst_decode; the mask layout is
+ *                  [B, Hkv, ceil(max_seq_len / 64)] and blocks past a
+ *                  sequence's end are not written
+ * The block table and the lengths live on the device, so they are checked
+ * there: before any copy of a split is issued, its kernel checks its
+ * sequence's length and every page id it will read.  A bad value is not
+ * read through; the split is abandoned (the sequence's o and lse are then
+ * undefined) and blasst_check_device_error() returns
+ * BLASST_ERR_INVALID_ARG with the sequence, position and value in
+ * blasst_last_error().
+ */
+blasst_status_t blasst_decode_paged(const void *q, const void *k_pages,
+                                    const void *v_pages, long long page_stride,
+                                    int num_pages, int page_size,
+                                    const int *block_table, int max_pages,
+                                    const int *seq_lens, int max_seq_len,
+                                    void *o, float *lse, int B, int Hq,
+                                    int Hkv, int d, float scale,
+                                    float ln_lambda, int per_length,
+                                    int num_splits, void *workspace,
+                                    size_t workspace_bytes,
+                                    const blasst_skip_stats_t *skip_stats,
+                                    void *stream);
+
 /* Bytes of decode workspace: B*Hq*S*(d+1) float32 values, rounded up to 256.
  * num_splits must be the resolved value (>= 1). */
 size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits);
@@ -233,10 +301,14 @@ blasst_status_t blasst_skip_stats_reset(unsigned long long *counters,
                                         void *stream);
 
 /* Reads and clears the library's device error word for the current device
- * (set by a kernel that abandoned a bounded wait).  Synchronises the device.
- * Returns BLASST_OK or BLASST_ERR_TIMEOUT; *where_out (may be NULL) receives
- * the code of the wait that gave up, and blasst_last_error() then describes
- * the first failed wait (block, step, parity, slot). */
+ * (set by a kernel that abandoned a bounded wait, or by the paged decode on
+ * a bad length or page id).  Synchronises the device.  Returns BLASST_OK,
+ * BLASST_ERR_TIMEOUT (a wait gave up: blasst_last_error() describes the
+ * first one -- block, step, parity, slot) or BLASST_ERR_INVALID_ARG (a
+ * device-resident argument was out of range: blasst_last_error() names the
+ * sequence, the position and the value).  *where_out (may be NULL)
+ * receives the code recorded first: 1..99 a wait, 100 a sequence length,
+ * 101 a page id. */
 blasst_status_t blasst_check_device_error(int *where_out);
 
 /* Diagnostic: launches one CTA that waits on an mbarrier nothing arrives

@@ -150,3 +150,47 @@ def test_reference_arm_split_policy_matches_library(lib):
     for B, H, L in itertools.product([1, 2, 3, 8, 32, 148], [1, 8],
                                      [64, 1000, 32768, 131072]):
         assert bench.auto_splits(B, H, L, 64) == m.blasst_decode_splits(B, H, L, 64)
+
+
+def _paged(lib, q=0x1000, kp=0x1000, vp=0x1000, stride=None, P=8, ps=64,
+           bt=0x3000, maxp=4, sl=0x4000, maxlen=256, o=0x2000, B=2, Hq=8,
+           Hkv=2, d=128, scale=0.088, lnl=-1.0, per_length=0, S=1):
+    f = lib.blasst_decode_paged
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_longlong, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_void_p,
+                                          ctypes.c_int, ctypes.c_void_p,
+                                          ctypes.c_int, ctypes.c_void_p,
+                                          ctypes.c_void_p] + [ctypes.c_int] * 4 + [
+        ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+    if stride is None:
+        stride = Hkv * ps * d
+    # a workspace of 0 bytes: every shape that passes validation stops at
+    # BLASST_ERR_WORKSPACE (7) before any CUDA call
+    return f(q, kp, vp, stride, P, ps, bt, maxp, sl, maxlen, o, None, B, Hq,
+             Hkv, d, scale, lnl, per_length, S, None, 0, None, None)
+
+
+def test_paged_decode_validation(lib):
+    assert _paged(lib) == 7                            # valid up to workspace
+    assert _paged(lib, bt=None) == 1
+    assert _paged(lib, sl=None) == 1
+    assert _paged(lib, ps=48) == 2                     # page size not built
+    assert _paged(lib, ps=8) == 2
+    for ps in (16, 32, 64, 128, 256):
+        assert _paged(lib, ps=ps, maxp=max(1, 256 // ps)) == 7
+    assert _paged(lib, maxlen=257) == 1                # beyond the table
+    assert _paged(lib, stride=2 * 64 * 128 - 8) == 1   # pages overlap
+    assert _paged(lib, stride=2 * 64 * 128 + 4) == 1   # not 16-byte multiple
+    assert _paged(lib, stride=2 * 2 * 64 * 128) == 7   # interleaved K/V pool
+    assert _paged(lib, lnl=0.5) == 1                   # ln lambda > 0 ...
+    assert _paged(lib, lnl=3.5, per_length=1) == 7     # ... but ln a may be
+    assert _paged(lib, lnl=float("nan"), per_length=1) == 1
+    assert _paged(lib, lnl=float("inf"), per_length=1) == 1
+    assert _paged(lib, lnl=-math.inf, per_length=1) == 7
+    assert _paged(lib, S=5) == 1                       # more splits than blocks
+    assert _paged(lib, Hq=24, Hkv=2) == 2              # G = 12 not built
+    assert _paged(lib, d=64) == 2
+    assert _paged(lib, kp=0x1008) == 3                 # misaligned pool
+    assert _paged(lib, P=0) == 1

@@ -1,0 +1,271 @@
+"""GPU parity of the paged, variable-length decode against the CPU oracle,
+called through the C ABI.
+
+The logical caches are seeded planted-gap inputs; the test scatters them
+into a page pool in a seeded random order and fills every pool row that no
+sequence owns with poison (large K and V values), so that a read outside a
+sequence's own rows changes its output visibly.  Checks: outputs within
+max 2e-2 / mean 2e-3, lse, skip decisions bit-exact except near-ties,
+counters, the statistics-only pass, page sizes 16..256, every GQA ratio,
+empty and one-token sequences, splits with no blocks, the interleaved K/V
+pool, the per-sequence threshold lambda = a / L_b, agreement bit for bit
+with the contiguous kernel on the same tokens, out-of-range lengths and
+page ids reported as invalid arguments, and the full-size decode workload
+(batch 32, 32K cache) in a shuffled pool.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import config_seed, paginate, planted_gap, planted_gap_kv_inplace
+from tests import _parity as P
+
+pytestmark = pytest.mark.gpu
+
+POISON = (6.0, 500.0)
+
+
+@pytest.fixture(scope="module")
+def blasst():
+    import dynamic_block_sparse_fa_b200 as m
+    return m
+
+
+def _pool(pk, layout):
+    """Separate K and V pools, or one interleaved pool [P, 2, Hkv, ps, d]."""
+    if layout == "separate":
+        return pk.k_pages, pk.v_pages
+    both = torch.stack([pk.k_pages, pk.v_pages], dim=1).contiguous()
+    return both[:, 0], both[:, 1]
+
+
+def _check_paged(m, q, kp, vp, pk, lens, ln_lambda, S_req, per_length,
+                 max_seq_len=None):
+    B, Hq, d = q.shape
+    Hkv = kp.shape[1]
+    if max_seq_len is None:
+        max_seq_len = pk.block_table.shape[1] * pk.page_size
+    nk_max = -(-max_seq_len // 64)
+    S = S_req if S_req > 0 else m.blasst_decode_splits(B, Hkv, max_seq_len, 64)
+    scale = 1.0 / math.sqrt(d)
+    stats = m.Stats(mask_numel=B * Hkv * nk_max)
+    o, lse = m.blasst_decode_paged(q, kp, vp, pk.block_table, pk.seq_lens,
+                                   max_seq_len=max_seq_len, scale=scale,
+                                   ln_lambda=ln_lambda, per_length=per_length,
+                                   num_splits=S_req, stats=stats)
+    torch.cuda.synchronize()
+    st, where = m.blasst_check_device_error()
+    assert st == 0, f"device error word set ({where})"
+    ref = oracle.decode_paged(q, pk.k_pages, pk.v_pages, pk.block_table,
+                              pk.seq_lens, scale, ln_lambda, S,
+                              per_length=per_length, nk_max=nk_max)
+    og, lg = P.to_np(o), P.to_np(lse)
+    live = [b for b in range(B) if lens[b] > 0]
+    for b in range(B):
+        if lens[b] == 0:
+            assert np.all(og[b] == 0.0) and np.all(np.isneginf(lg[b]))
+    P.check_out(og[live], ref["o"][live], "paged o")
+    P.check_lse(lg[live], ref["lse"][live], "paged lse")
+    mask = stats.mask.cpu().numpy().reshape(B, Hkv, nk_max)
+    ties = P.check_mask(mask, ref["mask"], ref["margin"], "paged mask")
+    vis, skp = stats.read()
+    assert vis == Hkv * sum(-(-L // 64) for L in lens)
+    assert skp == int((mask == 2).sum())
+    if ties == 0:
+        assert (vis, skp) == (ref["visited"], ref["skipped"])
+    st2 = m.Stats(mask_numel=B * Hkv * nk_max)
+    r2 = m.blasst_decode_paged(q, kp, vp, pk.block_table, pk.seq_lens,
+                               max_seq_len=max_seq_len, scale=scale,
+                               ln_lambda=ln_lambda, per_length=per_length,
+                               num_splits=S_req, stats=st2, stats_only=True)
+    assert r2 == (None, None)
+    assert torch.equal(st2.mask, stats.mask)
+    assert st2.read() == (vis, skp)
+    return o, lse, mask
+
+
+PAGED_CASES = [
+    # Hq, Hkv, lens, page_size, ln_lambda, splits, per_length, layout
+    (32, 8, [1000, 64, 65, 4096], 16, -3.0, 0, False, "separate"),
+    (8, 2, [777, 2048, 1], 32, -2.0, 3, False, "separate"),
+    (16, 8, [3000, 1500], 64, -4.0, 4, False, "interleaved"),
+    (64, 8, [2048, 0, 300], 128, -3.0, 2, False, "separate"),
+    (4, 1, [5000, 130], 256, math.log(60.0), 5, True, "separate"),
+    (8, 8, [63, 64, 129, 1000], 64, -math.inf, 2, False, "separate"),
+    (32, 8, [4096, 4096], 64, 0.0, 7, False, "interleaved"),
+    (32, 8, [2500, 40, 7000, 64, 3333], 16, math.log(20.0), 0, True,
+     "interleaved"),
+]
+
+
+@pytest.mark.parametrize("case", PAGED_CASES)
+def test_paged_decode_matches_oracle(blasst, case):
+    Hq, Hkv, lens, ps, ln_lambda, S, per_length, layout = case
+    B = len(lens)
+    Lmax = max(max(lens), 1)
+    x = planted_gap(B, Hq, Hkv, 1, Lmax, 128, decode=True, block=64, gap=8.0,
+                    heavy_frac=0.03, seed=config_seed(1, 7 * Lmax + Hq + ps),
+                    device="cuda")
+    pk = paginate(x.k, x.v, lens, ps, seed=Lmax + ps, spare_pages=7,
+                  poison=POISON)
+    kp, vp = _pool(pk, layout)
+    o, lse, mask = _check_paged(blasst, x.q, kp, vp, pk, lens, ln_lambda, S,
+                                per_length)
+    if ln_lambda == -math.inf:
+        assert (mask == 2).sum() == 0
+
+
+@pytest.mark.parametrize("ps", [16, 64, 256])
+def test_paged_equals_contiguous_bitwise(blasst, ps):
+    """Same tokens, same splits: the paged kernel reads the same bytes in the
+    same order as the contiguous one, so the results agree bit for bit."""
+    m = blasst
+    B, Hq, Hkv, L = 6, 32, 8, 4096 + 64 * 3
+    x = planted_gap(B, Hq, Hkv, 1, L, 128, decode=True, block=64, gap=8.0,
+                    heavy_frac=0.03, seed=config_seed(1, 99), device="cuda")
+    pk = paginate(x.k, x.v, [L] * B, ps, seed=3, spare_pages=2,
+                  poison=POISON)
+    for lnl in (-math.inf, -3.0):
+        o1, l1 = m.blasst_decode(x.q, x.k, x.v, ln_lambda=lnl, num_splits=3)
+        o2, l2 = m.blasst_decode_paged(x.q, pk.k_pages, pk.v_pages,
+                                       pk.block_table, pk.seq_lens,
+                                       max_seq_len=L, ln_lambda=lnl,
+                                       num_splits=3)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_paged_bad_table_and_length_are_reported(blasst):
+    """Out-of-range values in the device-resident table and lengths are
+    caught by the kernel before any copy through them is issued."""
+    m = blasst
+    B, Hq, Hkv, L = 2, 8, 2, 1000
+    x = planted_gap(B, Hq, Hkv, 1, L, 128, decode=True, block=64, gap=8.0,
+                    heavy_frac=0.03, seed=5, device="cuda")
+    pk = paginate(x.k, x.v, [L, L], 64, seed=1, poison=POISON)
+    bt = pk.block_table.clone()
+    bt[1, 3] = pk.num_pages + 5
+    m.blasst_decode_paged(x.q, pk.k_pages, pk.v_pages, bt, pk.seq_lens,
+                          ln_lambda=-2.0)
+    st, where = m.blasst_check_device_error()
+    assert st == 1 and "page id" in where and "sequence 1" in where
+    bt[1, 3] = -1
+    m.blasst_decode_paged(x.q, pk.k_pages, pk.v_pages, bt, pk.seq_lens,
+                          ln_lambda=-2.0)
+    st, where = m.blasst_check_device_error()
+    assert st == 1 and "page id" in where
+    lens = torch.tensor([L, 16 * 64 + 1], dtype=torch.int32, device="cuda")
+    m.blasst_decode_paged(x.q, pk.k_pages, pk.v_pages, pk.block_table, lens,
+                          ln_lambda=-2.0)
+    st, where = m.blasst_check_device_error()
+    assert st == 1 and "length" in where
+    # the context is still usable and a good call is clean afterwards
+    m.blasst_decode_paged(x.q, pk.k_pages, pk.v_pages, pk.block_table,
+                          pk.seq_lens, ln_lambda=-2.0)
+    assert m.blasst_check_device_error()[0] == 0
+
+
+def test_paged_rejects_bad_arguments(blasst):
+    m = blasst
+    q = torch.zeros(1, 4, 128, dtype=torch.bfloat16, device="cuda")
+    kp = torch.zeros(4, 1, 64, 128, dtype=torch.bfloat16, device="cuda")
+    bt = torch.zeros(1, 4, dtype=torch.int32, device="cuda")
+    sl = torch.tensor([100], dtype=torch.int32, device="cuda")
+    with pytest.raises(blasst.BlasstError, match="INVALID_ARG"):
+        m.blasst_decode_paged(q, kp, kp, bt, sl, ln_lambda=0.5)
+    with pytest.raises(blasst.BlasstError, match="INVALID_ARG"):
+        m.blasst_decode_paged(q, kp, kp, bt, sl, max_seq_len=257)
+    kp48 = torch.zeros(4, 1, 48, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(blasst.BlasstError, match="UNSUPPORTED"):
+        m.blasst_decode_paged(q, kp48, kp48, bt, sl)
+    with pytest.raises(ValueError):
+        m.blasst_decode_paged(q, kp, kp, bt.long(), sl)
+
+
+def test_paged_full_size_shuffled_pool(blasst):
+    """Batch 32, Hq 32 / Hkv 8, 32K cache, d 128 in a shuffled pool of
+    64-token pages, lambda calibrated to 70% sparsity on the contiguous
+    cache: decisions and outputs equal the contiguous kernel's bit for bit,
+    and 3 sampled sequences match the oracle."""
+    m = blasst
+    B, Hq, Hkv, L, d = 32, 32, 8, 32768, 128
+    q = torch.empty(B, Hq, d, dtype=torch.bfloat16, device="cuda")
+    k = torch.empty(B, Hkv, L, d, dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    planted_gap_kv_inplace(k, v, q, block=64, gap=8.0, heavy_frac=0.03,
+                           seed=config_seed(1))
+    cal = m.blasst_calibrate(0.70, mode="decode", q=q, k=k, v=v, Bc=64)
+    lnl = cal["ln_lambda"]
+    nk = L // 64
+    pk = paginate(k, v, [L] * B, 64, seed=11, spare_pages=64)
+    s1 = m.Stats(mask_numel=B * Hkv * nk)
+    s2 = m.Stats(mask_numel=B * Hkv * nk)
+    o1, l1 = m.blasst_decode(q, k, v, ln_lambda=lnl, stats=s1)
+    o2, l2 = m.blasst_decode_paged(q, pk.k_pages, pk.v_pages, pk.block_table,
+                                   pk.seq_lens, max_seq_len=L, ln_lambda=lnl,
+                                   stats=s2)
+    torch.cuda.synchronize()
+    assert m.blasst_check_device_error()[0] == 0
+    assert torch.equal(s1.mask, s2.mask) and s1.read() == s2.read()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    del k, v
+    S = m.blasst_decode_splits(B, Hkv, L, 64)
+    mask = s2.mask.cpu().numpy().reshape(B, Hkv, nk)
+    for b in (0, 17, 31):
+        ids = pk.block_table[b].long()
+        kb = pk.k_pages[ids].transpose(0, 1).reshape(1, Hkv, L, d)
+        vb = pk.v_pages[ids].transpose(0, 1).reshape(1, Hkv, L, d)
+        ref = oracle.decode(q[b:b + 1], kb, vb, 1 / math.sqrt(d), lnl, 64, S)
+        P.check_out(P.to_np(o2[b:b + 1]), ref["o"], f"seq {b}")
+        P.check_lse(P.to_np(l2[b:b + 1]), ref["lse"], f"seq {b}")
+        P.check_mask(mask[b:b + 1], ref["mask"], ref["margin"], f"seq {b}")
+
+
+def test_paged_varlen_per_length_sampled(blasst):
+    """Batch 32 of lengths 1K..64K (mean about 32K) in a shuffled pool of
+    16-token pages, per-sequence threshold lambda = a / L_b with a the value
+    calibrated for 70% at 32K; 3 sampled sequences against the oracle."""
+    m = blasst
+    B, Hq, Hkv, d = 32, 32, 8, 128
+    g = torch.Generator().manual_seed(config_seed(6))
+    lens = torch.randint(1024, 65536 + 1, (B,), generator=g).tolist()
+    lens[0], lens[1] = 65536, 1023
+    Lmax = max(lens)
+    q = torch.empty(B, Hq, d, dtype=torch.bfloat16, device="cuda")
+    k = torch.empty(B, Hkv, Lmax, d, dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    planted_gap_kv_inplace(k, v, q, block=64, gap=8.0, heavy_frac=0.03,
+                           seed=config_seed(6, 1))
+    ln_a = math.log(math.exp(-8.0) * 32768)  # any a: parity is what counts
+    pk = paginate(k, v, lens, 16, seed=12, spare_pages=100, poison=POISON)
+    del k, v
+    nk_max = -(-Lmax // 64)
+    stats = m.Stats(mask_numel=B * Hkv * nk_max)
+    o, lse = m.blasst_decode_paged(q, pk.k_pages, pk.v_pages, pk.block_table,
+                                   pk.seq_lens, max_seq_len=Lmax,
+                                   ln_lambda=ln_a, per_length=True,
+                                   stats=stats)
+    torch.cuda.synchronize()
+    assert m.blasst_check_device_error()[0] == 0
+    vis, skp = stats.read()
+    assert vis == Hkv * sum(-(-L // 64) for L in lens)
+    S = m.blasst_decode_splits(B, Hkv, Lmax, 64)
+    mask = stats.mask.cpu().numpy().reshape(B, Hkv, nk_max)
+    for b in (0, 1, 20):
+        L = lens[b]
+        npg = -(-L // 16)
+        ids = pk.block_table[b, :npg].long()
+        kb = pk.k_pages[ids].transpose(0, 1).reshape(Hkv, npg * 16, d)[:, :L]
+        vb = pk.v_pages[ids].transpose(0, 1).reshape(Hkv, npg * 16, d)[:, :L]
+        lnl = min(0.0, ln_a - math.log(L))
+        ref = oracle.decode(q[b:b + 1], kb[None], vb[None], 1 / math.sqrt(d),
+                            lnl, 64, S)
+        P.check_out(P.to_np(o[b:b + 1]), ref["o"], f"seq {b}")
+        P.check_lse(P.to_np(lse[b:b + 1]), ref["lse"], f"seq {b}")
+        nk = -(-L // 64)
+        P.check_mask(mask[b:b + 1, :, :nk], ref["mask"], ref["margin"],
+                     f"seq {b}")
+        assert np.all(mask[b, :, nk:] == 0)
