@@ -519,7 +519,7 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
     if args.prefill_lnl is not None:
         out["fixed"] = measure(args.prefill_lnl)
         r = out["fixed"]
-        return out, {"bound": "tensor", "kernel": "prefill_kernel<128,128,128>",
+        return out, {"bound": "tensor", "kernel": "prefill2_kernel<128>",
                      "achieved": r["executed_tflops"], "peak": tf_peak,
                      "peak_kind": peak_kind + " bf16 burst", "unit": "TFLOP/s",
                      "frac": r["tensor_frac"], "traffic": None}
@@ -533,7 +533,7 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
         r["speedup_vs_dense"] = round(dense["us"] / r["us"], 4)
         out[key] = r
     best = out["s70"]
-    roof = {"bound": "tensor", "kernel": "prefill_kernel<128,128,128> at 70%",
+    roof = {"bound": "tensor", "kernel": "prefill2_kernel<128> at 70%",
             "achieved": best["executed_tflops"], "peak": tf_peak,
             "peak_kind": peak_kind + " bf16 burst", "unit": "TFLOP/s",
             "frac": best["tensor_frac"], "traffic": None}

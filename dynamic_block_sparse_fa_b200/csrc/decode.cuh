@@ -72,7 +72,12 @@ struct DecodeSmem {
   static constexpr int kA = kM + 2 * 4 * 8 * 4;                  // [NV][8] f32
   static constexpr int kL = kA + kDecNV * 8 * 4;                 // [4 warps][8] f32
   static constexpr int kNV = kL + 4 * 8 * 4;                     // [NV] int
-  static constexpr int kBar = (kNV + kDecNV * 4 + 15) & ~15;     // [NK+NV] u64
+  // paged cache, 2 chunks of 32 blocks, up to 4 copies a block: element
+  // offsets of each copy's source in the pool, and the page ids they are
+  // computed from
+  static constexpr int kOff = (kNV + kDecNV * 4 + 7) & ~7;       // [64][4] i64
+  static constexpr int kPid = kOff + 64 * 4 * 8;                 // [64][4] int
+  static constexpr int kBar = (kPid + 64 * 4 * 4 + 15) & ~15;    // [NK+NV] u64
   static constexpr int kTotal = kBar + (kDecNK + kDecNV) * 8;
   // The end-of-split reduction [8 key groups][G][D] f32 reuses the K and V
   // rings (all copies into them have been consumed by then).
@@ -157,20 +162,50 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
   const int j0 = (int)(((long long)s * nk_b) / a.S);
   const int j1 = (int)(((long long)(s + 1) * nk_b) / a.S);
   const int nblk = j1 - j0;
+  // Paged cache: a block of 64 keys is npb copies of 2^seg_l2 rows, each
+  // from one page.  The source offsets of the copies of blocks r (relative
+  // to j0) are kept in a shared ring sOff[r mod 64][copy], filled 32 blocks
+  // ahead, so the thread that issues a copy reads a ready address.
+  long long* sOff = reinterpret_cast<long long*>(smem + L::kOff);
+  int* sPid = reinterpret_cast<int*>(smem + L::kPid);
   const int* bt_row = nullptr;
+  const int seg_l2 = a.log2_page < 6 ? a.log2_page : 6;
+  const int npb = 1 << (6 - seg_l2);
+  // element offset of the copy of block r (relative) that starts at token
+  // tok, in page id
+  auto src_off = [&](int id, int tok) -> long long {
+    return (long long)id * a.page_stride +
+           ((long long)hkv << (a.log2_page + 7)) +
+           (long long)(tok & ((1 << a.log2_page) - 1)) * kDecD;
+  };
   if constexpr (PAGED) {
-    // Every page id this split will read is checked before its first copy.
+    // Every page id this split will read is checked before its first copy;
+    // the copies of its first 64 blocks go into the ring.
     bt_row = a.block_table + (size_t)b * a.max_pages;
-    const int t0 = j0 * kDecBc;
-    const int t1 = min(j1 * kDecBc, Lb);
-    const int p0 = t0 >> a.log2_page;
-    const int p1 = t1 > t0 ? ((t1 - 1) >> a.log2_page) + 1 : p0;
     bool bad = false;
-    for (int p = p0 + tid; p < p1; p += kDecThreads) {
-      const int id = __ldg(bt_row + p);
-      if (id < 0 || id >= a.num_pages) {
-        bad = true;
-        record_error(kBadPageId, (unsigned)b, (unsigned)p, (unsigned)id);
+    for (int e = tid; e < 64 * 4; e += kDecThreads) {
+      const int r = e >> 2, i = e & 3;
+      const int tok = (j0 + r) * kDecBc + (i << seg_l2);
+      if (r < nblk && i < npb && tok < Lb) {
+        const int p = tok >> a.log2_page;
+        const int id = __ldg(bt_row + p);
+        if (id < 0 || id >= a.num_pages) {
+          bad = true;
+          record_error(kBadPageId, (unsigned)b, (unsigned)p, (unsigned)id);
+        }
+        sOff[e] = src_off(id, tok);
+      }
+    }
+    const int t0 = (j0 + min(nblk, 64)) * kDecBc;
+    const int t1 = min(j1 * kDecBc, Lb);
+    if (t1 > t0) {
+      const int p1 = ((t1 - 1) >> a.log2_page) + 1;
+      for (int p = (t0 >> a.log2_page) + tid; p < p1; p += kDecThreads) {
+        const int id = __ldg(bt_row + p);
+        if (id < 0 || id >= a.num_pages) {
+          bad = true;
+          record_error(kBadPageId, (unsigned)b, (unsigned)p, (unsigned)id);
+        }
       }
     }
     if (__syncthreads_or(bad)) return;
@@ -186,13 +221,13 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
   uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* vfull = kfull + kDecNK;
 
-  // contiguous: the (b, hkv) cache; paged: the pool, offset to head hkv
+  // contiguous: the (b, hkv) cache; paged: the pool (the ring's offsets
+  // include the head)
   const __nv_bfloat16* kbase;
   const __nv_bfloat16* vbase;
   if constexpr (PAGED) {
-    const size_t hoff = (size_t)hkv * ((size_t)kDecD << a.log2_page);
-    kbase = a.k + hoff;
-    vbase = a.v + hoff;
+    kbase = a.k;
+    vbase = a.v;
   } else {
     kbase = a.k + (size_t)bh * a.Lkv * kDecD;
     vbase = a.v + (size_t)bh * a.Lkv * kDecD;
@@ -217,16 +252,14 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
       bulk_load(dst, base + (size_t)j * kDecBc * kDecD,
                 (uint32_t)n * kDecRowBytes, bar, pol);
     } else {
-      const int ps = 1 << a.log2_page;
-      const int seg = ps < kDecBc ? ps : kDecBc;  // rows per copy
-      for (int t = 0; t < n; t += seg) {
-        const int tok = j * kDecBc + t;
-        const int id = __ldg(bt_row + (tok >> a.log2_page));
-        const __nv_bfloat16* src = base + (size_t)id * a.page_stride +
-                                   (size_t)(tok & (ps - 1)) * kDecD;
-        const int c = min(seg, n - t);
-        bulk_load(dst + t * kDecRowBytes, src, (uint32_t)c * kDecRowBytes,
-                  bar, pol);
+      const long long* offs = sOff + ((j - j0) & 63) * 4;
+      if (npb == 1) {
+        bulk_load(dst, base + offs[0], (uint32_t)n * kDecRowBytes, bar, pol);
+      } else {
+        const int seg = 1 << seg_l2;  // rows per copy
+        for (int t = 0, i = 0; t < n; t += seg, ++i)
+          bulk_load(dst + t * kDecRowBytes, base + offs[i],
+                    (uint32_t)min(seg, n - t) * kDecRowBytes, bar, pol);
       }
     }
   };
@@ -394,6 +427,38 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
     }
     if (__syncthreads_or(!ok)) { ok = false; break; }
     if (tid == 0 && r + kDecNK < nblk) issue_k(r + kDecNK);
+    if constexpr (PAGED) {
+      // Ring refill, by the last warp, lane l for block 32(c+1) + l: at
+      // block 32c (c >= 1) it copies the page ids of chunk c+1 into sPid
+      // asynchronously; at block 32c+1 it waits for them and writes the
+      // copies' offsets into the sOff slots chunk c-1 used (their last
+      // reader, the V copy of block 32c-1, was issued before the barrier of
+      // block 32c).  The first reader of chunk c+1 (the K copy of block
+      // 32c+32, issued at block 32c+30) comes after many more barriers.
+      if (warp == kDecThreads / 32 - 1 && r >= 32 && (r & 31) <= 1) {
+        const int rr = (r & ~31) + 32 + lane;
+        if ((r & 31) == 0) {
+          if (rr < nblk) {
+            for (int i = 0; i < npb; ++i) {
+              const int tok = (j0 + rr) * kDecBc + (i << seg_l2);
+              if (tok < Lb)
+                cp_async_4(sPid + (rr & 63) * 4 + i,
+                           bt_row + (tok >> a.log2_page));
+            }
+          }
+          cp_async_commit();
+        } else {
+          cp_async_wait_all();
+          if (rr < nblk) {
+            for (int i = 0; i < npb; ++i) {
+              const int tok = (j0 + rr) * kDecBc + (i << seg_l2);
+              if (tok < Lb)
+                sOff[(rr & 63) * 4 + i] = src_off(sPid[(rr & 63) * 4 + i], tok);
+            }
+          }
+        }
+      }
+    }
 
     // ---- decision, identical in every thread: skip block j iff every
     // head's block max lies more than |ln lambda| below its running max.
@@ -449,6 +514,10 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
       ok = pv(kept_done);
       ++kept_done;
     }
+  }
+  if constexpr (PAGED) {
+    // no ring copy may still be landing when the CTA leaves
+    if (warp == kDecThreads / 32 - 1) cp_async_wait_all();
   }
   if (__syncthreads_or(!ok)) ok = false;
   while (ok && kept_done < kept_issued) {
