@@ -260,40 +260,43 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
       }
       mma_commit(&bar[C::B_SF + t]);
     };
-    bool ok = __all_sync(FULL, mbar_wait(&bar[C::B_Q], 0, kWaitPrefillMma, 0, 0));
-    if (ok)
-      ok = __all_sync(FULL, mbar_wait(&bar[C::B_KF], 0, kWaitPrefillMma, 0, 0));
-    tc_fence_after();
-    if (ok) {
-      if (leader) {
+    // One lane issues.  All waits of a tile's step come before its MMAs, so
+    // the P.V and the next QK^T of a tile go to the tensor core back to back.
+    if (leader) {
+      bool ok = mbar_wait(&bar[C::B_Q], 0, kWaitPrefillMma, 0, 0) &&
+                mbar_wait(&bar[C::B_KF], 0, kWaitPrefillMma, 0, 0);
+      tc_fence_after();
+      if (ok) {
         for (int t = 0; t < 2; ++t)
           if (nblk_t[t] > 0) qk(t, 0);
         mma_commit(&bar[C::B_KE]);
       }
-      __syncwarp();
-    }
-    int vcount = 0;
-    int npv[2] = {0, 0};
-    for (int j = 0; j < nblk && ok; ++j) {
-      int vslot = -1;
+      int vcount = 0;
+      int npv[2] = {0, 0};
+      for (int j = 0; j < nblk && ok; ++j) {
+        int vslot = -1;
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (!ok || j >= nblk_t[t]) continue;
-        ok = __all_sync(FULL, mbar_wait(&bar[C::B_PF + t], j & 1,
-                                        kWaitPrefillMma, j, 300 + t));
-        if (!ok) break;
-        const bool kept = dec_flag[t * C::R + j % C::R] != 0;
-        if (kept && !stats_only) {
-          if (vslot < 0) {
+        for (int t = 0; t < 2; ++t) {
+          if (!ok || j >= nblk_t[t]) continue;
+          ok = mbar_wait(&bar[C::B_PF + t], j & 1, kWaitPrefillMma, j, 300 + t);
+          if (!ok) break;
+          const bool kept = !stats_only && dec_flag[t * C::R + j % C::R] != 0;
+          if (kept && vslot < 0) {
             vslot = vcount % C::NVS;
-            ok = __all_sync(FULL, mbar_wait(&bar[C::B_VF + vslot],
-                                            (vcount / C::NVS) & 1,
-                                            kWaitPrefillMma, j, 200 + vslot));
+            ok = mbar_wait(&bar[C::B_VF + vslot], (vcount / C::NVS) & 1,
+                           kWaitPrefillMma, j, 200 + vslot);
             ++vcount;
             if (!ok) break;
           }
+          const bool more = j + 1 < nblk_t[t];
+          if (more) {
+            ok = mbar_wait(&bar[C::B_KF + (j + 1) % C::NKS],
+                           ((j + 1) / C::NKS) & 1, kWaitPrefillMma, j + 1,
+                           (j + 1) % C::NKS);
+            if (!ok) break;
+          }
           tc_fence_after();
-          if (leader) {
+          if (kept) {
             const uint32_t a_p = tmem + C::COL_S + t * 128;
 #pragma unroll
             for (int k = 0; k < BN / 16; ++k) {
@@ -302,29 +305,19 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
               mma_ts(tmem + C::COL_O + t * 128, a_p + k * 8, db, idesc_o,
                      (npv[t] > 0 || k > 0) ? 1u : 0u);
             }
+            ++npv[t];
           }
-          ++npv[t];
+          if (more)
+            qk(t, j + 1);
+          else
+            mma_commit(&bar[C::B_OD + t]);  // tile t has issued its last MMA
         }
-        if (j + 1 < nblk_t[t]) {
-          ok = __all_sync(FULL, mbar_wait(&bar[C::B_KF + (j + 1) % C::NKS],
-                                          ((j + 1) / C::NKS) & 1,
-                                          kWaitPrefillMma, j + 1,
-                                          (j + 1) % C::NKS));
-          if (!ok) break;
-          tc_fence_after();
-          if (leader) qk(t, j + 1);
-        } else if (leader) {
-          mma_commit(&bar[C::B_OD + t]);  // tile t has issued its last MMA
-        }
-        __syncwarp();
-      }
-      if (!ok) break;
-      if (leader) {
+        if (!ok) break;
         if (vslot >= 0) mma_commit(&bar[C::B_VE + vslot]);
         if (j + 1 < nblk) mma_commit(&bar[C::B_KE + (j + 1) % C::NKS]);
       }
-      __syncwarp();
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------------
     // Softmax: warps 2 .. 2+WPT-1 tile 0, the next WPT warps tile 1.  A row
@@ -388,13 +381,19 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
       }
       float mt;
       {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        // 8 chains of three-input maxima (two comparisons per instruction)
+        float m8[8];
 #pragma unroll
-        for (int c = 0; c < CPT / 32; ++c)
+        for (int x = 0; x < 8; ++x)
+          m8[x] = fmaxf(__uint_as_float(sr[0][x]), __uint_as_float(sr[0][x + 8]));
 #pragma unroll
-          for (int x = 0; x < 32; ++x)
-            m4[x & 3] = fmaxf(m4[x & 3], __uint_as_float(sr[c][x]));
-        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        for (int i = 16; i + 16 <= CPT; i += 16)
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            m8[x] = fmax3(m8[x], __uint_as_float(sr[i >> 5][(i & 31) + x]),
+                          __uint_as_float(sr[(i + 8) >> 5][((i + 8) & 31) + x]));
+        mt = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                   fmaxf(m8[6], m8[7]));
       }
       float* xm = xmax + (((j & 1) * 2 + t) * NH) * 128;
       if (NH > 1) xm[half * 128 + rr] = mt;

@@ -239,6 +239,14 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return x < -126.0f ? 0.0f : r;
 }
 
+// max(a, b, c) in one instruction (sm_100): two comparisons for the issue
+// cost of one two-input max.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // bf16x2 word -> two floats (exact: a bf16 is the top half of an f32).
 __device__ __forceinline__ float bf16lo(uint32_t w) {
   return __uint_as_float(w << 16);
