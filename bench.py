@@ -43,7 +43,31 @@ METRIC = ("sparse attn latency & dense-equiv TFLOP/s vs λ=0 at 50/70% "
           "sparsity; decode GB/s")
 
 DEC = dict(B=32, Hq=32, Hkv=8, Lkv=32768, d=128, Bc=64, target=0.70)
+
+# DRAM traffic of the dominant decode kernel per launch, relative to the
+# algorithmic bytes of that launch, from one ncu capture of a smaller case
+# (profiles/decode_split_kernel_B8_Lkv32k.md: dram__bytes_read.sum +
+# dram__bytes_write.sum = 955.6 MB for 957.8 MB of algorithmic bytes).  The
+# kernel reads K once and V only for kept blocks, so traffic grows with the
+# algorithmic bytes; the ratio is applied to the benchmarked launch.  It holds
+# only for the kernel source it was measured on (sha256 prefix below).
+DECODE_TRAFFIC = dict(source="dynamic_block_sparse_fa_b200/csrc/decode.cuh",
+                      sha256_16="e61d605edef51723", ratio=955.6 / 957.8)
 PRE = dict(B=1, Hq=32, Hkv=8, L=32768, d=128, Br=128, Bc=128)
+
+
+def _measured_traffic(spec, algorithmic_bytes):
+    """Bytes of DRAM traffic per launch, or None once the kernel source has
+    changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, spec["source"]), "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if h != spec["sha256_16"]:
+        return None
+    return int(round(spec["ratio"] * algorithmic_bytes))
 
 
 def _peaks():
@@ -349,8 +373,9 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
         "accumulate": "f32",
         "data": "synthetic planted-gap (seeded; gap 8 nats, sink + 3% heavy blocks)",
         "config": {
-            "workload": (f"decode B{B} Hq{Hq} Hkv{Hkv} Lkv{Lkv} d{d} Bc{Bc}, "
-                         f"lambda calibrated to {DEC['target']:.0%} sparsity"),
+            "workload": (f"decode B{B} Hq{Hq} Hkv{Hkv} Lkv{Lkv} d{d} Bc{Bc}, " + (
+                f"lambda calibrated to {DEC['target']:.0%} sparsity"
+                if args.decode_lnl is None else f"fixed ln lambda {lnl}")),
             "global_batch": B * world, "seq_len": Lkv,
             "parallelism": f"replicas{world}", "splits": S,
             "ln_lambda": lnl, "a": cal["a"], "sparsity": skp / vis,
@@ -370,7 +395,9 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
             "bound": "hbm", "kernel": "decode_split_kernel (+ merge)",
             "achieved": round(achieved, 1), "peak": hbm_peak,
             "peak_kind": peak_kind + " copy bandwidth", "unit": "GB/s",
-            "frac": round(achieved / hbm_peak, 4), "traffic": None,
+            "frac": round(achieved / hbm_peak, 4),
+            "traffic": _measured_traffic(DECODE_TRAFFIC, by_call),
+            "traffic_unit": "bytes per launch",
         },
         "e2e": {"value": _r(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
