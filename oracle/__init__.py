@@ -44,6 +44,20 @@ def _load():
             ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
             ctypes.c_double, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, _i32p, _dp, _dp, _u8p, _dp, _i64p, ctypes.c_int]
+        lib.oracle_prefill_window.restype = ctypes.c_int
+        lib.oracle_prefill_window.argtypes = [
+            _u16p, _u16p, _u16p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+            ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, _i32p, _dp, _dp, _u8p, _dp, _i64p, ctypes.c_int]
+        lib.oracle_decode_window.restype = ctypes.c_int
+        lib.oracle_decode_window.argtypes = [
+            _u16p, _u16p, _u16p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_double,
+            ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp, _u8p, _dp, _i64p,
+            ctypes.c_int]
         lib.oracle_decode.restype = ctypes.c_int
         lib.oracle_decode.argtypes = [
             _u16p, _u16p, _u16p,
@@ -87,8 +101,11 @@ def n_threads_default():
 
 
 def prefill(q, k, v, scale, causal, ln_lambda, Br, Bc, units=None,
-            n_threads=0):
+            n_threads=0, window=0):
     """BLASST prefill forward for query tiles ``units`` (list of (b, hq, i)).
+
+    ``window`` > 0 (causal only): query r sees the ``window`` keys ending at
+    its diagonal (sliding-window attention); 0 = no window.
 
     q [B,Hq,Lq,d], k/v [B,Hkv,Lkv,d] bf16.  Returns a dict with
     ``o`` [n_units,Br,d] f64, ``lse`` [n_units,Br], ``mask`` [n_units,nk] u8,
@@ -111,9 +128,9 @@ def prefill(q, k, v, scale, causal, ln_lambda, Br, Bc, units=None,
     mask = np.zeros((n, nk), np.uint8)
     margin = np.zeros((n, nk), np.float64)
     counts = np.zeros(2, np.int64)
-    rc = lib.oracle_prefill(
+    rc = lib.oracle_prefill_window(
         _ptr(qb, _u16p), _ptr(kb, _u16p), _ptr(vb, _u16p),
-        B, Hq, Hkv, Lq, Lkv, d, float(scale), int(bool(causal)),
+        B, Hq, Hkv, Lq, Lkv, d, float(scale), int(bool(causal)), int(window),
         float(ln_lambda), Br, Bc, n, _ptr(ua, _i32p),
         _ptr(o, _dp), _ptr(lse, _dp), _ptr(mask, _u8p), _ptr(margin, _dp),
         _ptr(counts, _i64p), int(n_threads))
@@ -125,8 +142,11 @@ def prefill(q, k, v, scale, causal, ln_lambda, Br, Bc, units=None,
                 units=ua, threads=threads)
 
 
-def decode(q, k, v, scale, ln_lambda, Bc, num_splits, n_threads=0):
+def decode(q, k, v, scale, ln_lambda, Bc, num_splits, n_threads=0, window=0):
     """BLASST decode forward with split-KV and log-sum-exp merge.
+
+    ``window`` > 0: the token sees only the last ``window`` keys (sliding
+    window); the splits divide the blocks holding them.
 
     q [B,Hq,d], k/v [B,Hkv,Lkv,d] bf16.  Returns ``o`` [B,Hq,d], ``lse``
     [B,Hq], ``o_part`` [B,Hq,S,d], ``lse_part`` [B,Hq,S], ``mask``
@@ -145,9 +165,9 @@ def decode(q, k, v, scale, ln_lambda, Bc, num_splits, n_threads=0):
     mask = np.zeros((B, Hkv, nk), np.uint8)
     margin = np.zeros((B, Hkv, nk), np.float64)
     counts = np.zeros(2, np.int64)
-    rc = lib.oracle_decode(
+    rc = lib.oracle_decode_window(
         _ptr(qb, _u16p), _ptr(kb, _u16p), _ptr(vb, _u16p),
-        B, Hq, Hkv, Lkv, d, float(scale), float(ln_lambda), Bc, S,
+        B, Hq, Hkv, Lkv, d, float(scale), int(window), float(ln_lambda), Bc, S,
         _ptr(o, _dp), _ptr(lse, _dp), _ptr(op, _dp), _ptr(lp, _dp),
         _ptr(mask, _u8p), _ptr(margin, _dp), _ptr(counts, _i64p),
         int(n_threads))

@@ -33,11 +33,12 @@ int oracle_split_begin(int nk, int S, int s) {
  * One query tile against KV blocks [j0, j1) of one KV head.
  *
  * The tile's rows are the query vectors qrows[r] (already converted to
- * float64); row r may attend to keys 0..limit[r] (inclusive).  State m, l,
- * acc is the blockwise online-softmax state, initialised here.
+ * float64); row r may attend to keys first[r]..limit[r] (inclusive; first
+ * may be NULL, meaning 0).  State m, l, acc is the blockwise online-softmax
+ * state, initialised here.
  *
  * Block j (keys c in [j*Bc, min((j+1)*Bc, Lkv))):
- *   S[r][c]  = scale * q_r . k_c, or -inf when c > limit[r]
+ *   S[r][c]  = scale * q_r . k_c, or -inf when c > limit[r] or c < first[r]
  *   visited  = some S[r][c] is finite
  *   mt[r]    = max_c S[r][c]                         (block-local row max)
  *   skip     = ln_lambda > -inf and for every row:  mt[r] == -inf  or
@@ -47,8 +48,8 @@ int oracle_split_begin(int nk, int S, int s) {
  *              acc = alpha*acc + sum_c p_c v_c;  m = m_new
  *   skipped  : no exp, no V, no P.V; m, l, acc unchanged
  */
-static void run_tile(int nrows, const double *qrows, const int *limit,
-                     const uint16_t *kh, const uint16_t *vh, int Lkv, int d,
+static void run_tile(int nrows, const double *qrows, const int *first,
+                     const int *limit, const uint16_t *kh, const uint16_t *vh, int Lkv, int d,
                      double scale, double ln_lambda, int Bc, int j0, int j1,
                      double *m, double *l, double *acc, uint8_t *mask,
                      double *margin, int64_t *n_visited, int64_t *n_skipped) {
@@ -70,8 +71,12 @@ static void run_tile(int nrows, const double *qrows, const int *limit,
 
         /* Is any entry of this (tile, block) pair unmasked? */
         int visited = 0;
-        for (int r = 0; r < nrows; ++r)
-            if (limit[r] >= c0) visited = 1;
+        for (int r = 0; r < nrows; ++r) {
+            int lo = first ? first[r] : 0;
+            if (lo < c0) lo = c0;
+            int hi = limit[r] < c1 - 1 ? limit[r] : c1 - 1;
+            if (lo <= hi) visited = 1;
+        }
         if (!visited) {
             if (mask) mask[j] = ORACLE_NOT_VISITED;
             if (margin) margin[j] = NAN;
@@ -88,7 +93,7 @@ static void run_tile(int nrows, const double *qrows, const int *limit,
             mt[r] = -INFINITY;
             for (int c = 0; c < nc; ++c) {
                 double s;
-                if (c0 + c > limit[r]) {
+                if (c0 + c > limit[r] || (first && c0 + c < first[r])) {
                     s = -INFINITY;
                 } else {
                     double dot = 0.0;
@@ -164,8 +169,21 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                    int n_units, const int32_t *units,
                    double *o, double *lse, uint8_t *mask, double *margin,
                    int64_t *counts, int n_threads) {
+    return oracle_prefill_window(q, k, v, B, Hq, Hkv, Lq, Lkv, d, scale,
+                                 causal, 0, ln_lambda, Br, Bc, n_units, units,
+                                 o, lse, mask, margin, counts, n_threads);
+}
+
+int oracle_prefill_window(const uint16_t *q, const uint16_t *k,
+                          const uint16_t *v, int B, int Hq, int Hkv, int Lq,
+                          int Lkv, int d, double scale, int causal,
+                          int window, double ln_lambda, int Br, int Bc,
+                          int n_units, const int32_t *units, double *o,
+                          double *lse, uint8_t *mask, double *margin,
+                          int64_t *counts, int n_threads) {
     if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || Lq < 1 || Lkv < 1 ||
-        d < 1 || Br < 1 || Bc < 1 || n_units < 0 || !(ln_lambda <= 0.0))
+        d < 1 || Br < 1 || Bc < 1 || n_units < 0 || !(ln_lambda <= 0.0) ||
+        window < 0 || (window > 0 && !causal))
         return -1;
     int nq = (Lq + Br - 1) / Br;
     int nk = (Lkv + Bc - 1) / Bc;
@@ -187,6 +205,7 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         int nrows = r1 - r0;
         double *qrows = (double *)malloc(sizeof(double) * (size_t)nrows * d);
         int *limit = (int *)malloc(sizeof(int) * (size_t)nrows);
+        int *first = (int *)malloc(sizeof(int) * (size_t)nrows);
         double *m = (double *)malloc(sizeof(double) * (size_t)nrows);
         double *l = (double *)malloc(sizeof(double) * (size_t)nrows);
         double *acc = (double *)malloc(sizeof(double) * (size_t)nrows * d);
@@ -198,14 +217,18 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 qrows[(size_t)r * d + x] =
                     oracle_bf16_to_double(qh[(size_t)(r0 + r) * d + x]);
             int lim = Lkv - 1;
+            int lo = 0;
             if (causal) {
                 int diag = r0 + r + (Lkv - Lq); /* bottom-right alignment */
                 if (diag < lim) lim = diag;
+                /* sliding window: the `window` keys ending at the diagonal */
+                if (window > 0 && diag - window + 1 > 0) lo = diag - window + 1;
             }
             limit[r] = lim;
+            first[r] = lo;
         }
         int64_t uv = 0, us = 0;
-        run_tile(nrows, qrows, limit, kh, vh, Lkv, d, scale, ln_lambda, Bc, 0,
+        run_tile(nrows, qrows, first, limit, kh, vh, Lkv, d, scale, ln_lambda, Bc, 0,
                  nk, m, l, acc, mask ? mask + (size_t)u * nk : NULL,
                  margin ? margin + (size_t)u * nk : NULL, &uv, &us);
         vis += uv;
@@ -224,6 +247,7 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         }
         free(qrows);
         free(limit);
+        free(first);
         free(m);
         free(l);
         free(acc);
@@ -265,10 +289,25 @@ int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                   double *o, double *lse, double *o_part, double *lse_part,
                   uint8_t *mask, double *margin, int64_t *counts,
                   int n_threads) {
+    return oracle_decode_window(q, k, v, B, Hq, Hkv, Lkv, d, scale, 0,
+                                ln_lambda, Bc, num_splits, o, lse, o_part,
+                                lse_part, mask, margin, counts, n_threads);
+}
+
+int oracle_decode_window(const uint16_t *q, const uint16_t *k,
+                         const uint16_t *v, int B, int Hq, int Hkv, int Lkv,
+                         int d, double scale, int window, double ln_lambda,
+                         int Bc, int num_splits, double *o, double *lse,
+                         double *o_part, double *lse_part, uint8_t *mask,
+                         double *margin, int64_t *counts, int n_threads) {
     if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || Lkv < 1 || d < 1 ||
-        Bc < 1 || num_splits < 1 || !(ln_lambda <= 0.0))
+        Bc < 1 || num_splits < 1 || !(ln_lambda <= 0.0) || window < 0)
         return -1;
     int nk = (Lkv + Bc - 1) / Bc;
+    /* sliding window: the decode token (position Lkv - 1) sees the last
+     * `window` keys; the splits divide the blocks that hold them */
+    int key_lo = (window > 0 && Lkv - window > 0) ? Lkv - window : 0;
+    int jlo = key_lo / Bc;
     int G = Hq / Hkv;
     int S = num_splits;
     double *op = (double *)malloc(sizeof(double) * (size_t)B * Hq * S * d);
@@ -281,6 +320,7 @@ int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         int b = bh / Hkv, hkv = bh % Hkv;
         double *qrows = (double *)malloc(sizeof(double) * (size_t)G * d);
         int *limit = (int *)malloc(sizeof(int) * (size_t)G);
+        int *first = (int *)malloc(sizeof(int) * (size_t)G);
         double *m = (double *)malloc(sizeof(double) * (size_t)G);
         double *l = (double *)malloc(sizeof(double) * (size_t)G);
         double *acc = (double *)malloc(sizeof(double) * (size_t)G * d);
@@ -289,17 +329,23 @@ int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             for (int x = 0; x < d; ++x)
                 qrows[(size_t)g * d + x] = oracle_bf16_to_double(qg[x]);
             limit[g] = Lkv - 1; /* the decode token sees the whole cache */
+            first[g] = key_lo;  /* ... or its last `window` keys */
         }
+        if (mask)
+            for (int j = 0; j < jlo; ++j)
+                mask[(size_t)bh * nk + j] = ORACLE_NOT_VISITED;
+        if (margin)
+            for (int j = 0; j < jlo; ++j) margin[(size_t)bh * nk + j] = NAN;
         const uint16_t *kh = k + (size_t)bh * Lkv * d;
         const uint16_t *vh = v + (size_t)bh * Lkv * d;
         uint8_t *mk = mask ? mask + (size_t)bh * nk : NULL;
         double *mg = margin ? margin + (size_t)bh * nk : NULL;
         for (int s = 0; s < S; ++s) {
-            int j0 = oracle_split_begin(nk, S, s);
-            int j1 = oracle_split_begin(nk, S, s + 1);
+            int j0 = jlo + oracle_split_begin(nk - jlo, S, s);
+            int j1 = jlo + oracle_split_begin(nk - jlo, S, s + 1);
             int64_t uv = 0, us = 0;
-            run_tile(G, qrows, limit, kh, vh, Lkv, d, scale, ln_lambda, Bc,
-                     j0, j1, m, l, acc, mk, mg, &uv, &us);
+            run_tile(G, qrows, first, limit, kh, vh, Lkv, d, scale, ln_lambda,
+                     Bc, j0, j1, m, l, acc, mk, mg, &uv, &us);
             vis += uv;
             skp += us;
             for (int g = 0; g < G; ++g) {
@@ -316,6 +362,7 @@ int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         }
         free(qrows);
         free(limit);
+        free(first);
         free(m);
         free(l);
         free(acc);
@@ -411,7 +458,7 @@ int oracle_decode_paged(const uint16_t *q, const uint16_t *k_pool,
             int j0 = oracle_split_begin(nk, S, s);
             int j1 = oracle_split_begin(nk, S, s + 1);
             int64_t uv = 0, us = 0;
-            run_tile(G, qrows, limit, kh, vh, L, d, scale, lnl, Bc, j0, j1, m,
+            run_tile(G, qrows, NULL, limit, kh, vh, L, d, scale, lnl, Bc, j0, j1, m,
                      l, acc, mk, mg, &uv, &us);
             vis += uv;
             skp += us;

@@ -80,6 +80,22 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                    int64_t *counts, int n_threads);
 
 /*
+ * Prefill with a causal sliding window (the attention-variant row of the
+ * method's supported forms): query r sees the `window` keys ending at its
+ * diagonal, c in [diag_r - window + 1, diag_r] with diag_r = r + Lkv - Lq.
+ * window = 0 is plain causal/non-causal attention (oracle_prefill); a
+ * window needs causal = 1.  Blocks wholly outside every row's window are
+ * not visited; a row with no visible key in a block votes "skippable" there.
+ */
+int oracle_prefill_window(const uint16_t *q, const uint16_t *k,
+                          const uint16_t *v, int B, int Hq, int Hkv, int Lq,
+                          int Lkv, int d, double scale, int causal,
+                          int window, double ln_lambda, int Br, int Bc,
+                          int n_units, const int32_t *units, double *o,
+                          double *lse, uint8_t *mask, double *margin,
+                          int64_t *counts, int n_threads);
+
+/*
  * Decode forward: one query token per sequence, the G = Hq/Hkv query heads
  * of a KV head form the rows of one tile.
  *
@@ -97,6 +113,20 @@ int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                   double *o, double *lse, double *o_part, double *lse_part,
                   uint8_t *mask, double *margin, int64_t *counts,
                   int n_threads);
+
+/*
+ * Decode with a sliding window: the token (position Lkv - 1) sees keys
+ * [max(0, Lkv - window), Lkv).  The blocks holding them,
+ * [jlo, nk) with jlo = floor(max(0, Lkv - window) / Bc), are divided into
+ * the S splits as oracle_decode divides [0, nk); blocks before jlo are not
+ * visited.  window = 0 is oracle_decode.
+ */
+int oracle_decode_window(const uint16_t *q, const uint16_t *k,
+                         const uint16_t *v, int B, int Hq, int Hkv, int Lkv,
+                         int d, double scale, int window, double ln_lambda,
+                         int Bc, int num_splits, double *o, double *lse,
+                         double *o_part, double *lse_part, uint8_t *mask,
+                         double *margin, int64_t *counts, int n_threads);
 
 /*
  * Paged, variable-length decode (block-table indirection).

@@ -93,3 +93,21 @@ def prefill_scores(q, k, scale, causal, b, hq, G):
     if causal:
         s = np.where(causal_visible(q.shape[2], k.shape[2]), s, -np.inf)
     return s
+
+
+def window_visible(Lq, Lkv, W):
+    """[Lq, Lkv] bool: causal sliding window of W keys ending at the
+    (bottom-right aligned) diagonal: diag - W < c <= diag."""
+    r = np.arange(Lq)[:, None]
+    c = np.arange(Lkv)[None, :]
+    diag = r + (Lkv - Lq)
+    return (c <= diag) & (c > diag - W)
+
+
+def dense_masked(qh, kh, vh, scale, vis):
+    """One head: softmax(scale q k^T where vis, else -inf) v, float64."""
+    s = np.where(vis, scale * (qh @ kh.T), -np.inf)
+    mx = s.max(axis=1, keepdims=True)
+    p = np.exp(s - mx)
+    den = p.sum(axis=1, keepdims=True)
+    return (p @ vh) / den, (mx + np.log(den))[:, 0]
