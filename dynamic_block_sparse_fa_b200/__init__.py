@@ -7,16 +7,19 @@ been built (``python dynamic_block_sparse_fa_b200/build.py``).
 from .blasst import (BlasstError, Stats, blasst_calibrate,
                      blasst_check_device_error, blasst_decode,
                      blasst_decode_noalloc, blasst_decode_paged,
-                     blasst_decode_splits, blasst_decode_workspace_size,
+                     blasst_decode_splits, blasst_decode_window,
+                     blasst_decode_workspace_size,
                      blasst_fit_a, blasst_last_error, blasst_prefill,
+                     blasst_prefill_window,
                      blasst_selftest_wait_timeout, blasst_skip_stats_reset,
                      blasst_strerror, blasst_version)
 
 __all__ = ["BlasstError", "Stats", "blasst_calibrate",
            "blasst_check_device_error", "blasst_decode",
            "blasst_decode_noalloc", "blasst_decode_paged",
-           "blasst_decode_splits",
+           "blasst_decode_splits", "blasst_decode_window",
            "blasst_decode_workspace_size", "blasst_fit_a", "blasst_last_error",
-           "blasst_prefill", "blasst_selftest_wait_timeout",
+           "blasst_prefill", "blasst_prefill_window",
+           "blasst_selftest_wait_timeout",
            "blasst_skip_stats_reset", "blasst_strerror",
            "blasst_version"]

@@ -73,10 +73,18 @@ _lib.blasst_prefill.restype = _i
 _lib.blasst_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                 _i, _f, _i, _f, _i, _i,
                                 ctypes.POINTER(SkipStats), _vp]
+_lib.blasst_prefill_window.restype = _i
+_lib.blasst_prefill_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                       _i, _i, _f, _i, _i, _f, _i, _i,
+                                       ctypes.POINTER(SkipStats), _vp]
 _lib.blasst_decode.restype = _i
 _lib.blasst_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                _f, _f, _i, _i, _vp, _sz,
                                ctypes.POINTER(SkipStats), _vp]
+_lib.blasst_decode_window.restype = _i
+_lib.blasst_decode_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                      _i, _f, _i, _f, _i, _i, _vp, _sz,
+                                      ctypes.POINTER(SkipStats), _vp]
 _lib.blasst_decode_paged.restype = _i
 _lib.blasst_decode_paged.argtypes = [_vp, _vp, _vp, ctypes.c_longlong, _i, _i,
                                      _vp, _i, _vp, _i, _vp, _vp, _i, _i, _i,
@@ -199,11 +207,13 @@ def blasst_selftest_wait_timeout(limit_cycles=1_000_000, stream=None):
 
 def blasst_prefill(q, k, v, *, scale=None, causal=True, ln_lambda=-math.inf,
                    Br=128, Bc=128, o=None, lse=None, want_lse=True,
-                   stats: Stats | None = None, stats_only=False, stream=None):
+                   stats: Stats | None = None, stats_only=False, stream=None,
+                   window=0):
     """BLASST prefill forward.  q [B,Hq,Lq,d], k/v [B,Hkv,Lkv,d] bf16 CUDA.
 
-    Returns (o, lse); both None when stats_only (decisions and counters
-    only)."""
+    window > 0 (causal, 128x128 tiles): each query sees the ``window`` keys
+    ending at its diagonal (blasst_prefill_window).  Returns (o, lse); both
+    None when stats_only (decisions and counters only)."""
     B, Hq, Lq, d = q.shape
     _, Hkv, Lkv, _ = k.shape
     if scale is None:
@@ -215,12 +225,22 @@ def blasst_prefill(q, k, v, *, scale=None, causal=True, ln_lambda=-math.inf,
             lse = torch.empty(B, Hq, Lq, dtype=torch.float32, device=q.device)
     else:
         o, lse = None, None
-    st = _lib.blasst_prefill(
+    st = _lib.blasst_prefill_window(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lkv, d,
-        float(scale), int(bool(causal)), float(ln_lambda), Br, Bc,
+        float(scale), int(bool(causal)), int(window), float(ln_lambda), Br, Bc,
         stats.c_struct if stats is not None else None, _stream(stream))
-    _check(st, "blasst_prefill")
+    _check(st, "blasst_prefill_window")
     return o, lse
+
+
+def blasst_prefill_window(q, k, v, *, window, **kw):
+    """blasst_prefill with a causal sliding window of ``window`` keys."""
+    return blasst_prefill(q, k, v, window=window, **kw)
+
+
+def blasst_decode_window(q, k, v, *, window, **kw):
+    """blasst_decode over the last ``window`` keys of the cache."""
+    return blasst_decode(q, k, v, window=window, **kw)
 
 
 def blasst_decode_workspace_size(B, Hq, d, num_splits) -> int:
@@ -234,15 +254,18 @@ def blasst_decode_splits(B, Hkv, Lkv, Bc=64) -> int:
 def blasst_decode(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
                   num_splits=0, o=None, lse=None, want_lse=True,
                   workspace=None, stats: Stats | None = None,
-                  stats_only=False, stream=None):
+                  stats_only=False, stream=None, window=0):
     """BLASST decode forward.  q [B,Hq,d], k/v [B,Hkv,Lkv,d] bf16 CUDA.
 
-    Returns (o, lse); both None when stats_only."""
+    window > 0: the token sees only the last ``window`` keys
+    (blasst_decode_window).  Returns (o, lse); both None when stats_only."""
     B, Hq, d = q.shape
     _, Hkv, Lkv, _ = k.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    S = num_splits if num_splits > 0 else blasst_decode_splits(B, Hkv, Lkv, Bc)
+    jlo = (Lkv - window) // Bc if 0 < window < Lkv else 0
+    S = (num_splits if num_splits > 0
+         else blasst_decode_splits(B, Hkv, Lkv - jlo * Bc, Bc))
     ws_bytes = 0
     if not stats_only:
         if o is None:
@@ -255,11 +278,12 @@ def blasst_decode(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
         ws_bytes = workspace.numel() * workspace.element_size()
     else:
         o, lse, workspace = None, None, None
-    st = _lib.blasst_decode(
+    st = _lib.blasst_decode_window(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lkv, d,
-        float(scale), float(ln_lambda), Bc, S, _ptr(workspace), ws_bytes,
-        stats.c_struct if stats is not None else None, _stream(stream))
-    _check(st, "blasst_decode")
+        float(scale), int(window), float(ln_lambda), Bc, S, _ptr(workspace),
+        ws_bytes, stats.c_struct if stats is not None else None,
+        _stream(stream))
+    _check(st, "blasst_decode_window")
     return o, lse
 
 

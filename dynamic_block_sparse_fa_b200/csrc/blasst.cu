@@ -238,8 +238,21 @@ blasst_status_t blasst_decode(const void* q, const void* k_cache,
                               void* workspace, size_t workspace_bytes,
                               const blasst_skip_stats_t* skip_stats,
                               void* stream) {
+  return blasst_decode_window(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Lkv, d,
+                              scale, 0, ln_lambda, Bc, num_splits, workspace,
+                              workspace_bytes, skip_stats, stream);
+}
+
+blasst_status_t blasst_decode_window(const void* q, const void* k_cache,
+                                     const void* v_cache, void* o, float* lse,
+                                     int B, int Hq, int Hkv, int Lkv, int d,
+                                     float scale, int window, float ln_lambda,
+                                     int Bc, int num_splits, void* workspace,
+                                     size_t workspace_bytes,
+                                     const blasst_skip_stats_t* skip_stats,
+                                     void* stream) {
   if (!q || !k_cache || !v_cache) return BLASST_ERR_INVALID_ARG;
-  if (B < 1 || Hq < 1 || Hkv < 1 || Lkv < 1 || Hq % Hkv != 0)
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lkv < 1 || Hq % Hkv != 0 || window < 0)
     return BLASST_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !valid_ln_lambda(ln_lambda))
     return BLASST_ERR_INVALID_ARG;
@@ -251,9 +264,12 @@ blasst_status_t blasst_decode(const void* q, const void* k_cache,
       (o && !aligned16(o)))
     return BLASST_ERR_MISALIGNED;
   const int nk = (Lkv + Bc - 1) / Bc;
-  const int S = num_splits == 0 ? blasst_decode_splits(B, Hkv, Lkv, Bc)
-                                : num_splits;
-  if (S < 1 || S > nk) return BLASST_ERR_INVALID_ARG;
+  // blocks that hold the visible keys (all of them without a window)
+  const int jlo = (window > 0 && Lkv > window) ? (Lkv - window) / Bc : 0;
+  const int S = num_splits == 0
+                    ? blasst_decode_splits(B, Hkv, Lkv - jlo * Bc, Bc)
+                    : num_splits;
+  if (S < 1 || S > nk - jlo) return BLASST_ERR_INVALID_ARG;
   const long long grid = (long long)B * Hkv * S;
   if (grid > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED_SHAPE;
   const bool stats_only = (o == nullptr);
@@ -279,6 +295,7 @@ blasst_status_t blasst_decode(const void* q, const void* k_cache,
   a.scale = scale;
   a.ln_lambda = ln_lambda;
   a.stats_only = stats_only ? 1 : 0;
+  a.window = window;
 
   return launch_decode(a, G, false, grid, stats_only, o, lse, B * Hq, S,
                        static_cast<cudaStream_t>(stream));
@@ -441,9 +458,24 @@ blasst_status_t blasst_prefill(const void* q, const void* k, const void* v,
                                float ln_lambda, int Br, int Bc,
                                const blasst_skip_stats_t* skip_stats,
                                void* stream) {
+  return blasst_prefill_window(q, k, v, o, lse, B, Hq, Hkv, Lq, Lkv, d, scale,
+                               causal, 0, ln_lambda, Br, Bc, skip_stats,
+                               stream);
+}
+
+blasst_status_t blasst_prefill_window(const void* q, const void* k,
+                                      const void* v, void* o, float* lse,
+                                      int B, int Hq, int Hkv, int Lq, int Lkv,
+                                      int d, float scale, int causal,
+                                      int window, float ln_lambda, int Br,
+                                      int Bc,
+                                      const blasst_skip_stats_t* skip_stats,
+                                      void* stream) {
   if (!q || !k || !v) return BLASST_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lkv < 1 || Hq % Hkv != 0)
     return BLASST_ERR_INVALID_ARG;
+  if (window < 0 || (window > 0 && !causal)) return BLASST_ERR_INVALID_ARG;
+  if (window > 0 && Br != 128) return BLASST_ERR_UNSUPPORTED_SHAPE;
   if (!std::isfinite(scale) || !valid_ln_lambda(ln_lambda))
     return BLASST_ERR_INVALID_ARG;
   if (causal && Lq > Lkv) return BLASST_ERR_INVALID_ARG;
@@ -471,6 +503,7 @@ blasst_status_t blasst_prefill(const void* q, const void* k, const void* v,
   p.Bc = Bc;
   p.counters = skip_stats ? skip_stats->counters : nullptr;
   p.mask = skip_stats ? skip_stats->mask : nullptr;
+  p.window = window;
   cudaError_t e = blasst::launch_prefill(p, static_cast<cudaStream_t>(stream));
   return cuda_status(e, "prefill launch");
 }

@@ -48,6 +48,9 @@ struct DecodeArgs {
   long long page_stride;   // elements
   int log2_page, max_pages, num_pages;
   int per_length;  // ln_lambda is ln a; sequence b uses min(0, ln a - ln L_b)
+  // sliding window: the token sees only the last `window` keys (0 = all);
+  // the splits divide the blocks that hold them
+  int window;
 };
 
 constexpr int kDecD = 128;       // head dimension
@@ -159,9 +162,14 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
       ln_lambda = fminf(0.f, ln_lambda - logf((float)Lb));
   }
   const int nk_b = (Lb + kDecBc - 1) / kDecBc;
-  const int j0 = (int)(((long long)s * nk_b) / a.S);
-  const int j1 = (int)(((long long)(s + 1) * nk_b) / a.S);
+  // first visible key and its block (sliding window)
+  const int key_lo = (a.window > 0 && Lb > a.window) ? Lb - a.window : 0;
+  const int jlo = key_lo / kDecBc;
+  const int j0 = jlo + (int)(((long long)s * (nk_b - jlo)) / a.S);
+  const int j1 = jlo + (int)(((long long)(s + 1) * (nk_b - jlo)) / a.S);
   const int nblk = j1 - j0;
+  if (a.mask && s == 0)  // blocks left of the window are not visited
+    for (int j = tid; j < jlo; j += kDecThreads) a.mask[(size_t)bh * a.nk + j] = 0;
   // Paged cache: a block of 64 keys is npb copies of 2^seg_l2 rows, each
   // from one page.  The source offsets of the copies of blocks r (relative
   // to j0) are kept in a shared ring sOff[r mod 64][copy], filled 32 blocks
@@ -416,7 +424,8 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
           }
         }
         const float tot = reduce8_transpose<G>(part, lane);
-        sc[i] = (c < nvalid) ? tot * a.scale : -INFINITY;
+        sc[i] = (c < nvalid && j * kDecBc + c >= key_lo) ? tot * a.scale
+                                                         : -INFINITY;
       }
       float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));

@@ -47,6 +47,7 @@ struct PrefillProblem {
   int Br, Bc;
   unsigned long long* counters;
   unsigned char* mask;
+  int window;  // 0 = none
 };
 
 struct __align__(64) PrefillParams {
@@ -58,6 +59,9 @@ struct __align__(64) PrefillParams {
   int B, Hq, Hkv, Lq, Lkv, nq, nk, G;
   float scale, ln_lambda;
   int causal, stats_only;
+  // causal sliding window: row r sees keys [diag_r - window + 1, diag_r]
+  // (0 = no window; 128x128 tiles only)
+  int window;
 };
 
 template <int D, int BN, int BRL>

@@ -111,10 +111,15 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
   const int b = kvi / p.Hkv;
   const int hkv = kvi - b * p.Hkv;
   const int hq = hkv * p.G + (rem - (rem / p.G) * p.G);
-  int nblk_t[2];
+  // Tile t visits blocks [jlo_t[t], nblk_t[t]): up to its last row's
+  // diagonal, and from the block holding its first row's first key when a
+  // sliding window is set.  The CTA walks [jlo, nblk); ring slots and
+  // barrier phases count blocks from jlo (K, V) or from jlo_t (per tile).
+  int nblk_t[2], jlo_t[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int tile = 2 * pair + t;
+    jlo_t[t] = 0;
     if (tile >= p.nq) {
       nblk_t[t] = 0;
     } else {
@@ -122,9 +127,13 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
       const int kmax = p.causal ? min(p.Lkv - 1, last_row + (p.Lkv - p.Lq))
                                 : p.Lkv - 1;
       nblk_t[t] = kmax / BN + 1;
+      if (p.window > 0)
+        jlo_t[t] = max(0, tile * 128 + (p.Lkv - p.Lq) - p.window + 1) / BN;
     }
   }
   const int nblk = max(nblk_t[0], nblk_t[1]);
+  const int jlo = jlo_t[0];
+  auto in_range = [&](int t, int j) { return j >= jlo_t[t] && j < nblk_t[t]; };
 
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sK = smem + C::OFF_K;
@@ -172,7 +181,7 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
     const int zq = b * p.Hq + hq;
     const int zk = b * p.Hkv + hkv;
     auto issue_k = [&](int j) {
-      const int st = j % C::NKS;
+      const int st = (j - jlo) % C::NKS;
       mbar_arrive_expect_tx(&bar[C::B_KF + st], C::KBYTES);
 #pragma unroll
       for (int c = 0; c < D / 64; ++c)
@@ -190,25 +199,26 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(sQ + t * C::QBYTES + c * C::BOX_Q, &p.tq, &bar[C::B_Q],
                       c * 64, (2 * pair + t) * 128, zq, pol_q);
-      const int n0 = nblk < C::NKS ? nblk : C::NKS;
-      for (int j = 0; j < n0; ++j) issue_k(j);
+      const int n0 = nblk - jlo < C::NKS ? nblk - jlo : C::NKS;
+      for (int j = jlo; j < jlo + n0; ++j) issue_k(j);
     }
     __syncwarp();
     // Per block: first the V load (needed by the P.V right after the exp of
     // this block), then the K prefetch two blocks ahead (needed only by the
     // next block's QK, and blocked until this block's QKs release a slot).
     int vcount = 0;
-    for (int j = 0; j < nblk; ++j) {
+    for (int j = jlo; j < nblk; ++j) {
       if (!stats_only) {
         bool need = false, ok = true;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (need || j >= nblk_t[t]) continue;
-          const bool w = mbar_wait(&bar[C::B_DEC + t * C::R + j % C::R],
-                                   (j / C::R) & 1, kWaitPrefillLoad, j,
-                                   100 + t * C::R + j % C::R);
+          if (need || !in_range(t, j)) continue;
+          const int jt = j - jlo_t[t];
+          const bool w = mbar_wait(&bar[C::B_DEC + t * C::R + jt % C::R],
+                                   (jt / C::R) & 1, kWaitPrefillLoad, j,
+                                   100 + t * C::R + jt % C::R);
           if (!__all_sync(FULL, w)) { ok = false; break; }
-          need = dec_flag[t * C::R + j % C::R] != 0;
+          need = dec_flag[t * C::R + jt % C::R] != 0;
         }
         if (!ok) break;
         if (need) {
@@ -230,8 +240,9 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
         }
       }
       if (j + C::NKS < nblk) {
-        const bool w = mbar_wait(&bar[C::B_KE + j % C::NKS], (j / C::NKS) & 1,
-                                 kWaitPrefillLoad, j, j % C::NKS);
+        const int jr = j - jlo;
+        const bool w = mbar_wait(&bar[C::B_KE + jr % C::NKS], (jr / C::NKS) & 1,
+                                 kWaitPrefillLoad, j, jr % C::NKS);
         if (!__all_sync(FULL, w)) break;
         if (leader) issue_k(j + C::NKS);
         __syncwarp();
@@ -247,7 +258,7 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
     const uint32_t aK = smem_u32(sK);
     const uint32_t aV = smem_u32(sV);
     auto qk = [&](int t, int j) {
-      const int st = j % C::NKS;
+      const int st = (j - jlo) % C::NKS;
       const uint32_t d_s = tmem + C::COL_S + t * 128;
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
@@ -268,19 +279,26 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
       tc_fence_after();
       if (ok) {
         for (int t = 0; t < 2; ++t)
-          if (nblk_t[t] > 0) qk(t, 0);
+          if (in_range(t, jlo)) qk(t, jlo);
         mma_commit(&bar[C::B_KE]);
       }
       int vcount = 0;
       int npv[2] = {0, 0};
-      for (int j = 0; j < nblk && ok; ++j) {
+      for (int j = jlo; j < nblk && ok; ++j) {
         int vslot = -1;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (!ok || j >= nblk_t[t]) continue;
-          ok = mbar_wait(&bar[C::B_PF + t], j & 1, kWaitPrefillMma, j, 300 + t);
-          if (!ok) break;
-          const bool kept = !stats_only && dec_flag[t * C::R + j % C::R] != 0;
+          const bool cur = in_range(t, j);
+          const bool more = in_range(t, j + 1);
+          if (!ok || !(cur || more)) continue;
+          const int jt = j - jlo_t[t];
+          bool kept = false;
+          if (cur) {
+            ok = mbar_wait(&bar[C::B_PF + t], jt & 1, kWaitPrefillMma, j,
+                           300 + t);
+            if (!ok) break;
+            kept = !stats_only && dec_flag[t * C::R + jt % C::R] != 0;
+          }
           if (kept && vslot < 0) {
             vslot = vcount % C::NVS;
             ok = mbar_wait(&bar[C::B_VF + vslot], (vcount / C::NVS) & 1,
@@ -288,11 +306,10 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
             ++vcount;
             if (!ok) break;
           }
-          const bool more = j + 1 < nblk_t[t];
           if (more) {
-            ok = mbar_wait(&bar[C::B_KF + (j + 1) % C::NKS],
-                           ((j + 1) / C::NKS) & 1, kWaitPrefillMma, j + 1,
-                           (j + 1) % C::NKS);
+            const int jr1 = j + 1 - jlo;
+            ok = mbar_wait(&bar[C::B_KF + jr1 % C::NKS], (jr1 / C::NKS) & 1,
+                           kWaitPrefillMma, j + 1, jr1 % C::NKS);
             if (!ok) break;
           }
           tc_fence_after();
@@ -314,7 +331,7 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
         }
         if (!ok) break;
         if (vslot >= 0) mma_commit(&bar[C::B_VE + vslot]);
-        if (j + 1 < nblk) mma_commit(&bar[C::B_KE + (j + 1) % C::NKS]);
+        if (j + 1 < nblk) mma_commit(&bar[C::B_KE + (j + 1 - jlo) % C::NKS]);
       }
     }
     __syncwarp();
@@ -341,6 +358,10 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
     const bool active = nb > 0 && row_g < p.Lq;
     const int lim = p.causal ? min(row_g + (p.Lkv - p.Lq), p.Lkv - 1)
                              : p.Lkv - 1;
+    // first key of the row's sliding window (0 without a window)
+    const int first = p.window > 0
+                          ? max(0, row_g + (p.Lkv - p.Lq) - p.window + 1)
+                          : 0;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t col_s = C::COL_S + t * 128 + half * CPT;      // my scores
     const uint32_t col_p = C::COL_S + t * 128 + half * (CPT / 2);  // my P
@@ -361,8 +382,9 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
     unsigned long long n_vis = 0, n_skp = 0;
     bool ok = true;
 
-    for (int j = 0; j < nb; ++j) {
-      if (!mbar_wait(&bar[C::B_SF + t], j & 1, kWaitPrefillSoftmax, j, 400 + t))
+    for (int j = jlo_t[t]; j < nb; ++j) {
+      const int jt = j - jlo_t[t];  // blocks this tile has visited before j
+      if (!mbar_wait(&bar[C::B_SF + t], jt & 1, kWaitPrefillSoftmax, j, 400 + t))
         abort_t[t] = 1;  // read by every thread of the tile after the vote
       tc_fence_after();
       uint32_t sr[CPT / 32][32];
@@ -372,12 +394,13 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
       tc_wait_ld();
 
       const int col0 = j * BN + half * CPT;  // first score column of mine
-      if (col0 + CPT - 1 > lim) {
+      if (col0 + CPT - 1 > lim || col0 < first) {
 #pragma unroll
         for (int c = 0; c < CPT / 32; ++c)
 #pragma unroll
           for (int x = 0; x < 32; ++x)
-            if (col0 + c * 32 + x > lim) sr[c][x] = __float_as_uint(-INFINITY);
+            if (col0 + c * 32 + x > lim || col0 + c * 32 + x < first)
+              sr[c][x] = __float_as_uint(-INFINITY);
       }
       float mt;
       {
@@ -414,8 +437,8 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
         ++n_vis;
         if (skip) ++n_skp;
         if (p.mask) p.mask[mask_row + j] = skip ? 2 : 1;
-        dec_flag[t * C::R + j % C::R] = skip ? 0 : 1;
-        mbar_arrive(&bar[C::B_DEC + t * C::R + j % C::R]);
+        dec_flag[t * C::R + jt % C::R] = skip ? 0 : 1;
+        mbar_arrive(&bar[C::B_DEC + t * C::R + jt % C::R]);
       }
       if (skip || stats_only) {
         __syncwarp();
@@ -481,7 +504,8 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
         atomicAdd(&p.counters[1], n_skp);
       }
       if (p.mask)
-        for (int j = nb; j < p.nk; ++j) p.mask[mask_row + j] = 0;
+        for (int j = 0; j < p.nk; ++j)
+          if (j < jlo_t[t] || j >= nb) p.mask[mask_row + j] = 0;
     }
     if (ok && !stats_only && nb > 0) {
       const bool w = mbar_wait(&bar[C::B_OD + t], 0, kWaitPrefillEpilogue, nb,
@@ -560,6 +584,7 @@ cudaError_t launch_prefill2(const PrefillProblem& pr, cudaStream_t st) {
   p.ln_lambda = pr.ln_lambda;
   p.causal = pr.causal;
   p.stats_only = pr.o == nullptr ? 1 : 0;
+  p.window = pr.window;
   const long long grid = (long long)((p.nq + 1) / 2) * pr.B * pr.Hq;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(prefill2_kernel<D>,

@@ -107,6 +107,32 @@ blasst_status_t blasst_prefill(const void *q, const void *k, const void *v,
                                void *stream);
 
 /*
+ * blasst_prefill_window -- blasst_prefill with a causal sliding window (the
+ * attention variants the method is stated to support: MLSys'26 reading
+ * notes, claims on sliding-window / GQA / MLA forms; gist.science summary,
+ * section 3).  Query r attends to keys c with
+ *     diag_r - window < c <= diag_r,   diag_r = r + Lkv - Lq
+ * (the `window` keys ending at its bottom-right aligned diagonal).  A
+ * (tile, block) pair none of whose entries is inside the window is not
+ * visited (no load, no MMA, not counted, mask byte 0); a row with no
+ * visible key in a visited block votes "skippable" there, so a block in
+ * which a row sees its first keys is never skipped.
+ *
+ *  causal   must be 1 when window > 0
+ *  window   >= 0; 0 (or >= Lkv) is blasst_prefill exactly
+ *  Br, Bc   128, 128 when window > 0 (else BLASST_ERR_UNSUPPORTED_SHAPE)
+ *  other arguments, layouts, ownership and errors as blasst_prefill.
+ */
+blasst_status_t blasst_prefill_window(const void *q, const void *k,
+                                      const void *v, void *o, float *lse,
+                                      int B, int Hq, int Hkv, int Lq, int Lkv,
+                                      int d, float scale, int causal,
+                                      int window, float ln_lambda, int Br,
+                                      int Bc,
+                                      const blasst_skip_stats_t *skip_stats,
+                                      void *stream);
+
+/*
  * blasst_decode -- one query token per sequence against a contiguous bf16
  * KV cache, split-KV with a log-sum-exp merge.
  *
@@ -135,6 +161,32 @@ blasst_status_t blasst_decode(const void *q, const void *k_cache,
                               void *workspace, size_t workspace_bytes,
                               const blasst_skip_stats_t *skip_stats,
                               void *stream);
+
+/*
+ * blasst_decode_window -- blasst_decode with a sliding attention window (the
+ * attention variants the method is stated to support: MLSys'26 reading
+ * notes, claims on sliding-window / GQA / MLA forms; gist.science summary,
+ * section 3).  The token at position Lkv - 1 attends only to keys
+ * [max(0, Lkv - window), Lkv).  The 64-key blocks that hold them,
+ * [jlo, nk) with jlo = floor(max(0, Lkv - window) / 64), are divided into the
+ * splits as blasst_decode divides [0, nk) (split s covers
+ * [jlo + floor(s (nk - jlo) / S), jlo + floor((s + 1)(nk - jlo) / S))); keys
+ * of block jlo before the window are masked; blocks before jlo are neither
+ * read nor counted, and their mask bytes are written 0 (not visited).
+ *
+ *  window       >= 0; 0 (or >= Lkv) is blasst_decode exactly
+ *  num_splits   1 .. nk - jlo, or 0 = blasst_decode_splits(B, Hkv,
+ *               Lkv - 64 jlo, 64)
+ *  other arguments, layouts, ownership and errors as blasst_decode.
+ */
+blasst_status_t blasst_decode_window(const void *q, const void *k_cache,
+                                     const void *v_cache, void *o, float *lse,
+                                     int B, int Hq, int Hkv, int Lkv, int d,
+                                     float scale, int window, float ln_lambda,
+                                     int Bc, int num_splits, void *workspace,
+                                     size_t workspace_bytes,
+                                     const blasst_skip_stats_t *skip_stats,
+                                     void *stream);
 
 /*
  * blasst_decode_noalloc -- blasst_decode for callers that may not allocate
