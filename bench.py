@@ -42,7 +42,8 @@ if ROOT not in sys.path:
 METRIC = ("sparse attn latency & dense-equiv TFLOP/s vs λ=0 at 50/70% "
           "sparsity; decode GB/s")
 
-DEC = dict(B=32, Hq=32, Hkv=8, Lkv=32768, d=128, Bc=64, target=0.70)
+DEC = dict(B=32, Hq=32, Hkv=8, Lkv=32768, d=128, Bc=64, target=0.70,
+           window=4096)
 
 # DRAM traffic of the dominant decode kernel per launch, relative to the
 # algorithmic bytes of that launch, from one ncu capture of a smaller case
@@ -53,7 +54,7 @@ DEC = dict(B=32, Hq=32, Hkv=8, Lkv=32768, d=128, Bc=64, target=0.70)
 # only for the kernel source it was measured on (sha256 prefix below).
 DECODE_TRAFFIC = dict(source="dynamic_block_sparse_fa_b200/csrc/decode.cuh",
                       sha256_16="e61d605edef51723", ratio=955.6 / 957.8)
-PRE = dict(B=1, Hq=32, Hkv=8, L=32768, d=128, Br=128, Bc=128)
+PRE = dict(B=1, Hq=32, Hkv=8, L=32768, d=128, Br=128, Bc=128, window=4096)
 
 
 def _measured_traffic(spec, algorithmic_bytes):
@@ -412,6 +413,9 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
         line["decode_paged"] = run_decode_paged(args, bl, dev, stream, q, k, v,
                                                 lnl, cal["a"], S, ms_max / K,
                                                 by_call)
+    if not args.no_window:
+        line["decode_window"] = run_decode_window(args, bl, q, k, v, lnl,
+                                                  stream)
 
     # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -559,12 +563,86 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
         r["a"] = cal["a"]
         r["speedup_vs_dense"] = round(dense["us"] / r["us"], 4)
         out[key] = r
+    if not args.no_window:
+        out["window"] = run_prefill_window(args, bl, q, k, v, o, lse,
+                                           out["s70"]["ln_lambda"], stream,
+                                           tf_peak)
     best = out["s70"]
     roof = {"bound": "tensor", "kernel": "prefill2_kernel<128> at 70%",
             "achieved": best["executed_tflops"], "peak": tf_peak,
             "peak_kind": peak_kind + " bf16 burst", "unit": "TFLOP/s",
             "frac": best["tensor_frac"], "traffic": None}
     return out, roof
+
+
+def run_prefill_window(args, bl, q, k, v, o, lse, lnl, stream, tf_peak):
+    """Sliding-window prefill on the same inputs: window WIN keys, dense and
+    at the ln lambda calibrated for 70% on the full causal problem."""
+    B, Hq, L, d = q.shape
+    Br = Bc = 128
+    K, W = args.prefill_steps, args.warmup
+    win = PRE["window"]
+    # dense-equivalent FLOPs: 4 d per visible (query, key) pair
+    pairs = sum(min(r + 1, win) for r in range(L))
+    dense_eq = 4.0 * B * Hq * d * pairs
+    res = {"window": win}
+    for key, x in (("dense", -math.inf), ("lnl_s70", lnl)):
+        st = bl.Stats(device=q.device)
+        bl.blasst_prefill_window(q, k, v, window=win, ln_lambda=x, o=o,
+                                 lse=lse, stats=st)
+        torch.cuda.synchronize()
+        vis, skp = st.read()
+        fn = lambda: bl.blasst_prefill_window(q, k, v, window=win,
+                                              ln_lambda=x, o=o, lse=lse)
+        ms = time_calls(fn, K, W, stream) / K
+        ex = prefill_flops(vis, vis - skp, Br, Bc, d)
+        res[key] = {"ln_lambda": x, "sparsity": skp / vis,
+                    "us": round(ms * 1e3, 1),
+                    "dense_equiv_tflops": round(dense_eq / (ms / 1e3) / 1e12, 1),
+                    "executed_tflops": round(ex / (ms / 1e3) / 1e12, 1),
+                    "tensor_frac": round(ex / (ms / 1e3) / 1e12 / tf_peak, 4)}
+    res["lnl_s70"]["speedup_vs_dense"] = round(
+        res["dense"]["us"] / res["lnl_s70"]["us"], 4)
+    return res
+
+
+def run_decode_window(args, bl, q, k, v, lnl, stream):
+    """Sliding-window decode on the decode workload's cache: the last WIN
+    keys, at the calibrated ln lambda and dense."""
+    B, Hq, d = q.shape
+    Hkv, Lkv = k.shape[1], k.shape[2]
+    Bc = DEC["Bc"]
+    win = DEC["window"]
+    K, W = args.steps, args.warmup
+    jlo = (Lkv - win) // Bc if 0 < win < Lkv else 0
+    S = bl.blasst_decode_splits(B, Hkv, Lkv - jlo * Bc, Bc)
+    nk = -(-Lkv // Bc)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    ws = torch.empty(bl.blasst_decode_workspace_size(B, Hq, d, S),
+                     dtype=torch.uint8, device=q.device)
+    res = {"window": win, "splits": S}
+    for key, x in (("dense", -math.inf), ("lnl_s70", lnl)):
+        st = bl.Stats(device=q.device, mask_numel=B * Hkv * nk)
+        bl.blasst_decode_window(q, k, v, window=win, ln_lambda=x, o=o, lse=lse,
+                                workspace=ws, stats=st)
+        torch.cuda.synchronize()
+        vis, skp = st.read()
+        mask = st.mask.view(B, Hkv, nk)
+        kept_rows = int((mask == 1).sum().item()) * Bc
+        by = (2 * d * B * Hkv * (Lkv - jlo * Bc) + 2 * d * kept_rows
+              + 2 * B * Hq * d + B * Hq * S * (d + 1) * 4 * 2
+              + B * Hq * (2 * d + 4))
+        fn = lambda: bl.blasst_decode_window(q, k, v, window=win, ln_lambda=x,
+                                             o=o, lse=lse, workspace=ws)
+        ms = time_calls(fn, K, W, stream) / K
+        res[key] = {"ln_lambda": x, "sparsity": skp / vis,
+                    "us": round(ms * 1e3, 2),
+                    "GBps": round(by / (ms / 1e3) / 1e9, 1),
+                    "bytes_per_call": by}
+    res["lnl_s70"]["speedup_vs_dense"] = round(
+        res["dense"]["us"] / res["lnl_s70"]["us"], 4)
+    return res
 
 
 # ---------------------------------------------------------------------------
@@ -655,6 +733,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-window", action="store_true",
+                    help="skip the sliding-window measurements")
     ap.add_argument("--no-paged", action="store_true",
                     help="skip the paged-cache decode measurements")
     ap.add_argument("--decode-batch", type=int, default=DEC["B"],
