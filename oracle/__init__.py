@@ -58,6 +58,13 @@ def _load():
             ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_double,
             ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp, _u8p, _dp, _i64p,
             ctypes.c_int]
+        lib.oracle_decode_batched.restype = ctypes.c_int
+        lib.oracle_decode_batched.argtypes = [
+            _u16p, _u16p, _u16p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_double, ctypes.c_double, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp, _u8p, _dp, _i64p,
+            ctypes.c_int]
         lib.oracle_decode.restype = ctypes.c_int
         lib.oracle_decode.argtypes = [
             _u16p, _u16p, _u16p,
@@ -173,6 +180,39 @@ def decode(q, k, v, scale, ln_lambda, Bc, num_splits, n_threads=0, window=0):
         int(n_threads))
     if rc != 0:
         raise ValueError("oracle_decode rejected its arguments")
+    threads = n_threads if n_threads > 0 else n_threads_default()
+    return dict(o=o, lse=lse, o_part=op, lse_part=lp, mask=mask,
+                margin=margin, visited=int(counts[0]),
+                skipped=int(counts[1]), threads=threads)
+
+
+def decode_batched(q, k, v, scale, ln_lambda, Bc, num_splits, batch,
+                   n_threads=0):
+    """Decode with the batched decision rule: blocks of each split are judged
+    in batches of ``batch`` against the max over all earlier blocks and the
+    whole batch.  ``batch`` = 1 is :func:`decode`.  Same outputs as
+    :func:`decode`."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, Hq, d = qb.shape
+    _, Hkv, Lkv, _ = kb.shape
+    nk = -(-Lkv // Bc)
+    S = int(num_splits)
+    o = np.zeros((B, Hq, d), np.float64)
+    lse = np.zeros((B, Hq), np.float64)
+    op = np.zeros((B, Hq, S, d), np.float64)
+    lp = np.zeros((B, Hq, S), np.float64)
+    mask = np.zeros((B, Hkv, nk), np.uint8)
+    margin = np.zeros((B, Hkv, nk), np.float64)
+    counts = np.zeros(2, np.int64)
+    rc = lib.oracle_decode_batched(
+        _ptr(qb, _u16p), _ptr(kb, _u16p), _ptr(vb, _u16p),
+        B, Hq, Hkv, Lkv, d, float(scale), float(ln_lambda), Bc, S, int(batch),
+        _ptr(o, _dp), _ptr(lse, _dp), _ptr(op, _dp), _ptr(lp, _dp),
+        _ptr(mask, _u8p), _ptr(margin, _dp), _ptr(counts, _i64p),
+        int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_decode_batched rejected its arguments")
     threads = n_threads if n_threads > 0 else n_threads_default()
     return dict(o=o, lse=lse, o_part=op, lse_part=lp, mask=mask,
                 margin=margin, visited=int(counts[0]),

@@ -153,6 +153,188 @@ static void run_tile(int nrows, const double *qrows, const int *first,
     free(vd);
 }
 
+static int set_threads(int n_threads);
+
+/*
+ * One decode tile (the G heads of a KV head, every key visible) against
+ * blocks [j0, j1) with the batched decision rule ("batched load
+ * scheduling": the Q.K products of a batch of `batch` consecutive blocks are
+ * formed before any of their V loads is decided).  Per batch
+ * [jb, min(jb + batch, j1)):
+ *   mt[r](j)  block-local row maxima of every block of the batch
+ *   Mb[r]     = max(M[r], max over the batch of mt[r](j)), M[r] the max over
+ *               all blocks before the batch (-inf at the start)
+ *   skip(j)   = ln_lambda > -inf and for every row mt[r](j) - Mb[r] < ln_lambda
+ *   kept j    : the online-softmax update of run_tile (m is the max over
+ *               kept blocks, the reference of l and acc)
+ *   M[r]      = Mb[r] after the batch.
+ * With batch = 1, Mb = max(M, mt(j)) and the decisions are run_tile's.
+ * margin[j] = max_r(mt[r](j) - Mb[r]) - ln_lambda.
+ */
+static void run_tile_batched(int nrows, const double *qrows,
+                             const uint16_t *kh, const uint16_t *vh, int Lkv,
+                             int d, double scale, double ln_lambda, int Bc,
+                             int j0, int j1, int batch, double *m, double *l,
+                             double *acc, uint8_t *mask, double *margin,
+                             int64_t *n_visited, int64_t *n_skipped) {
+    double *S = (double *)malloc(sizeof(double) * (size_t)batch * nrows * Bc);
+    double *mt = (double *)malloc(sizeof(double) * (size_t)batch * nrows);
+    double *M = (double *)malloc(sizeof(double) * (size_t)nrows);
+    double *Mb = (double *)malloc(sizeof(double) * (size_t)nrows);
+    double *vd = (double *)malloc(sizeof(double) * (size_t)Bc * d);
+
+    for (int r = 0; r < nrows; ++r) {
+        m[r] = -INFINITY;
+        l[r] = 0.0;
+        M[r] = -INFINITY;
+        for (int x = 0; x < d; ++x) acc[(size_t)r * d + x] = 0.0;
+    }
+    for (int jb = j0; jb < j1; jb += batch) {
+        int je = jb + batch < j1 ? jb + batch : j1;
+        /* 1. scores and block maxima of the whole batch */
+        for (int j = jb; j < je; ++j) {
+            int c0 = j * Bc;
+            int nc = (c0 + Bc < Lkv ? c0 + Bc : Lkv) - c0;
+            double *Sj = S + (size_t)(j - jb) * nrows * Bc;
+            double *mj = mt + (size_t)(j - jb) * nrows;
+            for (int r = 0; r < nrows; ++r) {
+                mj[r] = -INFINITY;
+                for (int c = 0; c < nc; ++c) {
+                    double dot = 0.0;
+                    for (int x = 0; x < d; ++x)
+                        dot += qrows[(size_t)r * d + x] *
+                               oracle_bf16_to_double(kh[(size_t)(c0 + c) * d + x]);
+                    double sc = scale * dot;
+                    Sj[(size_t)r * Bc + c] = sc;
+                    if (sc > mj[r]) mj[r] = sc;
+                }
+            }
+        }
+        /* 2. the batch's criterion max */
+        for (int r = 0; r < nrows; ++r) {
+            Mb[r] = M[r];
+            for (int j = jb; j < je; ++j) {
+                double v = mt[(size_t)(j - jb) * nrows + r];
+                if (v > Mb[r]) Mb[r] = v;
+            }
+        }
+        /* 3. decisions in block order; kept blocks update the state */
+        for (int j = jb; j < je; ++j) {
+            int c0 = j * Bc;
+            int nc = (c0 + Bc < Lkv ? c0 + Bc : Lkv) - c0;
+            const double *Sj = S + (size_t)(j - jb) * nrows * Bc;
+            const double *mj = mt + (size_t)(j - jb) * nrows;
+            *n_visited += 1;
+            int skip = ln_lambda > -INFINITY;
+            double mu = -INFINITY;
+            for (int r = 0; r < nrows; ++r) {
+                double diff = mj[r] - Mb[r];
+                if (!(diff < ln_lambda)) skip = 0;
+                if (diff > mu) mu = diff;
+            }
+            if (margin) margin[j] = mu - ln_lambda;
+            if (skip) {
+                *n_skipped += 1;
+                if (mask) mask[j] = ORACLE_SKIPPED;
+                continue;
+            }
+            if (mask) mask[j] = ORACLE_KEPT;
+            for (int c = 0; c < nc; ++c)
+                for (int x = 0; x < d; ++x)
+                    vd[(size_t)c * d + x] =
+                        oracle_bf16_to_double(vh[(size_t)(c0 + c) * d + x]);
+            for (int r = 0; r < nrows; ++r) {
+                double m_new = m[r] > mj[r] ? m[r] : mj[r];
+                double alpha = (m[r] == -INFINITY) ? 0.0 : exp(m[r] - m_new);
+                double psum = 0.0;
+                double *a = acc + (size_t)r * d;
+                for (int x = 0; x < d; ++x) a[x] *= alpha;
+                for (int c = 0; c < nc; ++c) {
+                    double p = exp(Sj[(size_t)r * Bc + c] - m_new);
+                    psum += p;
+                    for (int x = 0; x < d; ++x) a[x] += p * vd[(size_t)c * d + x];
+                }
+                l[r] = alpha * l[r] + psum;
+                m[r] = m_new;
+            }
+        }
+        for (int r = 0; r < nrows; ++r) M[r] = Mb[r];
+    }
+    free(S);
+    free(mt);
+    free(M);
+    free(Mb);
+    free(vd);
+}
+
+int oracle_decode_batched(const uint16_t *q, const uint16_t *k,
+                          const uint16_t *v, int B, int Hq, int Hkv, int Lkv,
+                          int d, double scale, double ln_lambda, int Bc,
+                          int num_splits, int batch, double *o, double *lse,
+                          double *o_part, double *lse_part, uint8_t *mask,
+                          double *margin, int64_t *counts, int n_threads) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || Lkv < 1 || d < 1 ||
+        Bc < 1 || num_splits < 1 || batch < 1 || !(ln_lambda <= 0.0))
+        return -1;
+    int nk = (Lkv + Bc - 1) / Bc;
+    int G = Hq / Hkv;
+    int S = num_splits;
+    double *op = (double *)malloc(sizeof(double) * (size_t)B * Hq * S * d);
+    double *lp = (double *)malloc(sizeof(double) * (size_t)B * Hq * S);
+    set_threads(n_threads);
+    int64_t vis = 0, skp = 0;
+
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : vis, skp)
+    for (int bh = 0; bh < B * Hkv; ++bh) {
+        int b = bh / Hkv, hkv = bh % Hkv;
+        double *qrows = (double *)malloc(sizeof(double) * (size_t)G * d);
+        double *m = (double *)malloc(sizeof(double) * (size_t)G);
+        double *l = (double *)malloc(sizeof(double) * (size_t)G);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)G * d);
+        for (int g = 0; g < G; ++g) {
+            const uint16_t *qg = q + ((size_t)b * Hq + hkv * G + g) * d;
+            for (int x = 0; x < d; ++x)
+                qrows[(size_t)g * d + x] = oracle_bf16_to_double(qg[x]);
+        }
+        const uint16_t *kh = k + (size_t)bh * Lkv * d;
+        const uint16_t *vh = v + (size_t)bh * Lkv * d;
+        uint8_t *mk = mask ? mask + (size_t)bh * nk : NULL;
+        double *mg = margin ? margin + (size_t)bh * nk : NULL;
+        for (int s = 0; s < S; ++s) {
+            int j0 = oracle_split_begin(nk, S, s);
+            int j1 = oracle_split_begin(nk, S, s + 1);
+            int64_t uv = 0, us = 0;
+            run_tile_batched(G, qrows, kh, vh, Lkv, d, scale, ln_lambda, Bc,
+                             j0, j1, batch, m, l, acc, mk, mg, &uv, &us);
+            vis += uv;
+            skp += us;
+            for (int g = 0; g < G; ++g) {
+                size_t row = ((size_t)b * Hq + hkv * G + g) * S + s;
+                if (l[g] > 0.0) {
+                    for (int x = 0; x < d; ++x)
+                        op[row * d + x] = acc[(size_t)g * d + x] / l[g];
+                    lp[row] = m[g] + log(l[g]);
+                } else { /* empty split */
+                    for (int x = 0; x < d; ++x) op[row * d + x] = 0.0;
+                    lp[row] = -INFINITY;
+                }
+            }
+        }
+        free(qrows);
+        free(m);
+        free(l);
+        free(acc);
+    }
+    oracle_combine(op, lp, B * Hq, S, d, o, lse);
+    if (o_part) memcpy(o_part, op, sizeof(double) * (size_t)B * Hq * S * d);
+    if (lse_part) memcpy(lse_part, lp, sizeof(double) * (size_t)B * Hq * S);
+    free(op);
+    free(lp);
+    counts[0] = vis;
+    counts[1] = skp;
+    return 0;
+}
+
 static int set_threads(int n_threads) {
 #ifdef _OPENMP
     if (n_threads > 0) omp_set_num_threads(n_threads);

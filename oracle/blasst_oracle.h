@@ -129,6 +129,24 @@ int oracle_decode_window(const uint16_t *q, const uint16_t *k,
                          double *margin, int64_t *counts, int n_threads);
 
 /*
+ * Decode with the batched decision rule (the Hindi summary's "batched load
+ * scheduling", section 2 kernel optimisation: several Q.K products are
+ * formed before the V loads are decided).  Each split's blocks are taken in
+ * batches of `batch` consecutive blocks; every block of a batch is judged
+ * against Mb = max(max over all earlier blocks, max over the whole batch):
+ *   skip(j) <=> for every head g:  mt_g(j) - Mb_g < ln_lambda.
+ * Kept blocks update the online softmax as in oracle_decode.  batch = 1 is
+ * oracle_decode exactly; a larger batch skips a superset of its blocks, and
+ * every skipped weight stays below lambda times the split's final max.
+ */
+int oracle_decode_batched(const uint16_t *q, const uint16_t *k,
+                          const uint16_t *v, int B, int Hq, int Hkv, int Lkv,
+                          int d, double scale, double ln_lambda, int Bc,
+                          int num_splits, int batch, double *o, double *lse,
+                          double *o_part, double *lse_part, uint8_t *mask,
+                          double *margin, int64_t *counts, int n_threads);
+
+/*
  * Paged, variable-length decode (block-table indirection).
  *
  * Sequence b holds seq_lens[b] tokens.  Its token t lives in page
