@@ -416,6 +416,8 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
     if not args.no_window:
         line["decode_window"] = run_decode_window(args, bl, q, k, v, lnl,
                                                   stream)
+        line["decode_batched"] = run_decode_batched(args, bl, q, k, v, lnl, S,
+                                                    ws, ms_max / K)
 
     # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -604,6 +606,32 @@ def run_prefill_window(args, bl, q, k, v, o, lse, lnl, stream, tf_peak):
     res["lnl_s70"]["speedup_vs_dense"] = round(
         res["dense"]["us"] / res["lnl_s70"]["us"], 4)
     return res
+
+
+def run_decode_batched(args, bl, q, k, v, lnl, S, ws, ms_seq):
+    """The batched decision rule (pairs of blocks scored before either is
+    decided) on the decode workload at the same ln lambda."""
+    B, Hq, d = q.shape
+    Hkv, Lkv = k.shape[1], k.shape[2]
+    Bc = DEC["Bc"]
+    nk = -(-Lkv // Bc)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    st = bl.Stats(device=q.device, mask_numel=B * Hkv * nk)
+    bl.blasst_decode_batched(q, k, v, batch=2, ln_lambda=lnl, num_splits=S,
+                             o=o, lse=lse, workspace=ws, stats=st)
+    torch.cuda.synchronize()
+    vis, skp = st.read()
+    kept_rows = kept_rows_from_mask(st.mask.view(B, Hkv, nk), Lkv, Bc)
+    by = decode_bytes(B, Hq, Hkv, Lkv, d, Bc, S, kept_rows)
+    fn = lambda: bl.blasst_decode_batched(q, k, v, batch=2, ln_lambda=lnl,
+                                          num_splits=S, o=o, lse=lse,
+                                          workspace=ws)
+    ms = time_calls(fn, args.steps, args.warmup, torch.cuda.current_stream()) / args.steps
+    return {"batch": 2, "ln_lambda": lnl, "sparsity": skp / vis,
+            "us": round(ms * 1e3, 2), "GBps": round(by / (ms / 1e3) / 1e9, 1),
+            "bytes_per_call": by,
+            "speedup_vs_sequential_rule": round(ms_seq / ms, 4)}
 
 
 def run_decode_window(args, bl, q, k, v, lnl, stream):

@@ -6,7 +6,8 @@ been built (``python dynamic_block_sparse_fa_b200/build.py``).
 """
 from .blasst import (BlasstError, Stats, blasst_calibrate,
                      blasst_check_device_error, blasst_decode,
-                     blasst_decode_noalloc, blasst_decode_paged,
+                     blasst_decode_batched, blasst_decode_noalloc,
+                     blasst_decode_paged,
                      blasst_decode_splits, blasst_decode_window,
                      blasst_decode_workspace_size,
                      blasst_fit_a, blasst_last_error, blasst_prefill,
@@ -16,7 +17,8 @@ from .blasst import (BlasstError, Stats, blasst_calibrate,
 
 __all__ = ["BlasstError", "Stats", "blasst_calibrate",
            "blasst_check_device_error", "blasst_decode",
-           "blasst_decode_noalloc", "blasst_decode_paged",
+           "blasst_decode_batched", "blasst_decode_noalloc",
+           "blasst_decode_paged",
            "blasst_decode_splits", "blasst_decode_window",
            "blasst_decode_workspace_size", "blasst_fit_a", "blasst_last_error",
            "blasst_prefill", "blasst_prefill_window",

@@ -85,6 +85,10 @@ _lib.blasst_decode_window.restype = _i
 _lib.blasst_decode_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                       _i, _f, _i, _f, _i, _i, _vp, _sz,
                                       ctypes.POINTER(SkipStats), _vp]
+_lib.blasst_decode_batched.restype = _i
+_lib.blasst_decode_batched.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                       _i, _f, _f, _i, _i, _i, _vp, _sz,
+                                       ctypes.POINTER(SkipStats), _vp]
 _lib.blasst_decode_paged.restype = _i
 _lib.blasst_decode_paged.argtypes = [_vp, _vp, _vp, ctypes.c_longlong, _i, _i,
                                      _vp, _i, _vp, _i, _vp, _vp, _i, _i, _i,
@@ -241,6 +245,40 @@ def blasst_prefill_window(q, k, v, *, window, **kw):
 def blasst_decode_window(q, k, v, *, window, **kw):
     """blasst_decode over the last ``window`` keys of the cache."""
     return blasst_decode(q, k, v, window=window, **kw)
+
+
+def blasst_decode_batched(q, k, v, *, batch=2, scale=None,
+                          ln_lambda=-math.inf, Bc=64, num_splits=0, o=None,
+                          lse=None, want_lse=True, workspace=None,
+                          stats: Stats | None = None, stats_only=False,
+                          stream=None):
+    """Decode with the batched decision rule: blocks are scored in pairs
+    and each is judged against the max over earlier blocks and the pair
+    (batch = 2; batch = 1 is blasst_decode).  Returns (o, lse)."""
+    B, Hq, d = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    S = num_splits if num_splits > 0 else blasst_decode_splits(B, Hkv, Lkv, Bc)
+    ws_bytes = 0
+    if not stats_only:
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and want_lse:
+            lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+        need = blasst_decode_workspace_size(B, Hq, d, S)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    else:
+        o, lse, workspace = None, None, None
+    st = _lib.blasst_decode_batched(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lkv, d,
+        float(scale), float(ln_lambda), Bc, S, int(batch), _ptr(workspace),
+        ws_bytes, stats.c_struct if stats is not None else None,
+        _stream(stream))
+    _check(st, "blasst_decode_batched")
+    return o, lse
 
 
 def blasst_decode_workspace_size(B, Hq, d, num_splits) -> int:

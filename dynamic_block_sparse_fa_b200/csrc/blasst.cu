@@ -164,28 +164,30 @@ namespace {
 // Split kernel, then (unless statistics only) the merge, launched as a
 // programmatic dependent of the split kernel so its launch overlaps the
 // split kernel's tail (it waits on griddepcontrol).
-template <int G, bool PAGED>
+template <int G, bool PAGED, int BATCH = 1>
 cudaError_t launch_split(const blasst::DecodeArgs& a, long long grid,
                          cudaStream_t st) {
   const int smem = blasst::DecodeSmem<G>::kTotal;
   cudaError_t e = cudaFuncSetAttribute(
-      blasst::decode_split_kernel<G, PAGED>,
+      blasst::decode_split_kernel<G, PAGED, BATCH>,
       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  blasst::decode_split_kernel<G, PAGED>
+  blasst::decode_split_kernel<G, PAGED, BATCH>
       <<<(unsigned)grid, blasst::kDecThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
 blasst_status_t launch_decode(const blasst::DecodeArgs& a, int G, bool paged,
                               long long grid, bool stats_only, void* o,
-                              float* lse, int rows, int S, cudaStream_t st) {
+                              float* lse, int rows, int S, cudaStream_t st,
+                              int batch = 1) {
   cudaError_t e = cudaErrorInvalidValue;
   switch (G) {
 #define BLASST_LAUNCH_DECODE(GG)                                             \
   case GG:                                                                   \
     e = paged ? launch_split<GG, true>(a, grid, st)                          \
-              : launch_split<GG, false>(a, grid, st);                        \
+              : (batch == 2 ? launch_split<GG, false, 2>(a, grid, st)        \
+                            : launch_split<GG, false>(a, grid, st));         \
     break;
     BLASST_LAUNCH_DECODE(1)
     BLASST_LAUNCH_DECODE(2)
@@ -210,6 +212,15 @@ blasst_status_t launch_decode(const blasst::DecodeArgs& a, int G, bool paged,
                          static_cast<__nv_bfloat16*>(o), lse, a.S);
   return cuda_status(e, "decode merge launch");
 }
+
+blasst_status_t decode_contiguous(const void* q, const void* k_cache,
+                                  const void* v_cache, void* o, float* lse,
+                                  int B, int Hq, int Hkv, int Lkv, int d,
+                                  float scale, int window, int batch,
+                                  float ln_lambda, int Bc, int num_splits,
+                                  void* workspace, size_t workspace_bytes,
+                                  const blasst_skip_stats_t* skip_stats,
+                                  void* stream);
 
 // Split partials inside a caller workspace (layout of
 // blasst_decode_workspace_size).
@@ -251,6 +262,38 @@ blasst_status_t blasst_decode_window(const void* q, const void* k_cache,
                                      size_t workspace_bytes,
                                      const blasst_skip_stats_t* skip_stats,
                                      void* stream) {
+  return decode_contiguous(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Lkv, d,
+                           scale, window, 1, ln_lambda, Bc, num_splits,
+                           workspace, workspace_bytes, skip_stats, stream);
+}
+
+blasst_status_t blasst_decode_batched(const void* q, const void* k_cache,
+                                      const void* v_cache, void* o, float* lse,
+                                      int B, int Hq, int Hkv, int Lkv, int d,
+                                      float scale, float ln_lambda, int Bc,
+                                      int num_splits, int batch,
+                                      void* workspace, size_t workspace_bytes,
+                                      const blasst_skip_stats_t* skip_stats,
+                                      void* stream) {
+  if (batch != 1 && batch != 2) return BLASST_ERR_UNSUPPORTED_SHAPE;
+  return decode_contiguous(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Lkv, d,
+                           scale, 0, batch, ln_lambda, Bc, num_splits,
+                           workspace, workspace_bytes, skip_stats, stream);
+}
+
+}  // extern "C"
+
+namespace {
+// Contiguous-cache decode: the sliding window (window > 0) and the batched
+// decision rule (batch = 2) are variants of the same split kernel.
+blasst_status_t decode_contiguous(const void* q, const void* k_cache,
+                                  const void* v_cache, void* o, float* lse,
+                                  int B, int Hq, int Hkv, int Lkv, int d,
+                                  float scale, int window, int batch,
+                                  float ln_lambda, int Bc, int num_splits,
+                                  void* workspace, size_t workspace_bytes,
+                                  const blasst_skip_stats_t* skip_stats,
+                                  void* stream) {
   if (!q || !k_cache || !v_cache) return BLASST_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || Lkv < 1 || Hq % Hkv != 0 || window < 0)
     return BLASST_ERR_INVALID_ARG;
@@ -298,8 +341,11 @@ blasst_status_t blasst_decode_window(const void* q, const void* k_cache,
   a.window = window;
 
   return launch_decode(a, G, false, grid, stats_only, o, lse, B * Hq, S,
-                       static_cast<cudaStream_t>(stream));
+                       static_cast<cudaStream_t>(stream), batch);
 }
+}  // namespace
+
+extern "C" {
 
 // ---------------------------------------------------------------------------
 // Decode over a paged cache (block table + per-sequence lengths)

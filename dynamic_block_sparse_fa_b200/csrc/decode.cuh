@@ -71,8 +71,8 @@ struct DecodeSmem {
   static constexpr int kK = 0;                                  // [NK][Bc][D] bf16
   static constexpr int kV = kK + kDecNK * kDecBlockBytes;        // [NV][Bc][D] bf16
   static constexpr int kP = kV + kDecNV * kDecBlockBytes;        // [NV][Bc][G] f32
-  static constexpr int kM = kP + kDecNV * kDecBc * G * 4;        // [2][4 warps][8] f32
-  static constexpr int kA = kM + 2 * 4 * 8 * 4;                  // [NV][8] f32
+  static constexpr int kM = kP + kDecNV * kDecBc * G * 4;        // [4][4 warps][8] f32
+  static constexpr int kA = kM + 4 * 4 * 8 * 4;                  // [NV][8] f32
   static constexpr int kL = kA + kDecNV * 8 * 4;                 // [4 warps][8] f32
   static constexpr int kNV = kL + 4 * 8 * 4;                     // [NV] int
   // paged cache, 2 chunks of 32 blocks, up to 4 copies a block: element
@@ -135,7 +135,7 @@ __device__ __forceinline__ int head_of_lane(int lane) {
   return h;
 }
 
-template <int G, bool PAGED>
+template <int G, bool PAGED, int BATCH = 1>
 __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
     decode_split_kernel(const DecodeArgs a) {
   using L = DecodeSmem<G>;
@@ -382,13 +382,12 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
   };
 
   bool ok = true;
-  for (int r = 0; r < nblk; ++r) {
+  // Scores of block r of the split (kept in registers by the caller) and
+  // the per-warp head maxima, written to sMw[warp][head].
+  auto score_block = [&](int r, float (&sc)[kDecBc / 16], float* sMw) {
     const int j = j0 + r;
     const int stage = r % kDecNK;
     const int nvalid = rows_of(j);
-
-    // ---- scores of block j (kept in registers) and per-warp head maxima
-    float sc[kDecBc / 16];
     if (ok)
       ok = mbar_wait(&kfull[stage], (uint32_t)(r / kDecNK) & 1u, kWaitDecodeK,
                      r, stage);
@@ -430,10 +429,19 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
       float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      // per-warp maxima, double-buffered by block parity: a fast warp may
-      // write block j+1's while a slow one still reads block j's
-      if ((lane & (kDupMask | 24)) == 0) sM[(r & 1) * 32 + warp * 8 + my_head] = mx;
+      if ((lane & (kDupMask | 24)) == 0) sMw[warp * 8 + my_head] = mx;
     }
+  };
+  if constexpr (BATCH == 1) {
+  for (int r = 0; r < nblk; ++r) {
+    const int j = j0 + r;
+    const int nvalid = rows_of(j);
+
+    // ---- scores of block j (kept in registers) and per-warp head maxima
+    // (double-buffered by block parity: a fast warp may write block j+1's
+    // while a slow one still reads block j's)
+    float sc[kDecBc / 16];
+    score_block(r, sc, sM + (r & 1) * 32);
     if (__syncthreads_or(!ok)) { ok = false; break; }
     if (tid == 0 && r + kDecNK < nblk) issue_k(r + kDecNK);
     if constexpr (PAGED) {
@@ -523,6 +531,96 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<G>())
       ok = pv(kept_done);
       ++kept_done;
     }
+  }
+  } else {
+    // Batched decisions (contiguous cache): blocks r and r+1 are scored
+    // before either is decided, and each is judged against
+    //   Mb = max(running max over earlier blocks, maxima of both blocks);
+    // kept blocks use Mb as the reference of P (m_ref, which acc and l
+    // follow; it can move past m_run's old value through a skipped block).
+    static_assert(BATCH == 2 && !PAGED, "batched decisions: pairs, contiguous");
+    float m_ref[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) m_ref[g] = -INFINITY;
+    for (int r = 0; r < nblk; r += 2) {
+      const bool two = r + 1 < nblk;
+      float sc0[kDecBc / 16], sc1[kDecBc / 16];
+      // pair maxima double-buffered by pair parity
+      float* sMp = sM + ((r >> 1) & 1) * 64;
+      score_block(r, sc0, sMp);
+      if (two) score_block(r + 1, sc1, sMp + 32);
+      if (__syncthreads_or(!ok)) { ok = false; break; }
+      if (tid == 0) {
+        if (r + 2 < nblk) issue_k(r + 2);
+        if (r + 3 < nblk) issue_k(r + 3);
+      }
+      float mt0[G], mt1[G], Mb[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        mt0[g] = fmaxf(fmaxf(sMp[g], sMp[8 + g]), fmaxf(sMp[16 + g], sMp[24 + g]));
+        mt1[g] = two ? fmaxf(fmaxf(sMp[32 + g], sMp[40 + g]),
+                             fmaxf(sMp[48 + g], sMp[56 + g]))
+                     : -INFINITY;
+        Mb[g] = fmaxf(m_run[g], fmaxf(mt0[g], mt1[g]));
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (u == 1 && !two) break;
+        const int j = j0 + r + u;
+        const int nvalid = rows_of(j);
+        bool skip = ln_lambda > -INFINITY;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          if (!((u ? mt1[g] : mt0[g]) - Mb[g] < ln_lambda)) skip = false;
+        if (tid == 0) {
+          ++n_vis;
+          if (skip) ++n_skp;
+          if (a.mask) a.mask[(size_t)bh * a.nk + j] = skip ? 2 : 1;
+        }
+        if (!skip && !a.stats_only) {
+          const int slot = kept_issued % kDecNV;
+          if (tid == 0) {
+            sNV[slot] = nvalid;
+            copy_block(sV + slot * kDecBlockBytes, vbase, j, &vfull[slot]);
+          }
+          float mb_mine = 0.f, al_mine = 1.f;
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float al = (m_ref[g] == -INFINITY)
+                                 ? 0.f
+                                 : ex2_approx((m_ref[g] - Mb[g]) * kLog2e);
+            if (tid == 0) sA[slot * 8 + g] = al;
+            if (g == my_head) {
+              mb_mine = Mb[g];
+              al_mine = al;
+            }
+            m_ref[g] = Mb[g];
+          }
+          if (writer) {
+            float* ps = sP + slot * kDecBc * G;
+            float psum = 0.f;
+#pragma unroll
+            for (int i = 0; i < kDecBc / 16; ++i) {
+              const float pv_ =
+                  ex2_approx(((u ? sc1[i] : sc0[i]) - mb_mine) * kLog2e);
+              ps[(ks + 16 * i) * G + my_head] = pv_;
+              psum += pv_;
+            }
+            l_part = al_mine * l_part + psum;
+          }
+          ++kept_issued;
+          // the next kept block's V slot is the one kept block n-1 used
+          while (ok && kept_issued - kept_done > kDecLag) {
+            ok = pv(kept_done);
+            ++kept_done;
+          }
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) m_run[g] = Mb[g];
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) m_run[g] = m_ref[g];  // reference of l, acc
   }
   if constexpr (PAGED) {
     // no ring copy may still be landing when the CTA leaves

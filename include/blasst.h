@@ -189,6 +189,31 @@ blasst_status_t blasst_decode_window(const void *q, const void *k_cache,
                                      void *stream);
 
 /*
+ * blasst_decode_batched -- blasst_decode with the batched decision rule
+ * (Hindi summary, section 2 "kernel optimisation": the Q.K products of
+ * several blocks are formed before their V loads are decided, which keeps
+ * the conditional V loads from stalling the pipeline).  With batch = 2 each
+ * split's blocks are taken in pairs (j, j+1), both scored before either is
+ * decided, and each is skipped iff for every head g of the tile
+ *     m~_g(block) - max(m_g before the pair, m~_g(j), m~_g(j+1)) < ln lambda
+ * where m_g is the max over all earlier blocks of the split.  The block
+ * holding the pair's max is always kept; the rule skips every block the
+ * sequential rule (blasst_decode) skips and possibly more, and each skipped
+ * weight stays below lambda times the split's final max.
+ *
+ *  batch   1 (= blasst_decode) or 2 (else BLASST_ERR_UNSUPPORTED_SHAPE)
+ *  other arguments, layouts, ownership and errors as blasst_decode.
+ */
+blasst_status_t blasst_decode_batched(const void *q, const void *k_cache,
+                                      const void *v_cache, void *o, float *lse,
+                                      int B, int Hq, int Hkv, int Lkv, int d,
+                                      float scale, float ln_lambda, int Bc,
+                                      int num_splits, int batch,
+                                      void *workspace, size_t workspace_bytes,
+                                      const blasst_skip_stats_t *skip_stats,
+                                      void *stream);
+
+/*
  * blasst_decode_noalloc -- blasst_decode for callers that may not allocate
  * device memory at call time and have no workspace to pass: for example an
  * inference-engine plugin whose enqueue step must not allocate, or a
