@@ -48,12 +48,12 @@ DEC = dict(B=32, Hq=32, Hkv=8, Lkv=32768, d=128, Bc=64, target=0.70,
 # DRAM traffic of the dominant decode kernel per launch, relative to the
 # algorithmic bytes of that launch, from one ncu capture of a smaller case
 # (profiles/decode_split_kernel_B8_Lkv32k.md: dram__bytes_read.sum +
-# dram__bytes_write.sum = 955.6 MB for 957.8 MB of algorithmic bytes).  The
+# dram__bytes_write.sum = 956.4 MB for 957.8 MB of algorithmic bytes).  The
 # kernel reads K once and V only for kept blocks, so traffic grows with the
 # algorithmic bytes; the ratio is applied to the benchmarked launch.  It holds
 # only for the kernel source it was measured on (sha256 prefix below).
 DECODE_TRAFFIC = dict(source="dynamic_block_sparse_fa_b200/csrc/decode.cuh",
-                      sha256_16="e61d605edef51723", ratio=955.6 / 957.8)
+                      sha256_16="899b6e40fc275750", ratio=956.4 / 957.8)
 PRE = dict(B=1, Hq=32, Hkv=8, L=32768, d=128, Br=128, Bc=128, window=4096)
 
 
