@@ -149,20 +149,42 @@ def prefill(q, k, v, scale, causal, ln_lambda, Br, Bc, units=None,
                 units=ua, threads=threads)
 
 
-def decode(q, k, v, scale, ln_lambda, Bc, num_splits, n_threads=0, window=0):
+def _tile_heads(Hq, Hkv, tile_heads, *pools):
+    """Decode tiles of ``tile_heads`` query heads.  The tile of the method is
+    the group of query heads that share a KV head (their rows are voted on
+    together); with ``tile_heads`` < G = Hq/Hkv the group is cut into G /
+    tile_heads consecutive tiles, which is the same as giving each tile its
+    own copy of the KV head.  Returns the number of (virtual) KV heads and
+    the pools with each KV head repeated G / tile_heads times (axis 1)."""
+    G = Hq // Hkv
+    T = G if tile_heads is None else int(tile_heads)
+    if T < 1 or G % T != 0:
+        raise ValueError("tile_heads must divide Hq / Hkv")
+    r = G // T
+    if r == 1:
+        return Hkv, pools
+    return Hkv * r, tuple(np.ascontiguousarray(np.repeat(x, r, axis=1))
+                          for x in pools)
+
+
+def decode(q, k, v, scale, ln_lambda, Bc, num_splits, n_threads=0, window=0,
+           tile_heads=None):
     """BLASST decode forward with split-KV and log-sum-exp merge.
 
     ``window`` > 0: the token sees only the last ``window`` keys (sliding
-    window); the splits divide the blocks holding them.
+    window); the splits divide the blocks holding them.  ``tile_heads``:
+    query heads per decode tile (default: all Hq/Hkv heads of a KV head).
 
     q [B,Hq,d], k/v [B,Hkv,Lkv,d] bf16.  Returns ``o`` [B,Hq,d], ``lse``
     [B,Hq], ``o_part`` [B,Hq,S,d], ``lse_part`` [B,Hq,S], ``mask``
-    [B,Hkv,nk], ``margin`` [B,Hkv,nk], ``visited``, ``skipped``.
+    [B,Hkv',nk], ``margin`` [B,Hkv',nk] (Hkv' = Hq / tile_heads), ``visited``,
+    ``skipped``.
     """
     lib = _load()
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     B, Hq, d = qb.shape
-    _, Hkv, Lkv, _ = kb.shape
+    Hkv, (kb, vb) = _tile_heads(Hq, kb.shape[1], tile_heads, kb, vb)
+    Lkv = kb.shape[2]
     nk = -(-Lkv // Bc)
     S = int(num_splits)
     o = np.zeros((B, Hq, d), np.float64)
@@ -187,7 +209,7 @@ def decode(q, k, v, scale, ln_lambda, Bc, num_splits, n_threads=0, window=0):
 
 
 def decode_batched(q, k, v, scale, ln_lambda, Bc, num_splits, batch,
-                   n_threads=0):
+                   n_threads=0, tile_heads=None):
     """Decode with the batched decision rule: blocks of each split are judged
     in batches of ``batch`` against the max over all earlier blocks and the
     whole batch.  ``batch`` = 1 is :func:`decode`.  Same outputs as
@@ -195,7 +217,8 @@ def decode_batched(q, k, v, scale, ln_lambda, Bc, num_splits, batch,
     lib = _load()
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     B, Hq, d = qb.shape
-    _, Hkv, Lkv, _ = kb.shape
+    Hkv, (kb, vb) = _tile_heads(Hq, kb.shape[1], tile_heads, kb, vb)
+    Lkv = kb.shape[2]
     nk = -(-Lkv // Bc)
     S = int(num_splits)
     o = np.zeros((B, Hq, d), np.float64)
@@ -227,7 +250,7 @@ def _i32(x):
 
 def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale, ln_lambda,
                  num_splits, Bc=64, per_length=False, nk_max=None,
-                 page_stride=None, n_threads=0):
+                 page_stride=None, n_threads=0, tile_heads=None):
     """Paged, variable-length decode: gather, then the decode above.
 
     q [B,Hq,d] bf16.  k_pages / v_pages: either [num_pages,Hkv,page_size,d]
@@ -235,19 +258,26 @@ def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale, ln_lambda,
     (then pass ``(pool, num_pages, Hkv, page_size, d)`` tuples).
     block_table [B,max_pages] int32, seq_lens [B] int32.  ``per_length``:
     ln_lambda is ln a and sequence b uses min(0, ln a - ln L_b).
-    Returns the keys of ``decode`` with mask/margin [B,Hkv,nk_max].
+    Returns the keys of ``decode`` with mask/margin [B,Hkv',nk_max]
+    (``tile_heads`` as in :func:`decode`; 4-D pools only when it is set).
     """
     lib = _load()
     qb = _bits(q)
     B, Hq, d = qb.shape
     if isinstance(k_pages, tuple):
         kp, num_pages, Hkv, ps, d2 = k_pages
+        if tile_heads is not None and tile_heads != Hq // Hkv:
+            raise ValueError("tile_heads needs [num_pages,Hkv,page,d] pools")
         vp = v_pages[0]
         kb, vb = _bits(kp).reshape(-1), _bits(vp).reshape(-1)
         stride = int(page_stride)
     else:
         kb, vb = _bits(k_pages), _bits(v_pages)
-        num_pages, Hkv, ps, d2 = kb.shape
+        if (page_stride is not None and tile_heads is not None
+                and tile_heads != Hq // kb.shape[1]):
+            raise ValueError("tile_heads with a padded page stride")
+        Hkv, (kb, vb) = _tile_heads(Hq, kb.shape[1], tile_heads, kb, vb)
+        num_pages, _, ps, d2 = kb.shape
         stride = Hkv * ps * d2 if page_stride is None else int(page_stride)
     assert d2 == d
     bt = _i32(block_table)
