@@ -161,6 +161,12 @@ size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits) {
 }  // extern "C"
 
 namespace {
+// Query heads per KV head the decode kernel takes: 1, 2, 4 or 8 heads form
+// one tile; a larger power of two is cut into tiles of 8 heads.
+bool decode_group_ok(int G) {
+  return G >= 1 && G <= 256 && (G & (G - 1)) == 0;
+}
+
 // Split kernel, then (unless statistics only) the merge, launched as a
 // programmatic dependent of the split kernel so its launch overlaps the
 // split kernel's tail (it waits on griddepcontrol).
@@ -299,10 +305,11 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
     return BLASST_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !valid_ln_lambda(ln_lambda))
     return BLASST_ERR_INVALID_ARG;
-  const int G = Hq / Hkv;
-  if (d != blasst::kDecD || Bc != blasst::kDecBc ||
-      !(G == 1 || G == 2 || G == 4 || G == 8))
+  int G = Hq / Hkv;
+  if (d != blasst::kDecD || Bc != blasst::kDecBc || !decode_group_ok(G))
     return BLASST_ERR_UNSUPPORTED_SHAPE;
+  const int kv_div = G > 8 ? G / 8 : 1;  // tiles of 8 heads above 8
+  G /= kv_div;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
       (o && !aligned16(o)))
     return BLASST_ERR_MISALIGNED;
@@ -313,7 +320,7 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
                     ? blasst_decode_splits(B, Hkv, Lkv - jlo * Bc, Bc)
                     : num_splits;
   if (S < 1 || S > nk - jlo) return BLASST_ERR_INVALID_ARG;
-  const long long grid = (long long)B * Hkv * S;
+  const long long grid = (long long)B * Hkv * kv_div * S;
   if (grid > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED_SHAPE;
   const bool stats_only = (o == nullptr);
   float* o_part = nullptr;
@@ -331,7 +338,8 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
   a.lse_part = lse_part;
   a.counters = skip_stats ? skip_stats->counters : nullptr;
   a.mask = skip_stats ? skip_stats->mask : nullptr;
-  a.Hkv = Hkv;
+  a.Hkv = Hkv * kv_div;
+  a.kv_div = kv_div;
   a.Lkv = Lkv;
   a.nk = nk;
   a.S = S;
@@ -377,9 +385,11 @@ blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
   if (log2_page < 0) return BLASST_ERR_UNSUPPORTED_SHAPE;
   if ((long long)max_seq_len > (long long)max_pages * page_size)
     return BLASST_ERR_INVALID_ARG;
-  const int G = Hq / Hkv;
-  if (d != blasst::kDecD || !(G == 1 || G == 2 || G == 4 || G == 8))
+  int G = Hq / Hkv;
+  if (d != blasst::kDecD || !decode_group_ok(G))
     return BLASST_ERR_UNSUPPORTED_SHAPE;
+  const int kv_div = G > 8 ? G / 8 : 1;  // tiles of 8 heads above 8
+  G /= kv_div;
   if (page_stride < (long long)Hkv * page_size * d || page_stride % 8 != 0)
     return BLASST_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) ||
@@ -390,7 +400,7 @@ blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
   const int S = num_splits == 0 ? blasst_decode_splits(B, Hkv, max_seq_len, Bc)
                                 : num_splits;
   if (S < 1 || S > nk) return BLASST_ERR_INVALID_ARG;
-  const long long grid = (long long)B * Hkv * S;
+  const long long grid = (long long)B * Hkv * kv_div * S;
   if (grid > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED_SHAPE;
   const bool stats_only = (o == nullptr);
   float* o_part = nullptr;
@@ -408,7 +418,8 @@ blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
   a.lse_part = lse_part;
   a.counters = skip_stats ? skip_stats->counters : nullptr;
   a.mask = skip_stats ? skip_stats->mask : nullptr;
-  a.Hkv = Hkv;
+  a.Hkv = Hkv * kv_div;
+  a.kv_div = kv_div;
   a.Lkv = max_seq_len;
   a.nk = nk;
   a.S = S;

@@ -51,6 +51,10 @@ struct DecodeArgs {
   // sliding window: the token sees only the last `window` keys (0 = all);
   // the splits divide the blocks that hold them
   int window;
+  // decode tiles per KV head of the cache (>= 1): with G query heads per KV
+  // head above the tile's rows, the heads are cut into kv_div tiles of G /
+  // kv_div heads; Hkv then counts tiles (cache heads * kv_div)
+  int kv_div;
 };
 
 constexpr int kDecD = 128;       // head dimension
@@ -152,10 +156,11 @@ __global__ void __launch_bounds__(kDecThreads, BATCH == 1
   const int warp = tid >> 5;
 
   const int s = blockIdx.x % a.S;
-  const int bh = blockIdx.x / a.S;  // b * Hkv + hkv
+  const int bh = blockIdx.x / a.S;  // b * Hkv + hkv (tiles)
   const int Hq = a.Hkv * G;
   const int b = bh / a.Hkv;
   const int hkv = bh - b * a.Hkv;
+  const int hkv_c = hkv / a.kv_div;  // the cache head of this tile
   int Lb = a.Lkv;  // keys of this sequence
   float ln_lambda = a.ln_lambda;
   if constexpr (PAGED) {
@@ -190,7 +195,7 @@ __global__ void __launch_bounds__(kDecThreads, BATCH == 1
   // tok, in page id
   auto src_off = [&](int id, int tok) -> long long {
     return (long long)id * a.page_stride +
-           ((long long)hkv << (a.log2_page + 7)) +
+           ((long long)hkv_c << (a.log2_page + 7)) +
            (long long)(tok & ((1 << a.log2_page) - 1)) * kDecD;
   };
   if constexpr (PAGED) {
@@ -244,8 +249,8 @@ __global__ void __launch_bounds__(kDecThreads, BATCH == 1
     kbase = a.k;
     vbase = a.v;
   } else {
-    kbase = a.k + (size_t)bh * a.Lkv * kDecD;
-    vbase = a.v + (size_t)bh * a.Lkv * kDecD;
+    kbase = a.k + (size_t)(bh / a.kv_div) * a.Lkv * kDecD;  // (b, hkv_c)
+    vbase = a.v + (size_t)(bh / a.kv_div) * a.Lkv * kDecD;
   }
   const uint64_t pol = policy_evict_first();
 

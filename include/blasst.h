@@ -69,8 +69,10 @@ typedef enum {
  *  mask      optional device uint8 buffer (NULL = not written) receiving one
  *            decision per (tile, block): 0 not visited, 1 kept, 2 skipped.
  *            Prefill layout [B, Hq, ceil(Lq/Br), ceil(Lkv/Bc)];
- *            decode layout  [B, Hkv, ceil(Lkv/Bc)] (a block belongs to
- *            exactly one split).  Entries of pairs that are not visited are
+ *            decode layout  [B, Hkv * T, ceil(Lkv/Bc)] with T decode tiles
+ *            per KV head (1 when Hq/Hkv <= 8, else Hq/Hkv/8; a block
+ *            belongs to exactly one split).  The caller allocates the whole
+ *            layout: the library cannot check a device buffer's size.  Entries of pairs that are not visited are
  *            written as 0 by prefill only for tiles it runs; callers that
  *            need them zeroed clear the buffer first.
  * A NULL blasst_skip_stats_t* disables both.
@@ -137,7 +139,10 @@ blasst_status_t blasst_prefill_window(const void *q, const void *k,
  * KV cache, split-KV with a log-sum-exp merge.
  *
  * The G = Hq/Hkv query heads sharing a KV head form the rows of one tile, so
- * every K and V byte read serves all G heads.  The Lkv keys are cut into
+ * every K and V byte read serves all G heads.  A tile has at most 8 rows:
+ * for G = 16, 32, ... (MQA with many heads) the heads of a KV head are cut
+ * into G/8 consecutive tiles of 8 heads, each with its own skip decisions,
+ * which read the same KV head (through L2 when they run together).  The Lkv keys are cut into
  * nk = ceil(Lkv/Bc) blocks and the blocks into num_splits contiguous splits
  * (split s covers blocks [floor(s*nk/S), floor((s+1)*nk/S))).  Each split
  * runs the blockwise forward independently (its running max starts at
@@ -147,7 +152,7 @@ blasst_status_t blasst_prefill_window(const void *q, const void *k,
  *  o           device bf16 [B,Hq,d], or NULL for a statistics-only pass
  *              (K is read and scored, V is never read)
  *  lse         device float32 [B,Hq] or NULL
- *  d           128;  Hq/Hkv in {1, 2, 4, 8};  Bc = 64
+ *  d           128;  Hq/Hkv a power of two up to 256;  Bc = 64
  *  num_splits  >= 1, or 0 for the automatic choice blasst_decode_splits()
  *  workspace   device buffer of at least blasst_decode_workspace_size()
  *              bytes (16-byte aligned) holding the per-split partials;
@@ -284,12 +289,12 @@ blasst_status_t blasst_decode_noalloc(const void *q, const void *k_cache,
  *                  (finite or -INFINITY), and sequence b uses
  *                  ln lambda_b = min(0, ln a - ln L_b), L_b its own length
  *                  (gist.science summary, section 2 "Calibracao Automatica")
- *  d = 128, Hq/Hkv in {1, 2, 4, 8}
+ *  d = 128, Hq/Hkv a power of two up to 256 (tiles as blasst_decode)
  *  num_splits      >= 1 (at most ceil(max_seq_len / 64)), or 0 = automatic
  *  workspace       as blasst_decode: blasst_decode_workspace_size(B, Hq, d,
  *                  resolved num_splits) bytes
  *  skip_stats      as blasst_decode; the mask layout is
- *                  [B, Hkv, ceil(max_seq_len / 64)] and blocks past a
+ *                  [B, Hkv * T, ceil(max_seq_len / 64)] and blocks past a
  *                  sequence's end are not written
  * The block table and the lengths live on the device, so they are checked
  * there: before any copy of a split is issued, its kernel checks its
