@@ -335,3 +335,6 @@ def lambda_fit(lambdas, lengths):
     """Least-squares fit of lambda = a / L in log space: a = exp(mean ln(lambda*L))."""
     vals = [math.log(lam * L) for lam, L in zip(lambdas, lengths)]
     return math.exp(sum(vals) / len(vals))
+
+
+from .backward import prefill_backward, restricted_forward  # noqa: E402,F401
