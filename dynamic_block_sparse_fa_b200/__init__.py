@@ -11,6 +11,8 @@ from .blasst import (BlasstError, Stats, blasst_calibrate,
                      blasst_decode_splits, blasst_decode_window,
                      blasst_decode_workspace_size,
                      blasst_fit_a, blasst_last_error, blasst_prefill,
+                     blasst_prefill_backward,
+                     blasst_prefill_backward_workspace_size,
                      blasst_prefill_window,
                      blasst_selftest_wait_timeout, blasst_skip_stats_reset,
                      blasst_strerror, blasst_version)
@@ -21,7 +23,8 @@ __all__ = ["BlasstError", "Stats", "blasst_calibrate",
            "blasst_decode_paged",
            "blasst_decode_splits", "blasst_decode_window",
            "blasst_decode_workspace_size", "blasst_fit_a", "blasst_last_error",
-           "blasst_prefill", "blasst_prefill_window",
+           "blasst_prefill", "blasst_prefill_backward",
+           "blasst_prefill_backward_workspace_size", "blasst_prefill_window",
            "blasst_selftest_wait_timeout",
            "blasst_skip_stats_reset", "blasst_strerror",
            "blasst_version"]

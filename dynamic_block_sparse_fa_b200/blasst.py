@@ -98,6 +98,12 @@ _lib.blasst_decode_noalloc.restype = _i
 _lib.blasst_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                        _i, _f, _f, _i, _i,
                                        ctypes.POINTER(SkipStats), _vp]
+_lib.blasst_prefill_backward.restype = _i
+_lib.blasst_prefill_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                         _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                         _i, _f, _i, _i, _i, _vp, _sz, _vp]
+_lib.blasst_prefill_backward_workspace_size.restype = _sz
+_lib.blasst_prefill_backward_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.blasst_decode_workspace_size.restype = _sz
 _lib.blasst_decode_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.blasst_decode_splits.restype = _i
@@ -240,6 +246,37 @@ def blasst_prefill(q, k, v, *, scale=None, causal=True, ln_lambda=-math.inf,
 def blasst_prefill_window(q, k, v, *, window, **kw):
     """blasst_prefill with a causal sliding window of ``window`` keys."""
     return blasst_prefill(q, k, v, window=window, **kw)
+
+
+def blasst_prefill_backward_workspace_size(B, Hq, Lq, d=128) -> int:
+    return int(_lib.blasst_prefill_backward_workspace_size(B, Hq, Lq, d))
+
+
+def blasst_prefill_backward(q, k, v, o, lse, dout, *, mask=None, scale=None,
+                            causal=True, Br=128, Bc=128, dq=None, dk=None,
+                            dv=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of a blasst_prefill forward with its decisions
+    held fixed.  q [B,Hq,Lq,d], k/v [B,Hkv,Lkv,d], o/dout [B,Hq,Lq,d] bf16,
+    lse [B,Hq,Lq] f32 (the forward's), mask: the forward's decision bytes
+    (Stats.mask) or None for the dense backward."""
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = blasst_prefill_backward_workspace_size(B, Hq, Lq, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8,
+                                device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _lib.blasst_prefill_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(mask),
+        _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, Lq, Lkv, d, float(scale),
+        int(bool(causal)), Br, Bc, _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "blasst_prefill_backward")
+    return dq, dk, dv
 
 
 def blasst_decode_window(q, k, v, *, window, **kw):

@@ -1,0 +1,494 @@
+// backward.cuh -- backward of the BLASST prefill forward on sm_100a, with the
+// forward's skip decisions held fixed (128x128 tiles, d = 128).
+//
+// Fine-tuning with BLASST active ("BLASST: Dynamic BLocked Attention
+// Sparsity via Softmax Thresholding", gist.science summary, section 2,
+// "Treinamento Consciente de Esparsidade"; Hindi summary, algorithm design)
+// differentiates the forward as it ran.  With its decisions fixed that
+// forward is softmax attention restricted, per query tile, to its kept
+// blocks, so only the kept (tile, block) pairs enter the backward:
+//   D_r = dO_r . O_r;  P = exp(scale q k^T - lse);  dV += P^T dO;
+//   dP = dO V^T;  dS = P o (dP - D);  dK += scale dS^T Q;  dQ += scale dS K
+// A pair the forward skipped (or did not visit) does no MMA and loads
+// nothing.
+//
+// Three kernels:
+//   bwd_prep_kernel     D per query row (from O and dO), zeroes the f32 dQ
+//                       accumulator
+//   bwd_dkdv_kernel     one CTA per (sequence, KV head, key block j): K_j and
+//                       V_j stay in shared memory while the kept query tiles
+//                       of the G query heads stream through; dK_j, dV_j
+//                       accumulate in tensor memory, each pair's dQ tile is
+//                       added to the f32 accumulator with vector reductions
+//   bwd_dq_kernel       dQ = bf16(scale * accumulator)
+// bwd_dkdv_kernel: warp 0 TMA producer (Q_i, dO_i ring of 2), warp 1 MMA
+// issuer (one lane), warps 2..5 one thread per tensor-memory lane.  Per kept
+// pair the MMAs are
+//   S^T  = K_j Q_i^T      (SS, K-major A and B)        -> TMEM [0, 128)
+//   dP^T = V_j dO_i^T     (SS)                         -> TMEM [128, 256)
+//   (threads: P^T, dS^T as bf16 into TMEM [0, 64), [128, 192) and dS^T into
+//    shared memory)
+//   dV  += P^T dO_i       (TS, A = P^T from TMEM, B = dO_i MN-major) -> [256, 384)
+//   dK  += dS^T Q_i       (TS, B = Q_i MN-major)       -> [384, 512)
+//   dQ_i = dS K_j         (SS, A = dS MN-major from shared memory,
+//                          B = K_j MN-major)           -> [0, 128)
+// Tensor memory is the whole 512 columns, so one CTA per SM; the steps of a
+// pair run one after the other (the producer prefetches the next pair).
+#pragma once
+
+#include "prefill.cuh"
+
+namespace blasst {
+
+struct BwdParams {
+  CUtensorMap tq, tk, tv, tdo;
+  const __nv_bfloat16* o;     // [B, Hq, Lq, D]
+  const __nv_bfloat16* dout;  // [B, Hq, Lq, D]
+  const float* lse;           // [B, Hq, Lq] natural log
+  const unsigned char* mask;  // [B, Hq, nq, nk]; 1 = kept (null: all kept)
+  float* dq_acc;              // [B, Hq, Lq, D]
+  float* delta;               // [B, Hq, Lq]
+  __nv_bfloat16* dq;          // [B, Hq, Lq, D]
+  __nv_bfloat16* dk;          // [B, Hkv, Lkv, D]
+  __nv_bfloat16* dv;          // [B, Hkv, Lkv, D]
+  int B, Hq, Hkv, Lq, Lkv, nq, nk, G, causal;
+  float scale;
+};
+
+constexpr int kBwdD = 128;
+constexpr int kBwdThreads = 192;
+
+struct BwdCfg {
+  static constexpr int TILE = 128 * kBwdD * 2;  // 32 KB, two 64-column boxes
+  static constexpr int BOX = 128 * 128;         // bytes of one box
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;     // [2]
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;  // [2]
+  static constexpr int OFF_DS = OFF_DO + 2 * TILE;  // dS^T [keys][queries]
+  static constexpr int OFF_LSE = OFF_DS + TILE;     // f32 [128] lse * log2 e
+  static constexpr int OFF_DEL = OFF_LSE + 512;     // f32 [128] D
+  static constexpr int OFF_BAR = OFF_DEL + 512;
+  static constexpr int B_KV = 0;
+  static constexpr int B_QF = 1;   // [2]
+  static constexpr int B_QE = 3;   // [2]
+  static constexpr int B_SP = 5;   // S^T and dP^T in TMEM
+  static constexpr int B_PDS = 6;  // P^T, dS^T written (one arrival per warp)
+  static constexpr int B_DQF = 7;  // dQ tile in TMEM
+  static constexpr int B_DQR = 8;  // dQ tile read out (one arrival per warp)
+  static constexpr int NBAR = 9;
+  static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_TMEM + 8;
+  static constexpr int SMEM_ALLOC = SMEM + 1024;
+  static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
+};
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c,
+                                           float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p),
+               "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// D_r = sum_e dO_re O_re (f32), and the row's dQ accumulator set to zero.
+// One warp per query row, 4 elements per lane.
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
+  const long long rows = (long long)p.B * p.Hq * p.Lq;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint2 a = reinterpret_cast<const uint2*>(p.o + row * kBwdD)[lane];
+  const uint2 g = reinterpret_cast<const uint2*>(p.dout + row * kBwdD)[lane];
+  float s = bf16lo(a.x) * bf16lo(g.x) + bf16hi(a.x) * bf16hi(g.x) +
+            bf16lo(a.y) * bf16lo(g.y) + bf16hi(a.y) * bf16hi(g.y);
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+  if (lane == 0) p.delta[row] = s;
+  reinterpret_cast<float4*>(p.dq_acc + row * kBwdD)[lane] =
+      make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// dQ = bf16(scale * accumulator), 8 elements per thread.
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p) {
+  const long long n8 = (long long)p.B * p.Hq * p.Lq * (kBwdD / 8);
+  const long long i = (long long)blockIdx.x * 256 + threadIdx.x;
+  if (i >= n8) return;
+  const float4 x = reinterpret_cast<const float4*>(p.dq_acc)[2 * i];
+  const float4 y = reinterpret_cast<const float4*>(p.dq_acc)[2 * i + 1];
+  const float sc = p.scale;
+  uint4 w;
+  w.x = pack_bf16x2(x.x * sc, x.y * sc);
+  w.y = pack_bf16x2(x.z * sc, x.w * sc);
+  w.z = pack_bf16x2(y.x * sc, y.y * sc);
+  w.w = pack_bf16x2(y.z * sc, y.w * sc);
+  reinterpret_cast<uint4*>(p.dq)[i] = w;
+}
+
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
+  using C = BwdCfg;
+  constexpr unsigned FULL = 0xffffffffu;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int jb = blockIdx.x % p.nk;  // key block
+  const int bk = blockIdx.x / p.nk;  // b * Hkv + hkv
+  const int b = bk / p.Hkv;
+  const int hkv = bk - b * p.Hkv;
+  const int off = p.Lkv - p.Lq;      // bottom-right causal alignment
+  // Pair (g, i) of query head hkv*G + g and query tile i enters the
+  // backward iff the forward kept it (and, causal, it is visible at all).
+  auto kept = [&](int g, int i) -> bool {
+    if (p.causal && min((i + 1) * 128, p.Lq) - 1 + off < jb * 128) return false;
+    if (!p.mask) return true;
+    const int hq = hkv * p.G + g;
+    return __ldg(p.mask + ((size_t)(b * p.Hq + hq) * p.nq + i) * p.nk + jb) == 1;
+  };
+
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[C::B_KV], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[C::B_QF + s], 1);
+      mbar_init(&bar[C::B_QE + s], 1);
+    }
+    mbar_init(&bar[C::B_SP], 1);
+    mbar_init(&bar[C::B_PDS], 4);
+    mbar_init(&bar[C::B_DQF], 1);
+    mbar_init(&bar[C::B_DQR], 4);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      const uint64_t pol_kv = policy_evict_first();
+      const uint64_t pol_q = policy_evict_last();
+      prefetch_tmap(&p.tq);
+      prefetch_tmap(&p.tk);
+      prefetch_tmap(&p.tv);
+      prefetch_tmap(&p.tdo);
+      mbar_arrive_expect_tx(&bar[C::B_KV], 2 * C::TILE);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        tma_load_3d(smem + C::OFF_K + c * C::BOX, &p.tk, &bar[C::B_KV], c * 64,
+                    jb * 128, bk, pol_kv);
+        tma_load_3d(smem + C::OFF_V + c * C::BOX, &p.tv, &bar[C::B_KV], c * 64,
+                    jb * 128, bk, pol_kv);
+      }
+      int n = 0;
+      bool ok = true;
+      for (int g = 0; g < p.G && ok; ++g) {
+        const int zq = b * p.Hq + hkv * p.G + g;
+        for (int i = 0; i < p.nq; ++i) {
+          if (!kept(g, i)) continue;
+          const int s = n & 1;
+          if (n >= 2 &&
+              !mbar_wait(&bar[C::B_QE + s], ((n >> 1) - 1) & 1, kWaitBackward,
+                         n, s)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar[C::B_QF + s], 2 * C::TILE);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            tma_load_3d(smem + C::OFF_Q + s * C::TILE + c * C::BOX, &p.tq,
+                        &bar[C::B_QF + s], c * 64, i * 128, zq, pol_q);
+            tma_load_3d(smem + C::OFF_DO + s * C::TILE + c * C::BOX, &p.tdo,
+                        &bar[C::B_QF + s], c * 64, i * 128, zq, pol_q);
+          }
+          ++n;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t id_kk = idesc_bf16(128, 128, 0, 0);  // K-major A, B
+      constexpr uint32_t id_km = idesc_bf16(128, 128, 0, 1);  // B MN-major
+      constexpr uint32_t id_mm = idesc_bf16(128, 128, 1, 1);  // A, B MN-major
+      const uint32_t aK = smem_u32(smem + C::OFF_K);
+      const uint32_t aV = smem_u32(smem + C::OFF_V);
+      const uint32_t aQ = smem_u32(smem + C::OFF_Q);
+      const uint32_t aDO = smem_u32(smem + C::OFF_DO);
+      const uint32_t aDS = smem_u32(smem + C::OFF_DS);
+      // K-major operand (128 rows x 128 elements, two 64-column boxes):
+      // the 16-element step k is box k/4, 32 bytes k%4 into the row.
+      auto kmaj = [&](uint32_t base, int k) {
+        return smem_desc(base + (k >> 2) * C::BOX + (k & 3) * 32, 16, 1024, 2);
+      };
+      // MN-major operand (K runs down the rows): step k is rows 16k..16k+15,
+      // the two 64-column boxes are C::BOX apart.
+      auto mnmaj = [&](uint32_t base, int k) {
+        return smem_desc(base + k * 2048, C::BOX, 1024, 2);
+      };
+      bool ok = mbar_wait(&bar[C::B_KV], 0, kWaitBackward, 0, 20);
+      int n = 0;
+      for (int g = 0; g < p.G && ok; ++g) {
+        for (int i = 0; i < p.nq && ok; ++i) {
+          if (!kept(g, i)) continue;
+          const int s = n & 1;
+          ok = mbar_wait(&bar[C::B_QF + s], (n >> 1) & 1, kWaitBackward, n,
+                         21 + s);
+          if (ok && n > 0)  // the previous dQ tile has left TMEM [0, 128)
+            ok = mbar_wait(&bar[C::B_DQR], (n - 1) & 1, kWaitBackward, n, 23);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t q_s = aQ + s * C::TILE, do_s = aDO + s * C::TILE;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mma_ss(tmem + 0, kmaj(aK, k), kmaj(q_s, k), id_kk, k > 0 ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mma_ss(tmem + 128, kmaj(aV, k), kmaj(do_s, k), id_kk,
+                   k > 0 ? 1u : 0u);
+          mma_commit(&bar[C::B_SP]);
+          ok = mbar_wait(&bar[C::B_PDS], n & 1, kWaitBackward, n, 24);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mma_ts(tmem + 256, tmem + 0 + k * 8, mnmaj(do_s, k), id_km,
+                   (n > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mma_ts(tmem + 384, tmem + 128 + k * 8, mnmaj(q_s, k), id_km,
+                   (n > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mma_ss(tmem + 0, mnmaj(aDS, k), mnmaj(aK, k), id_mm,
+                   k > 0 ? 1u : 0u);
+          mma_commit(&bar[C::B_DQF]);
+          mma_commit(&bar[C::B_QE + s]);
+          ++n;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ----------------------------------------------------------- threads
+    const int quad = warp & 3;
+    const int rr = quad * 32 + lane;  // TMEM lane of this thread
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
+    float* del_s = reinterpret_cast<float*>(smem + C::OFF_DEL);
+    uint8_t* sDS = smem + C::OFF_DS;
+    const int key = jb * 128 + rr;
+    const bool key_ok = key < p.Lkv;
+    const float sl2 = p.scale * kPrefLog2e;
+    int n = 0;
+    bool ok = true, stop = false;
+    for (int g = 0; g < p.G && !stop; ++g) {
+      const int hq = hkv * p.G + g;
+      const size_t rowbase = (size_t)(b * p.Hq + hq) * p.Lq;
+      for (int i = 0; i < p.nq; ++i) {
+        if (!kept(g, i)) continue;
+        // All four warps leave together: a wait that gave up in any of them
+        // ends the loop for all at this barrier (never between barriers).
+        if (!named_sync_and(1, 128, ok)) { ok = false; stop = true; break; }
+        // this pair's lse (log2 units) and D per query column
+        {
+          const int qr = i * 128 + rr;
+          lse_s[rr] = qr < p.Lq ? __ldg(p.lse + rowbase + qr) * kPrefLog2e
+                                : INFINITY;
+          del_s[rr] = qr < p.Lq ? p.delta[rowbase + qr] : 0.f;
+        }
+        named_sync(1, 128);
+        const bool w1 = mbar_wait(&bar[C::B_SP], n & 1, kWaitBackward, n, 30);
+        ok = __all_sync(FULL, w1);
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < 4 && ok; ++cc) {
+          uint32_t s[32], dp[32];
+          tmem_ld32(lane_base + 0 + cc * 32, s);
+          tmem_ld32(lane_base + 128 + cc * 32, dp);
+          tc_wait_ld();
+          uint32_t pk[16], dk16[16];
+#pragma unroll
+          for (int x = 0; x < 32; x += 2) {
+            float pv[2], dv2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = cc * 32 + x + e;  // query column in the tile
+              const int qr = i * 128 + c;
+              const bool valid = key_ok && qr < p.Lq &&
+                                 (!p.causal || key <= qr + off);
+              const float pr = valid ? ex2_approx(fmaf(__uint_as_float(s[x + e]),
+                                                       sl2, -lse_s[c]))
+                                     : 0.f;
+              pv[e] = pr;
+              dv2[e] = pr * (__uint_as_float(dp[x + e]) - del_s[c]);
+            }
+            pk[x >> 1] = pack_bf16x2(pv[0], pv[1]);
+            dk16[x >> 1] = pack_bf16x2(dv2[0], dv2[1]);
+          }
+          tmem_st16(lane_base + 0 + cc * 16, pk);
+          tmem_st16(lane_base + 128 + cc * 16, dk16);
+          // dS^T row rr, query columns 32cc..32cc+31: box cc/2, 16-byte
+          // chunks (cc%2)*4 .. +3 of the 128-byte row, 128-byte swizzle
+          uint8_t* row = sDS + (cc >> 1) * C::BOX + rr * 128;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int ch = ((cc & 1) * 4 + u) ^ (rr & 7);
+            *reinterpret_cast<uint4*>(row + ch * 16) =
+                make_uint4(dk16[4 * u], dk16[4 * u + 1], dk16[4 * u + 2],
+                           dk16[4 * u + 3]);
+          }
+        }
+        tc_wait_st();
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(&bar[C::B_PDS]);
+        // dQ tile: TMEM lane = query row
+        const bool w2 =
+            ok && mbar_wait(&bar[C::B_DQF], n & 1, kWaitBackward, n, 31);
+        ok = __all_sync(FULL, w2);
+        tc_fence_after();
+        const int qr = i * 128 + rr;
+        float* dst = p.dq_acc + (rowbase + qr) * kBwdD;
+#pragma unroll 1
+        for (int cc = 0; cc < 4 && ok; ++cc) {
+          uint32_t a[32];
+          tmem_ld32(lane_base + 0 + cc * 32, a);
+          tc_wait_ld();
+          if (qr < p.Lq) {
+#pragma unroll
+            for (int x = 0; x < 32; x += 4)
+              red_add_v4(dst + cc * 32 + x, __uint_as_float(a[x]),
+                         __uint_as_float(a[x + 1]), __uint_as_float(a[x + 2]),
+                         __uint_as_float(a[x + 3]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(&bar[C::B_DQR]);
+        ++n;
+      }
+    }
+    // dK_j, dV_j (TMEM lane = key row); zero when no pair was kept.  The
+    // tensor-memory loads are warp-collective, so every lane takes part and
+    // only the stores depend on the row (a warp can straddle the cache end).
+    if (ok) {
+      __nv_bfloat16* dvr = p.dv + ((size_t)bk * p.Lkv + key) * kBwdD;
+      __nv_bfloat16* dkr = p.dk + ((size_t)bk * p.Lkv + key) * kBwdD;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        const uint32_t col = half == 0 ? 256u : 384u;
+        const float f = half == 0 ? 1.f : p.scale;
+        __nv_bfloat16* out = half == 0 ? dvr : dkr;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t a[32];
+          if (n > 0) {
+            tmem_ld32(lane_base + col + cc * 32, a);
+            tc_wait_ld();
+          } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) a[x] = 0u;
+          }
+          if (key_ok) {
+#pragma unroll
+            for (int x = 0; x < 32; x += 8) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(a[x]) * f, __uint_as_float(a[x + 1]) * f);
+              w.y = pack_bf16x2(__uint_as_float(a[x + 2]) * f, __uint_as_float(a[x + 3]) * f);
+              w.z = pack_bf16x2(__uint_as_float(a[x + 4]) * f, __uint_as_float(a[x + 5]) * f);
+              w.w = pack_bf16x2(__uint_as_float(a[x + 6]) * f, __uint_as_float(a[x + 7]) * f);
+              *reinterpret_cast<uint4*>(out + cc * 32 + x) = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+struct BwdProblem {
+  const void *q, *k, *v, *o, *dout;
+  const float* lse;
+  const unsigned char* mask;
+  void *dq, *dk, *dv;
+  float* workspace;  // dQ accumulator [B*Hq*Lq*D] then D [B*Hq*Lq]
+  int B, Hq, Hkv, Lq, Lkv, causal;
+  float scale;
+};
+
+inline size_t bwd_workspace_bytes(int B, int Hq, int Lq) {
+  const size_t rows = (size_t)B * Hq * Lq;
+  return rows * kBwdD * 4 + ((rows * 4 + 255) & ~(size_t)255);
+}
+
+inline cudaError_t launch_backward(const BwdProblem& pr, cudaStream_t st) {
+  BwdParams p;
+  memset(&p, 0, sizeof p);
+  if (!encode_map(&p.tq, pr.q, kBwdD, pr.Lq, (long long)pr.B * pr.Hq, 128) ||
+      !encode_map(&p.tdo, pr.dout, kBwdD, pr.Lq, (long long)pr.B * pr.Hq, 128) ||
+      !encode_map(&p.tk, pr.k, kBwdD, pr.Lkv, (long long)pr.B * pr.Hkv, 128) ||
+      !encode_map(&p.tv, pr.v, kBwdD, pr.Lkv, (long long)pr.B * pr.Hkv, 128))
+    return cudaErrorInvalidValue;
+  p.o = static_cast<const __nv_bfloat16*>(pr.o);
+  p.dout = static_cast<const __nv_bfloat16*>(pr.dout);
+  p.lse = pr.lse;
+  p.mask = pr.mask;
+  const size_t rows = (size_t)pr.B * pr.Hq * pr.Lq;
+  p.dq_acc = pr.workspace;
+  p.delta = pr.workspace + rows * kBwdD;
+  p.dq = static_cast<__nv_bfloat16*>(pr.dq);
+  p.dk = static_cast<__nv_bfloat16*>(pr.dk);
+  p.dv = static_cast<__nv_bfloat16*>(pr.dv);
+  p.B = pr.B;
+  p.Hq = pr.Hq;
+  p.Hkv = pr.Hkv;
+  p.Lq = pr.Lq;
+  p.Lkv = pr.Lkv;
+  p.nq = (pr.Lq + 127) / 128;
+  p.nk = (pr.Lkv + 127) / 128;
+  p.G = pr.Hq / pr.Hkv;
+  p.causal = pr.causal;
+  p.scale = pr.scale;
+  const long long prep_blocks = (long long)((rows + 7) / 8);
+  const long long grid = (long long)pr.B * pr.Hkv * p.nk;
+  const long long conv_blocks = (long long)((rows * (kBwdD / 8) + 255) / 256);
+  if (prep_blocks > 0x7fffffffLL || grid > 0x7fffffffLL ||
+      conv_blocks > 0x7fffffffLL)
+    return cudaErrorInvalidConfiguration;
+  bwd_prep_kernel<<<(unsigned)prep_blocks, 256, 0, st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_dkdv_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           BwdCfg::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  bwd_dkdv_kernel<<<(unsigned)grid, kBwdThreads, BwdCfg::SMEM_ALLOC, st>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_dq_kernel<<<(unsigned)conv_blocks, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace blasst

@@ -11,6 +11,7 @@
 #include "decode.cuh"
 #include "prefill.cuh"
 #include "prefill2.cuh"
+#include "backward.cuh"
 
 namespace {
 
@@ -563,6 +564,56 @@ blasst_status_t blasst_prefill_window(const void* q, const void* k,
   p.window = window;
   cudaError_t e = blasst::launch_prefill(p, static_cast<cudaStream_t>(stream));
   return cuda_status(e, "prefill launch");
+}
+
+size_t blasst_prefill_backward_workspace_size(int B, int Hq, int Lq, int d) {
+  if (B < 1 || Hq < 1 || Lq < 1 || d != blasst::kBwdD) return 0;
+  return blasst::bwd_workspace_bytes(B, Hq, Lq);
+}
+
+blasst_status_t blasst_prefill_backward(
+    const void* q, const void* k, const void* v, const void* o,
+    const void* dout, const float* lse, const unsigned char* mask, void* dq,
+    void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lkv, int d,
+    float scale, int causal, int Br, int Bc, void* workspace,
+    size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv)
+    return BLASST_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lkv < 1 || Hq % Hkv != 0)
+    return BLASST_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return BLASST_ERR_INVALID_ARG;
+  if (causal && Lq > Lkv) return BLASST_ERR_INVALID_ARG;
+  if (d != blasst::kBwdD || Br != 128 || Bc != 128)
+    return BLASST_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return BLASST_ERR_MISALIGNED;
+  if (!workspace ||
+      workspace_bytes < blasst::bwd_workspace_bytes(B, Hq, Lq))
+    return BLASST_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return BLASST_ERR_MISALIGNED;
+  blasst::BwdProblem p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.dout = dout;
+  p.lse = lse;
+  p.mask = mask;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.workspace = static_cast<float*>(workspace);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Lq = Lq;
+  p.Lkv = Lkv;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  cudaError_t e = blasst::launch_backward(p, static_cast<cudaStream_t>(stream));
+  return cuda_status(e, "backward launch");
 }
 
 // ---------------------------------------------------------------------------

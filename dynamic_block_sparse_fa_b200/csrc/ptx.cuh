@@ -26,6 +26,7 @@ enum : unsigned int {
   kWaitPrefillMma = 11,
   kWaitPrefillSoftmax = 12,
   kWaitPrefillEpilogue = 13,
+  kWaitBackward = 14,
   kWaitSelfTest = 99,
   // Device-resident arguments found out of range (paged decode); these are
   // reported as invalid arguments, not as waits that gave up.

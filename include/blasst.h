@@ -135,6 +135,45 @@ blasst_status_t blasst_prefill_window(const void *q, const void *k,
                                       void *stream);
 
 /*
+ * blasst_prefill_backward -- gradients of a blasst_prefill forward with the
+ * decisions that forward took held fixed (sparsity-aware fine-tuning with
+ * the method active: gist.science summary, section 2, "Treinamento
+ * Consciente de Esparsidade"; Hindi summary, algorithm design).  With its
+ * decisions fixed the forward is softmax attention restricted, per query
+ * tile, to its kept blocks; a decision is a step function, so its gradient
+ * is that of the restricted attention:
+ *     D_r = dO_r . O_r,  P = exp(scale q k^T - lse) on kept pairs (else 0),
+ *     dV = P^T dO,  dS = P o (dO V^T - D),  dQ = scale dS K,
+ *     dK = scale dS^T Q  (dK, dV summed over the G heads of a KV head).
+ * Pairs the forward skipped or did not visit issue no load and no MMA.
+ *
+ *  q, k, v     the forward's inputs (device bf16, layouts as blasst_prefill)
+ *  o, lse      the forward's outputs: o bf16 [B,Hq,Lq,d], lse float32
+ *              [B,Hq,Lq] (required)
+ *  dout        device bf16 [B,Hq,Lq,d], the gradient of o
+ *  mask        the forward's decision bytes (skip_stats.mask layout
+ *              [B,Hq,ceil(Lq/128),ceil(Lkv/128)], 1 = kept), or NULL for
+ *              the dense backward (every visible pair kept)
+ *  dq          device bf16 [B,Hq,Lq,d] (written)
+ *  dk, dv      device bf16 [B,Hkv,Lkv,d] (written)
+ *  d = 128, Br = Bc = 128 (else BLASST_ERR_UNSUPPORTED_SHAPE); causal with
+ *              Lq > Lkv is rejected
+ *  workspace   device buffer of blasst_prefill_backward_workspace_size()
+ *              bytes, 256-byte aligned, caller-owned (f32 dQ accumulator and
+ *              the per-row D); contents need not be initialised
+ * Asynchronous on `stream`; three kernel launches; allocates nothing.
+ * Errors as blasst_prefill (BLASST_ERR_WORKSPACE for a missing or small
+ * workspace).
+ */
+size_t blasst_prefill_backward_workspace_size(int B, int Hq, int Lq, int d);
+blasst_status_t blasst_prefill_backward(
+    const void *q, const void *k, const void *v, const void *o,
+    const void *dout, const float *lse, const unsigned char *mask, void *dq,
+    void *dk, void *dv, int B, int Hq, int Hkv, int Lq, int Lkv, int d,
+    float scale, int causal, int Br, int Bc, void *workspace,
+    size_t workspace_bytes, void *stream);
+
+/*
  * blasst_decode -- one query token per sequence against a contiguous bf16
  * KV cache, split-KV with a log-sum-exp merge.
  *

@@ -183,3 +183,10 @@ def planted_gap_kv_inplace(k, v, q, *, block=64, gap=8.0, heavy_frac=0.03,
 
 def config_seed(index: int, extra: int = 0) -> int:
     return CONFIG_SEED_BASE + index + extra
+
+
+def output_gradient(shape, seed, device="cpu") -> torch.Tensor:
+    """A seeded standard-normal bf16 tensor: the loss gradient dO fed to the
+    backward (drawn on the CPU so that every device gets the same values)."""
+    g = _gen("cpu", seed)
+    return torch.randn(*shape, generator=g).to(torch.bfloat16).to(device)
