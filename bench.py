@@ -569,12 +569,56 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
         out["window"] = run_prefill_window(args, bl, q, k, v, o, lse,
                                            out["s70"]["ln_lambda"], stream,
                                            tf_peak)
+    if not args.no_backward:
+        out["backward"] = run_prefill_backward(args, bl, q, k, v,
+                                               out["s70"]["ln_lambda"], stream,
+                                               tf_peak)
     best = out["s70"]
     roof = {"bound": "tensor", "kernel": "prefill2_kernel<128> at 70%",
             "achieved": best["executed_tflops"], "peak": tf_peak,
             "peak_kind": peak_kind + " bf16 burst", "unit": "TFLOP/s",
             "frac": best["tensor_frac"], "traffic": None}
     return out, roof
+
+
+def run_prefill_backward(args, bl, q, k, v, lnl, stream, tf_peak):
+    """blasst_prefill_backward on the prefill workload: the dense backward
+    (every visible pair) and the backward of the forward at the ln lambda
+    calibrated for 70% (its decision bytes as the mask).  Executed FLOPs
+    = 5 GEMMs of 128 x 128 x d per kept pair (S^T, dP^T, dV, dK, dQ)."""
+    from synth import config_seed, output_gradient
+    B, Hq, Lq, d = q.shape
+    Br = 128
+    nq, nk = -(-Lq // Br), -(-k.shape[2] // Br)
+    dout = output_gradient((B, Hq, Lq, d), config_seed(2, 1), device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(bl.blasst_prefill_backward_workspace_size(B, Hq, Lq, d),
+                     dtype=torch.uint8, device=q.device)
+    K, W = max(3, args.prefill_steps // 2), args.warmup
+    res = {"what": "dQ, dK, dV of the forward with its decisions fixed; "
+                   "f32 dQ accumulated with vector reductions"}
+    dense_ms = None
+    for key, l in (("dense", -math.inf), ("s70", lnl)):
+        st = bl.Stats(device=q.device, mask_numel=B * Hq * nq * nk)
+        o, lse = bl.blasst_prefill(q, k, v, ln_lambda=l, stats=st)
+        torch.cuda.synchronize()
+        vis, skp = st.read()
+        mask = None if key == "dense" else st.mask
+
+        def fn():
+            bl.blasst_prefill_backward(q, k, v, o, lse, dout, mask=mask, dq=dq,
+                                       dk=dk, dv=dv, workspace=ws)
+        ms = time_calls(fn, K, W, stream) / K
+        ex = 10.0 * Br * Br * d * (vis - skp)
+        r = {"us": round(ms * 1e3, 1), "sparsity": skp / vis,
+             "executed_tflops": round(ex / (ms / 1e3) / 1e12, 1),
+             "tensor_frac": round(ex / (ms / 1e3) / 1e12 / tf_peak, 4)}
+        if key == "dense":
+            dense_ms = ms
+        else:
+            r["speedup_vs_dense"] = round(dense_ms / ms, 4)
+        res[key] = r
+    return res
 
 
 def run_prefill_window(args, bl, q, k, v, o, lse, lnl, stream, tf_peak):
@@ -763,6 +807,8 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-window", action="store_true",
                     help="skip the sliding-window measurements")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the prefill backward measurements")
     ap.add_argument("--no-paged", action="store_true",
                     help="skip the paged-cache decode measurements")
     ap.add_argument("--decode-batch", type=int, default=DEC["B"],

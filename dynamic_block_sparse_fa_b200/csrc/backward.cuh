@@ -19,21 +19,24 @@
 //                       V_j stay in shared memory while the kept query tiles
 //                       of the G query heads stream through; dK_j, dV_j
 //                       accumulate in tensor memory, each pair's dQ tile is
-//                       added to the f32 accumulator with vector reductions
+//                       staged in shared memory and added to the f32
+//                       accumulator by TMA bulk reductions
 //   bwd_dq_kernel       dQ = bf16(scale * accumulator)
 // bwd_dkdv_kernel: warp 0 TMA producer (Q_i, dO_i ring of 2), warp 1 MMA
 // issuer (one lane), warps 2..5 one thread per tensor-memory lane.  Per kept
 // pair the MMAs are
 //   S^T  = K_j Q_i^T      (SS, K-major A and B)        -> TMEM [0, 128)
 //   dP^T = V_j dO_i^T     (SS)                         -> TMEM [128, 256)
-//   (threads: P^T, dS^T as bf16 into TMEM [0, 64), [128, 192) and dS^T into
-//    shared memory)
-//   dV  += P^T dO_i       (TS, A = P^T from TMEM, B = dO_i MN-major) -> [256, 384)
-//   dK  += dS^T Q_i       (TS, B = Q_i MN-major)       -> [384, 512)
+//   dV  += P^T dO_i       (TS, A = P^T (bf16) from TMEM [0, 64),
+//                          B = dO_i MN-major)          -> [256, 384)
+//   dK  += dS^T Q_i       (TS, A = dS^T from TMEM [128, 192),
+//                          B = Q_i MN-major)           -> [384, 512)
 //   dQ_i = dS K_j         (SS, A = dS MN-major from shared memory,
-//                          B = K_j MN-major)           -> [0, 128)
-// Tensor memory is the whole 512 columns, so one CTA per SM; the steps of a
-// pair run one after the other (the producer prefetches the next pair).
+//                          B = K_j MN-major)           -> [128, 256)
+// and the threads signal P^T and dS^T separately, so the dV product runs
+// while dS is computed, and the next pair's S^T product runs while the dQ
+// tile is read out (it lands in the dP^T columns, which the next dP^T waits
+// for).  Tensor memory is the whole 512 columns: one CTA per SM.
 #pragma once
 
 #include "prefill.cuh"
@@ -42,6 +45,7 @@ namespace blasst {
 
 struct BwdParams {
   CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tdq;  // f32 dQ accumulator [B*Hq][Lq][D], box 32 x 128
   const __nv_bfloat16* o;     // [B, Hq, Lq, D]
   const __nv_bfloat16* dout;  // [B, Hq, Lq, D]
   const float* lse;           // [B, Hq, Lq] natural log
@@ -70,28 +74,44 @@ struct BwdCfg {
   static constexpr int OFF_DEL = OFF_LSE + 512;     // f32 [128] D
   static constexpr int OFF_BAR = OFF_DEL + 512;
   static constexpr int B_KV = 0;
-  static constexpr int B_QF = 1;   // [2]
-  static constexpr int B_QE = 3;   // [2]
-  static constexpr int B_SP = 5;   // S^T and dP^T in TMEM
-  static constexpr int B_PDS = 6;  // P^T, dS^T written (one arrival per warp)
-  static constexpr int B_DQF = 7;  // dQ tile in TMEM
-  static constexpr int B_DQR = 8;  // dQ tile read out (one arrival per warp)
-  static constexpr int NBAR = 9;
+  static constexpr int B_QF = 1;    // [2]
+  static constexpr int B_QE = 3;    // [2]
+  static constexpr int B_SF = 5;    // S^T in TMEM
+  static constexpr int B_DPF = 6;   // dP^T in TMEM
+  static constexpr int B_PR = 7;    // P^T written (one arrival per warp)
+  static constexpr int B_DSR = 8;   // dS^T written (one arrival per warp)
+  static constexpr int B_DQF = 9;   // dQ tile in TMEM
+  static constexpr int B_DQR = 10;  // dQ tile read out (one arrival per warp)
+  static constexpr int NBAR = 11;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_TMEM + 8;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
   static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
 };
 
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c,
-                                           float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p),
-               "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// global[box at (c0, c1, c2)] += shared box (f32 add), as a bulk group.
+__device__ __forceinline__ void tma_reduce_add_3d(const void* tmap,
+                                                  const void* src, int c0,
+                                                  int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group "
+      "[%0, {%2, %3, %4}], [%1];" ::"l"(tmap),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the shared-memory sources of every committed bulk group have been read
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // D_r = sum_e dO_re O_re (f32), and the row's dQ accumulator set to zero.
@@ -138,8 +158,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int jb = blockIdx.x % p.nk;  // key block
-  const int bk = blockIdx.x / p.nk;  // b * Hkv + hkv
+  // Causal key block j has the most query tiles for j = 0: CTAs go out in
+  // ascending j over all (sequence, KV head), longest first.
+  const int nbk = p.B * p.Hkv;
+  const int jb = blockIdx.x / nbk;   // key block
+  const int bk = blockIdx.x - jb * nbk;  // b * Hkv + hkv
   const int b = bk / p.Hkv;
   const int hkv = bk - b * p.Hkv;
   const int off = p.Lkv - p.Lq;      // bottom-right causal alignment
@@ -160,8 +183,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bar[C::B_QF + s], 1);
       mbar_init(&bar[C::B_QE + s], 1);
     }
-    mbar_init(&bar[C::B_SP], 1);
-    mbar_init(&bar[C::B_PDS], 4);
+    mbar_init(&bar[C::B_SF], 1);
+    mbar_init(&bar[C::B_DPF], 1);
+    mbar_init(&bar[C::B_PR], 4);
+    mbar_init(&bar[C::B_DSR], 4);
     mbar_init(&bar[C::B_DQF], 1);
     mbar_init(&bar[C::B_DQR], 4);
     fence_mbar_init();
@@ -184,6 +209,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       prefetch_tmap(&p.tk);
       prefetch_tmap(&p.tv);
       prefetch_tmap(&p.tdo);
+      prefetch_tmap(&p.tdq);
       mbar_arrive_expect_tx(&bar[C::B_KV], 2 * C::TILE);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -240,44 +266,70 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         return smem_desc(base + k * 2048, C::BOX, 1024, 2);
       };
       bool ok = mbar_wait(&bar[C::B_KV], 0, kWaitBackward, 0, 20);
+      // S^T of pair n is issued at the end of pair n-1's step (or here).
+      auto issue_s = [&](int n) {
+        const int s = n & 1;
+        ok = ok && mbar_wait(&bar[C::B_QF + s], (n >> 1) & 1, kWaitBackward,
+                             n, 21 + s);
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t q_s = aQ + s * C::TILE;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ss(tmem + 0, kmaj(aK, k), kmaj(q_s, k), id_kk, k > 0 ? 1u : 0u);
+        mma_commit(&bar[C::B_SF]);
+      };
       int n = 0;
+      bool pending = false;  // S^T of pair n issued
       for (int g = 0; g < p.G && ok; ++g) {
         for (int i = 0; i < p.nq && ok; ++i) {
           if (!kept(g, i)) continue;
           const int s = n & 1;
-          ok = mbar_wait(&bar[C::B_QF + s], (n >> 1) & 1, kWaitBackward, n,
-                         21 + s);
-          if (ok && n > 0)  // the previous dQ tile has left TMEM [0, 128)
+          if (!pending) issue_s(n);
+          pending = false;
+          // dP^T overwrites the columns the previous dQ tile was read from
+          if (ok && n > 0)
             ok = mbar_wait(&bar[C::B_DQR], (n - 1) & 1, kWaitBackward, n, 23);
           if (!ok) break;
           tc_fence_after();
           const uint32_t q_s = aQ + s * C::TILE, do_s = aDO + s * C::TILE;
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            mma_ss(tmem + 0, kmaj(aK, k), kmaj(q_s, k), id_kk, k > 0 ? 1u : 0u);
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
             mma_ss(tmem + 128, kmaj(aV, k), kmaj(do_s, k), id_kk,
                    k > 0 ? 1u : 0u);
-          mma_commit(&bar[C::B_SP]);
-          ok = mbar_wait(&bar[C::B_PDS], n & 1, kWaitBackward, n, 24);
+          mma_commit(&bar[C::B_DPF]);
+          ok = mbar_wait(&bar[C::B_PR], n & 1, kWaitBackward, n, 24);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             mma_ts(tmem + 256, tmem + 0 + k * 8, mnmaj(do_s, k), id_km,
                    (n > 0 || k > 0) ? 1u : 0u);
+          ok = mbar_wait(&bar[C::B_DSR], n & 1, kWaitBackward, n, 25);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             mma_ts(tmem + 384, tmem + 128 + k * 8, mnmaj(q_s, k), id_km,
                    (n > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            mma_ss(tmem + 0, mnmaj(aDS, k), mnmaj(aK, k), id_mm,
+            mma_ss(tmem + 128, mnmaj(aDS, k), mnmaj(aK, k), id_mm,
                    k > 0 ? 1u : 0u);
           mma_commit(&bar[C::B_DQF]);
           mma_commit(&bar[C::B_QE + s]);
           ++n;
+          // the next kept pair's S^T now, behind this pair's dQ product
+          int g2 = g, i2 = i + 1;
+          while (g2 < p.G) {
+            if (i2 >= p.nq) { ++g2; i2 = 0; continue; }
+            if (kept(g2, i2)) break;
+            ++i2;
+          }
+          if (g2 < p.G) {
+            issue_s(n);
+            pending = ok;
+          }
         }
       }
     }
@@ -311,35 +363,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           del_s[rr] = qr < p.Lq ? p.delta[rowbase + qr] : 0.f;
         }
         named_sync(1, 128);
-        const bool w1 = mbar_wait(&bar[C::B_SP], n & 1, kWaitBackward, n, 30);
+        // P^T (thread = key row, 128 query columns) into TMEM [0, 64) as
+        // bf16; the packed values stay in registers for dS.
+        uint32_t pk[64];
+        const bool w1 = mbar_wait(&bar[C::B_SF], n & 1, kWaitBackward, n, 30);
         ok = __all_sync(FULL, w1);
         tc_fence_after();
-#pragma unroll 1
-        for (int cc = 0; cc < 4 && ok; ++cc) {
-          uint32_t s[32], dp[32];
-          tmem_ld32(lane_base + 0 + cc * 32, s);
-          tmem_ld32(lane_base + 128 + cc * 32, dp);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          if (!ok) break;
+          uint32_t sv[32];
+          tmem_ld32(lane_base + 0 + cc * 32, sv);
           tc_wait_ld();
-          uint32_t pk[16], dk16[16];
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
-            float pv[2], dv2[2];
+            float pv[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int c = cc * 32 + x + e;  // query column in the tile
               const int qr = i * 128 + c;
               const bool valid = key_ok && qr < p.Lq &&
                                  (!p.causal || key <= qr + off);
-              const float pr = valid ? ex2_approx(fmaf(__uint_as_float(s[x + e]),
-                                                       sl2, -lse_s[c]))
-                                     : 0.f;
-              pv[e] = pr;
-              dv2[e] = pr * (__uint_as_float(dp[x + e]) - del_s[c]);
+              pv[e] = valid ? ex2_approx(fmaf(__uint_as_float(sv[x + e]), sl2,
+                                              -lse_s[c]))
+                            : 0.f;
             }
-            pk[x >> 1] = pack_bf16x2(pv[0], pv[1]);
-            dk16[x >> 1] = pack_bf16x2(dv2[0], dv2[1]);
+            pk[cc * 16 + (x >> 1)] = pack_bf16x2(pv[0], pv[1]);
           }
-          tmem_st16(lane_base + 0 + cc * 16, pk);
+          uint32_t st16[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) st16[u] = pk[cc * 16 + u];
+          tmem_st16(lane_base + 0 + cc * 16, st16);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(&bar[C::B_PR]);
+        // dS^T = P^T o (dP^T - D) into TMEM [128, 192) and shared memory
+        const bool w2 =
+            ok && mbar_wait(&bar[C::B_DPF], n & 1, kWaitBackward, n, 31);
+        ok = __all_sync(FULL, w2);
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          if (!ok) break;
+          uint32_t dp[32];
+          tmem_ld32(lane_base + 128 + cc * 32, dp);
+          tc_wait_ld();
+          uint32_t dk16[16];
+#pragma unroll
+          for (int x = 0; x < 32; x += 2) {
+            const uint32_t pw = pk[cc * 16 + (x >> 1)];
+            const int c = cc * 32 + x;
+            dk16[x >> 1] = pack_bf16x2(
+                bf16lo(pw) * (__uint_as_float(dp[x]) - del_s[c]),
+                bf16hi(pw) * (__uint_as_float(dp[x + 1]) - del_s[c + 1]));
+          }
           tmem_st16(lane_base + 128 + cc * 16, dk16);
           // dS^T row rr, query columns 32cc..32cc+31: box cc/2, 16-byte
           // chunks (cc%2)*4 .. +3 of the 128-byte row, 128-byte swizzle
@@ -356,30 +435,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (ok && lane == 0) mbar_arrive(&bar[C::B_PDS]);
-        // dQ tile: TMEM lane = query row
-        const bool w2 =
-            ok && mbar_wait(&bar[C::B_DQF], n & 1, kWaitBackward, n, 31);
-        ok = __all_sync(FULL, w2);
-        tc_fence_after();
-        const int qr = i * 128 + rr;
-        float* dst = p.dq_acc + (rowbase + qr) * kBwdD;
+        if (ok && lane == 0) mbar_arrive(&bar[C::B_DSR]);
+        // dQ tile (TMEM lane = query row) from [128, 256): staged in the dS
+        // buffer (free once the dQ product is done) as two rounds of two
+        // 32-column boxes (128-byte swizzle), each added to the f32
+        // accumulator by TMA reductions issued by one thread.
+        const bool w3 =
+            ok && mbar_wait(&bar[C::B_DQF], n & 1, kWaitBackward, n, 32);
+        ok = named_sync_and(1, 128, __all_sync(FULL, w3));
+        if (ok) {
+          tc_fence_after();
 #pragma unroll 1
-        for (int cc = 0; cc < 4 && ok; ++cc) {
-          uint32_t a[32];
-          tmem_ld32(lane_base + 0 + cc * 32, a);
-          tc_wait_ld();
-          if (qr < p.Lq) {
+          for (int h = 0; h < 2; ++h) {
 #pragma unroll
-            for (int x = 0; x < 32; x += 4)
-              red_add_v4(dst + cc * 32 + x, __uint_as_float(a[x]),
-                         __uint_as_float(a[x + 1]), __uint_as_float(a[x + 2]),
-                         __uint_as_float(a[x + 3]));
+            for (int u = 0; u < 2; ++u) {
+              uint32_t a[32];
+              tmem_ld32(lane_base + 128 + h * 64 + u * 32, a);
+              tc_wait_ld();
+              uint8_t* row = sDS + u * (C::TILE / 2) + rr * 128;
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(row + ((c ^ (rr & 7)) * 16)) =
+                    make_uint4(a[4 * c], a[4 * c + 1], a[4 * c + 2],
+                               a[4 * c + 3]);
+            }
+            if (h == 1) {  // TMEM [128, 256) is free for the next dP^T
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bar[C::B_DQR]);
+            }
+            fence_async_smem();
+            named_sync(1, 128);
+            if (warp == 2 && lane == 0) {
+#pragma unroll
+              for (int u = 0; u < 2; ++u)
+                tma_reduce_add_3d(&p.tdq, sDS + u * (C::TILE / 2),
+                                  h * 64 + u * 32, i * 128, b * p.Hq + hq);
+              bulk_commit_group();
+              bulk_wait_read_all();
+            }
+            named_sync(1, 128);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (ok && lane == 0) mbar_arrive(&bar[C::B_DQR]);
         ++n;
       }
     }
@@ -420,12 +517,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   }
 
+  if (warp == 2 && lane == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// 3-D map over the f32 dQ accumulator [planes, rows, 128], box 32 columns
+// (128 bytes) x 128 rows, 128-byte swizzle; rows past the end are clipped.
+inline bool encode_map_f32(CUtensorMap* m, void* base, int rows,
+                           long long planes) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kBwdD, (cuuint64_t)rows,
+                        (cuuint64_t)planes};
+  cuuint64_t strides[2] = {(cuuint64_t)kBwdD * 4,
+                           (cuuint64_t)rows * kBwdD * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 struct BwdProblem {
@@ -458,6 +575,8 @@ inline cudaError_t launch_backward(const BwdProblem& pr, cudaStream_t st) {
   const size_t rows = (size_t)pr.B * pr.Hq * pr.Lq;
   p.dq_acc = pr.workspace;
   p.delta = pr.workspace + rows * kBwdD;
+  if (!encode_map_f32(&p.tdq, p.dq_acc, pr.Lq, (long long)pr.B * pr.Hq))
+    return cudaErrorInvalidValue;
   p.dq = static_cast<__nv_bfloat16*>(pr.dq);
   p.dk = static_cast<__nv_bfloat16*>(pr.dk);
   p.dv = static_cast<__nv_bfloat16*>(pr.dv);
