@@ -48,12 +48,12 @@ DEC = dict(B=32, Hq=32, Hkv=8, Lkv=32768, d=128, Bc=64, target=0.70,
 # DRAM traffic of the dominant decode kernel per launch, relative to the
 # algorithmic bytes of that launch, from one ncu capture of a smaller case
 # (profiles/decode_split_kernel_B8_Lkv32k.md: dram__bytes_read.sum +
-# dram__bytes_write.sum = 956.4 MB for 957.8 MB of algorithmic bytes).  The
+# dram__bytes_write.sum = 955.2 MB for 957.8 MB of algorithmic bytes).  The
 # kernel reads K once and V only for kept blocks, so traffic grows with the
 # algorithmic bytes; the ratio is applied to the benchmarked launch.  It holds
 # only for the kernel source it was measured on (sha256 prefix below).
 DECODE_TRAFFIC = dict(source="dynamic_block_sparse_fa_b200/csrc/decode.cuh",
-                      sha256_16="899b6e40fc275750", ratio=956.4 / 957.8)
+                      sha256_16="436b7fe2e10bdb6c", ratio=955.2 / 957.8)
 PRE = dict(B=1, Hq=32, Hkv=8, L=32768, d=128, Br=128, Bc=128, window=4096)
 
 
@@ -596,7 +596,7 @@ def run_prefill_backward(args, bl, q, k, v, lnl, stream, tf_peak):
                      dtype=torch.uint8, device=q.device)
     K, W = max(3, args.prefill_steps // 2), args.warmup
     res = {"what": "dQ, dK, dV of the forward with its decisions fixed; "
-                   "f32 dQ accumulated with vector reductions"}
+                   "f32 dQ accumulated by TMA bulk reductions"}
     dense_ms = None
     for key, l in (("dense", -math.inf), ("s70", lnl)):
         st = bl.Stats(device=q.device, mask_numel=B * Hq * nq * nk)
