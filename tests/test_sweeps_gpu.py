@@ -13,8 +13,8 @@ Prefill sparsity / calibration sweep: B 1, Hq 32 / Hkv 8, d 128, causal,
 the deviation |s(a/L) - target| is reported; the 4K case is compared with
 the oracle in full.
 
-Each test appends a JSON record of what it measured to
-gpurun_out/sweeps.jsonl when that directory exists.
+Each test appends a JSON record of what it measured to the file named by
+the BLASST_SWEEP_RECORD environment variable, when it is set.
 """
 import json
 import math
@@ -30,13 +30,10 @@ from tests import _parity as P
 
 pytestmark = pytest.mark.gpu
 
-ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-
-
 def _record(obj):
-    out = os.path.join(ROOT, "gpurun_out")
-    if os.path.isdir(out):
-        with open(os.path.join(out, "sweeps.jsonl"), "a") as f:
+    path = os.environ.get("BLASST_SWEEP_RECORD")
+    if path:
+        with open(path, "a") as f:
             f.write(json.dumps(obj) + "\n")
 
 
