@@ -139,7 +139,9 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sV = smem + C::OFF_V;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  volatile int* dec_flag = reinterpret_cast<volatile int*>(smem + C::OFF_DEC);
+  // Decision words [2][R]: ((jt + 1) << 1) | skip for block jt of a tile,
+  // published with a release store right after the vote.
+  uint32_t* dec_word = reinterpret_cast<uint32_t*>(smem + C::OFF_DEC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
 
   if (threadIdx.x == 0) {
@@ -154,10 +156,11 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar[C::B_SF + t], 1);
-      mbar_init(&bar[C::B_PF + t], C::WPT);  // one arrival per softmax warp
+      mbar_init(&bar[C::B_PF + t], C::WPT);  // P written: one arrival per softmax warp, kept blocks only
       mbar_init(&bar[C::B_OD + t], 1);
       for (int i = 0; i < C::R; ++i) mbar_init(&bar[C::B_DEC + t * C::R + i], 1);
     }
+    for (int i = 0; i < 2 * C::R; ++i) dec_word[i] = 0u;
     reinterpret_cast<volatile int*>(smem + C::OFF_ABORT)[0] = 0;
     reinterpret_cast<volatile int*>(smem + C::OFF_ABORT)[1] = 0;
     fence_mbar_init();
@@ -218,7 +221,7 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
                                    (jt / C::R) & 1, kWaitPrefillLoad, j,
                                    100 + t * C::R + jt % C::R);
           if (!__all_sync(FULL, w)) { ok = false; break; }
-          need = dec_flag[t * C::R + jt % C::R] != 0;
+          need = (ld_acquire_shared(&dec_word[t * C::R + jt % C::R]) & 1u) == 0;
         }
         if (!ok) break;
         if (need) {
@@ -283,7 +286,7 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
         mma_commit(&bar[C::B_KE]);
       }
       int vcount = 0;
-      int npv[2] = {0, 0};
+      int npv[2] = {0, 0};  // kept blocks of each tile so far
       for (int j = jlo; j < nblk && ok; ++j) {
         int vslot = -1;
 #pragma unroll
@@ -294,10 +297,29 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
           const int jt = j - jlo_t[t];
           bool kept = false;
           if (cur) {
-            ok = mbar_wait(&bar[C::B_PF + t], jt & 1, kWaitPrefillMma, j,
-                           300 + t);
-            if (!ok) break;
-            kept = !stats_only && dec_flag[t * C::R + jt % C::R] != 0;
+            // The decision word: a skipped block needs nothing more (its
+            // scores were read before the vote), a kept one its P (B_PF,
+            // one phase per kept block).
+            const uint32_t want = (uint32_t)(jt + 1) << 1;
+            uint32_t w = ld_acquire_shared(&dec_word[t * C::R + jt % C::R]);
+            if ((w & ~1u) != want) {
+              const long long t0 = clock64();
+              while (((w = ld_acquire_shared(
+                           &dec_word[t * C::R + jt % C::R])) & ~1u) != want) {
+                if (clock64() - t0 > kWaitLimitCycles) {
+                  record_error(kWaitPrefillMma, j, 0, 310 + t);
+                  ok = false;
+                  break;
+                }
+              }
+              if (!ok) break;
+            }
+            kept = !stats_only && (w & 1u) == 0;
+            if (kept) {
+              ok = mbar_wait(&bar[C::B_PF + t], npv[t] & 1, kWaitPrefillMma, j,
+                             300 + t);
+              if (!ok) break;
+            }
           }
           if (kept && vslot < 0) {
             vslot = vcount % C::NVS;
@@ -437,12 +459,11 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
         ++n_vis;
         if (skip) ++n_skp;
         if (p.mask) p.mask[mask_row + j] = skip ? 2 : 1;
-        dec_flag[t * C::R + jt % C::R] = skip ? 0 : 1;
+        st_release_shared(&dec_word[t * C::R + jt % C::R],
+                          ((uint32_t)(jt + 1) << 1) | (skip ? 1u : 0u));
         mbar_arrive(&bar[C::B_DEC + t * C::R + jt % C::R]);
       }
-      if (skip || stats_only) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[C::B_PF + t]);
+      if (skip || stats_only) {  // the issuer reads the decision word
         if (active) m_crit = fmaxf(m_crit, mt_s);
         continue;
       }

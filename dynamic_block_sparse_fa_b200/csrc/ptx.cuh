@@ -175,6 +175,22 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
+// Release store / acquire load of a shared-memory word (a flag one thread
+// publishes and another polls).
+__device__ __forceinline__ void st_release_shared(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)),
+               "r"(v)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_shared(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];"
+               : "=r"(v)
+               : "r"(smem_u32(p))
+               : "memory");
+  return v;
+}
+
 // ---------------------------------------------------------------------------
 // Named barriers (subsets of the CTA).
 // ---------------------------------------------------------------------------
