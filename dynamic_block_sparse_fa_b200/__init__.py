@@ -10,7 +10,9 @@ from .blasst import (BlasstError, Stats, blasst_calibrate,
                      blasst_decode_paged,
                      blasst_decode_splits, blasst_decode_window,
                      blasst_decode_workspace_size,
-                     blasst_fit_a, blasst_last_error, blasst_prefill,
+                     blasst_fit_a, blasst_last_error, blasst_mla_decode,
+                     blasst_mla_decode_splits,
+                     blasst_mla_decode_workspace_size, blasst_prefill,
                      blasst_prefill_backward,
                      blasst_prefill_backward_workspace_size,
                      blasst_prefill_window,
@@ -23,6 +25,8 @@ __all__ = ["BlasstError", "Stats", "blasst_calibrate",
            "blasst_decode_paged",
            "blasst_decode_splits", "blasst_decode_window",
            "blasst_decode_workspace_size", "blasst_fit_a", "blasst_last_error",
+           "blasst_mla_decode", "blasst_mla_decode_splits",
+           "blasst_mla_decode_workspace_size",
            "blasst_prefill", "blasst_prefill_backward",
            "blasst_prefill_backward_workspace_size", "blasst_prefill_window",
            "blasst_selftest_wait_timeout",

@@ -98,6 +98,13 @@ _lib.blasst_decode_noalloc.restype = _i
 _lib.blasst_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                        _i, _f, _f, _i, _i,
                                        ctypes.POINTER(SkipStats), _vp]
+_lib.blasst_mla_decode.restype = _i
+_lib.blasst_mla_decode.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f,
+                                   _f, _i, _vp, _sz, _vp, _vp]
+_lib.blasst_mla_decode_workspace_size.restype = _sz
+_lib.blasst_mla_decode_workspace_size.argtypes = [_i, _i, _i]
+_lib.blasst_mla_decode_splits.restype = _i
+_lib.blasst_mla_decode_splits.argtypes = [_i, _i]
 _lib.blasst_prefill_backward.restype = _i
 _lib.blasst_prefill_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                          _vp, _vp, _vp, _i, _i, _i, _i, _i,
@@ -246,6 +253,47 @@ def blasst_prefill(q, k, v, *, scale=None, causal=True, ln_lambda=-math.inf,
 def blasst_prefill_window(q, k, v, *, window, **kw):
     """blasst_prefill with a causal sliding window of ``window`` keys."""
     return blasst_prefill(q, k, v, window=window, **kw)
+
+
+def blasst_mla_decode_splits(B, L) -> int:
+    return int(_lib.blasst_mla_decode_splits(B, L))
+
+
+def blasst_mla_decode_workspace_size(B, H, num_splits) -> int:
+    return int(_lib.blasst_mla_decode_workspace_size(B, H, num_splits))
+
+
+def blasst_mla_decode(q, cache, *, d_v=512, scale=None, ln_lambda=-math.inf,
+                      num_splits=0, o=None, lse=None, want_lse=True,
+                      workspace=None, stats: Stats | None = None,
+                      stats_only=False, stream=None):
+    """MLA decode.  q [B,H,576], cache [B,L,576] bf16 CUDA (one shared
+    latent row per key; value = its first d_v = 512 columns).  Returns
+    (o [B,H,512], lse [B,H]); both None when stats_only."""
+    B, H, dqk = q.shape
+    L = cache.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(dqk)
+    S = num_splits if num_splits > 0 else blasst_mla_decode_splits(B, L)
+    ws_bytes = 0
+    if not stats_only:
+        if o is None:
+            o = torch.empty(B, H, d_v, dtype=q.dtype, device=q.device)
+        if lse is None and want_lse:
+            lse = torch.empty(B, H, dtype=torch.float32, device=q.device)
+        need = blasst_mla_decode_workspace_size(B, H, S)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8,
+                                    device=q.device)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    else:
+        o, lse, workspace = None, None, None
+    st = _lib.blasst_mla_decode(
+        _ptr(q), _ptr(cache), _ptr(o), _ptr(lse), B, H, L, dqk, d_v,
+        float(scale), float(ln_lambda), S, _ptr(workspace), ws_bytes,
+        stats.c_struct if stats is not None else None, _stream(stream))
+    _check(st, "blasst_mla_decode")
+    return o, lse
 
 
 def blasst_prefill_backward_workspace_size(B, Hq, Lq, d=128) -> int:

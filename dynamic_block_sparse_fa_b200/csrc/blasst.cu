@@ -12,6 +12,7 @@
 #include "prefill.cuh"
 #include "prefill2.cuh"
 #include "backward.cuh"
+#include "mla.cuh"
 
 namespace {
 
@@ -564,6 +565,87 @@ blasst_status_t blasst_prefill_window(const void* q, const void* k,
   p.window = window;
   cudaError_t e = blasst::launch_prefill(p, static_cast<cudaStream_t>(stream));
   return cuda_status(e, "prefill launch");
+}
+
+int blasst_mla_decode_splits(int B, int L) {
+  if (B < 1 || L < 1) return 1;
+  const long long nk = (L + (long long)blasst::kMlaBc - 1) / blasst::kMlaBc;
+  // about two waves of one CTA per SM (4 value quarters per split), at
+  // least 8 blocks per split
+  const long long per = (long long)B * blasst::kMlaParts;
+  long long s = (2LL * kNumSmB200 + per - 1) / per;
+  const long long s_max = nk / 8 > 1 ? nk / 8 : 1;
+  if (s > s_max) s = s_max;
+  return (int)(s < 1 ? 1 : s);
+}
+
+size_t blasst_mla_decode_workspace_size(int B, int H, int num_splits) {
+  if (B < 1 || H < 1 || num_splits < 1) return 0;
+  const size_t rows = (size_t)B * H * num_splits;
+  return ((rows * blasst::kMlaDv * 4 + 255) & ~(size_t)255) +
+         ((rows * 4 + 255) & ~(size_t)255);
+}
+
+blasst_status_t blasst_mla_decode(const void* q, const void* cache, void* o,
+                                  float* lse, int B, int H, int L, int d_qk,
+                                  int d_v, float scale, float ln_lambda,
+                                  int num_splits, void* workspace,
+                                  size_t workspace_bytes,
+                                  const blasst_skip_stats_t* skip_stats,
+                                  void* stream) {
+  if (!q || !cache) return BLASST_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || L < 1 || num_splits < 0) return BLASST_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !valid_ln_lambda(ln_lambda))
+    return BLASST_ERR_INVALID_ARG;
+  if (d_qk != blasst::kMlaDqk || d_v != blasst::kMlaDv ||
+      H > blasst::kMlaRows)
+    return BLASST_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(cache) || (o && !aligned16(o)))
+    return BLASST_ERR_MISALIGNED;
+  const int nk = (L + blasst::kMlaBc - 1) / blasst::kMlaBc;
+  const int S = num_splits == 0 ? blasst_mla_decode_splits(B, L) : num_splits;
+  if (S < 1 || S > nk) return BLASST_ERR_INVALID_ARG;
+  const long long grid = (long long)B * S * blasst::kMlaParts;
+  if (grid > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED_SHAPE;
+  const bool stats_only = (o == nullptr);
+  blasst::MlaArgs a;
+  memset(&a, 0, sizeof a);
+  if (!stats_only) {
+    const size_t need = blasst_mla_decode_workspace_size(B, H, S);
+    if (!workspace || workspace_bytes < need) return BLASST_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return BLASST_ERR_MISALIGNED;
+    const size_t rows = (size_t)B * H * S;
+    a.o_part = static_cast<float*>(workspace);
+    a.lse_part = reinterpret_cast<float*>(
+        static_cast<char*>(workspace) +
+        ((rows * blasst::kMlaDv * 4 + 255) & ~(size_t)255));
+  }
+  if (!blasst::encode_map(&a.tc, cache, blasst::kMlaDqk, L, B, 64))
+    return cuda_status(cudaErrorInvalidValue, "mla tensor map");
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.counters = skip_stats ? skip_stats->counters : nullptr;
+  a.mask = skip_stats ? skip_stats->mask : nullptr;
+  a.B = B;
+  a.H = H;
+  a.L = L;
+  a.nk = nk;
+  a.S = S;
+  a.scale = scale;
+  a.ln_lambda = ln_lambda;
+  a.stats_only = stats_only ? 1 : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaFuncSetAttribute(blasst::mla_split_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       blasst::MlaCfg::SMEM_ALLOC);
+  if (e != cudaSuccess) return cuda_status(e, "mla attribute");
+  blasst::mla_split_kernel<<<(unsigned)grid, blasst::kMlaThreads,
+                             blasst::MlaCfg::SMEM_ALLOC, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || stats_only) return cuda_status(e, "mla split launch");
+  blasst::mla_combine_kernel<<<(unsigned)((long long)B * H), 128, 0, st>>>(
+      a.o_part, a.lse_part, static_cast<__nv_bfloat16*>(o), lse, S);
+  return cuda_status(cudaGetLastError(), "mla merge launch");
 }
 
 size_t blasst_prefill_backward_workspace_size(int B, int Hq, int Lq, int d) {

@@ -1,0 +1,397 @@
+// mla.cuh -- BLASST decode over a multi-head latent (MLA) cache on sm_100a.
+//
+// Every query head h of a token scores the shared latent cache row c_t
+// (d_qk = 576: 512 latent + 64 rope dimensions) as scale * q_h . c_t, and the
+// value is the latent part c_t[0:512] (the attention forms the method is
+// stated to support: MLSys'26 reading notes; gist.science summary, section
+// 3).  The H heads of a token form one decode tile (rows), blocks of 64 keys,
+// the decode criterion and online softmax per split, split-KV merged by
+// log-sum-exp: the same algorithm as decode.cuh with K = c and V = c[:512].
+//
+// One CTA per (sequence, split, value quarter): the 512 value columns are
+// cut into 4 quarters of 128 so that a CTA's output fits in tensor memory
+// next to Q; the 4 CTAs of a (sequence, split) score the same blocks (the
+// second to fourth read them from L2) and take identical decisions.
+//   warp 0      TMA producer: cache blocks [64 keys x 576] (9 boxes of 64
+//               columns), ring of 2
+//   warp 1      MMA issuer (one lane): S = Q c^T (TS: A = Q from TMEM),
+//               then, for a kept block, O += P V (TS: A = P from TMEM,
+//               B = the quarter's value columns, MN-major)
+//   warps 2..5  one thread per head (TMEM lane): Q into TMEM, row max,
+//               vote, exp, P, lazy O rescale, epilogue
+// Tensor memory: Q [0, 288) (bf16 pairs), S [320, 384) (P over its first 32
+// columns), O [384, 512).  Per block the steps run in order (S, decision,
+// P, P.V); the producer keeps the next block in flight.
+#pragma once
+
+#include "prefill.cuh"
+
+namespace blasst {
+
+constexpr int kMlaDqk = 576;
+constexpr int kMlaDv = 512;
+constexpr int kMlaBc = 64;
+constexpr int kMlaParts = 4;   // value quarters of 128 columns
+constexpr int kMlaRows = 128;  // heads per tile (at most)
+constexpr int kMlaThreads = 192;
+
+struct MlaArgs {
+  CUtensorMap tc;            // cache [B][L][576], box 64 x 64
+  const __nv_bfloat16* q;    // [B, H, 576]
+  float* o_part;             // [B*H, S, 512] normalised split outputs
+  float* lse_part;           // [B*H, S]
+  unsigned long long* counters;
+  unsigned char* mask;       // [B, nk]
+  int B, H, L, nk, S;
+  float scale, ln_lambda;
+  int stats_only;
+};
+
+struct MlaCfg {
+  static constexpr int BOX = 64 * 128;           // 64 rows x 128 bytes
+  static constexpr int KBLOCK = 9 * BOX;         // 73728 bytes
+  static constexpr int NK = 2;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_BAR = OFF_K + NK * KBLOCK;
+  static constexpr int B_KF = 0;   // [NK]
+  static constexpr int B_KE = 2;   // [NK]
+  static constexpr int B_QR = 4;   // Q in TMEM (one arrival per head warp)
+  static constexpr int B_SF = 5;   // S in TMEM
+  static constexpr int B_PF = 6;   // P written (kept blocks; per warp)
+  static constexpr int B_OD = 7;   // last MMA done
+  static constexpr int NBAR = 8;
+  static constexpr int R = 4;      // decision-word ring
+  static constexpr int OFF_DEC = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_TMEM = OFF_DEC + R * 4;
+  static constexpr int SMEM = OFF_TMEM + 8;
+  static constexpr int SMEM_ALLOC = SMEM + 1024;
+  static constexpr uint32_t COL_Q = 0, COL_S = 320, COL_O = 384;
+  static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
+};
+
+__global__ void __launch_bounds__(kMlaThreads, 1)
+    mla_split_kernel(const __grid_constant__ MlaArgs a) {
+  using C = MlaCfg;
+  constexpr unsigned FULL = 0xffffffffu;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int part = blockIdx.x % kMlaParts;
+  const int bs = blockIdx.x / kMlaParts;  // b * S + s
+  const int s = bs % a.S;
+  const int b = bs / a.S;
+  const int j0 = (int)(((long long)s * a.nk) / a.S);
+  const int j1 = (int)(((long long)(s + 1) * a.nk) / a.S);
+  const int nb = j1 - j0;
+  const bool recorder = part == 0;  // one CTA of the four records stats
+
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint32_t* dec_word = reinterpret_cast<uint32_t*>(smem + C::OFF_DEC);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NK; ++i) {
+      mbar_init(&bar[C::B_KF + i], 1);
+      mbar_init(&bar[C::B_KE + i], 1);
+    }
+    mbar_init(&bar[C::B_QR], 4);
+    mbar_init(&bar[C::B_SF], 1);
+    mbar_init(&bar[C::B_PF], 4);
+    mbar_init(&bar[C::B_OD], 1);
+    for (int i = 0; i < C::R; ++i) dec_word[i] = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool stats_only = a.stats_only != 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();  // read by the 4 quarters
+      prefetch_tmap(&a.tc);
+      for (int jj = 0; jj < nb; ++jj) {
+        const int sl = jj % C::NK;
+        if (jj >= C::NK &&
+            !mbar_wait(&bar[C::B_KE + sl], ((jj / C::NK) - 1) & 1,
+                       kWaitMla, jj, sl))
+          break;
+        mbar_arrive_expect_tx(&bar[C::B_KF + sl], C::KBLOCK);
+#pragma unroll 1
+        for (int c = 0; c < 9; ++c)
+          tma_load_3d(smem + C::OFF_K + sl * C::KBLOCK + c * C::BOX, &a.tc,
+                      &bar[C::B_KF + sl], c * 64, (j0 + jj) * kMlaBc, b, pol);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0 && nb > 0) {
+      constexpr uint32_t id_s = idesc_bf16(128, kMlaBc, 0, 0);
+      constexpr uint32_t id_o = idesc_bf16(128, 128, 0, 1);
+      const uint32_t aK = smem_u32(smem + C::OFF_K);
+      bool ok = mbar_wait(&bar[C::B_QR], 0, kWaitMla, 0, 10);
+      int npv = 0;
+      for (int jj = 0; jj < nb && ok; ++jj) {
+        const int sl = jj % C::NK;
+        ok = mbar_wait(&bar[C::B_KF + sl], (jj / C::NK) & 1, kWaitMla, jj,
+                       11 + sl);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kb = aK + sl * C::KBLOCK;
+#pragma unroll 4
+        for (int k = 0; k < kMlaDqk / 16; ++k)
+          mma_ts(tmem + C::COL_S, tmem + C::COL_Q + k * 8,
+                 smem_desc(kb + (k >> 2) * C::BOX + (k & 3) * 32, 16, 1024, 2),
+                 id_s, k > 0 ? 1u : 0u);
+        mma_commit(&bar[C::B_SF]);
+        // the tile's decision on this block (published after the vote)
+        const uint32_t want = (uint32_t)(jj + 1) << 1;
+        uint32_t w = ld_acquire_shared(&dec_word[jj % C::R]);
+        if ((w & ~1u) != want) {
+          const long long t0 = clock64();
+          while (((w = ld_acquire_shared(&dec_word[jj % C::R])) & ~1u) != want) {
+            if (clock64() - t0 > kWaitLimitCycles) {
+              record_error(kWaitMla, jj, 0, 13);
+              ok = false;
+              break;
+            }
+          }
+          if (!ok) break;
+        }
+        if (!stats_only && (w & 1u) == 0) {
+          ok = mbar_wait(&bar[C::B_PF], npv & 1, kWaitMla, jj, 14);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < kMlaBc / 16; ++k)
+            mma_ts(tmem + C::COL_O, tmem + C::COL_S + k * 8,
+                   smem_desc(kb + (2 * part) * C::BOX + k * 2048, C::BOX, 1024,
+                             2),
+                   id_o, (npv > 0 || k > 0) ? 1u : 0u);
+          ++npv;
+        }
+        mma_commit(&bar[C::B_KE + sl]);
+      }
+      mma_commit(&bar[C::B_OD]);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------- head rows
+    const int quad = warp & 3;
+    const int h = quad * 32 + lane;  // head = TMEM lane
+    const bool active = h < a.H;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const bool elected = (quad == 0 && lane == 0);
+    // Q row into TMEM [0, 288): 9 chunks of 64 bf16 (32 columns)
+    {
+      // padding rows (h >= H) read head 0's row and store zeros: no branch
+      // before the warp-collective TMEM stores
+      const uint4* qrow = reinterpret_cast<const uint4*>(
+          a.q + ((size_t)b * a.H + (active ? h : 0)) * kMlaDqk);
+      const uint32_t keep = active ? 0xffffffffu : 0u;
+#pragma unroll 1
+      for (int c = 0; c < 9; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = __ldg(qrow + c * 8 + u);
+          r[4 * u] = v.x & keep;
+          r[4 * u + 1] = v.y & keep;
+          r[4 * u + 2] = v.z & keep;
+          r[4 * u + 3] = v.w & keep;
+        }
+        __syncwarp();
+        tmem_st32(lane_base + C::COL_Q + c * 32, r);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[C::B_QR]);
+    }
+    const float scale = a.scale, ln_lambda = a.ln_lambda;
+    const float sl2 = scale * kPrefLog2e;
+    float m_crit = -INFINITY, m_ref = -INFINITY, l = 0.f;
+    unsigned long long n_vis = 0, n_skp = 0;
+    bool ok = true;
+    for (int jj = 0; jj < nb; ++jj) {
+      const int j = j0 + jj;
+      const bool w = mbar_wait(&bar[C::B_SF], jj & 1, kWaitMla, jj, 20);
+      tc_fence_after();
+      uint32_t sr[2][32];
+      tmem_ld32(lane_base + C::COL_S, sr[0]);
+      tmem_ld32(lane_base + C::COL_S + 32, sr[1]);
+      tc_wait_ld();
+      const int valid = min(kMlaBc, a.L - j * kMlaBc);  // keys of the block
+      if (valid < kMlaBc) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            if (c * 32 + x >= valid) sr[c][x] = __float_as_uint(-INFINITY);
+      }
+      float m8[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x)
+        m8[x] = fmaxf(__uint_as_float(sr[0][x]), __uint_as_float(sr[0][x + 8]));
+#pragma unroll
+      for (int i = 16; i < 64; i += 16)
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+          m8[x] = fmax3(m8[x], __uint_as_float(sr[i >> 5][(i & 31) + x]),
+                        __uint_as_float(sr[(i + 8) >> 5][((i + 8) & 31) + x]));
+      const float mt = fmax3(fmax3(m8[0], m8[1], m8[2]),
+                             fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+      const float mt_s = mt * scale;
+      const bool pred = !active || mt_s == -INFINITY ||
+                        (mt_s - m_crit < ln_lambda);
+      tc_fence_before();
+      // the vote also carries a failed wait: every thread then leaves
+      const bool all = named_sync_and(1, 128, pred && w);
+      const bool any_fail = !named_sync_and(1, 128, w);
+      if (any_fail) { ok = false; break; }
+      const bool skip = all && (ln_lambda > -INFINITY);
+      if (elected) {
+        st_release_shared(&dec_word[jj % C::R],
+                          ((uint32_t)(jj + 1) << 1) | (skip ? 1u : 0u));
+        ++n_vis;
+        if (skip) ++n_skp;
+        if (recorder && a.mask) a.mask[(size_t)b * a.nk + j] = skip ? 2 : 1;
+      }
+      if (skip || stats_only) {
+        if (active) m_crit = fmaxf(m_crit, mt_s);
+        continue;
+      }
+      float alpha = 1.f;
+      bool rescale = false;
+      if (active && mt_s != -INFINITY) {
+        const float m_new = fmaxf(m_crit, mt_s);
+        if (m_ref == -INFINITY || m_new > m_ref + kRescaleNats) {
+          alpha = (m_ref == -INFINITY) ? 0.f
+                                       : ex2_approx((m_ref - m_new) * kPrefLog2e);
+          m_ref = m_new;
+          rescale = true;
+        }
+      }
+      const float mb = (active && m_ref != -INFINITY) ? m_ref * kPrefLog2e
+                                                      : INFINITY;
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][x]), sl2, -mb));
+          const float p1 =
+              ex2_approx(fmaf(__uint_as_float(sr[c][x + 1]), sl2, -mb));
+          rs += p0 + p1;
+          pk[x / 2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(lane_base + C::COL_S + c * 16, pk);
+      }
+      l = alpha * l + rs;
+      tc_wait_st();
+      // O is idle here (S of this block arrived after the previous P.V)
+      if (__any_sync(FULL, rescale)) {
+        const float f = rescale ? alpha : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t orow[32];
+          tmem_ld32(lane_base + C::COL_O + c * 32, orow);
+          tc_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            orow[x] = __float_as_uint(__uint_as_float(orow[x]) * f);
+          tmem_st32(lane_base + C::COL_O + c * 32, orow);
+        }
+        tc_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[C::B_PF]);
+      if (active) m_crit = fmaxf(m_crit, mt_s);
+    }
+    if (ok && elected && recorder && a.counters && nb > 0) {
+      atomicAdd(&a.counters[0], n_vis);
+      atomicAdd(&a.counters[1], n_skp);
+    }
+    if (ok && !stats_only) {
+      const size_t row = (size_t)b * a.H + h;
+      bool w2 = true;
+      if (nb > 0) w2 = mbar_wait(&bar[C::B_OD], 0, kWaitMla, nb, 21);
+      tc_fence_after();
+      // warp-wide: every lane takes part (padding heads included)
+      const bool done = __all_sync(FULL, w2) && nb > 0;
+      const bool have = done && l > 0.f;
+      const float inv_l = have ? 1.f / l : 0.f;
+      float* dst = a.o_part + (row * a.S + s) * kMlaDv + part * 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t orow[32];
+        if (done) {
+          tmem_ld32(lane_base + C::COL_O + c * 32, orow);
+          tc_wait_ld();
+        }
+        if (active) {
+#pragma unroll
+          for (int x = 0; x < 32; x += 4)
+            *reinterpret_cast<float4*>(dst + c * 32 + x) =
+                have ? make_float4(__uint_as_float(orow[x]) * inv_l,
+                                   __uint_as_float(orow[x + 1]) * inv_l,
+                                   __uint_as_float(orow[x + 2]) * inv_l,
+                                   __uint_as_float(orow[x + 3]) * inv_l)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      if (active && part == 0)
+        a.lse_part[row * a.S + s] = have ? m_ref + __logf(l) : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// lse = ln sum_s exp(lse_s), o = sum_s exp(lse_s - lse) o_s -> bf16.  One
+// CTA of 128 threads per (sequence, head), 4 value columns per thread.
+__global__ void __launch_bounds__(128) mla_combine_kernel(
+    const float* o_part, const float* lse_part, __nv_bfloat16* o, float* lse,
+    int S) {
+  const size_t row = blockIdx.x;
+  const float* lp = lse_part + row * S;
+  float mx = -INFINITY;
+  for (int s = 0; s < S; ++s) mx = fmaxf(mx, lp[s]);
+  float den = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (mx > -INFINITY) {
+    for (int s = 0; s < S; ++s) {
+      const float wgt = lp[s] == -INFINITY ? 0.f : __expf(lp[s] - mx);
+      den += wgt;
+      const float4 v =
+          reinterpret_cast<const float4*>(o_part + (row * S + s) * kMlaDv)[threadIdx.x];
+      acc.x += wgt * v.x;
+      acc.y += wgt * v.y;
+      acc.z += wgt * v.z;
+      acc.w += wgt * v.w;
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  uint2 w;
+  w.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+  w.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+  reinterpret_cast<uint2*>(o + row * kMlaDv)[threadIdx.x] = w;
+  if (threadIdx.x == 0 && lse) lse[row] = den > 0.f ? mx + __logf(den) : -INFINITY;
+}
+
+}  // namespace blasst

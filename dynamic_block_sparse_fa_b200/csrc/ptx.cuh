@@ -27,6 +27,7 @@ enum : unsigned int {
   kWaitPrefillSoftmax = 12,
   kWaitPrefillEpilogue = 13,
   kWaitBackward = 14,
+  kWaitMla = 15,
   kWaitSelfTest = 99,
   // Device-resident arguments found out of range (paged decode); these are
   // reported as invalid arguments, not as waits that gave up.

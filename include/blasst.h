@@ -369,6 +369,43 @@ size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits);
 int blasst_decode_splits(int B, int Hkv, int Lkv, int Bc);
 
 /*
+ * blasst_mla_decode -- decode over a multi-head latent (MLA) cache: each
+ * of the H query heads of a token scores the shared latent row c_t of every
+ * key as scale * q_h . c_t (d_qk = 576: 512 latent + 64 rope dimensions)
+ * and takes the latent part c_t[0:512] as value (the attention forms the
+ * method is stated to support: MLSys'26 reading notes; gist.science
+ * summary, section 3).  The H heads form one decode tile; blocks of 64 keys
+ * with the decode criterion and online softmax per split (split s covers
+ * blocks [floor(s*nk/S), floor((s+1)*nk/S))), merged by log-sum-exp as in
+ * blasst_decode.  Only the P.V product and the exp are saved by a skip: the
+ * value is part of the row the score already read.
+ *
+ *  q           device bf16 [B, H, 576]
+ *  cache       device bf16 [B, L, 576] (one latent row per key)
+ *  o           device bf16 [B, H, 512], or NULL for a statistics-only pass
+ *  lse         device float32 [B, H] or NULL
+ *  H           1..128;  d_qk = 576, d_v = 512 (else UNSUPPORTED_SHAPE)
+ *  num_splits  >= 1 (at most ceil(L/64)), or 0 = blasst_mla_decode_splits
+ *  workspace   blasst_mla_decode_workspace_size(B, H, resolved splits)
+ *              bytes, 256-byte aligned, caller-owned (NULL allowed when o
+ *              is NULL)
+ *  skip_stats  counters as blasst_decode; mask layout [B, ceil(L/64)]
+ * Asynchronous on `stream`; two kernel launches; allocates nothing.
+ */
+blasst_status_t blasst_mla_decode(const void *q, const void *cache, void *o,
+                                  float *lse, int B, int H, int L, int d_qk,
+                                  int d_v, float scale, float ln_lambda,
+                                  int num_splits, void *workspace,
+                                  size_t workspace_bytes,
+                                  const blasst_skip_stats_t *skip_stats,
+                                  void *stream);
+/* Bytes of MLA decode workspace (split outputs and their lse). */
+size_t blasst_mla_decode_workspace_size(int B, int H, int num_splits);
+/* The automatic MLA split count: about two waves of one CTA per SM (four
+ * CTAs per split), at least 8 blocks per split. */
+int blasst_mla_decode_splits(int B, int L);
+
+/*
  * Calibration of the threshold lambda = a / L for a target sparsity
  * (gist.science summary, section 2 "Calibracao Automatica"; MLSys'26 reading
  * notes, observation 2: a is fitted on calibration data, not universal).
