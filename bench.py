@@ -277,6 +277,10 @@ def run_blasst(args):
         line = {"metric": METRIC, "value": None, "unit": "GB/s",
                 "n_gpus": world, "note": "decode leg skipped"}
 
+    # ---------------- MLA decode (rank 0) ----------------
+    if rank == 0 and not args.no_mla and not args.no_decode:
+        line["decode_mla"] = run_mla(args, bl, dev, stream, hbm_peak, tf_burst)
+
     # ---------------- prefill workload (rank 0) ----------------
     if rank == 0 and not args.no_prefill:
         line["prefill"], line["roofline_prefill"] = run_prefill(
@@ -581,6 +585,63 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
     return out, roof
 
 
+def run_mla(args, bl, dev, stream, hbm_peak, tf_peak):
+    """MLA decode: B 32 tokens x 128 heads against a 32K-key latent cache
+    (576 wide, value = first 512 columns), planted-gap rows; dense and at the
+    ln lambda (bisection over statistics-only passes) that skips ~50%.
+    Algorithmic bytes = the cache (read once; the value is part of the row)
+    + q + split partials written and read + o and lse."""
+    from synth import config_seed, planted_gap_kv_inplace
+    B, H, L, dqk, dv = 32, 128, 32768, 576, 512
+    q = torch.empty(B, H, dqk, dtype=torch.bfloat16, device=dev)
+    c4 = torch.empty(B, 1, L, dqk, dtype=torch.bfloat16, device=dev)
+    planted_gap_kv_inplace(c4, torch.empty_like(c4), q, block=64, gap=8.0,
+                           heavy_frac=0.03, seed=config_seed(31))
+    cache = c4[:, 0]
+    nk = -(-L // 64)
+    S = bl.blasst_mla_decode_splits(B, L)
+    st = bl.Stats(device=dev, mask_numel=B * nk)
+
+    def sparsity(lnl):
+        st.reset()
+        bl.blasst_mla_decode(q, cache, ln_lambda=lnl, stats=st, stats_only=True)
+        torch.cuda.synchronize()
+        v, s_ = st.read()
+        return s_ / v
+    lo, hi = -64.0, 0.0
+    for _ in range(16):
+        mid = 0.5 * (lo + hi)
+        if sparsity(mid) < 0.5:
+            lo = mid
+        else:
+            hi = mid
+    lnl = hi
+    o = torch.empty(B, H, dv, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, H, dtype=torch.float32, device=dev)
+    ws = torch.empty(bl.blasst_mla_decode_workspace_size(B, H, S),
+                     dtype=torch.uint8, device=dev)
+    out = {"workload": f"MLA decode B{B} H{H} L{L} d_qk {dqk} d_v {dv} Bc 64",
+           "splits": S}
+    K, W = args.steps, args.warmup
+    for key, l in (("dense", -math.inf), ("sparse", lnl)):
+        sp = sparsity(l)
+        fn = lambda: bl.blasst_mla_decode(q, cache, ln_lambda=l, o=o, lse=lse,
+                                          workspace=ws)
+        ms = time_calls(fn, K, W, stream) / K
+        byts = (B * L * dqk * 2 + B * H * dqk * 2 + 2 * B * H * S * (dv + 1) * 4
+                + B * H * (dv * 2 + 4))
+        kept = (1.0 - sp) * B * nk
+        # tensor work issued: 4 CTAs score each block, one P.V quarter each
+        issued = (4 * 2.0 * 128 * 64 * dqk * B * nk + 2.0 * 128 * 64 * dv * kept)
+        out[key] = {"ln_lambda": l, "sparsity": sp, "us": round(ms * 1e3, 1),
+                    "GBps": round(byts / (ms / 1e3) / 1e9, 1),
+                    "hbm_frac": round(byts / (ms / 1e3) / 1e9 / hbm_peak, 4),
+                    "issued_tflops": round(issued / (ms / 1e3) / 1e12, 1),
+                    "tensor_frac_issued": round(issued / (ms / 1e3) / 1e12 / tf_peak, 4)}
+    out["sparse"]["speedup_vs_dense"] = round(out["dense"]["us"] / out["sparse"]["us"], 4)
+    return out
+
+
 def run_prefill_backward(args, bl, q, k, v, lnl, stream, tf_peak):
     """blasst_prefill_backward on the prefill workload: the dense backward
     (every visible pair) and the backward of the forward at the ln lambda
@@ -807,6 +868,8 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-window", action="store_true",
                     help="skip the sliding-window measurements")
+    ap.add_argument("--no-mla", action="store_true",
+                    help="skip the MLA decode measurements")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the prefill backward measurements")
     ap.add_argument("--no-paged", action="store_true",
