@@ -98,6 +98,9 @@ _lib.blasst_decode_noalloc.restype = _i
 _lib.blasst_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                        _i, _f, _f, _i, _i,
                                        ctypes.POINTER(SkipStats), _vp]
+_lib.blasst_decode_wide.restype = _i
+_lib.blasst_decode_wide.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                    _i, _f, _f, _i, _i, _vp, _sz, _vp, _vp]
 _lib.blasst_mla_decode.restype = _i
 _lib.blasst_mla_decode.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f,
                                    _f, _i, _vp, _sz, _vp, _vp]
@@ -407,6 +410,38 @@ def blasst_decode(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
         ws_bytes, stats.c_struct if stats is not None else None,
         _stream(stream))
     _check(st, "blasst_decode_window")
+    return o, lse
+
+
+def blasst_decode_wide(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
+                       num_splits=0, o=None, lse=None, want_lse=True,
+                       workspace=None, stats: Stats | None = None,
+                       stats_only=False, stream=None):
+    """Decode on the tensor core with all G = Hq/Hkv (<= 128) heads of a KV
+    head as one tile (blasst_decode_wide).  Same arguments and results as
+    blasst_decode; the mask layout is [B, Hkv, nk]."""
+    B, Hq, d = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    S = num_splits if num_splits > 0 else blasst_decode_splits(B, Hkv, Lkv, Bc)
+    ws_bytes = 0
+    if not stats_only:
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and want_lse:
+            lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+        need = blasst_decode_workspace_size(B, Hq, d, S)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    else:
+        o, lse, workspace = None, None, None
+    st = _lib.blasst_decode_wide(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lkv, d,
+        float(scale), float(ln_lambda), Bc, S, _ptr(workspace), ws_bytes,
+        stats.c_struct if stats is not None else None, _stream(stream))
+    _check(st, "blasst_decode_wide")
     return o, lse
 
 

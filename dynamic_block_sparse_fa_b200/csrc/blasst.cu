@@ -13,6 +13,7 @@
 #include "prefill2.cuh"
 #include "backward.cuh"
 #include "mla.cuh"
+#include "decode_wide.cuh"
 
 namespace {
 
@@ -565,6 +566,71 @@ blasst_status_t blasst_prefill_window(const void* q, const void* k,
   p.window = window;
   cudaError_t e = blasst::launch_prefill(p, static_cast<cudaStream_t>(stream));
   return cuda_status(e, "prefill launch");
+}
+
+blasst_status_t blasst_decode_wide(const void* q, const void* k_cache,
+                                   const void* v_cache, void* o, float* lse,
+                                   int B, int Hq, int Hkv, int Lkv, int d,
+                                   float scale, float ln_lambda, int Bc,
+                                   int num_splits, void* workspace,
+                                   size_t workspace_bytes,
+                                   const blasst_skip_stats_t* skip_stats,
+                                   void* stream) {
+  if (!q || !k_cache || !v_cache) return BLASST_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lkv < 1 || Hq % Hkv != 0 ||
+      num_splits < 0)
+    return BLASST_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !valid_ln_lambda(ln_lambda))
+    return BLASST_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (d != blasst::kWideD || Bc != blasst::kWideBc || G > 128)
+    return BLASST_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (o && !aligned16(o)))
+    return BLASST_ERR_MISALIGNED;
+  const int nk = (Lkv + Bc - 1) / Bc;
+  const int S = num_splits == 0 ? blasst_decode_splits(B, Hkv, Lkv, Bc)
+                                : num_splits;
+  if (S < 1 || S > nk) return BLASST_ERR_INVALID_ARG;
+  const long long grid = (long long)B * Hkv * S;
+  if (grid > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED_SHAPE;
+  const bool stats_only = (o == nullptr);
+  blasst::WideArgs a;
+  memset(&a, 0, sizeof a);
+  if (!stats_only) {
+    const blasst_status_t ws = carve_workspace(workspace, workspace_bytes, B,
+                                               Hq, d, S, &a.o_part,
+                                               &a.lse_part);
+    if (ws != BLASST_OK) return ws;
+  }
+  if (!blasst::encode_map(&a.tk, k_cache, d, Lkv, (long long)B * Hkv, 64) ||
+      !blasst::encode_map(&a.tv, v_cache, d, Lkv, (long long)B * Hkv, 64))
+    return cuda_status(cudaErrorInvalidValue, "wide decode tensor maps");
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.counters = skip_stats ? skip_stats->counters : nullptr;
+  a.mask = skip_stats ? skip_stats->mask : nullptr;
+  a.Hkv = Hkv;
+  a.G = G;
+  a.Lkv = Lkv;
+  a.nk = nk;
+  a.S = S;
+  a.scale = scale;
+  a.ln_lambda = ln_lambda;
+  a.stats_only = stats_only ? 1 : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaFuncSetAttribute(blasst::decode_wide_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       blasst::WideCfg::SMEM_ALLOC);
+  if (e != cudaSuccess) return cuda_status(e, "wide decode attribute");
+  blasst::decode_wide_kernel<<<(unsigned)grid, blasst::kWideThreads,
+                               blasst::WideCfg::SMEM_ALLOC, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || stats_only)
+    return cuda_status(e, "wide decode split launch");
+  blasst::decode_combine_kernel<<<(unsigned)((long long)B * Hq), blasst::kDecD,
+                                  0, st>>>(
+      a.o_part, a.lse_part, static_cast<__nv_bfloat16*>(o), lse, S);
+  return cuda_status(cudaGetLastError(), "wide decode merge launch");
 }
 
 int blasst_mla_decode_splits(int B, int L) {

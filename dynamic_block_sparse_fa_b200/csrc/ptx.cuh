@@ -28,6 +28,7 @@ enum : unsigned int {
   kWaitPrefillEpilogue = 13,
   kWaitBackward = 14,
   kWaitMla = 15,
+  kWaitDecodeWide = 16,
   kWaitSelfTest = 99,
   // Device-resident arguments found out of range (paged decode); these are
   // reported as invalid arguments, not as waits that gave up.

@@ -369,6 +369,29 @@ size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits);
 int blasst_decode_splits(int B, int Hkv, int Lkv, int Bc);
 
 /*
+ * blasst_decode_wide -- blasst_decode on the tensor core for wide head
+ * groups: all G = Hq/Hkv (1..128) query heads of a KV head form one tile
+ * (the rows of 128 x 64 score and 128 x 128 P.V MMAs; G < 128 is padded),
+ * with the decode criterion, V read only for kept blocks and the split/merge
+ * of blasst_decode.  For MQA and large GQA ratios, where G x d FMAs per key
+ * outgrow the memory time of the CUDA-core kernel.  Unlike blasst_decode
+ * with G > 8 (tiles of 8 heads), the whole group votes together; the mask
+ * layout is [B, Hkv, ceil(Lkv/64)].
+ *
+ *  d = 128, Bc = 64, 1 <= Hq/Hkv <= 128 (else UNSUPPORTED_SHAPE); other
+ *  arguments, workspace (blasst_decode_workspace_size), ownership and
+ *  errors as blasst_decode.
+ */
+blasst_status_t blasst_decode_wide(const void *q, const void *k_cache,
+                                   const void *v_cache, void *o, float *lse,
+                                   int B, int Hq, int Hkv, int Lkv, int d,
+                                   float scale, float ln_lambda, int Bc,
+                                   int num_splits, void *workspace,
+                                   size_t workspace_bytes,
+                                   const blasst_skip_stats_t *skip_stats,
+                                   void *stream);
+
+/*
  * blasst_mla_decode -- decode over a multi-head latent (MLA) cache: each
  * of the H query heads of a token scores the shared latent row c_t of every
  * key as scale * q_h . c_t (d_qk = 576: 512 latent + 64 rope dimensions)
