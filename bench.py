@@ -277,8 +277,9 @@ def run_blasst(args):
         line = {"metric": METRIC, "value": None, "unit": "GB/s",
                 "n_gpus": world, "note": "decode leg skipped"}
 
-    # ---------------- MLA decode (rank 0) ----------------
+    # ---------------- MQA and MLA decode (rank 0) ----------------
     if rank == 0 and not args.no_mla and not args.no_decode:
+        line["decode_mqa"] = run_mqa(args, bl, dev, stream, hbm_peak)
         line["decode_mla"] = run_mla(args, bl, dev, stream, hbm_peak, tf_burst)
 
     # ---------------- prefill workload (rank 0) ----------------
@@ -583,6 +584,39 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
             "peak_kind": peak_kind + " bf16 burst", "unit": "TFLOP/s",
             "frac": best["tensor_frac"], "traffic": None}
     return out, roof
+
+
+def run_mqa(args, bl, dev, stream, hbm_peak):
+    """MQA decode, B 32 x 32 query heads on one KV head, 32K keys, d 128:
+    blasst_decode (CUDA cores, tiles of 8 heads) against blasst_decode_wide
+    (tensor cores, the 32 heads as one tile), dense and at ln lambda -2.
+    GB/s counts K and the V of kept blocks."""
+    from synth import config_seed, planted_gap_kv_inplace
+    B, Hq, Hkv, L, d = 32, 32, 1, 32768, 128
+    q = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev)
+    k = torch.empty(B, Hkv, L, d, dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    planted_gap_kv_inplace(k, v, q, block=64, gap=8.0, heavy_frac=0.03,
+                           seed=config_seed(10, 4))
+    nk = L // 64
+    K, W = args.steps, args.warmup
+    out = {"workload": f"MQA decode B{B} Hq{Hq} Hkv{Hkv} Lkv{L} d{d} Bc 64"}
+    for name, fn, rows in (("tiles_of_8", bl.blasst_decode, Hkv * Hq // 8),
+                           ("wide", bl.blasst_decode_wide, Hkv)):
+        r = {}
+        for key, lnl in (("dense", -math.inf), ("lnl_-2", -2.0)):
+            st = bl.Stats(device=dev, mask_numel=B * rows * nk)
+            o, lse = fn(q, k, v, ln_lambda=lnl, stats=st)
+            torch.cuda.synchronize()
+            vis, skp = st.read()
+            ms = time_calls(lambda: fn(q, k, v, ln_lambda=lnl, o=o, lse=lse),
+                            K, W, stream) / K
+            byts = B * Hkv * L * d * 2 * (2.0 - skp / vis)
+            r[key] = {"us": round(ms * 1e3, 1), "sparsity": skp / vis,
+                      "GBps": round(byts / (ms / 1e3) / 1e9, 1),
+                      "hbm_frac": round(byts / (ms / 1e3) / 1e9 / hbm_peak, 4)}
+        out[name] = r
+    return out
 
 
 def run_mla(args, bl, dev, stream, hbm_peak, tf_peak):
