@@ -9,12 +9,16 @@
 // cannot feed fast enough once G x d FMAs per key exceed the memory time.
 //   warp 0      producer: K blocks (2-slot ring) ahead of the scores; V of
 //               a block as soon as the tile's decision keeps it (2 slots)
-//   warp 1      MMA issuer (one lane): S = Q K^T (TS, A = Q from TMEM),
-//               O += P V (TS, A = P from TMEM, B = V MN-major)
-//   warps 2..5  one thread per head: Q into TMEM, row max, vote, exp, P,
-//               lazy O rescale, epilogue
-// Tensor memory: Q [0, 64) (bf16 pairs), S [64, 128) (P over its first 32
-// columns), O [128, 256): 256 columns, two CTAs per SM.
+//   warp 1      MMA issuer (one lane): S = Q K^T (TS, A = Q from TMEM);
+//               O += P V (SS, P from shared memory, V MN-major) one block
+//               behind: the P.V of a kept block goes out after the next
+//               block's S, so its V load overlaps that block's score and
+//               vote
+//   warps 2..5  one thread per head: Q into TMEM, row max, vote, exp, P
+//               (bf16, two shared-memory slots), lazy O rescale (after the
+//               pending P.V is done), epilogue
+// Tensor memory: Q [0, 64) (bf16 pairs), S [64, 128), O [128, 256): 256
+// columns, two CTAs per SM.
 #pragma once
 
 #include "prefill.cuh"
@@ -43,16 +47,20 @@ struct WideCfg {
   static constexpr int NK = 2, NV = 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + NK * TILE;
-  static constexpr int OFF_BAR = OFF_V + NV * TILE;
+  static constexpr int PT = 128 * kWideBc * 2;  // P tile: 128 rows x 64 keys
+  static constexpr int OFF_P = OFF_V + NV * TILE;  // [2] P tiles
+  static constexpr int OFF_BAR = OFF_P + 2 * PT;
   static constexpr int B_KF = 0;   // [NK]
   static constexpr int B_KE = 2;   // [NK]
   static constexpr int B_VF = 4;   // [NV]
   static constexpr int B_VE = 6;   // [NV]
   static constexpr int B_QR = 8;   // Q in TMEM (one arrival per row warp)
   static constexpr int B_SF = 9;   // S in TMEM
-  static constexpr int B_PF = 10;  // P written (kept blocks; per warp)
-  static constexpr int B_OD = 11;  // last MMA done
-  static constexpr int NBAR = 12;
+  static constexpr int B_PF = 10;  // [2] P slot written (one arrival per warp)
+  static constexpr int B_PE = 12;  // [2] P slot read by its P.V
+  static constexpr int B_PVD = 14; // a P.V done (one phase per kept block)
+  static constexpr int B_OD = 15;  // last MMA done
+  static constexpr int NBAR = 16;
   static constexpr int R = 4;      // decision-word ring
   static constexpr int OFF_DEC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_TMEM = OFF_DEC + R * 4;
@@ -105,7 +113,11 @@ __global__ void __launch_bounds__(kWideThreads, 2)
     }
     mbar_init(&bar[C::B_QR], 4);
     mbar_init(&bar[C::B_SF], 1);
-    mbar_init(&bar[C::B_PF], 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[C::B_PF + i], 4);
+      mbar_init(&bar[C::B_PE + i], 1);
+    }
+    mbar_init(&bar[C::B_PVD], 1);
     mbar_init(&bar[C::B_OD], 1);
     for (int i = 0; i < C::R; ++i) dec_word[i] = 0u;
     fence_mbar_init();
@@ -171,8 +183,32 @@ __global__ void __launch_bounds__(kWideThreads, 2)
       constexpr uint32_t id_o = idesc_bf16(128, kWideD, 0, 1);
       const uint32_t aK = smem_u32(smem + C::OFF_K);
       const uint32_t aV = smem_u32(smem + C::OFF_V);
+      const uint32_t aP = smem_u32(smem + C::OFF_P);
       bool ok = mbar_wait(&bar[C::B_QR], 0, kWaitDecodeWide, 0, 10);
-      int npv = 0;
+      int npv = 0;           // P.V products issued
+      bool pending = false;  // a kept block whose P.V is not issued yet
+      // P.V of kept block number npv: P and V slot npv % 2
+      auto issue_pv = [&]() {
+        const int sl = npv % 2;
+        ok = ok &&
+             mbar_wait(&bar[C::B_PF + sl], (npv / 2) & 1, kWaitDecodeWide, npv,
+                       13) &&
+             mbar_wait(&bar[C::B_VF + sl], (npv / C::NV) & 1, kWaitDecodeWide,
+                       npv, 14);
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t vb = aV + sl * C::TILE, pb = aP + sl * C::PT;
+#pragma unroll
+        for (int k = 0; k < kWideBc / 16; ++k)
+          mma_ss(tmem + C::COL_O,
+                 smem_desc(pb + k * 32, 16, 1024, 2),  // P: K-major, 128 B rows
+                 smem_desc(vb + k * 2048, C::BOX, 1024, 2), id_o,
+                 (npv > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&bar[C::B_PE + sl]);
+        mma_commit(&bar[C::B_VE + sl]);
+        mma_commit(&bar[C::B_PVD]);
+        ++npv;
+      };
       for (int jj = 0; jj < nb && ok; ++jj) {
         const int sl = jj % C::NK;
         ok = mbar_wait(&bar[C::B_KF + sl], (jj / C::NK) & 1, kWaitDecodeWide,
@@ -186,26 +222,17 @@ __global__ void __launch_bounds__(kWideThreads, 2)
                  smem_desc(kb + (k >> 2) * C::BOX + (k & 3) * 32, 16, 1024, 2),
                  id_s, k > 0 ? 1u : 0u);
         mma_commit(&bar[C::B_SF]);
+        mma_commit(&bar[C::B_KE + sl]);
+        if (pending) {  // the previous kept block, behind this block's S
+          issue_pv();
+          pending = false;
+          if (!ok) break;
+        }
         const uint32_t w = wide_decision(&dec_word[jj % C::R], jj, 12);
         if (w == 0u) { ok = false; break; }
-        if (!stats_only && (w & 1u) == 0) {
-          const int vs = npv % C::NV;
-          ok = mbar_wait(&bar[C::B_PF], npv & 1, kWaitDecodeWide, jj, 13) &&
-               mbar_wait(&bar[C::B_VF + vs], (npv / C::NV) & 1,
-                         kWaitDecodeWide, jj, 14);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t vb = aV + vs * C::TILE;
-#pragma unroll
-          for (int k = 0; k < kWideBc / 16; ++k)
-            mma_ts(tmem + C::COL_O, tmem + C::COL_S + k * 8,
-                   smem_desc(vb + k * 2048, C::BOX, 1024, 2), id_o,
-                   (npv > 0 || k > 0) ? 1u : 0u);
-          mma_commit(&bar[C::B_VE + vs]);
-          ++npv;
-        }
-        mma_commit(&bar[C::B_KE + sl]);
+        pending = !stats_only && (w & 1u) == 0;
       }
+      if (ok && pending) issue_pv();
       mma_commit(&bar[C::B_OD]);
     }
     __syncwarp();
@@ -248,6 +275,8 @@ __global__ void __launch_bounds__(kWideThreads, 2)
     const float sl2 = scale * kPrefLog2e;
     float m_crit = -INFINITY, m_ref = -INFINITY, l = 0.f;
     unsigned long long n_vis = 0, n_skp = 0;
+    int kp = 0;  // kept blocks so far (their P slot is kp % 2)
+    uint8_t* sP = smem + C::OFF_P;
     bool ok = true;
     for (int jj = 0; jj < nb; ++jj) {
       const int j = j0 + jj;
@@ -309,25 +338,38 @@ __global__ void __launch_bounds__(kWideThreads, 2)
       }
       const float mb = (active && m_ref != -INFINITY) ? m_ref * kPrefLog2e
                                                       : INFINITY;
+      // P (bf16, this row's 64 keys = one 128-byte swizzled row) into P
+      // slot kp % 2, once the P.V two kept blocks back has read it
+      const int psl = kp & 1;
+      bool wp = true;
+      if (kp >= 2)
+        wp = mbar_wait(&bar[C::B_PE + psl], ((kp >> 1) - 1) & 1,
+                       kWaitDecodeWide, jj, 22);
       float rs = 0.f;
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][x]), sl2, -mb));
-          const float p1 =
-              ex2_approx(fmaf(__uint_as_float(sr[c][x + 1]), sl2, -mb));
-          rs += p0 + p1;
-          pk[x / 2] = pack_bf16x2(p0, p1);
-        }
-        __syncwarp();
-        tmem_st16(lane_base + C::COL_S + c * 16, pk);
+      for (int x = 0; x < 64; x += 2) {
+        const float p0 =
+            ex2_approx(fmaf(__uint_as_float(sr[x >> 5][x & 31]), sl2, -mb));
+        const float p1 =
+            ex2_approx(fmaf(__uint_as_float(sr[x >> 5][(x & 31) + 1]), sl2, -mb));
+        rs += p0 + p1;
+        pk[x / 2] = pack_bf16x2(p0, p1);
       }
       l = alpha * l + rs;
-      tc_wait_st();
-      // O is idle here: S of this block arrived after the previous P.V
+      uint8_t* prow = sP + psl * C::PT + h * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) * 16)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_async_smem();
+      // The O rescale waits for the P.V of the previous kept block (it may
+      // still be running: P.V goes out one block behind).
       if (__any_sync(FULL, rescale)) {
+        bool wv = true;
+        if (kp >= 1)
+          wv = mbar_wait(&bar[C::B_PVD], (kp - 1) & 1, kWaitDecodeWide, jj, 23);
+        tc_fence_after();
         const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -340,10 +382,12 @@ __global__ void __launch_bounds__(kWideThreads, 2)
           tmem_st32(lane_base + C::COL_O + c * 32, orow);
         }
         tc_wait_st();
+        wp = wp && wv;
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[C::B_PF]);
+      const bool wall = __all_sync(FULL, wp);  // every lane votes
+      if (lane == 0 && wall) mbar_arrive(&bar[C::B_PF + psl]);
+      ++kp;
       if (active) m_crit = fmaxf(m_crit, mt_s);
     }
     if (ok && elected && a.counters && nb > 0) {
