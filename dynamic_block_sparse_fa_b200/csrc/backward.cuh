@@ -89,10 +89,6 @@ struct BwdCfg {
   static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
 };
 
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // global[box at (c0, c1, c2)] += shared box (f32 add), as a bulk group.
 __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap,
                                                   const void* src, int c0,

@@ -177,6 +177,12 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads (TMA stores, tensor-core operand reads).
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Release store / acquire load of a shared-memory word (a flag one thread
 // publishes and another polls).
 __device__ __forceinline__ void st_release_shared(uint32_t* p, uint32_t v) {
