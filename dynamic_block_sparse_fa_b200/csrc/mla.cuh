@@ -19,9 +19,12 @@
 //               B = the quarter's value columns, MN-major)
 //   warps 2..5  one thread per head (TMEM lane): Q into TMEM, row max,
 //               vote, exp, P, lazy O rescale, epilogue
-// Tensor memory: Q [0, 288) (bf16 pairs), S [320, 384) (P over its first 32
-// columns), O [384, 512).  Per block the steps run in order (S, decision,
-// P, P.V); the producer keeps the next block in flight.
+// Tensor memory: Q [0, 288) (bf16 pairs), P [288, 320), S [320, 384),
+// O [384, 512).  P has columns of its own, so S(j+1) is issued as soon as
+// the head threads have read S(j) (B_SR) and runs during the vote and the
+// exp of block j; P.V(j) follows it, and the head threads wait for that
+// P.V (B_PVD) before they write the next P or rescale O.  A ring of 3
+// cache blocks keeps block j+2 in flight meanwhile.
 #pragma once
 
 #include "prefill.cuh"
@@ -50,22 +53,24 @@ struct MlaArgs {
 struct MlaCfg {
   static constexpr int BOX = 64 * 128;           // 64 rows x 128 bytes
   static constexpr int KBLOCK = 9 * BOX;         // 73728 bytes
-  static constexpr int NK = 2;
+  static constexpr int NK = 3;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_BAR = OFF_K + NK * KBLOCK;
-  static constexpr int B_KF = 0;   // [NK]
-  static constexpr int B_KE = 2;   // [NK]
-  static constexpr int B_QR = 4;   // Q in TMEM (one arrival per head warp)
-  static constexpr int B_SF = 5;   // S in TMEM
-  static constexpr int B_PF = 6;   // P written (kept blocks; per warp)
-  static constexpr int B_OD = 7;   // last MMA done
-  static constexpr int NBAR = 8;
+  static constexpr int B_KF = 0;       // [NK]
+  static constexpr int B_KE = NK;      // [NK]
+  static constexpr int B_QR = 2 * NK;  // Q in TMEM (one arrival per head warp)
+  static constexpr int B_SF = B_QR + 1;   // S in TMEM
+  static constexpr int B_SR = B_SF + 1;   // S read (one arrival per head warp)
+  static constexpr int B_PF = B_SR + 1;   // P written (kept blocks; per warp)
+  static constexpr int B_PVD = B_PF + 1;  // a P.V done
+  static constexpr int B_OD = B_PVD + 1;  // last MMA done
+  static constexpr int NBAR = B_OD + 1;
   static constexpr int R = 4;      // decision-word ring
   static constexpr int OFF_DEC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_TMEM = OFF_DEC + R * 4;
   static constexpr int SMEM = OFF_TMEM + 8;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
-  static constexpr uint32_t COL_Q = 0, COL_S = 320, COL_O = 384;
+  static constexpr uint32_t COL_Q = 0, COL_P = 288, COL_S = 320, COL_O = 384;
   static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
 };
 
@@ -97,7 +102,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     }
     mbar_init(&bar[C::B_QR], 4);
     mbar_init(&bar[C::B_SF], 1);
+    mbar_init(&bar[C::B_SR], 4);
     mbar_init(&bar[C::B_PF], 4);
+    mbar_init(&bar[C::B_PVD], 1);
     mbar_init(&bar[C::B_OD], 1);
     for (int i = 0; i < C::R; ++i) dec_word[i] = 0u;
     fence_mbar_init();
@@ -138,20 +145,34 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       constexpr uint32_t id_o = idesc_bf16(128, 128, 0, 1);
       const uint32_t aK = smem_u32(smem + C::OFF_K);
       bool ok = mbar_wait(&bar[C::B_QR], 0, kWaitMla, 0, 10);
-      int npv = 0;
-      for (int jj = 0; jj < nb && ok; ++jj) {
-        const int sl = jj % C::NK;
-        ok = mbar_wait(&bar[C::B_KF + sl], (jj / C::NK) & 1, kWaitMla, jj,
-                       11 + sl);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t kb = aK + sl * C::KBLOCK;
+      // S(jj) = Q c_jj^T into the S columns (36 TS products, K = 576)
+      auto score = [&](int jj) {
+        const uint32_t kb = aK + (jj % C::NK) * C::KBLOCK;
 #pragma unroll 4
         for (int k = 0; k < kMlaDqk / 16; ++k)
           mma_ts(tmem + C::COL_S, tmem + C::COL_Q + k * 8,
                  smem_desc(kb + (k >> 2) * C::BOX + (k & 3) * 32, 16, 1024, 2),
                  id_s, k > 0 ? 1u : 0u);
         mma_commit(&bar[C::B_SF]);
+      };
+      if (ok) {
+        ok = mbar_wait(&bar[C::B_KF], 0, kWaitMla, 0, 11);
+        tc_fence_after();
+        if (ok) score(0);
+      }
+      int npv = 0;
+      for (int jj = 0; jj < nb && ok; ++jj) {
+        const int sl = jj % C::NK;
+        if (jj + 1 < nb) {
+          // S(jj) has been read: the next block's score overwrites it
+          const int sn = (jj + 1) % C::NK;
+          ok = mbar_wait(&bar[C::B_SR], jj & 1, kWaitMla, jj, 16) &&
+               mbar_wait(&bar[C::B_KF + sn], ((jj + 1) / C::NK) & 1, kWaitMla,
+                         jj + 1, 11 + sn);
+          if (!ok) break;
+          tc_fence_after();
+          score(jj + 1);
+        }
         // the tile's decision on this block (published after the vote)
         const uint32_t want = (uint32_t)(jj + 1) << 1;
         uint32_t w = ld_acquire_shared(&dec_word[jj % C::R]);
@@ -170,13 +191,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           ok = mbar_wait(&bar[C::B_PF], npv & 1, kWaitMla, jj, 14);
           if (!ok) break;
           tc_fence_after();
+          const uint32_t kb = aK + sl * C::KBLOCK;
 #pragma unroll
           for (int k = 0; k < kMlaBc / 16; ++k)
-            mma_ts(tmem + C::COL_O, tmem + C::COL_S + k * 8,
+            mma_ts(tmem + C::COL_O, tmem + C::COL_P + k * 8,
                    smem_desc(kb + (2 * part) * C::BOX + k * 2048, C::BOX, 1024,
                              2),
                    id_o, (npv > 0 || k > 0) ? 1u : 0u);
           ++npv;
+          mma_commit(&bar[C::B_PVD]);
         }
         mma_commit(&bar[C::B_KE + sl]);
       }
@@ -221,14 +244,19 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     float m_crit = -INFINITY, m_ref = -INFINITY, l = 0.f;
     unsigned long long n_vis = 0, n_skp = 0;
     bool ok = true;
+    int npv = 0;         // kept blocks so far (one P.V each)
+    bool wfail = false;  // a P.V wait gave up: leave at the next vote
     for (int jj = 0; jj < nb; ++jj) {
       const int j = j0 + jj;
-      const bool w = mbar_wait(&bar[C::B_SF], jj & 1, kWaitMla, jj, 20);
+      const bool w = mbar_wait(&bar[C::B_SF], jj & 1, kWaitMla, jj, 20) && !wfail;
       tc_fence_after();
       uint32_t sr[2][32];
       tmem_ld32(lane_base + C::COL_S, sr[0]);
       tmem_ld32(lane_base + C::COL_S + 32, sr[1]);
       tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[C::B_SR]);  // S(jj+1) may overwrite S
       const int valid = min(kMlaBc, a.L - j * kMlaBc);  // keys of the block
       if (valid < kMlaBc) {
 #pragma unroll
@@ -269,6 +297,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         if (active) m_crit = fmaxf(m_crit, mt_s);
         continue;
       }
+      // P and O are free once the previous P.V is done
+      if (npv > 0 && !mbar_wait(&bar[C::B_PVD], (npv - 1) & 1, kWaitMla, jj, 22))
+        wfail = true;
+      tc_fence_after();
       float alpha = 1.f;
       bool rescale = false;
       if (active && mt_s != -INFINITY) {
@@ -294,11 +326,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           rs += p0 + p1;
           pk[x / 2] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(lane_base + C::COL_S + c * 16, pk);
+        tmem_st16(lane_base + C::COL_P + c * 16, pk);
       }
       l = alpha * l + rs;
       tc_wait_st();
-      // O is idle here (S of this block arrived after the previous P.V)
       if (__any_sync(FULL, rescale)) {
         const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
@@ -316,6 +347,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[C::B_PF]);
+      ++npv;
       if (active) m_crit = fmaxf(m_crit, mt_s);
     }
     if (ok && elected && recorder && a.counters && nb > 0) {
