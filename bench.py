@@ -665,8 +665,9 @@ def run_mla(args, bl, dev, stream, hbm_peak, tf_peak):
         byts = (B * L * dqk * 2 + B * H * dqk * 2 + 2 * B * H * S * (dv + 1) * 4
                 + B * H * (dv * 2 + 4))
         kept = (1.0 - sp) * B * nk
-        # tensor work issued: 4 CTAs score each block, one P.V quarter each
-        issued = (4 * 2.0 * 128 * 64 * dqk * B * nk + 2.0 * 128 * 64 * dv * kept)
+        # tensor work issued: each block scored once (its 576 columns split
+        # over a CTA pair), P.V of kept blocks (512 value columns, split too)
+        issued = (2.0 * 128 * 64 * dqk * B * nk + 2.0 * 128 * 64 * dv * kept)
         out[key] = {"ln_lambda": l, "sparsity": sp, "us": round(ms * 1e3, 1),
                     "GBps": round(byts / (ms / 1e3) / 1e9, 1),
                     "hbm_frac": round(byts / (ms / 1e3) / 1e9 / hbm_peak, 4),

@@ -636,13 +636,22 @@ blasst_status_t blasst_decode_wide(const void* q, const void* k_cache,
 int blasst_mla_decode_splits(int B, int L) {
   if (B < 1 || L < 1) return 1;
   const long long nk = (L + (long long)blasst::kMlaBc - 1) / blasst::kMlaBc;
-  // about two waves of one CTA per SM (4 value quarters per split), at
-  // least 8 blocks per split
-  const long long per = (long long)B * blasst::kMlaParts;
-  long long s = (2LL * kNumSmB200 + per - 1) / per;
+  const long long per = 2LL * B;  // a cluster pair of CTAs per split
+  // one CTA per SM: the split count with the least time in waves of SMs
+  // (waves / splits), among those of at most two waves and 8 blocks or
+  // more per split; the smaller on a tie (fewer partials to merge)
   const long long s_max = nk / 8 > 1 ? nk / 8 : 1;
-  if (s > s_max) s = s_max;
-  return (int)(s < 1 ? 1 : s);
+  long long best = 1;
+  double best_cost = 1e30;
+  for (long long s = 1; s <= s_max && per * s <= 2LL * kNumSmB200; ++s) {
+    const long long waves = (per * s + kNumSmB200 - 1) / kNumSmB200;
+    const double cost = (double)waves / (double)s;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return (int)best;
 }
 
 size_t blasst_mla_decode_workspace_size(int B, int H, int num_splits) {
@@ -671,7 +680,7 @@ blasst_status_t blasst_mla_decode(const void* q, const void* cache, void* o,
   const int nk = (L + blasst::kMlaBc - 1) / blasst::kMlaBc;
   const int S = num_splits == 0 ? blasst_mla_decode_splits(B, L) : num_splits;
   if (S < 1 || S > nk) return BLASST_ERR_INVALID_ARG;
-  const long long grid = (long long)B * S * blasst::kMlaParts;
+  const long long grid = 2LL * B * S;  // cluster pairs
   if (grid > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED_SHAPE;
   const bool stats_only = (o == nullptr);
   blasst::MlaArgs a;
@@ -701,12 +710,12 @@ blasst_status_t blasst_mla_decode(const void* q, const void* cache, void* o,
   a.ln_lambda = ln_lambda;
   a.stats_only = stats_only ? 1 : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaFuncSetAttribute(blasst::mla_split_kernel,
+  cudaError_t e = cudaFuncSetAttribute(blasst::mla_pair_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       blasst::MlaCfg::SMEM_ALLOC);
+                                       blasst::MlaPairCfg::SMEM_ALLOC);
   if (e != cudaSuccess) return cuda_status(e, "mla attribute");
-  blasst::mla_split_kernel<<<(unsigned)grid, blasst::kMlaThreads,
-                             blasst::MlaCfg::SMEM_ALLOC, st>>>(a);
+  blasst::mla_pair_kernel<<<(unsigned)grid, blasst::kMlaPairThreads,
+                            blasst::MlaPairCfg::SMEM_ALLOC, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess || stats_only) return cuda_status(e, "mla split launch");
   blasst::mla_combine_kernel<<<(unsigned)((long long)B * H), 128, 0, st>>>(

@@ -8,23 +8,27 @@
 // the decode criterion and online softmax per split, split-KV merged by
 // log-sum-exp: the same algorithm as decode.cuh with K = c and V = c[:512].
 //
-// One CTA per (sequence, split, value quarter): the 512 value columns are
-// cut into 4 quarters of 128 so that a CTA's output fits in tensor memory
-// next to Q; the 4 CTAs of a (sequence, split) score the same blocks (the
-// second to fourth read them from L2) and take identical decisions.
-//   warp 0      TMA producer: cache blocks [64 keys x 576] (9 boxes of 64
-//               columns), ring of 2
-//   warp 1      MMA issuer (one lane): S = Q c^T (TS: A = Q from TMEM),
-//               then, for a kept block, O += P V (TS: A = P from TMEM,
-//               B = the quarter's value columns, MN-major)
-//   warps 2..5  one thread per head (TMEM lane): Q into TMEM, row max,
-//               vote, exp, P, lazy O rescale, epilogue
-// Tensor memory: Q [0, 288) (bf16 pairs), P [288, 320), S [320, 384),
-// O [384, 512).  P has columns of its own, so S(j+1) is issued as soon as
-// the head threads have read S(j) (B_SR) and runs during the vote and the
-// exp of block j; P.V(j) follows it, and the head threads wait for that
-// P.V (B_PVD) before they write the next P or rescale O.  A ring of 3
-// cache blocks keeps block j+2 in flight meanwhile.
+// One CTA pair (a cluster of 2) per (sequence, split), the work cut so that
+// no cache byte is loaded twice and no score product is issued twice:
+//   rank 0 scores columns [0, 256) of c_t (4 boxes of 64) and accumulates
+//          value columns [0, 256): the same 4 boxes;
+//   rank 1 scores columns [256, 576) (5 boxes) and accumulates value
+//          columns [256, 512): the first 4 of its boxes.
+// Each CTA's head threads read their partial scores from tensor memory,
+// store them into the other CTA's shared memory (distributed shared memory,
+// as [4-key group][head] float4s so that a warp's stores are contiguous),
+// and add the other CTA's partial to their own.  IEEE addition commutes, so
+// both CTAs hold the same scores bit for bit and take the same decisions
+// without exchanging them.
+//   warp 0      TMA producer: this rank's boxes of each cache block, ring of 3
+//   warp 1      MMA issuer (one lane): partial S = Q_r c_r^T (TS, 16 or 20
+//               products, N = 64), issued as soon as the previous S has been
+//               read; for a kept block O_r += P V_r (TS, 4 products, N = 256)
+//   warps 2..5  one thread per head (TMEM lane): Q_r into TMEM, partial
+//               score exchange, row max, vote, exp, P, lazy O rescale,
+//               epilogue
+// Tensor memory: Q_r [0, 160) (bf16 pairs), P [160, 192), S [192, 256),
+// O_r [256, 512).
 #pragma once
 
 #include "prefill.cuh"
@@ -34,9 +38,7 @@ namespace blasst {
 constexpr int kMlaDqk = 576;
 constexpr int kMlaDv = 512;
 constexpr int kMlaBc = 64;
-constexpr int kMlaParts = 4;   // value quarters of 128 columns
 constexpr int kMlaRows = 128;  // heads per tile (at most)
-constexpr int kMlaThreads = 192;
 
 struct MlaArgs {
   CUtensorMap tc;            // cache [B][L][576], box 64 x 64
@@ -50,47 +52,56 @@ struct MlaArgs {
   int stats_only;
 };
 
-struct MlaCfg {
-  static constexpr int BOX = 64 * 128;           // 64 rows x 128 bytes
-  static constexpr int KBLOCK = 9 * BOX;         // 73728 bytes
-  static constexpr int NK = 3;
+constexpr int kMlaPairThreads = 192;
+
+struct MlaPairCfg {
+  static constexpr int BOX = 64 * 128;        // 64 keys x 64 columns (bf16)
+  static constexpr int NBX = 5;               // boxes per ring slot (rank 1)
+  static constexpr int SLOT = NBX * BOX;      // 40960 bytes
+  static constexpr int NK = 3;                // ring slots
+  static constexpr int XBYTES = 64 * 128 * 4; // a partial score block, f32
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_BAR = OFF_K + NK * KBLOCK;
-  static constexpr int B_KF = 0;       // [NK]
-  static constexpr int B_KE = NK;      // [NK]
-  static constexpr int B_QR = 2 * NK;  // Q in TMEM (one arrival per head warp)
-  static constexpr int B_SF = B_QR + 1;   // S in TMEM
-  static constexpr int B_SR = B_SF + 1;   // S read (one arrival per head warp)
-  static constexpr int B_PF = B_SR + 1;   // P written (kept blocks; per warp)
-  static constexpr int B_PVD = B_PF + 1;  // a P.V done
-  static constexpr int B_OD = B_PVD + 1;  // last MMA done
-  static constexpr int NBAR = B_OD + 1;
-  static constexpr int R = 4;      // decision-word ring
+  static constexpr int OFF_X = OFF_K + NK * SLOT;  // [2] partials from the peer
+  static constexpr int OFF_BAR = OFF_X + 2 * XBYTES;
+  static constexpr int B_KF = 0;            // [NK]
+  static constexpr int B_KE = NK;           // [NK]
+  static constexpr int B_QR = 2 * NK;       // Q in TMEM (per head warp)
+  static constexpr int B_SF = B_QR + 1;     // partial S in TMEM
+  static constexpr int B_SR = B_SF + 1;     // partial S read (per head warp)
+  static constexpr int B_PF = B_SR + 1;     // P written (per head warp)
+  static constexpr int B_PVD = B_PF + 1;    // a P.V done
+  static constexpr int B_OD = B_PVD + 1;    // last MMA done
+  static constexpr int B_XF = B_OD + 1;     // [2] my X[b] holds the peer's partial
+  static constexpr int NBAR = B_XF + 2;
+  static constexpr int R = 4;               // decision-word ring
   static constexpr int OFF_DEC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_TMEM = OFF_DEC + R * 4;
   static constexpr int SMEM = OFF_TMEM + 8;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
-  static constexpr uint32_t COL_Q = 0, COL_P = 288, COL_S = 320, COL_O = 384;
+  static constexpr uint32_t COL_Q = 0, COL_P = 160, COL_S = 192, COL_O = 256;
   static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
 };
 
-__global__ void __launch_bounds__(kMlaThreads, 1)
-    mla_split_kernel(const __grid_constant__ MlaArgs a) {
-  using C = MlaCfg;
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaPairThreads, 1)
+    mla_pair_kernel(const __grid_constant__ MlaArgs a) {
+  using C = MlaPairCfg;
   constexpr unsigned FULL = 0xffffffffu;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int part = blockIdx.x % kMlaParts;
-  const int bs = blockIdx.x / kMlaParts;  // b * S + s
+  const uint32_t rank = cluster_rank();
+  const uint32_t peer = rank ^ 1u;
+  const int bs = blockIdx.x >> 1;  // b * S + s
   const int s = bs % a.S;
   const int b = bs / a.S;
   const int j0 = (int)(((long long)s * a.nk) / a.S);
   const int j1 = (int)(((long long)(s + 1) * a.nk) / a.S);
   const int nb = j1 - j0;
-  const bool recorder = part == 0;  // one CTA of the four records stats
+  const int box0 = rank ? 4 : 0;  // first cache box (64 columns) of mine
+  const int nbx = rank ? 5 : 4;   // boxes I score
+  const bool recorder = rank == 0;
 
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint32_t* dec_word = reinterpret_cast<uint32_t*>(smem + C::OFF_DEC);
@@ -106,15 +117,20 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     mbar_init(&bar[C::B_PF], 4);
     mbar_init(&bar[C::B_PVD], 1);
     mbar_init(&bar[C::B_OD], 1);
+    // X[b]'s phases: one arrival (this CTA arming the phase with the bytes
+    // it expects) plus the peer's 32 KB of st.async transactions
+    for (int i = 0; i < 2; ++i) mbar_init(&bar[C::B_XF + i], 1);
     for (int i = 0; i < C::R; ++i) dec_word[i] = 0u;
     fence_mbar_init();
+    for (int i = 0; i < 2; ++i) mbar_arrive_expect_tx(&bar[C::B_XF + i], C::XBYTES);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  // both CTAs' barriers are initialised before either arrives remotely
+  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const bool stats_only = a.stats_only != 0;
@@ -122,19 +138,20 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA
     if (lane == 0) {
-      const uint64_t pol = policy_evict_last();  // read by the 4 quarters
+      const uint64_t pol = policy_evict_first();  // each box is read once
       prefetch_tmap(&a.tc);
       for (int jj = 0; jj < nb; ++jj) {
         const int sl = jj % C::NK;
         if (jj >= C::NK &&
             !mbar_wait(&bar[C::B_KE + sl], ((jj / C::NK) - 1) & 1,
-                       kWaitMla, jj, sl))
+                       kWaitMlaPair, jj, sl))
           break;
-        mbar_arrive_expect_tx(&bar[C::B_KF + sl], C::KBLOCK);
+        mbar_arrive_expect_tx(&bar[C::B_KF + sl], nbx * C::BOX);
 #pragma unroll 1
-        for (int c = 0; c < 9; ++c)
-          tma_load_3d(smem + C::OFF_K + sl * C::KBLOCK + c * C::BOX, &a.tc,
-                      &bar[C::B_KF + sl], c * 64, (j0 + jj) * kMlaBc, b, pol);
+        for (int c = 0; c < nbx; ++c)
+          tma_load_3d(smem + C::OFF_K + sl * C::SLOT + c * C::BOX, &a.tc,
+                      &bar[C::B_KF + sl], (box0 + c) * 64, (j0 + jj) * kMlaBc,
+                      b, pol);
       }
     }
     __syncwarp();
@@ -142,45 +159,42 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // ------------------------------------------------------------ MMA
     if (lane == 0 && nb > 0) {
       constexpr uint32_t id_s = idesc_bf16(128, kMlaBc, 0, 0);
-      constexpr uint32_t id_o = idesc_bf16(128, 128, 0, 1);
+      constexpr uint32_t id_o = idesc_bf16(128, 256, 0, 1);
       const uint32_t aK = smem_u32(smem + C::OFF_K);
-      bool ok = mbar_wait(&bar[C::B_QR], 0, kWaitMla, 0, 10);
-      // S(jj) = Q c_jj^T into the S columns (36 TS products, K = 576)
+      const int nmma = nbx * 4;  // K = 64 columns per box, 16 per product
       auto score = [&](int jj) {
-        const uint32_t kb = aK + (jj % C::NK) * C::KBLOCK;
+        const uint32_t kb = aK + (jj % C::NK) * C::SLOT;
 #pragma unroll 4
-        for (int k = 0; k < kMlaDqk / 16; ++k)
+        for (int k = 0; k < nmma; ++k)
           mma_ts(tmem + C::COL_S, tmem + C::COL_Q + k * 8,
                  smem_desc(kb + (k >> 2) * C::BOX + (k & 3) * 32, 16, 1024, 2),
                  id_s, k > 0 ? 1u : 0u);
         mma_commit(&bar[C::B_SF]);
       };
-      if (ok) {
-        ok = mbar_wait(&bar[C::B_KF], 0, kWaitMla, 0, 11);
-        tc_fence_after();
-        if (ok) score(0);
-      }
+      bool ok = mbar_wait(&bar[C::B_QR], 0, kWaitMlaPair, 0, 10) &&
+                mbar_wait(&bar[C::B_KF], 0, kWaitMlaPair, 0, 11);
+      tc_fence_after();
+      if (ok) score(0);
       int npv = 0;
       for (int jj = 0; jj < nb && ok; ++jj) {
         const int sl = jj % C::NK;
         if (jj + 1 < nb) {
-          // S(jj) has been read: the next block's score overwrites it
+          // my partial S(jj) has been read: S(jj+1) overwrites it
           const int sn = (jj + 1) % C::NK;
-          ok = mbar_wait(&bar[C::B_SR], jj & 1, kWaitMla, jj, 16) &&
-               mbar_wait(&bar[C::B_KF + sn], ((jj + 1) / C::NK) & 1, kWaitMla,
-                         jj + 1, 11 + sn);
+          ok = mbar_wait(&bar[C::B_SR], jj & 1, kWaitMlaPair, jj, 16) &&
+               mbar_wait(&bar[C::B_KF + sn], ((jj + 1) / C::NK) & 1,
+                         kWaitMlaPair, jj + 1, 11 + sn);
           if (!ok) break;
           tc_fence_after();
           score(jj + 1);
         }
-        // the tile's decision on this block (published after the vote)
         const uint32_t want = (uint32_t)(jj + 1) << 1;
         uint32_t w = ld_acquire_shared(&dec_word[jj % C::R]);
         if ((w & ~1u) != want) {
           const long long t0 = clock64();
           while (((w = ld_acquire_shared(&dec_word[jj % C::R])) & ~1u) != want) {
             if (clock64() - t0 > kWaitLimitCycles) {
-              record_error(kWaitMla, jj, 0, 13);
+              record_error(kWaitMlaPair, jj, 0, 13);
               ok = false;
               break;
             }
@@ -188,16 +202,16 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           if (!ok) break;
         }
         if (!stats_only && (w & 1u) == 0) {
-          ok = mbar_wait(&bar[C::B_PF], npv & 1, kWaitMla, jj, 14);
+          ok = mbar_wait(&bar[C::B_PF], npv & 1, kWaitMlaPair, jj, 14);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t kb = aK + sl * C::KBLOCK;
+          // my 256 value columns: the slot's first 4 boxes, MN-major
+          const uint32_t kb = aK + sl * C::SLOT;
 #pragma unroll
           for (int k = 0; k < kMlaBc / 16; ++k)
             mma_ts(tmem + C::COL_O, tmem + C::COL_P + k * 8,
-                   smem_desc(kb + (2 * part) * C::BOX + k * 2048, C::BOX, 1024,
-                             2),
-                   id_o, (npv > 0 || k > 0) ? 1u : 0u);
+                   smem_desc(kb + k * 2048, C::BOX, 1024, 2), id_o,
+                   (npv > 0 || k > 0) ? 1u : 0u);
           ++npv;
           mma_commit(&bar[C::B_PVD]);
         }
@@ -213,15 +227,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     const bool active = h < a.H;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const bool elected = (quad == 0 && lane == 0);
-    // Q row into TMEM [0, 288): 9 chunks of 64 bf16 (32 columns)
+    // my part of the Q row into TMEM: nbx chunks of 64 bf16 (32 columns);
+    // padding rows (h >= H) read head 0's row and store zeros (no branch
+    // before the warp-collective TMEM stores)
     {
-      // padding rows (h >= H) read head 0's row and store zeros: no branch
-      // before the warp-collective TMEM stores
       const uint4* qrow = reinterpret_cast<const uint4*>(
-          a.q + ((size_t)b * a.H + (active ? h : 0)) * kMlaDqk);
+          a.q + ((size_t)b * a.H + (active ? h : 0)) * kMlaDqk) + box0 * 8;
       const uint32_t keep = active ? 0xffffffffu : 0u;
 #pragma unroll 1
-      for (int c = 0; c < 9; ++c) {
+      for (int c = 0; c < nbx; ++c) {
         uint32_t r[32];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -239,16 +253,25 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[C::B_QR]);
     }
+    // the exchange buffers: mine (written by the peer) and the peer's.
+    // X[b] is written again (block jj+2) only after the peer has received
+    // my partial of block jj+1, which I send after reading X[b] for block
+    // jj: the two CTAs' steps interlock, so X[b] needs no "free" signal.
+    const uint32_t x_mine = smem_u32(smem + C::OFF_X);
+    const uint32_t x_peer = map_shared(x_mine, peer);
+    const uint32_t xf_peer = map_shared(smem_u32(&bar[C::B_XF]), peer);
+    const bool armer = quad == 0 && lane == 0;  // re-arms X[b]'s next phase
     const float scale = a.scale, ln_lambda = a.ln_lambda;
     const float sl2 = scale * kPrefLog2e;
     float m_crit = -INFINITY, m_ref = -INFINITY, l = 0.f;
     unsigned long long n_vis = 0, n_skp = 0;
     bool ok = true;
     int npv = 0;         // kept blocks so far (one P.V each)
-    bool wfail = false;  // a P.V wait gave up: leave at the next vote
+    bool wfail = false;  // a wait after the vote gave up: leave at the next one
     for (int jj = 0; jj < nb; ++jj) {
       const int j = j0 + jj;
-      const bool w = mbar_wait(&bar[C::B_SF], jj & 1, kWaitMla, jj, 20) && !wfail;
+      const int xb = jj & 1;
+      bool w = mbar_wait(&bar[C::B_SF], jj & 1, kWaitMlaPair, jj, 20) && !wfail;
       tc_fence_after();
       uint32_t sr[2][32];
       tmem_ld32(lane_base + C::COL_S, sr[0]);
@@ -257,6 +280,34 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[C::B_SR]);  // S(jj+1) may overwrite S
+      // my partial into the peer's X[xb] as [4-key group][head] float4s,
+      // counted on the peer's X[xb] barrier
+      const uint32_t xp = x_peer + xb * C::XBYTES + h * 16;
+#pragma unroll
+      for (int q4 = 0; q4 < 16; ++q4) {
+        const uint32_t* v = &sr[q4 >> 3][(q4 & 7) * 4];
+        st_async_v4(xp + q4 * 2048, v[0], v[1], v[2], v[3], xf_peer + xb * 8);
+      }
+      // the peer's partial, added to mine (the peer adds in the other
+      // order: the same sums)
+      if (!mbar_wait_cluster(&bar[C::B_XF + xb], (jj >> 1) & 1, kWaitMlaPair,
+                             jj, 32 + xb))
+        w = false;
+      // X[xb]'s phase for block jj is complete (this thread has seen it):
+      // arm the phase of block jj+2
+      if (armer && jj + 2 < nb)
+        mbar_arrive_expect_tx(&bar[C::B_XF + xb], C::XBYTES);
+      const float4* xm =
+          reinterpret_cast<const float4*>(smem + C::OFF_X + xb * C::XBYTES) + h;
+#pragma unroll
+      for (int q4 = 0; q4 < 16; ++q4) {
+        const float4 o4 = xm[q4 * 128];
+        uint32_t* v = &sr[q4 >> 3][(q4 & 7) * 4];
+        v[0] = __float_as_uint(__uint_as_float(v[0]) + o4.x);
+        v[1] = __float_as_uint(__uint_as_float(v[1]) + o4.y);
+        v[2] = __float_as_uint(__uint_as_float(v[2]) + o4.z);
+        v[3] = __float_as_uint(__uint_as_float(v[3]) + o4.w);
+      }
       const int valid = min(kMlaBc, a.L - j * kMlaBc);  // keys of the block
       if (valid < kMlaBc) {
 #pragma unroll
@@ -298,7 +349,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         continue;
       }
       // P and O are free once the previous P.V is done
-      if (npv > 0 && !mbar_wait(&bar[C::B_PVD], (npv - 1) & 1, kWaitMla, jj, 22))
+      if (npv > 0 &&
+          !mbar_wait(&bar[C::B_PVD], (npv - 1) & 1, kWaitMlaPair, jj, 22))
         wfail = true;
       tc_fence_after();
       float alpha = 1.f;
@@ -333,7 +385,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       if (__any_sync(FULL, rescale)) {
         const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 8; ++c) {
           uint32_t orow[32];
           tmem_ld32(lane_base + C::COL_O + c * 32, orow);
           tc_wait_ld();
@@ -357,15 +409,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     if (ok && !stats_only) {
       const size_t row = (size_t)b * a.H + h;
       bool w2 = true;
-      if (nb > 0) w2 = mbar_wait(&bar[C::B_OD], 0, kWaitMla, nb, 21);
+      if (nb > 0) w2 = mbar_wait(&bar[C::B_OD], 0, kWaitMlaPair, nb, 21);
       tc_fence_after();
       // warp-wide: every lane takes part (padding heads included)
       const bool done = __all_sync(FULL, w2) && nb > 0;
       const bool have = done && l > 0.f;
       const float inv_l = have ? 1.f / l : 0.f;
-      float* dst = a.o_part + (row * a.S + s) * kMlaDv + part * 128;
+      float* dst = a.o_part + (row * a.S + s) * kMlaDv + rank * 256;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 8; ++c) {
         uint32_t orow[32];
         if (done) {
           tmem_ld32(lane_base + C::COL_O + c * 32, orow);
@@ -382,7 +434,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                      : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
-      if (active && part == 0)
+      if (active && rank == 0)
         a.lse_part[row * a.S + s] = have ? m_ref + __logf(l) : -INFINITY;
     }
   }
@@ -393,6 +445,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // the peer's stores and arrivals into this CTA's shared memory are over
+  // before either CTA exits
+  cluster_sync_all();
 }
 
 // lse = ln sum_s exp(lse_s), o = sum_s exp(lse_s - lse) o_s -> bf16.  One

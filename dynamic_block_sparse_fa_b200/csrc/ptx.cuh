@@ -29,6 +29,7 @@ enum : unsigned int {
   kWaitBackward = 14,
   kWaitMla = 15,
   kWaitDecodeWide = 16,
+  kWaitMlaPair = 17,
   kWaitSelfTest = 99,
   // Device-resident arguments found out of range (paged decode); these are
   // reported as invalid arguments, not as waits that gave up.
@@ -113,6 +114,76 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     }
   }
   return true;
+}
+
+// The same wait with cluster-scope acquire: for phases completed by the
+// other CTA of a cluster (remote arrivals that release its writes into this
+// CTA's shared memory).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar,
+                                                      uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(
+    uint64_t* bar, uint32_t parity, unsigned int where,
+    unsigned int step = 0xffffffffu, unsigned int slot = 0,
+    long long limit = kWaitLimitCycles) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  long long t0 = clock64();
+  while (!mbar_try_wait_cluster(bar, parity)) {
+    if (clock64() - t0 > limit) {
+      record_error(where, step, parity, slot);
+      return false;
+    }
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// Thread-block clusters: rank, the peer's shared-memory addresses, remote
+// stores, and the cluster-wide barrier.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address in CTA `rank`'s shared memory of this CTA's shared address `a`.
+__device__ __forceinline__ uint32_t map_shared(uint32_t a, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(r)
+               : "r"(a), "r"(rank));
+  return r;
+}
+
+// 16 bytes into another CTA's shared memory (mapped address `a`), counted
+// as transaction bytes on that CTA's barrier `bar_cluster` (mapped), which
+// then needs no arrival from the writer.
+__device__ __forceinline__ void st_async_v4(uint32_t a, uint32_t x, uint32_t y,
+                                            uint32_t z, uint32_t w,
+                                            uint32_t bar_cluster) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], "
+      "{%1, %2, %3, %4}, [%5];" ::"r"(a),
+      "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar_cluster)
+      : "memory");
+}
+
+// Every thread of every CTA of the cluster.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
