@@ -116,6 +116,26 @@ def test_split_policy_and_workspace(lib):
     assert ws >= rows * 129 * 4 and ws % 256 == 0
 
 
+def test_mla_split_policy(lib):
+    """One CTA pair per (sequence, split), one CTA per SM: the count with the
+    fewest SM waves per split, at most two waves, 8 blocks per split or
+    more, the smaller on a tie."""
+    import math
+    import dynamic_block_sparse_fa_b200 as m
+    assert m.blasst_mla_decode_splits(32, 32768) == 2    # 128 CTAs, one wave
+    assert m.blasst_mla_decode_splits(74, 32768) == 1    # 148 CTAs, one wave
+    assert m.blasst_mla_decode_splits(200, 32768) == 1   # above two waves
+    assert m.blasst_mla_decode_splits(1, 32768) == 64    # capped at nk / 8
+    assert m.blasst_mla_decode_splits(1, 640) == 1       # 10 blocks
+    for B, L in [(1, 10 ** 6), (3, 4096), (16, 65536), (37, 9000)]:
+        s = m.blasst_mla_decode_splits(B, L)
+        nk = -(-L // 64)
+        assert 1 <= s <= max(1, nk // 8)
+        best = min(math.ceil(2 * B * t / 148) / t
+                   for t in range(1, max(1, nk // 8) + 1) if 2 * B * t <= 296)
+        assert math.ceil(2 * B * s / 148) / s == pytest.approx(best)
+
+
 def test_fit_a_and_strings(lib):
     import dynamic_block_sparse_fa_b200 as m
     assert m.blasst_fit_a([50 / 4096, 50 / 65536], [4096, 65536]) == \
