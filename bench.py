@@ -620,13 +620,14 @@ def run_mqa(args, bl, dev, stream, hbm_peak):
 
 
 def run_mla(args, bl, dev, stream, hbm_peak, tf_peak):
-    """MLA decode: B 32 tokens x 128 heads against a 32K-key latent cache
-    (576 wide, value = first 512 columns), planted-gap rows; dense and at the
-    ln lambda (bisection over statistics-only passes) that skips ~50%.
+    """MLA decode: B 32 tokens x 128 heads against a latent cache of
+    --mla-len keys (32K by default; 576 wide, value = first 512 columns),
+    planted-gap rows; dense and at the ln lambda (bisection over
+    statistics-only passes) that skips ~50%.
     Algorithmic bytes = the cache (read once; the value is part of the row)
     + q + split partials written and read + o and lse."""
     from synth import config_seed, planted_gap_kv_inplace
-    B, H, L, dqk, dv = 32, 128, 32768, 576, 512
+    B, H, L, dqk, dv = 32, 128, args.mla_len, 576, 512
     q = torch.empty(B, H, dqk, dtype=torch.bfloat16, device=dev)
     c4 = torch.empty(B, 1, L, dqk, dtype=torch.bfloat16, device=dev)
     planted_gap_kv_inplace(c4, torch.empty_like(c4), q, block=64, gap=8.0,
@@ -905,6 +906,8 @@ def main():
                     help="skip the sliding-window measurements")
     ap.add_argument("--no-mla", action="store_true",
                     help="skip the MLA decode measurements")
+    ap.add_argument("--mla-len", type=int, default=32768,
+                    help="latent rows per sequence in the MLA decode leg")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the prefill backward measurements")
     ap.add_argument("--no-paged", action="store_true",
