@@ -4,8 +4,9 @@ MLA decode, through the C ABI.
 The H query heads of a token score one shared latent row per key (d_qk =
 576) and take its first 512 columns as value.  Checks outputs (max 2e-2 /
 mean 2e-3), lse, masks [B, nk] bit-exact except near-ties, counters, the
-statistics-only pass, fewer heads than the tile's 128 rows, ragged caches,
-automatic and explicit split counts, and argument checks.
+statistics-only pass, fewer heads than the tile's 128 rows (down to one,
+and a warp that mixes real and padding heads), ragged caches, automatic and
+explicit split counts, and argument checks.
 """
 import math
 
@@ -41,6 +42,8 @@ MLA_CASES = [
     (3, 128, 65, -1.0, 2),       # two blocks, the second holds one key
     (1, 128, 4096, -4.0, 0),
     (2, 32, 1500, 0.0, 5),
+    (1, 1, 300, -2.0, 0),        # one head: 127 padding rows
+    (2, 100, 2000, -3.0, 0),     # a warp of real and padding heads
 ]
 
 
