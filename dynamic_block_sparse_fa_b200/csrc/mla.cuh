@@ -15,9 +15,10 @@
 //   rank 1 scores columns [256, 576) (5 boxes) and accumulates value
 //          columns [256, 512): the first 4 of its boxes.
 // Each CTA's head threads read their partial scores from tensor memory,
-// store them into the other CTA's shared memory (distributed shared memory,
-// as [4-key group][head] float4s so that a warp's stores are contiguous),
-// and add the other CTA's partial to their own.  IEEE addition commutes, so
+// store them into the other CTA's shared memory with st.async (distributed
+// shared memory, as [4-key group][head] float4s so that a warp's stores are
+// contiguous, counted as transaction bytes on the other CTA's barrier), and
+// add the other CTA's partial to their own.  IEEE addition commutes, so
 // both CTAs hold the same scores bit for bit and take the same decisions
 // without exchanging them.
 //   warp 0      TMA producer: this rank's boxes of each cache block, ring of 3
