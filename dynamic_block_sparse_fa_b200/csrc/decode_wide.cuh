@@ -120,6 +120,8 @@ __global__ void __launch_bounds__(kWideThreads, 2)
     mbar_init(&bar[C::B_PVD], 1);
     mbar_init(&bar[C::B_OD], 1);
     for (int i = 0; i < C::R; ++i) dec_word[i] = 0u;
+    // a wait that gave up in any head thread, read by all after the vote
+    *reinterpret_cast<volatile int*>(smem + C::OFF_TMEM + 4) = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -310,9 +312,11 @@ __global__ void __launch_bounds__(kWideThreads, 2)
       const bool pred = !active || mt_s == -INFINITY ||
                         (mt_s - m_crit < ln_lambda);
       tc_fence_before();
-      // a failed wait in any thread ends the loop for all, at a barrier
+      // a failed wait in any thread ends the loop for all, after the vote
+      volatile int* abort_w = reinterpret_cast<volatile int*>(smem + C::OFF_TMEM + 4);
+      if (!w) *abort_w = 1;
       const bool all = named_sync_and(1, 128, pred && w);
-      if (!named_sync_and(1, 128, w)) { ok = false; break; }
+      if (*abort_w) { ok = false; break; }
       const bool skip = all && (ln_lambda > -INFINITY);
       if (elected) {
         st_release_shared(&dec_word[jj % C::R],

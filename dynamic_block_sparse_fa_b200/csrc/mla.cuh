@@ -122,6 +122,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaPairThreads, 1)
     // it expects) plus the peer's 32 KB of st.async transactions
     for (int i = 0; i < 2; ++i) mbar_init(&bar[C::B_XF + i], 1);
     for (int i = 0; i < C::R; ++i) dec_word[i] = 0u;
+    // a wait that gave up in any head thread, read by all after the vote
+    *reinterpret_cast<volatile int*>(smem + C::OFF_TMEM + 4) = 0;
     fence_mbar_init();
     for (int i = 0; i < 2; ++i) mbar_arrive_expect_tx(&bar[C::B_XF + i], C::XBYTES);
   }
@@ -333,10 +335,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaPairThreads, 1)
       const bool pred = !active || mt_s == -INFINITY ||
                         (mt_s - m_crit < ln_lambda);
       tc_fence_before();
-      // the vote also carries a failed wait: every thread then leaves
+      // a failed wait in any thread ends the loop for all, after the vote
+      volatile int* abort_w = reinterpret_cast<volatile int*>(smem + C::OFF_TMEM + 4);
+      if (!w) *abort_w = 1;
       const bool all = named_sync_and(1, 128, pred && w);
-      const bool any_fail = !named_sync_and(1, 128, w);
-      if (any_fail) { ok = false; break; }
+      if (*abort_w) { ok = false; break; }
       const bool skip = all && (ln_lambda > -INFINITY);
       if (elected) {
         st_release_shared(&dec_word[jj % C::R],
