@@ -424,8 +424,10 @@ blasst_status_t blasst_mla_decode(const void *q, const void *cache, void *o,
                                   void *stream);
 /* Bytes of MLA decode workspace (split outputs and their lse). */
 size_t blasst_mla_decode_workspace_size(int B, int H, int num_splits);
-/* The automatic MLA split count: about two waves of one CTA per SM (four
- * CTAs per split), at least 8 blocks per split. */
+/* The automatic MLA split count.  A split runs on a pair of CTAs (a cluster
+ * of 2, one CTA per SM); the count is the one with the fewest waves of SMs
+ * per split among counts of at most two waves and at least 8 blocks per
+ * split, the smaller on a tie. */
 int blasst_mla_decode_splits(int B, int L);
 
 /*

@@ -101,6 +101,85 @@ def test_decode_validation(lib):
     assert _decode(lib, ws=0x4000, ws_bytes=64) == 7   # too small
 
 
+def _mla(lib, q=0x1000, c=0x1000, o=0x2000, B=1, H=8, L=256, dqk=576,
+         dv=512, lnl=-1.0, S=1, ws=None, ws_bytes=0):
+    f = lib.blasst_mla_decode
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 5 + [
+        ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+        ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+    return f(q, c, o, None, B, H, L, dqk, dv, 0.04, lnl, S, ws, ws_bytes,
+             None, None)
+
+
+def test_mla_decode_validation(lib):
+    """Argument checks of blasst_mla_decode, all taken before any launch."""
+    assert _mla(lib, q=None) == 1
+    assert _mla(lib, B=0) == 1
+    assert _mla(lib, lnl=0.5) == 1                     # ln lambda > 0
+    assert _mla(lib, H=129) == 2                       # at most 128 heads
+    assert _mla(lib, dqk=512) == 2                     # d_qk 576 only
+    assert _mla(lib, dv=256) == 2                      # d_v 512 only
+    assert _mla(lib, c=0x1008) == 3                    # misaligned cache
+    assert _mla(lib, S=5) == 1                         # 4 blocks of 64 keys
+    assert _mla(lib) == 7                              # no workspace
+    need = 1 * 8 * 1 * (512 + 1) * 4
+    assert _mla(lib, ws=0x4004, ws_bytes=4 * need) == 3  # not 256-aligned
+
+
+def _wide(lib, q=0x1000, k=0x1000, v=0x1000, o=0x2000, B=1, Hq=32, Hkv=1,
+          Lkv=256, d=128, lnl=-1.0, Bc=64, S=1, ws=None, ws_bytes=0):
+    f = lib.blasst_decode_wide
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5 + [
+        ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+    return f(q, k, v, o, None, B, Hq, Hkv, Lkv, d, 0.088, lnl, Bc, S, ws,
+             ws_bytes, None, None)
+
+
+def test_decode_wide_validation(lib):
+    """Argument checks of blasst_decode_wide, all taken before any launch."""
+    assert _wide(lib, v=None) == 1
+    assert _wide(lib, Hq=12, Hkv=5) == 1               # Hq % Hkv
+    assert _wide(lib, lnl=float("nan")) == 1
+    assert _wide(lib, Hq=256) == 2                     # group above 128 heads
+    assert _wide(lib, d=64) == 2
+    assert _wide(lib, Bc=128) == 2
+    assert _wide(lib, q=0x1002) == 3
+    assert _wide(lib, S=5) == 1                        # 4 blocks of 64 keys
+    assert _wide(lib) == 7                             # no workspace
+
+
+def _bwd(lib, ptr=0x1000, dq=0x2000, B=1, Hq=4, Hkv=1, Lq=256, Lkv=256, d=128,
+         causal=1, Br=128, Bc=128, ws=None, ws_bytes=0):
+    f = lib.blasst_prefill_backward
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 10 + [ctypes.c_int] * 6 + [
+        ctypes.c_float] + [ctypes.c_int] * 3 + [
+        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    return f(ptr, ptr, ptr, ptr, ptr, ptr, None, dq, ptr, ptr, B, Hq, Hkv, Lq,
+             Lkv, d, 0.088, causal, Br, Bc, ws, ws_bytes, None)
+
+
+def test_prefill_backward_validation(lib):
+    """Argument checks of blasst_prefill_backward, before any launch."""
+    m_ws = lib.blasst_prefill_backward_workspace_size
+    m_ws.restype = ctypes.c_size_t
+    m_ws.argtypes = [ctypes.c_int] * 4
+    need = m_ws(1, 4, 256, 128)
+    assert need >= 4 * 256 * 128 * 4 and need % 256 == 0
+    assert _bwd(lib, dq=None) == 1
+    assert _bwd(lib, Hq=3, Hkv=2) == 1                 # Hq % Hkv
+    assert _bwd(lib, Lq=512) == 1                      # causal, Lq > Lkv
+    assert _bwd(lib, d=64) == 2                        # d 128 only
+    assert _bwd(lib, Br=64, Bc=64) == 2                # 128 x 128 only
+    assert _bwd(lib, dq=0x2004) == 3
+    assert _bwd(lib) == 7                              # no workspace
+    assert _bwd(lib, ws=0x4000, ws_bytes=need - 256) == 7
+    assert _bwd(lib, ws=0x4010, ws_bytes=need) == 3    # not 256-aligned
+
+
 def test_split_policy_and_workspace(lib):
     import dynamic_block_sparse_fa_b200 as m
     # batch 32 x 8 KV heads at 32K: 5 splits; batch 148: 1 split
