@@ -154,6 +154,23 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _arg(t, name, dtype=torch.bfloat16, contiguous=True):
+    """Device pointer of a tensor argument after checking what the C ABI
+    cannot see: a CUDA tensor, of the given dtype (None: any, for byte
+    workspaces), dense in memory (the ABI takes no strides)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor (got {t.device})")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -202,7 +219,8 @@ def blasst_last_error() -> str:
 
 
 def blasst_skip_stats_reset(counters: torch.Tensor, stream=None):
-    _check(_lib.blasst_skip_stats_reset(_ptr(counters), _stream(stream)),
+    _check(_lib.blasst_skip_stats_reset(_arg(counters, "counters", torch.int64),
+                                        _stream(stream)),
            "blasst_skip_stats_reset")
 
 
@@ -246,7 +264,8 @@ def blasst_prefill(q, k, v, *, scale=None, causal=True, ln_lambda=-math.inf,
     else:
         o, lse = None, None
     st = _lib.blasst_prefill_window(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lkv, d,
+        _arg(q, "q"), _arg(k, "k"), _arg(v, "v"), _arg(o, "o"),
+        _arg(lse, "lse", torch.float32), B, Hq, Hkv, Lq, Lkv, d,
         float(scale), int(bool(causal)), int(window), float(ln_lambda), Br, Bc,
         stats.c_struct if stats is not None else None, _stream(stream))
     _check(st, "blasst_prefill_window")
@@ -292,8 +311,10 @@ def blasst_mla_decode(q, cache, *, d_v=512, scale=None, ln_lambda=-math.inf,
     else:
         o, lse, workspace = None, None, None
     st = _lib.blasst_mla_decode(
-        _ptr(q), _ptr(cache), _ptr(o), _ptr(lse), B, H, L, dqk, d_v,
-        float(scale), float(ln_lambda), S, _ptr(workspace), ws_bytes,
+        _arg(q, "q"), _arg(cache, "cache"), _arg(o, "o"),
+        _arg(lse, "lse", torch.float32), B, H, L, dqk, d_v,
+        float(scale), float(ln_lambda), S, _arg(workspace, "workspace", None),
+        ws_bytes,
         stats.c_struct if stats is not None else None, _stream(stream))
     _check(st, "blasst_mla_decode")
     return o, lse
@@ -323,9 +344,12 @@ def blasst_prefill_backward(q, k, v, o, lse, dout, *, mask=None, scale=None,
                                 device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
     st = _lib.blasst_prefill_backward(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(mask),
-        _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, Lq, Lkv, d, float(scale),
-        int(bool(causal)), Br, Bc, _ptr(workspace), ws_bytes, _stream(stream))
+        _arg(q, "q"), _arg(k, "k"), _arg(v, "v"), _arg(o, "o"),
+        _arg(dout, "dout"), _arg(lse, "lse", torch.float32),
+        _arg(mask, "mask", torch.uint8), _arg(dq, "dq"), _arg(dk, "dk"),
+        _arg(dv, "dv"), B, Hq, Hkv, Lq, Lkv, d, float(scale),
+        int(bool(causal)), Br, Bc, _arg(workspace, "workspace", None), ws_bytes,
+        _stream(stream))
     _check(st, "blasst_prefill_backward")
     return dq, dk, dv
 
@@ -361,8 +385,10 @@ def blasst_decode_batched(q, k, v, *, batch=2, scale=None,
     else:
         o, lse, workspace = None, None, None
     st = _lib.blasst_decode_batched(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lkv, d,
-        float(scale), float(ln_lambda), Bc, S, int(batch), _ptr(workspace),
+        _arg(q, "q"), _arg(k, "k"), _arg(v, "v"), _arg(o, "o"),
+        _arg(lse, "lse", torch.float32), B, Hq, Hkv, Lkv, d,
+        float(scale), float(ln_lambda), Bc, S, int(batch),
+        _arg(workspace, "workspace", None),
         ws_bytes, stats.c_struct if stats is not None else None,
         _stream(stream))
     _check(st, "blasst_decode_batched")
@@ -405,8 +431,10 @@ def blasst_decode(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
     else:
         o, lse, workspace = None, None, None
     st = _lib.blasst_decode_window(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lkv, d,
-        float(scale), int(window), float(ln_lambda), Bc, S, _ptr(workspace),
+        _arg(q, "q"), _arg(k, "k"), _arg(v, "v"), _arg(o, "o"),
+        _arg(lse, "lse", torch.float32), B, Hq, Hkv, Lkv, d,
+        float(scale), int(window), float(ln_lambda), Bc, S,
+        _arg(workspace, "workspace", None),
         ws_bytes, stats.c_struct if stats is not None else None,
         _stream(stream))
     _check(st, "blasst_decode_window")
@@ -438,8 +466,10 @@ def blasst_decode_wide(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
     else:
         o, lse, workspace = None, None, None
     st = _lib.blasst_decode_wide(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lkv, d,
-        float(scale), float(ln_lambda), Bc, S, _ptr(workspace), ws_bytes,
+        _arg(q, "q"), _arg(k, "k"), _arg(v, "v"), _arg(o, "o"),
+        _arg(lse, "lse", torch.float32), B, Hq, Hkv, Lkv, d,
+        float(scale), float(ln_lambda), Bc, S,
+        _arg(workspace, "workspace", None), ws_bytes,
         stats.c_struct if stats is not None else None, _stream(stream))
     _check(st, "blasst_decode_wide")
     return o, lse
@@ -496,10 +526,13 @@ def blasst_decode_paged(q, k_pages, v_pages, block_table, seq_lens, *,
     else:
         o, lse, workspace = None, None, None
     st = _lib.blasst_decode_paged(
-        _ptr(q), _ptr(k_pages), _ptr(v_pages), int(k_pages.stride(0)), P, ps,
-        _ptr(block_table), max_pages, _ptr(seq_lens), int(max_seq_len),
-        _ptr(o), _ptr(lse), B, Hq, Hkv, d, float(scale), float(ln_lambda),
-        int(bool(per_length)), S, _ptr(workspace), ws_bytes,
+        _arg(q, "q"), _arg(k_pages, "k_pages", contiguous=False),
+        _arg(v_pages, "v_pages", contiguous=False), int(k_pages.stride(0)), P,
+        ps, _arg(block_table, "block_table", torch.int32), max_pages,
+        _arg(seq_lens, "seq_lens", torch.int32), int(max_seq_len),
+        _arg(o, "o"), _arg(lse, "lse", torch.float32), B, Hq, Hkv, d,
+        float(scale), float(ln_lambda), int(bool(per_length)), S,
+        _arg(workspace, "workspace", None), ws_bytes,
         stats.c_struct if stats is not None else None, _stream(stream))
     _check(st, "blasst_decode_paged")
     return o, lse
@@ -525,7 +558,8 @@ def blasst_decode_noalloc(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
     else:
         o, lse = None, None
     st = _lib.blasst_decode_noalloc(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lkv, d,
+        _arg(q, "q"), _arg(k, "k"), _arg(v, "v"), _arg(o, "o"),
+        _arg(lse, "lse", torch.float32), B, Hq, Hkv, Lkv, d,
         float(scale), float(ln_lambda), Bc, num_splits,
         stats.c_struct if stats is not None else None, _stream(stream))
     if st == 7:
@@ -551,12 +585,15 @@ def blasst_calibrate(target, *, mode, q, k, v, scale=None, causal=True,
         scale = 1.0 / math.sqrt(d)
     if counters is None:
         counters = torch.zeros(2, dtype=torch.int64, device=q.device)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _arg(t, n)
     smp = CalibSample(m, q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv,
                       Lq, Lkv, d, float(scale), int(bool(causal)), Br, Bc,
                       num_splits)
     res = CalibResult()
     st = _lib.blasst_calibrate(float(target), ctypes.byref(smp), float(tol),
-                               _ptr(counters), ctypes.byref(res),
+                               _arg(counters, "counters", torch.int64),
+                               ctypes.byref(res),
                                _stream(stream))
     if st != BLASST_OK and (st != 6 or raise_on_no_converge):
         _check(st, "blasst_calibrate")

@@ -180,6 +180,24 @@ def test_prefill_backward_validation(lib):
     assert _bwd(lib, ws=0x4010, ws_bytes=need) == 3    # not 256-aligned
 
 
+def test_binding_rejects_host_and_mistyped_tensors(lib):
+    """The binding passes raw device pointers, so it refuses before the call
+    what the C ABI cannot see: host tensors, wrong dtypes, non-tensors."""
+    import torch
+    import dynamic_block_sparse_fa_b200 as m
+    from dynamic_block_sparse_fa_b200 import blasst as b
+    q = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        m.blasst_prefill(q, q, q)
+    with pytest.raises(ValueError, match="CUDA"):
+        m.blasst_decode(q[:, :, 0].contiguous(), q, q)
+    with pytest.raises(TypeError, match="Tensor"):
+        b._arg([1, 2], "x")
+    assert b._arg(None, "x") is None
+    with pytest.raises(ValueError, match="CUDA"):
+        b._arg(torch.zeros(4, dtype=torch.float16), "x")
+
+
 def test_split_policy_and_workspace(lib):
     import dynamic_block_sparse_fa_b200 as m
     # batch 32 x 8 KV heads at 32K: 5 splits; batch 148: 1 split
