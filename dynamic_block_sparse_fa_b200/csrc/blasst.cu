@@ -457,22 +457,55 @@ static __device__ __align__(256) unsigned char
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
+// Per device: the context the address was looked up in, and the address.
+// The array moves when its module is loaded again (after cudaDeviceReset,
+// or in another context made current on the same device), so the address
+// is looked up again whenever the current context differs.
+void* g_noalloc_ctx[kMaxDevices] = {};
 void* g_noalloc_ptr[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn get_ctx_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault,
+                                &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+  }
+  return fn;
+}
 
 // Device address of g_noalloc_scratch on the current device.  In host code
 // the array's name only stands in for the symbol; its device address must be
-// asked of the runtime, once per device, with that device current.
+// asked of the runtime, with that device current: once per device and
+// context (the first call after the context was created, or re-created).
 blasst_status_t noalloc_scratch(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return BLASST_ERR_UNSUPPORTED_SHAPE;
+  CtxGetCurrentFn ctx_fn = get_ctx_fn();
+  if (!ctx_fn) {
+    snprintf(g_last_error, sizeof g_last_error,
+             "blasst_decode_noalloc: cuCtxGetCurrent is not available");
+    return BLASST_ERR_CUDA;
+  }
+  CUcontext ctx = nullptr;
+  if (ctx_fn(&ctx) != CUDA_SUCCESS) ctx = nullptr;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  if (!ctx || !g_noalloc_ptr[dev] || g_noalloc_ctx[dev] != (void*)ctx) {
+    // The runtime binds the device's primary context here if none is
+    // current yet, so the context is read again afterwards.
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(scratch)");
+    if (ctx_fn(&ctx) != CUDA_SUCCESS) ctx = nullptr;
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = (void*)ctx;
   }
   *out = g_noalloc_ptr[dev];
   return BLASST_OK;

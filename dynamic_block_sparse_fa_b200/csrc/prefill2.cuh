@@ -27,27 +27,13 @@
 
 #include "prefill.cuh"
 
-#ifndef BLASST_PREFILL2_NKS
-#define BLASST_PREFILL2_NKS 2
-#endif
-// Number of the four 32-column chunks of a kept score row whose exponentials
-// run on the FMA pipe (exp2_poly) instead of the MUFU pipe.
-#ifndef BLASST_PREFILL2_EXP_EMU
-#define BLASST_PREFILL2_EXP_EMU 0
-#endif
-// Threads per score row (1 or 2): with 2, each tile's softmax runs on 8
-// warps, each thread owning half of the row's score and output columns.
-#ifndef BLASST_PREFILL2_COL_SPLIT
-#define BLASST_PREFILL2_COL_SPLIT 1
-#endif
-
 namespace blasst {
 
 template <int D>
 struct Prefill2Cfg {
   static constexpr int BM = 128;
   static constexpr int BN = 128;
-  static constexpr int NKS = BLASST_PREFILL2_NKS;  // K ring depth
+  static constexpr int NKS = 2;  // K ring depth
   static constexpr int NVS = 2;
   static constexpr int R = 8;  // decision ring per tile (> NKS)
   static constexpr int BOX_Q = BM * 128;
@@ -71,13 +57,8 @@ struct Prefill2Cfg {
   static constexpr int OFF_DEC = OFF_BAR + NBAR * 8;  // int [2][R]
   static constexpr int OFF_TMEM = OFF_DEC + 2 * R * 4;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;      // int [2]
-  static constexpr int NH = BLASST_PREFILL2_COL_SPLIT;  // threads per row
-  static constexpr int WPT = 4 * NH;                  // softmax warps per tile
-  // row-part exchange buffers, needed only when a row is split (NH > 1)
-  static constexpr int XN = NH > 1 ? NH : 0;
-  static constexpr int OFF_XMAX = (OFF_ABORT + 8 + 15) & ~15;  // f32 [2][2][NH][128]
-  static constexpr int OFF_XSUM = OFF_XMAX + 2 * 2 * XN * 128 * 4;  // f32 [2][NH][128]
-  static constexpr int SMEM = OFF_XSUM + 2 * XN * 128 * 4;
+  static constexpr int WPT = 4;  // softmax warps per tile (thread = row)
+  static constexpr int SMEM = OFF_ABORT + 8;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
   static constexpr int TMEM_COLS = 512;
   static constexpr int COL_S = 0;    // tile t at COL_S + t * 128
@@ -87,7 +68,7 @@ struct Prefill2Cfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1)
+__global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
     prefill2_kernel(const __grid_constant__ PrefillParams p) {
   using C = Prefill2Cfg<D>;
   constexpr int BN = C::BN;
@@ -359,17 +340,14 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
     __syncwarp();
   } else {
     // ------------------------------------------------------------------
-    // Softmax: warps 2 .. 2+WPT-1 tile 0, the next WPT warps tile 1.  A row
-    // is shared by NH threads (warps with the same TMEM lane quadrant), each
-    // owning BN/NH score columns and D/NH output columns.
+    // Softmax: warps 2..5 tile 0, warps 6..9 tile 1; thread = row (the
+    // warp's TMEM lane quadrant is warp % 4).
     // ------------------------------------------------------------------
-    constexpr int NH = C::NH;
-    constexpr int CPT = BN / NH;      // score columns per thread
-    constexpr int OPT = D / NH;       // output columns per thread
+    constexpr int CPT = BN;  // score columns per thread
+    constexpr int OPT = D;   // output columns per thread
     const int gw = warp - 2;
     const int t = gw / C::WPT;
     const int wi = gw - t * C::WPT;
-    const int half = wi >> 2;
     const uint32_t bar_id = 1 + t;
     constexpr uint32_t kBarThreads = 32 * C::WPT;
     const int nb = nblk_t[t];
@@ -385,22 +363,20 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
                           ? max(0, row_g + (p.Lkv - p.Lq) - p.window + 1)
                           : 0;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t col_s = C::COL_S + t * 128 + half * CPT;      // my scores
-    const uint32_t col_p = C::COL_S + t * 128 + half * (CPT / 2);  // my P
-    const uint32_t col_o = C::COL_O + t * 128 + half * OPT;      // my O
+    const uint32_t col_s = C::COL_S + t * 128;  // the row's scores
+    const uint32_t col_p = C::COL_S + t * 128;  // its P (bf16 pairs)
+    const uint32_t col_o = C::COL_O + t * 128;  // its O
     const float scale = p.scale;
     const float ln_lambda = p.ln_lambda;
     const float sl2 = scale * kPrefLog2e;
     const bool elected = (wi == 0 && lane == 0);
     const size_t mask_row =
         ((size_t)(b * p.Hq + hq) * p.nq + tile) * (size_t)p.nk;
-    float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);  // [2][2][NH][128]
-    float* xsum = reinterpret_cast<float*>(smem + C::OFF_XSUM);  // [2][NH][128]
     volatile int* abort_t = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
 
     float m_crit = -INFINITY;
     float m_ref = -INFINITY;
-    float l = 0.f;  // this thread's part of the row normaliser
+    float l = 0.f;  // the row normaliser
     unsigned long long n_vis = 0, n_skp = 0;
     bool ok = true;
 
@@ -415,7 +391,7 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
         tmem_ld32(lane_base + col_s + c * 32, sr[c]);
       tc_wait_ld();
 
-      const int col0 = j * BN + half * CPT;  // first score column of mine
+      const int col0 = j * BN;  // the block's first key
       if (col0 + CPT - 1 > lim || col0 < first) {
 #pragma unroll
         for (int c = 0; c < CPT / 32; ++c)
@@ -440,21 +416,13 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
         mt = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
                    fmaxf(m8[6], m8[7]));
       }
-      float* xm = xmax + (((j & 1) * 2 + t) * NH) * 128;
-      if (NH > 1) xm[half * 128 + rr] = mt;
-      // A row passes the criterion iff each of its parts does, so the vote
-      // needs no exchange; the barrier also publishes the part maxima.
-      const float mt_part = mt * scale;
-      const bool pred = !active || mt_part == -INFINITY ||
-                        (mt_part - m_crit < ln_lambda);
+      const float mt_s = mt * scale;  // the row's block max
+      const bool pred = !active || mt_s == -INFINITY ||
+                        (mt_s - m_crit < ln_lambda);
       tc_fence_before();
       const bool skip =
           named_sync_and(bar_id, kBarThreads, pred) && (ln_lambda > -INFINITY);
       if (abort_t[t]) { ok = false; break; }
-#pragma unroll
-      for (int h = 0; h < NH; ++h)
-        if (h != half) mt = fmaxf(mt, xm[h * 128 + rr]);
-      const float mt_s = mt * scale;  // whole-row block max
       if (elected) {
         ++n_vis;
         if (skip) ++n_skp;
@@ -489,8 +457,8 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
         for (int x = 0; x < 32; x += 2) {
           const float a0 = fmaf(__uint_as_float(sr[c][x]), sl2, -mb);
           const float a1 = fmaf(__uint_as_float(sr[c][x + 1]), sl2, -mb);
-          const float p0 = c < BLASST_PREFILL2_EXP_EMU ? exp2_poly(a0) : ex2_approx(a0);
-          const float p1 = c < BLASST_PREFILL2_EXP_EMU ? exp2_poly(a1) : ex2_approx(a1);
+          const float p0 = ex2_approx(a0);
+          const float p1 = ex2_approx(a1);
           rs[(x >> 1) & 3] += p0 + p1;
           pk[x / 2] = pack_bf16x2(p0, p1);
         }
@@ -532,18 +500,11 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
       const bool w = mbar_wait(&bar[C::B_OD + t], 0, kWaitPrefillEpilogue, nb,
                                600 + t);
       tc_fence_after();
-      float lrow = l;
-      if (NH > 1) {
-        xsum[(t * NH + half) * 128 + rr] = l;
-        named_sync(bar_id, kBarThreads);
-        lrow = 0.f;
-#pragma unroll
-        for (int h = 0; h < NH; ++h) lrow += xsum[(t * NH + h) * 128 + rr];
-      }
+      const float lrow = l;
       if (__all_sync(FULL, w)) {
         const float inv_l = (lrow > 0.f) ? 1.f / lrow : 0.f;
         __nv_bfloat16* orow_g =
-            p.o + ((size_t)(b * p.Hq + hq) * p.Lq + row_g) * D + half * OPT;
+            p.o + ((size_t)(b * p.Hq + hq) * p.Lq + row_g) * D;
 #pragma unroll
         for (int c = 0; c < OPT / 32; ++c) {
           uint32_t orow[32];
@@ -566,7 +527,7 @@ __global__ void __launch_bounds__(64 + 2 * 4 * BLASST_PREFILL2_COL_SPLIT * 32, 1
             }
           }
         }
-        if (active && half == 0 && p.lse)
+        if (active && p.lse)
           p.lse[(size_t)(b * p.Hq + hq) * p.Lq + row_g] = m_ref + __logf(lrow);
       }
     }

@@ -316,25 +316,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= ~8: n = round(x) goes into the exponent
-// field, 2^f on f = x - n in [-1/2, 1/2] is a cubic fitted for minimum
-// maximum relative error (Remez exchange; csrc/exp2_poly_fit.py derives
-// the coefficients; max relative error 7.5e-5).  Arguments below -126
-// (masked entries included) give exactly 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float xc = fmaxf(x, -126.0f);
-  const float magic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to n
-  const float t = xc + magic;       // bits(t) = bits(magic) + n
-  const float n = t - magic;
-  const float f = xc - n;
-  float p = fmaf(5.517166906e-02f, f, 2.426111222e-01f);
-  p = fmaf(p, f, 6.932609855e-01f);
-  p = fmaf(p, f, 9.999280735e-01f);
-  // (bits(t) << 23) == n << 23 modulo 2^32: adds n to the exponent of p
-  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-  return x < -126.0f ? 0.0f : r;
-}
-
 // max(a, b, c) in one instruction (sm_100): two comparisons for the issue
 // cost of one two-input max.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

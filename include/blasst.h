@@ -269,8 +269,10 @@ blasst_status_t blasst_decode_batched(const void *q, const void *k_cache,
  * split partials go to an 8 MiB array that the library holds in device
  * memory on every GPU that loads it, until the process exits.
  *  - The first call on a device looks up that array's device address for
- *    the current device (once per device); make that first call before any
- *    stream capture.
+ *    the current device and context (once per device and context: a call
+ *    made after cudaDeviceReset, or with another context current on the
+ *    device, looks it up again, because the array then lives at a new
+ *    address); make that first call before any stream capture.
  *  - Shapes whose partials exceed 8 MiB (B*Hq*S*(d+1) float32 values plus
  *    alignment, see blasst_decode_workspace_size) are rejected with
  *    BLASST_ERR_WORKSPACE and a message in blasst_last_error().

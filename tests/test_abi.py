@@ -101,6 +101,29 @@ def test_decode_validation(lib):
     assert _decode(lib, ws=0x4000, ws_bytes=64) == 7   # too small
 
 
+def _noalloc(lib, B, Hq, Hkv, Lkv, S, d=128, o=0x2000):
+    f = lib.blasst_decode_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5 + [
+        ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_void_p]
+    return f(0x1000, 0x1000, 0x1000, o, None, B, Hq, Hkv, Lkv, d, 0.088,
+             -1.0, 64, S, None, None)
+
+
+def test_decode_noalloc_size_guard_needs_no_device(lib):
+    """Shapes whose split partials exceed the 8 MiB built-in scratch are
+    refused before the library asks the runtime for anything (no device
+    here), with a message naming both sizes."""
+    # 64 sequences x 64 heads x 8 splits x 129 floats = 16.9 MB of partials
+    assert _noalloc(lib, 64, 64, 8, 512, 8) == 7
+    lib.blasst_last_error.restype = ctypes.c_char_p
+    msg = lib.blasst_last_error().decode()
+    assert "scratch holds 8388608" in msg
+    assert _noalloc(lib, 0, 64, 8, 512, 8) == 1
+    assert _noalloc(lib, 1, 4, 1, 512, -1) == 1
+
+
 def _mla(lib, q=0x1000, c=0x1000, o=0x2000, B=1, H=8, L=256, dqk=576,
          dv=512, lnl=-1.0, S=1, ws=None, ws_bytes=0):
     f = lib.blasst_mla_decode

@@ -140,32 +140,54 @@ def test_paged_equals_contiguous_bitwise(blasst, ps):
 
 def test_paged_bad_table_and_length_are_reported(blasst):
     """Out-of-range values in the device-resident table and lengths are
-    caught by the kernel before any copy through them is issued."""
+    caught by the kernel before any copy through them is issued.  The pool
+    passed to the call is a view into a larger allocation with 8 poisoned
+    guard pages on each side, so that the bad page ids used here (-1 and
+    num_pages + 5) would still address allocated memory if the check ever
+    failed to stop a copy."""
     m = blasst
     B, Hq, Hkv, L = 2, 8, 2, 1000
     x = planted_gap(B, Hq, Hkv, 1, L, 128, decode=True, block=64, gap=8.0,
                     heavy_frac=0.03, seed=5, device="cuda")
     pk = paginate(x.k, x.v, [L, L], 64, seed=1, poison=POISON)
+    GUARD = 8
+    P_ = pk.num_pages
+    kg = torch.full((P_ + 2 * GUARD,) + tuple(pk.k_pages.shape[1:]),
+                    POISON[0], dtype=torch.bfloat16, device="cuda")
+    vg = torch.full_like(kg, POISON[1])
+    kg[GUARD:GUARD + P_] = pk.k_pages
+    vg[GUARD:GUARD + P_] = pk.v_pages
+    kp, vp = kg[GUARD:GUARD + P_], vg[GUARD:GUARD + P_]
+    assert kp.shape[0] == P_ and kp.data_ptr() > kg.data_ptr()
+    o_good, _ = m.blasst_decode_paged(x.q, kp, vp, pk.block_table,
+                                      pk.seq_lens, ln_lambda=-2.0)
+    assert m.blasst_check_device_error()[0] == 0
     bt = pk.block_table.clone()
-    bt[1, 3] = pk.num_pages + 5
-    m.blasst_decode_paged(x.q, pk.k_pages, pk.v_pages, bt, pk.seq_lens,
-                          ln_lambda=-2.0)
+    bt[1, 3] = P_ + 5
+    assert P_ + 5 < P_ + GUARD
+    m.blasst_decode_paged(x.q, kp, vp, bt, pk.seq_lens, ln_lambda=-2.0)
     st, where = m.blasst_check_device_error()
     assert st == 1 and "page id" in where and "sequence 1" in where
     bt[1, 3] = -1
-    m.blasst_decode_paged(x.q, pk.k_pages, pk.v_pages, bt, pk.seq_lens,
-                          ln_lambda=-2.0)
+    m.blasst_decode_paged(x.q, kp, vp, bt, pk.seq_lens, ln_lambda=-2.0)
     st, where = m.blasst_check_device_error()
     assert st == 1 and "page id" in where
+    # a length past what the table holds: the table is a view of a larger
+    # one (an extra row of -1), so an entry read past its end stays inside
+    # the allocation
+    tb = torch.full((B + 1, pk.block_table.shape[1]), -1, dtype=torch.int32,
+                    device="cuda")
+    tb[:B] = pk.block_table
     lens = torch.tensor([L, 16 * 64 + 1], dtype=torch.int32, device="cuda")
-    m.blasst_decode_paged(x.q, pk.k_pages, pk.v_pages, pk.block_table, lens,
-                          ln_lambda=-2.0)
+    assert pk.block_table.shape[1] * 64 == 16 * 64
+    m.blasst_decode_paged(x.q, kp, vp, tb[:B], lens, ln_lambda=-2.0)
     st, where = m.blasst_check_device_error()
     assert st == 1 and "length" in where
     # the context is still usable and a good call is clean afterwards
-    m.blasst_decode_paged(x.q, pk.k_pages, pk.v_pages, pk.block_table,
-                          pk.seq_lens, ln_lambda=-2.0)
+    o2, _ = m.blasst_decode_paged(x.q, kp, vp, pk.block_table, pk.seq_lens,
+                                  ln_lambda=-2.0)
     assert m.blasst_check_device_error()[0] == 0
+    assert torch.equal(o2, o_good)
 
 
 def test_paged_rejects_bad_arguments(blasst):

@@ -110,18 +110,34 @@ def test_prefill_rejects_bad_arguments(blasst):
         blasst.blasst_prefill(big, big, big)
 
 
-def test_prefill_full_size_sampled(blasst):
+@pytest.mark.parametrize("which", ["s70", "dense"])
+def test_prefill_full_size_sampled(blasst, which):
     """B 1, Hq 32, Hkv 8, L 32768, d 128, causal, 128x128 tiles, planted gap
-    8 with sink + 2% heavy blocks + 512-token window boost, lambda calibrated
-    to 70% sparsity; 12 tiles (first, second, middle and last of 3 heads)
-    compared with the oracle."""
+    8 with sink + 2% heavy blocks + 512-token window boost, at the lambda
+    calibrated to 70% sparsity and at the dense path; compared with the
+    oracle on every one of the 256 tiles of heads 0 and 17 (the middle of
+    the causal range included, where the long runs of skipped blocks and
+    the lazy rescales happen) and on 64 random tiles of the other heads."""
     m = blasst
     L = 32768
     x = planted_gap(1, 32, 8, L, L, 128, block=128, gap=8.0, heavy_frac=0.02,
                     window=512, seed=config_seed(2), device="cuda")
-    cal = m.blasst_calibrate(0.70, mode="prefill", q=x.q, k=x.k, v=x.v,
-                             Br=128, Bc=128)
-    assert abs(cal["achieved"] - 0.70) < 0.01
-    units = [(0, h, i) for h in (0, 17, 31) for i in (0, 1, 128, 255)]
-    _compare(m, x, True, 128, cal["ln_lambda"], units=units,
-             check_stats_only=False)
+    if which == "s70":
+        cal = m.blasst_calibrate(0.70, mode="prefill", q=x.q, k=x.k, v=x.v,
+                                 Br=128, Bc=128)
+        assert abs(cal["achieved"] - 0.70) < 0.01
+        lnl = cal["ln_lambda"]
+    else:
+        lnl = -math.inf
+    rng = np.random.default_rng(17)
+    others = [h for h in range(32) if h not in (0, 17)]
+    units = [(0, h, i) for h in (0, 17) for i in range(256)]
+    units += [(0, int(others[rng.integers(len(others))]),
+               int(rng.integers(256))) for _ in range(64)]
+    ref, mask, ties = _compare(m, x, True, 128, lnl, units=units,
+                               check_stats_only=False)
+    print(f"full-size prefill ({which}, ln lambda {lnl}): {len(units)} tiles, "
+          f"oracle sparsity {ref['skipped'] / ref['visited']:.4f}, "
+          f"near-ties {ties}")
+    if which == "dense":
+        assert (mask == 2).sum() == 0
