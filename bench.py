@@ -11,11 +11,20 @@ sparsity.  A step is one blasst_decode call (split kernel + merge kernel);
 `value` is the algorithmic bytes those calls read and write (all of K, the V
 of kept blocks, q, the split partials, o) per second, summed over ranks.
 
-The same line carries the prefill measurements (B 1, Hq 32 / Hkv 8, 32K
-tokens, d 128, causal, 128x128 tiles, lambda calibrated to 50% and 70%, and
-the dense path ln lambda = -inf), the roofline of the dominant kernel, the
-CPU oracle baseline, an end-to-end number with host buffers, and the SM
-clocks sampled (NVML) during the timed region.
+The same line carries:
+  * decode at the lambda calibrated for 50% and at the dense path, near-tie
+    counts of both from the oracle on sampled sequences;
+  * the decode length sweep (batch 148, 8K-128K keys, a fitted at 32K);
+  * the tiny prefill configuration (2 heads, 1024 tokens, d 64, ln lambda
+    -6) against the full CPU oracle on all host cores and on one;
+  * the prefill workload (B 1, Hq 32 / Hkv 8, 32K tokens, d 128, causal,
+    128x128 tiles, lambda calibrated to 50% and 70%, and the dense path
+    ln lambda = -inf), with the oracle timed on sampled tiles;
+  * the prefill calibration sweep (4K-64K, targets 0-90%, deviation of the
+    achieved sparsity from the target under lambda = a / L);
+  * the roofline of the dominant kernels, the CPU oracle baseline, an
+    end-to-end number with host buffers, and the SM clocks sampled (NVML)
+    during the timed region.
 
 Under torchrun each rank runs its own replica of the workload (independent
 sequences; no collective on the data path) and the reported time is the
@@ -47,13 +56,13 @@ DEC = dict(B=32, Hq=32, Hkv=8, Lkv=32768, d=128, Bc=64, target=0.70,
 
 # DRAM traffic of the dominant decode kernel per launch, relative to the
 # algorithmic bytes of that launch, from one ncu capture of a smaller case
-# (profiles/decode_split_kernel_B8_Lkv32k.md: dram__bytes_read.sum +
-# dram__bytes_write.sum = 955.2 MB for 957.8 MB of algorithmic bytes).  The
-# kernel reads K once and V only for kept blocks, so traffic grows with the
-# algorithmic bytes; the ratio is applied to the benchmarked launch.  It holds
-# only for the kernel source it was measured on (sha256 prefix below).
-DECODE_TRAFFIC = dict(source="dynamic_block_sparse_fa_b200/csrc/decode.cuh",
-                      sha256_16="436b7fe2e10bdb6c", ratio=955.2 / 957.8)
+# (dram__bytes_read.sum + dram__bytes_write.sum over the algorithmic bytes of
+# the captured launch).  The kernel reads K once and V only for kept blocks,
+# so traffic grows with the algorithmic bytes; the ratio is applied to the
+# benchmarked launch.  It holds only for the kernel source it was measured
+# on (sha256 prefix below); a source without a capture reports null.
+DECODE_TRAFFIC = dict(source="dynamic_block_sparse_fa_b200/csrc/decode_mma.cuh",
+                      sha256_16=None, ratio=None)
 PRE = dict(B=1, Hq=32, Hkv=8, L=32768, d=128, Br=128, Bc=128, window=4096)
 
 
@@ -66,7 +75,7 @@ def _measured_traffic(spec, algorithmic_bytes):
             h = hashlib.sha256(f.read()).hexdigest()[:16]
     except OSError:
         return None
-    if h != spec["sha256_16"]:
+    if spec["sha256_16"] is None or h != spec["sha256_16"]:
         return None
     return int(round(spec["ratio"] * algorithmic_bytes))
 
@@ -207,6 +216,31 @@ def time_calls(fn, steps, warmup, stream, barrier=None):
     return start.elapsed_time(end)
 
 
+def time_calls_flushed(fn, steps, warmup, stream, flush):
+    """Like time_calls for inputs that fit in L2: before each call the
+    `flush` buffer (larger than L2) is rewritten, and only the calls are
+    timed (a pair of CUDA events around each).  Returns the summed
+    milliseconds of the `steps` timed calls."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = []
+    for _ in range(steps):
+        flush.fill_(1)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev)
+
+
+def l2_flush_buffer(device, nbytes=256 << 20):
+    return torch.empty(nbytes // 4, dtype=torch.float32, device=device)
+
+
 def reduce_max(value, dist, device):
     """Maximum of a per-rank float over all ranks (the value itself when
     not distributed)."""
@@ -242,6 +276,31 @@ def cpu_oracle_decode_sample(q, k, v, ln_lambda, S, budget_s=10.0):
         f"{n} sequence passes over the batch of {B} (each: all {k.shape[1]} "
         f"KV heads x {k.shape[2]} keys), same splits and lambda, "
         f"~{budget_s:.0f} s budget")
+
+
+NEAR_TIE = 1e-3       # |margin| below this: the decision may differ by rounding
+DEC_TIE_SEQS = (0, 11, 22, 31)
+
+
+def _near(margin):
+    import numpy as np
+    m = np.nan_to_num(margin, nan=1.0, posinf=1.0, neginf=1.0)
+    return int((np.abs(m) < NEAR_TIE).sum())
+
+
+def decode_near_ties(q, k, v, ln_lambda, S, seqs):
+    """Near-tie count of the decode decisions on sampled sequences, from the
+    oracle's per-pair margins at this ln lambda."""
+    import oracle
+    d = q.shape[-1]
+    n = 0
+    for b in seqs:
+        if b >= q.shape[0]:
+            continue
+        r = oracle.decode(q[b:b + 1], k[b:b + 1], v[b:b + 1],
+                          1.0 / math.sqrt(d), ln_lambda, DEC["Bc"], S)
+        n += _near(r["margin"])
+    return n
 
 
 # ---------------------------------------------------------------------------
@@ -282,10 +341,16 @@ def run_blasst(args):
         line["decode_mqa"] = run_mqa(args, bl, dev, stream, hbm_peak)
         line["decode_mla"] = run_mla(args, bl, dev, stream, hbm_peak, tf_burst)
 
-    # ---------------- prefill workload (rank 0) ----------------
+    # ---------------- the remaining workloads (rank 0) ----------------
+    if rank == 0 and not args.no_sweeps and not args.no_decode:
+        line["decode_sweep"] = run_decode_sweep(args, bl, dev, stream, hbm_peak)
     if rank == 0 and not args.no_prefill:
+        line["tiny_prefill"] = run_tiny_prefill(args, bl, dev, stream, tf_burst)
         line["prefill"], line["roofline_prefill"] = run_prefill(
             args, bl, dev, stream, tf_burst, peak_kind)
+        if not args.no_sweeps:
+            line["prefill_sweep"] = run_prefill_sweep(args, bl, dev, stream,
+                                                      tf_burst)
     barrier()
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -398,7 +463,7 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
             "calibration_iterations": cal["iterations"],
         },
         "roofline": {
-            "bound": "hbm", "kernel": "decode_split_kernel (+ merge)",
+            "bound": "hbm", "kernel": "decode_mma_kernel (+ merge)",
             "achieved": round(achieved, 1), "peak": hbm_peak,
             "peak_kind": peak_kind + " copy bandwidth", "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4),
@@ -413,6 +478,36 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
         "gpu_launches": 2 * K,
         "clocks": clk.summary(),
     }
+
+    # ---------------- 50% calibrated sparsity, same inputs ----------------
+    cal50 = bl.blasst_calibrate(0.50, mode="decode", q=q, k=k, v=v, Bc=Bc,
+                                tol=0.002)
+    st50 = bl.Stats(device=dev, mask_numel=B * Hkv * nk)
+    bl.blasst_decode(q, k, v, ln_lambda=cal50["ln_lambda"], o=o, lse=lse,
+                     workspace=ws, stats=st50)
+    torch.cuda.synchronize()
+    v50, k50 = st50.read()
+    by50 = decode_bytes(B, Hq, Hkv, Lkv, d, Bc, S,
+                        kept_rows_from_mask(st50.mask.view(B, Hkv, nk), Lkv, Bc))
+    ms50 = time_calls(lambda: bl.blasst_decode(
+        q, k, v, ln_lambda=cal50["ln_lambda"], o=o, lse=lse, workspace=ws),
+        K, W, stream, barrier)
+    ms50 = reduce_max(ms50, dist, dev)
+    line["decode"]["s50"] = {
+        "ln_lambda": cal50["ln_lambda"], "a": cal50["a"],
+        "sparsity": k50 / v50, "us": round(ms50 / K * 1e3, 2),
+        "GBps": round(by50 / (ms50 / K / 1e3) / 1e9, 1),
+        "hbm_frac": round(by50 / (ms50 / K / 1e3) / 1e9 / hbm_peak, 4),
+        "speedup_vs_dense": _r(ms_dense / ms50, 4)}
+    line["decode"]["hbm_frac_dense"] = _r(
+        by_dense / (ms_dense / K / 1e3) / 1e9 / hbm_peak, 4)
+    if rank == 0 and not args.no_cpu:
+        line["decode"]["near_ties"] = {
+            key: decode_near_ties(q, k, v, l, S, DEC_TIE_SEQS)
+            for key, l in (("s70", lnl), ("s50", cal50["ln_lambda"]))}
+        line["decode"]["near_ties"]["sample"] = (
+            f"oracle margins of sequences {DEC_TIE_SEQS} (all heads); a pair "
+            f"is a near-tie when |max_r(m~ - m) - ln lambda| < {NEAR_TIE}")
 
     if not args.no_paged:
         line["decode_paged"] = run_decode_paged(args, bl, dev, stream, q, k, v,
@@ -563,6 +658,11 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
                      "frac": r["tensor_frac"], "traffic": None}
     dense = measure(-math.inf)
     out["dense"] = dense
+    # the skipping kernel at a threshold that never skips: the dense path
+    # with the vote and the decision hand-offs still in it
+    vote = measure(-3.4028234663852886e38)
+    out["dense_with_vote"] = vote
+    out["vote_overhead"] = round(vote["us"] / dense["us"] - 1.0, 4)
     for tgt, key in ((0.5, "s50"), (0.7, "s70")):
         cal = bl.blasst_calibrate(tgt, mode="prefill", q=q, k=k, v=v, Br=Br,
                                   Bc=Bc, tol=0.002)
@@ -570,6 +670,25 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
         r["a"] = cal["a"]
         r["speedup_vs_dense"] = round(dense["us"] / r["us"], 4)
         out[key] = r
+    if not args.no_cpu:
+        tiles = [(0, h, i) for h in (0, 17) for i in range(0, 256, 4)]
+        for key in ("s50", "s70"):
+            _, smp = prefill_oracle_sample(q, k, v, out[key]["ln_lambda"],
+                                           tiles, Br)
+            out[key]["near_ties_sample"] = smp["near_ties"]
+            if key == "s70":
+                total_vis = B * Hq * (L // Br) * (L // Br + 1) // 2
+                out["cpu_baseline_prefill"] = {
+                    "value": round(smp["tflops"], 6), "unit": "TFLOP/s executed",
+                    "kind": "oracle", "cores": smp["cores"],
+                    "seconds": smp["seconds"],
+                    "sample": f"{len(tiles)} query tiles (every 4th tile of "
+                              f"heads 0 and 17) at the 70% lambda: "
+                              f"{smp['visited']} of {total_vis} visited pairs "
+                              f"({smp['visited'] / total_vis:.2%})"}
+        out["near_ties_sample"] = (
+            "oracle margins on the CPU-baseline tiles; a pair is a near-tie "
+            f"when |max_r(m~ - m) - ln lambda| < {NEAR_TIE}")
     if not args.no_window:
         out["window"] = run_prefill_window(args, bl, q, k, v, o, lse,
                                            out["s70"]["ln_lambda"], stream,
@@ -586,11 +705,235 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
     return out, roof
 
 
+def prefill_oracle_sample(q, k, v, ln_lambda, units, Br=128):
+    """The CPU oracle (all host cores) on sampled query tiles of the
+    prefill workload: seconds, executed FLOPs per second and the near-tie
+    count of the sample, and the sample's share of the visited pairs."""
+    import oracle
+    d = q.shape[-1]
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    r = oracle.prefill(q, k, v, 1.0 / math.sqrt(d), True, ln_lambda, Br, Br,
+                       units=units, n_threads=threads)
+    secs = time.perf_counter() - t0
+    ex = prefill_flops(r["visited"], r["visited"] - r["skipped"], Br, Br, d)
+    return r, {"seconds": round(secs, 3), "cores": threads,
+               "tflops": ex / secs / 1e12, "visited": r["visited"],
+               "near_ties": _near(r["margin"])}
+
+
+def run_tiny_prefill(args, bl, dev, stream, tf_peak):
+    """The tiny prefill configuration: B 1, Hq = Hkv = 2, L 1024, d 64,
+    causal, 64 x 64 tiles, ln lambda = -6, planted gap 8 (sink + 3% heavy
+    blocks).  GPU time with L2 flushed between calls; the full CPU oracle
+    on all host cores and on one; parity of the GPU result."""
+    import numpy as np
+    import oracle
+    from synth import config_seed, planted_gap
+    B, H, L, d, T, lnl = 1, 2, 1024, 64, 64, -6.0
+    x = planted_gap(B, H, H, L, L, d, block=T, gap=8.0, heavy_frac=0.03,
+                    seed=config_seed(0), device=dev)
+    nq = nk = L // T
+    st = bl.Stats(device=dev, mask_numel=B * H * nq * nk)
+    o, lse = bl.blasst_prefill(x.q, x.k, x.v, ln_lambda=lnl, Br=T, Bc=T,
+                               stats=st)
+    torch.cuda.synchronize()
+    vis, skp = st.read()
+    flush = l2_flush_buffer(dev)
+    steps = max(args.steps, 100)
+    ms = time_calls_flushed(lambda: bl.blasst_prefill(
+        x.q, x.k, x.v, ln_lambda=lnl, Br=T, Bc=T, o=o, lse=lse),
+        steps, args.warmup, stream, flush) / steps
+    od, ld = torch.empty_like(o), torch.empty_like(lse)
+    ms_d = time_calls_flushed(lambda: bl.blasst_prefill(
+        x.q, x.k, x.v, Br=T, Bc=T, o=od, lse=ld),
+        steps, args.warmup, stream, flush) / steps
+    del flush
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    ref = oracle.prefill(x.q, x.k, x.v, 1.0 / math.sqrt(d), True, lnl, T, T,
+                         n_threads=threads)
+    t_all = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.prefill(x.q, x.k, x.v, 1.0 / math.sqrt(d), True, lnl, T, T,
+                   n_threads=1)
+    t_one = time.perf_counter() - t0
+    o_np = o.float().cpu().numpy()
+    err = np.concatenate([np.abs(o_np[b, h, i * T:(i + 1) * T] - ref["o"][u])
+                          .ravel() for u, (b, h, i) in enumerate(ref["units"])])
+    gm = st.mask.cpu().numpy().reshape(B, H, nq, nk)
+    got = np.stack([gm[b, h, i] for (b, h, i) in ref["units"]])
+    near = np.abs(np.nan_to_num(ref["margin"], nan=1, posinf=1)) < NEAR_TIE
+    ex = prefill_flops(vis, vis - skp, T, T, d)
+    dense_eq = dense_equiv_flops(B, H, L, d)
+    return {
+        "workload": f"prefill B{B} Hq{H} Hkv{H} L{L} d{d} causal {T}x{T}, "
+                    f"ln lambda {lnl}",
+        "l2": "L2 flushed (256 MB write) before every timed call",
+        "sparsity": skp / vis, "us": round(ms * 1e3, 2),
+        "dense_us": round(ms_d * 1e3, 2),
+        "speedup_vs_dense": round(ms_d / ms, 4),
+        "dense_equiv_tflops": round(dense_eq / (ms / 1e3) / 1e12, 3),
+        "executed_tflops": round(ex / (ms / 1e3) / 1e12, 3),
+        "tensor_frac": round(ex / (ms / 1e3) / 1e12 / tf_peak, 5),
+        "oracle_seconds_all_cores": round(t_all, 4), "oracle_cores": threads,
+        "oracle_seconds_one_core": round(t_one, 4),
+        "max_abs_err": float(err.max()), "mean_abs_err": float(err.mean()),
+        "mask_mismatch_outside_near_ties": int(((got != ref["mask"]) & ~near).sum()),
+        "near_ties": int(near.sum())}
+
+
+def run_decode_sweep(args, bl, dev, stream, hbm_peak):
+    """Decode length sweep: B 148, Hq 32 / Hkv 8, d 128, Bc 64, planted gap 8
+    (sink + 3% heavy blocks); a of lambda = a / L calibrated once at 32K for
+    70% sparsity and applied at every length.  Per length: achieved
+    sparsity, time against the dense path, algorithmic GB/s, near-ties and
+    error on 4 sampled sequences from the oracle."""
+    import numpy as np
+    import oracle
+    from synth import config_seed, planted_gap_kv_inplace
+    B, Hq, Hkv, d, Bc = 148, 32, 8, 128, 64
+    K, W = min(args.steps, 20), args.warmup
+
+    def make(L):
+        q = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev)
+        k = torch.empty(B, Hkv, L, d, dtype=torch.bfloat16, device=dev)
+        v = torch.empty_like(k)
+        planted_gap_kv_inplace(k, v, q, block=Bc, gap=8.0, heavy_frac=0.03,
+                               seed=config_seed(3, L))
+        return q, k, v
+
+    q, k, v = make(32768)
+    cal = bl.blasst_calibrate(0.70, mode="decode", q=q, k=k, v=v, Bc=Bc,
+                              tol=0.002)
+    a = cal["a"]
+    del q, k, v
+    torch.cuda.empty_cache()
+    out = {"workload": f"decode B{B} Hq{Hq} Hkv{Hkv} d{d} Bc{Bc}, lambda = a/L "
+                       f"with a fitted at 32K for 70%",
+           "a": a, "l2": "inputs larger than L2, no flush"}
+    seqs = (0, 37, 101, 147)
+    for L in args.sweep_lengths:
+        need = 2 * B * Hkv * L * d * 2
+        if torch.cuda.mem_get_info(dev)[0] < need * 1.1 + (2 << 30):
+            out[str(L)] = {"skipped": "not enough free device memory"}
+            continue
+        q, k, v = make(L)
+        lnl = min(0.0, math.log(a / L))
+        S = bl.blasst_decode_splits(B, Hkv, L, Bc)
+        nk = -(-L // Bc)
+        st = bl.Stats(device=dev, mask_numel=B * Hkv * nk)
+        o, lse = bl.blasst_decode(q, k, v, ln_lambda=lnl, stats=st)
+        torch.cuda.synchronize()
+        vis, skp = st.read()
+        mask = st.mask.view(B, Hkv, nk)
+        by = decode_bytes(B, Hq, Hkv, L, d, Bc, S,
+                          kept_rows_from_mask(mask, L, Bc))
+        ms = time_calls(lambda: bl.blasst_decode(q, k, v, ln_lambda=lnl, o=o,
+                                                 lse=lse), K, W, stream) / K
+        od = torch.empty_like(o)
+        ms_d = time_calls(lambda: bl.blasst_decode(q, k, v, o=od), K, W,
+                          stream) / K
+        ties, errs = 0, []
+        for b in seqs:
+            r = oracle.decode(q[b:b + 1], k[b:b + 1], v[b:b + 1],
+                              1.0 / math.sqrt(d), lnl, Bc, S)
+            ties += _near(r["margin"])
+            errs.append(np.abs(o[b:b + 1].float().cpu().numpy() - r["o"]).max())
+        gbs = by / (ms / 1e3) / 1e9
+        out[str(L)] = {"ln_lambda": lnl, "splits": S, "sparsity": skp / vis,
+                       "us": round(ms * 1e3, 1), "dense_us": round(ms_d * 1e3, 1),
+                       "speedup_vs_dense": round(ms_d / ms, 4),
+                       "GBps": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 4),
+                       "near_ties_4seq": ties,
+                       "max_abs_err_4seq": float(max(errs))}
+        del q, k, v, o, lse, od, st
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_prefill_sweep(args, bl, dev, stream, tf_peak):
+    """Prefill sparsity and calibration sweep: B 1, Hq 32 / Hkv 8, d 128,
+    causal, 128 x 128 tiles, gap per head uniform in [4, 12] nats, sink +
+    2% heavy blocks + 512-token window boost, L in {4K, 16K, 64K}.  For each
+    target sparsity a is fitted over the lengths whose calibration reaches
+    it (log-space fit of lambda = a / L), then each length runs at
+    lambda = a / L: achieved sparsity, deviation from the target, time
+    against the dense path.  The 4K case is compared with the oracle."""
+    import numpy as np
+    import oracle
+    from synth import config_seed, planted_gap
+    lengths, targets = args.prefill_sweep_lengths, (0.0, 0.3, 0.5, 0.7, 0.9)
+    flush = l2_flush_buffer(dev)
+    reps = 3
+    xs = {L: planted_gap(1, 32, 8, L, L, 128, block=128, gap_range=(4.0, 12.0),
+                         heavy_frac=0.02, window=512, seed=config_seed(4, L),
+                         device=dev) for L in lengths}
+    dense_ms = {}
+    for L, x in xs.items():
+        o = torch.empty_like(x.q)
+        dense_ms[L] = time_calls_flushed(lambda: bl.blasst_prefill(
+            x.q, x.k, x.v, o=o, want_lse=False), reps, 1, stream, flush) / reps
+    out = {"workload": "prefill B1 Hq32 Hkv8 d128 causal 128x128, gap per head "
+                       "U[4,12] nats, lambda = a/L with a fitted per target "
+                       "over the lengths (log space)",
+           "l2": "L2 flushed (256 MB write) before every timed call",
+           "dense_us": {str(L): round(t * 1e3, 1) for L, t in dense_ms.items()},
+           "runs": []}
+    devs = []
+    for tgt in targets:
+        cals = {L: bl.blasst_calibrate(tgt, mode="prefill", q=x.q, k=x.k,
+                                       v=x.v, Br=128, Bc=128, tol=0.002,
+                                       raise_on_no_converge=False)
+                for L, x in xs.items()}
+        fit_L = [L for L in lengths if cals[L]["status"] == 0]
+        a = None if (tgt == 0.0 or not fit_L) else bl.blasst_fit_a(
+            [cals[L]["lambda_"] for L in fit_L], fit_L)
+        for L, x in xs.items():
+            lnl = -math.inf if a is None else min(0.0, math.log(a / L))
+            st = bl.Stats(device=dev)
+            bl.blasst_prefill(x.q, x.k, x.v, ln_lambda=lnl, stats=st,
+                              stats_only=True)
+            torch.cuda.synchronize()
+            sp = st.sparsity()
+            o = torch.empty_like(x.q)
+            ms = time_calls_flushed(lambda: bl.blasst_prefill(
+                x.q, x.k, x.v, ln_lambda=lnl, o=o, want_lse=False),
+                reps, 1, stream, flush) / reps
+            rec = {"L": L, "target": tgt, "a": a, "ln_lambda": lnl,
+                   "sparsity": round(sp, 5), "deviation": round(abs(sp - tgt), 5),
+                   "calibration_reached_target_at_L": cals[L]["status"] == 0,
+                   "us": round(ms * 1e3, 1),
+                   "speedup_vs_dense": round(dense_ms[L] / ms, 4),
+                   "dense_equiv_tflops": round(dense_equiv_flops(1, 32, L, 128)
+                                               / (ms / 1e3) / 1e12, 1)}
+            if tgt > 0 and L == 4096 and a is not None and not args.no_cpu:
+                r = oracle.prefill(x.q, x.k, x.v, 1 / math.sqrt(128), True,
+                                   lnl, 128, 128)
+                og, _ = bl.blasst_prefill(x.q, x.k, x.v, ln_lambda=lnl)
+                g = og.float().cpu().numpy()
+                e = np.concatenate([np.abs(g[b, h, i * 128:(i + 1) * 128]
+                                           - r["o"][u]).ravel()
+                                    for u, (b, h, i) in enumerate(r["units"])])
+                rec.update(max_abs_err=float(e.max()),
+                           mean_abs_err=float(e.mean()),
+                           near_ties=_near(r["margin"]))
+            if tgt > 0 and cals[L]["status"] == 0:
+                devs.append(abs(sp - tgt))
+            out["runs"].append(rec)
+    out["mean_deviation"] = float(np.mean(devs)) if devs else None
+    out["max_deviation"] = float(np.max(devs)) if devs else None
+    del flush, xs
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_mqa(args, bl, dev, stream, hbm_peak):
     """MQA decode, B 32 x 32 query heads on one KV head, 32K keys, d 128:
-    blasst_decode (CUDA cores, tiles of 8 heads) against blasst_decode_wide
-    (tensor cores, the 32 heads as one tile), dense and at ln lambda -2.
-    GB/s counts K and the V of kept blocks."""
+    blasst_decode (tiles of 8 heads on the tensor core), the same tiles on
+    the CUDA cores (blasst_decode_batched with batch 1, one CTA per tile)
+    and blasst_decode_wide (the 32 heads as one tile), dense and at
+    ln lambda -2.  GB/s counts K and the V of kept blocks."""
     from synth import config_seed, planted_gap_kv_inplace
     B, Hq, Hkv, L, d = 32, 32, 1, 32768, 128
     q = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev)
@@ -601,7 +944,9 @@ def run_mqa(args, bl, dev, stream, hbm_peak):
     nk = L // 64
     K, W = args.steps, args.warmup
     out = {"workload": f"MQA decode B{B} Hq{Hq} Hkv{Hkv} Lkv{L} d{d} Bc 64"}
+    cuda_cores = lambda *a, **kw: bl.blasst_decode_batched(*a, batch=1, **kw)
     for name, fn, rows in (("tiles_of_8", bl.blasst_decode, Hkv * Hq // 8),
+                           ("tiles_of_8_cuda_cores", cuda_cores, Hkv * Hq // 8),
                            ("wide", bl.blasst_decode_wide, Hkv)):
         r = {}
         for key, lnl in (("dense", -math.inf), ("lnl_-2", -2.0)):
@@ -919,6 +1264,13 @@ def main():
     ap.add_argument("--prefill-L", type=int, default=PRE["L"])
     ap.add_argument("--prefill-lnl", type=float, default=None,
                     help="measure prefill only at this ln(lambda)")
+    ap.add_argument("--no-sweeps", action="store_true",
+                    help="skip the decode length and prefill calibration sweeps")
+    ap.add_argument("--sweep-lengths", type=int, nargs="+",
+                    default=[8192, 32768, 65536, 131072],
+                    help="cache lengths of the B148 decode sweep")
+    ap.add_argument("--prefill-sweep-lengths", type=int, nargs="+",
+                    default=[4096, 16384, 65536])
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="approximate CPU time budget of the oracle baseline")
     args = ap.parse_args()

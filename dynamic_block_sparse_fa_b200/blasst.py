@@ -366,7 +366,8 @@ def blasst_decode_batched(q, k, v, *, batch=2, scale=None,
                           stream=None):
     """Decode with the batched decision rule: blocks are scored in pairs
     and each is judged against the max over earlier blocks and the pair
-    (batch = 2; batch = 1 is blasst_decode).  Returns (o, lse)."""
+    (batch = 2; batch = 1 is the sequential rule of blasst_decode, always on
+    the CUDA-core kernel).  Returns (o, lse)."""
     B, Hq, d = q.shape
     _, Hkv, Lkv, _ = k.shape
     if scale is None:

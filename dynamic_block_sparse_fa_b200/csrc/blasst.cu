@@ -14,6 +14,7 @@
 #include "backward.cuh"
 #include "mla.cuh"
 #include "decode_wide.cuh"
+#include "decode_mma.cuh"
 
 namespace {
 
@@ -186,6 +187,49 @@ cudaError_t launch_split(const blasst::DecodeArgs& a, long long grid,
   return cudaGetLastError();
 }
 
+// The warp-MMA decode (decode_mma.cuh) for the sequential rule on a
+// contiguous cache with G <= 8, then the merge as for launch_decode.
+template <int G>
+cudaError_t launch_mma_split(const blasst::DecodeMmaArgs& a, long long grid,
+                             cudaStream_t st) {
+  using C = blasst::DecodeMmaCfg;
+  cudaError_t e = cudaFuncSetAttribute(
+      blasst::decode_mma_kernel<G>,
+      cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  blasst::decode_mma_kernel<G>
+      <<<(unsigned)grid, blasst::kDecThreads, C::SMEM_ALLOC, st>>>(a);
+  return cudaGetLastError();
+}
+
+blasst_status_t launch_decode_mma(const blasst::DecodeMmaArgs& a, int G,
+                                  long long grid, bool stats_only, void* o,
+                                  float* lse, int rows, cudaStream_t st) {
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (G) {
+    case 1: e = launch_mma_split<1>(a, grid, st); break;
+    case 2: e = launch_mma_split<2>(a, grid, st); break;
+    case 4: e = launch_mma_split<4>(a, grid, st); break;
+    case 8: e = launch_mma_split<8>(a, grid, st); break;
+  }
+  if (e != cudaSuccess) return cuda_status(e, "decode split launch");
+  if (stats_only) return BLASST_OK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)rows);
+  cfg.blockDim = dim3(blasst::kDecD);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, blasst::decode_combine_kernel,
+                         (const float*)a.o_part, (const float*)a.lse_part,
+                         static_cast<__nv_bfloat16*>(o), lse, a.S);
+  return cuda_status(e, "decode merge launch");
+}
+
 blasst_status_t launch_decode(const blasst::DecodeArgs& a, int G, bool paged,
                               long long grid, bool stats_only, void* o,
                               float* lse, int rows, int S, cudaStream_t st,
@@ -272,7 +316,7 @@ blasst_status_t blasst_decode_window(const void* q, const void* k_cache,
                                      const blasst_skip_stats_t* skip_stats,
                                      void* stream) {
   return decode_contiguous(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Lkv, d,
-                           scale, window, 1, ln_lambda, Bc, num_splits,
+                           scale, window, 0, ln_lambda, Bc, num_splits,
                            workspace, workspace_bytes, skip_stats, stream);
 }
 
@@ -293,8 +337,67 @@ blasst_status_t blasst_decode_batched(const void* q, const void* k_cache,
 }  // extern "C"
 
 namespace {
-// Contiguous-cache decode: the sliding window (window > 0) and the batched
-// decision rule (batch = 2) are variants of the same split kernel.
+// The tensor-core decode (decode_wide.cuh) for G = Hq / Hkv <= 128 heads
+// per KV head, in tiles of T heads (T = G, or 8 for G a multiple of 8);
+// arguments already validated, S resolved.
+blasst_status_t wide_launch(const void* q, const void* k_cache,
+                            const void* v_cache, void* o, float* lse, int B,
+                            int Hq, int Hkv, int Lkv, float scale, int window,
+                            int T, float ln_lambda, int S, void* workspace,
+                            size_t workspace_bytes,
+                            const blasst_skip_stats_t* skip_stats,
+                            void* stream) {
+  const int d = blasst::kWideD;
+  const int G = Hq / Hkv;
+  const int nk = (Lkv + blasst::kWideBc - 1) / blasst::kWideBc;
+  const long long grid = (long long)B * Hkv * S;
+  if (grid > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED_SHAPE;
+  const bool stats_only = (o == nullptr);
+  blasst::WideArgs a;
+  memset(&a, 0, sizeof a);
+  if (!stats_only) {
+    const blasst_status_t ws = carve_workspace(workspace, workspace_bytes, B,
+                                               Hq, d, S, &a.o_part,
+                                               &a.lse_part);
+    if (ws != BLASST_OK) return ws;
+  }
+  if (!blasst::encode_map(&a.tk, k_cache, d, Lkv, (long long)B * Hkv, 64) ||
+      !blasst::encode_map(&a.tv, v_cache, d, Lkv, (long long)B * Hkv, 64))
+    return cuda_status(cudaErrorInvalidValue, "wide decode tensor maps");
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.counters = skip_stats ? skip_stats->counters : nullptr;
+  a.mask = skip_stats ? skip_stats->mask : nullptr;
+  a.Hkv = Hkv;
+  a.G = G;
+  a.T = T;
+  a.window = window;
+  a.Lkv = Lkv;
+  a.nk = nk;
+  a.S = S;
+  a.scale = scale;
+  a.ln_lambda = ln_lambda;
+  a.stats_only = stats_only ? 1 : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaFuncSetAttribute(blasst::decode_wide_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       blasst::WideCfg::SMEM_ALLOC);
+  if (e != cudaSuccess) return cuda_status(e, "wide decode attribute");
+  blasst::decode_wide_kernel<<<(unsigned)grid, blasst::kWideThreads,
+                               blasst::WideCfg::SMEM_ALLOC, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || stats_only)
+    return cuda_status(e, "wide decode split launch");
+  blasst::decode_combine_kernel<<<(unsigned)((long long)B * Hq), blasst::kDecD,
+                                  0, st>>>(
+      a.o_part, a.lse_part, static_cast<__nv_bfloat16*>(o), lse, S);
+  return cuda_status(cudaGetLastError(), "wide decode merge launch");
+}
+
+// Contiguous-cache decode.  batch = 0: blasst_decode / blasst_decode_window
+// (the sequential rule on the fastest kernel for the group: the warp-MMA
+// kernel for G <= 8, the tensor-core tiles for 16 <= G <= 128, the
+// CUDA-core kernel above); batch = 1 or 2: blasst_decode_batched, always on
+// the CUDA-core split kernel (batch 1 = the sequential rule).
 blasst_status_t decode_contiguous(const void* q, const void* k_cache,
                                   const void* v_cache, void* o, float* lse,
                                   int B, int Hq, int Hkv, int Lkv, int d,
@@ -312,7 +415,6 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
   if (d != blasst::kDecD || Bc != blasst::kDecBc || !decode_group_ok(G))
     return BLASST_ERR_UNSUPPORTED_SHAPE;
   const int kv_div = G > 8 ? G / 8 : 1;  // tiles of 8 heads above 8
-  G /= kv_div;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
       (o && !aligned16(o)))
     return BLASST_ERR_MISALIGNED;
@@ -323,6 +425,44 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
                     ? blasst_decode_splits(B, Hkv, Lkv - jlo * Bc, Bc)
                     : num_splits;
   if (S < 1 || S > nk - jlo) return BLASST_ERR_INVALID_ARG;
+  // Wide groups (16 to 128 heads per KV head): the tiles of 8 run on the
+  // tensor core, one CTA per (sequence, KV head, split) for all of them;
+  // G x d FMAs per key would leave the CUDA-core kernel far below the
+  // memory time.  Same tiles, decisions and split policy.
+  if (batch == 0 && G > 8 && G <= 128)
+    return wide_launch(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Lkv, scale,
+                       window, 8, ln_lambda, S, workspace, workspace_bytes,
+                       skip_stats, stream);
+  const long long grid_mma = (long long)B * Hkv * S;
+  if (batch == 0 && G <= 8 && grid_mma <= 0x7fffffffLL) {
+    // the sequential rule on the warp-MMA kernel
+    const bool stats_only = (o == nullptr);
+    blasst::DecodeMmaArgs m;
+    memset(&m, 0, sizeof m);
+    if (!stats_only) {
+      const blasst_status_t ws = carve_workspace(workspace, workspace_bytes, B,
+                                                 Hq, d, S, &m.o_part,
+                                                 &m.lse_part);
+      if (ws != BLASST_OK) return ws;
+    }
+    if (!blasst::encode_map(&m.tk, k_cache, d, Lkv, (long long)B * Hkv, 64) ||
+        !blasst::encode_map(&m.tv, v_cache, d, Lkv, (long long)B * Hkv, 64))
+      return cuda_status(cudaErrorInvalidValue, "decode tensor maps");
+    m.q = static_cast<const __nv_bfloat16*>(q);
+    m.counters = skip_stats ? skip_stats->counters : nullptr;
+    m.mask = skip_stats ? skip_stats->mask : nullptr;
+    m.Hkv = Hkv;
+    m.Lkv = Lkv;
+    m.nk = nk;
+    m.S = S;
+    m.scale = scale;
+    m.ln_lambda = ln_lambda;
+    m.stats_only = stats_only ? 1 : 0;
+    m.window = window;
+    return launch_decode_mma(m, G, grid_mma, stats_only, o, lse, B * Hq,
+                             static_cast<cudaStream_t>(stream));
+  }
+  G /= kv_div;
   const long long grid = (long long)B * Hkv * kv_div * S;
   if (grid > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED_SHAPE;
   const bool stats_only = (o == nullptr);
@@ -625,45 +765,9 @@ blasst_status_t blasst_decode_wide(const void* q, const void* k_cache,
   const int S = num_splits == 0 ? blasst_decode_splits(B, Hkv, Lkv, Bc)
                                 : num_splits;
   if (S < 1 || S > nk) return BLASST_ERR_INVALID_ARG;
-  const long long grid = (long long)B * Hkv * S;
-  if (grid > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED_SHAPE;
-  const bool stats_only = (o == nullptr);
-  blasst::WideArgs a;
-  memset(&a, 0, sizeof a);
-  if (!stats_only) {
-    const blasst_status_t ws = carve_workspace(workspace, workspace_bytes, B,
-                                               Hq, d, S, &a.o_part,
-                                               &a.lse_part);
-    if (ws != BLASST_OK) return ws;
-  }
-  if (!blasst::encode_map(&a.tk, k_cache, d, Lkv, (long long)B * Hkv, 64) ||
-      !blasst::encode_map(&a.tv, v_cache, d, Lkv, (long long)B * Hkv, 64))
-    return cuda_status(cudaErrorInvalidValue, "wide decode tensor maps");
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.counters = skip_stats ? skip_stats->counters : nullptr;
-  a.mask = skip_stats ? skip_stats->mask : nullptr;
-  a.Hkv = Hkv;
-  a.G = G;
-  a.Lkv = Lkv;
-  a.nk = nk;
-  a.S = S;
-  a.scale = scale;
-  a.ln_lambda = ln_lambda;
-  a.stats_only = stats_only ? 1 : 0;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaFuncSetAttribute(blasst::decode_wide_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       blasst::WideCfg::SMEM_ALLOC);
-  if (e != cudaSuccess) return cuda_status(e, "wide decode attribute");
-  blasst::decode_wide_kernel<<<(unsigned)grid, blasst::kWideThreads,
-                               blasst::WideCfg::SMEM_ALLOC, st>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || stats_only)
-    return cuda_status(e, "wide decode split launch");
-  blasst::decode_combine_kernel<<<(unsigned)((long long)B * Hq), blasst::kDecD,
-                                  0, st>>>(
-      a.o_part, a.lse_part, static_cast<__nv_bfloat16*>(o), lse, S);
-  return cuda_status(cudaGetLastError(), "wide decode merge launch");
+  return wide_launch(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Lkv, scale, 0,
+                     G, ln_lambda, S, workspace, workspace_bytes, skip_stats,
+                     stream);
 }
 
 int blasst_mla_decode_splits(int B, int L) {

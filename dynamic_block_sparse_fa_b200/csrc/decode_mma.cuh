@@ -1,0 +1,359 @@
+// decode_mma.cuh -- BLASST decode with the scores and P.V on warp-level
+// tensor-core instructions (mma.sync m16n8k16, bf16 in, f32 accumulate):
+// contiguous bf16 KV cache, G <= 8 query heads per KV head, split-KV.
+//
+// Method as in decode.cuh ("BLASST: Dynamic BLocked Attention Sparsity via
+// Softmax Thresholding", gist.science summary, section 2 "Criterio de Pulo"
+// and "Acoes de Otimizacao", section 3: in the memory-bound decode the
+// saving is the V blocks never loaded): per (sequence, KV head, split) the
+// G heads are the rows of one tile, blocks of 64 keys in ascending order,
+// block j skipped when every head's block max lies more than |ln lambda|
+// below its running max, V read only for kept blocks, then the split
+// partials are merged by log-sum-exp (decode_combine_kernel).
+//
+// Why this form: the decode is bound by HBM, and the CUDA-core scoring of a
+// block (G x 64 x 128 FMAs plus the bf16 unpacking and the cross-lane
+// reductions, ~350 instructions a thread) left each CTA ~4k cycles per block,
+// far from the ~1k at which 3 CTAs per SM keep HBM busy when most V blocks
+// are skipped.  Here a warp scores its 16 keys of the block with 16 MMAs fed
+// by 8 ldmatrix loads, and the score fragment it holds is, after the exp,
+// exactly the A fragment of its 16-key slice of P.V, so P never leaves
+// registers.  A tcgen05 MMA would need the scores to go through tensor
+// memory and a cross-warp hand-off on every block (the wide kernel pays that
+// chain); at M = G <= 8 rows the warp-level instruction keeps the whole
+// per-block chain inside each warp.
+//
+// CTA = 4 warps per (b, hkv, split); warp w owns keys 16w .. 16w+15 of each
+// block.  K and V blocks arrive by TMA as two 64-column boxes with the
+// 128-byte swizzle (ldmatrix reads are then free of bank conflicts): a K
+// ring of two blocks and a V ring of two.  The P.V of a kept block runs
+// when the next kept block has been decided (its V load has had a block of
+// scoring to land); its P and rescale factor wait in registers.
+#pragma once
+
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace blasst {
+
+struct DecodeMmaArgs {
+  CUtensorMap tk, tv;        // [B*Hkv][Lkv][128] bf16, box 64 cols x 64 rows
+  const __nv_bfloat16* q;    // [B, Hq, 128]
+  float* o_part;             // [B*Hq, S, 128]
+  float* lse_part;           // [B*Hq, S]
+  unsigned long long* counters;
+  unsigned char* mask;       // [B*Hkv, nk]
+  int Hkv, Lkv, nk, S;
+  float scale, ln_lambda;
+  int stats_only;
+  int window;                // the last `window` keys (0 = all)
+};
+
+struct DecodeMmaCfg {
+  static constexpr int BOX = 64 * 128;      // 64 rows x 128 bytes
+  static constexpr int TILE = 2 * BOX;      // 64 keys x 128 dims, 16 KB
+  static constexpr int NK = 2, NV = 2;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + NK * TILE;
+  static constexpr int OFF_M = OFF_V + NV * TILE;   // f32 [2][8 heads][4 warps]
+  static constexpr int OFF_L = OFF_M + 2 * 8 * 4 * 4;  // f32 [4 warps][8]
+  static constexpr int OFF_BAR = OFF_L + 4 * 8 * 4;    // u64 [NK + NV]
+  static constexpr int SMEM = OFF_BAR + (NK + NV) * 8;
+  static constexpr int SMEM_ALLOC = SMEM + 1024;  // 1024-byte alignment
+  static_assert(4 * 8 * 128 * 4 <= NK * TILE, "reduction fits the K ring");
+};
+
+// D = A * B + C for one 16 x 8 x 16 step; rows 8..15 of A are zero (at most
+// 8 heads), so only D rows 0..7 (d0, d1) are kept.
+__device__ __forceinline__ void mma16816_top(float& d0, float& d1, uint32_t a0,
+                                             uint32_t a2, uint32_t b0,
+                                             uint32_t b1) {
+  [[maybe_unused]] float x2, x3;  // rows 8..15 of D: always zero, unused
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
+      : "=f"(d0), "=f"(d1), "=f"(x2), "=f"(x3)
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d0),
+        "f"(d1), "f"(0.f), "f"(0.f));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0,
+                                        uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile(
+      "ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+      : "r"(addr)
+      : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0,
+                                          uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile(
+      "ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+      : "r"(addr)
+      : "memory");
+}
+
+// Byte offset of the 16-byte chunk `chunk` (0..15: dims 8*chunk ..) of key
+// row `key` in a block stored as two 64-column boxes with the 128-byte
+// swizzle (chunk index XOR key % 8 within each 1024-byte group of rows).
+__device__ __forceinline__ uint32_t swz_off(int key, int chunk) {
+  return (uint32_t)((chunk >> 3) * DecodeMmaCfg::BOX + key * 128 +
+                    (((chunk & 7) ^ (key & 7)) << 4));
+}
+
+template <int G>
+__global__ void __launch_bounds__(kDecThreads, 3)
+    decode_mma_kernel(const __grid_constant__ DecodeMmaArgs a) {
+  static_assert(G >= 1 && G <= 8, "at most 8 heads per tile");
+  using C = DecodeMmaCfg;
+  constexpr unsigned FULL = 0xffffffffu;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+
+  const int s = blockIdx.x % a.S;
+  const int bh = blockIdx.x / a.S;  // b * Hkv + hkv
+  const int Hq = a.Hkv * G;
+  const int b = bh / a.Hkv;
+  const int hkv = bh - b * a.Hkv;
+  const int key_lo = (a.window > 0 && a.Lkv > a.window) ? a.Lkv - a.window : 0;
+  const int jlo = key_lo / kDecBc;
+  const int j0 = jlo + (int)(((long long)s * (a.nk - jlo)) / a.S);
+  const int j1 = jlo + (int)(((long long)(s + 1) * (a.nk - jlo)) / a.S);
+  const int nblk = j1 - j0;
+  if (a.mask && s == 0)  // blocks left of the window are not visited
+    for (int j = tid; j < jlo; j += kDecThreads) a.mask[(size_t)bh * a.nk + j] = 0;
+
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  float* sM = reinterpret_cast<float*>(smem + C::OFF_M);
+  float* sL = reinterpret_cast<float*>(smem + C::OFF_L);
+  uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* vfull = kfull + C::NK;
+  const bool stats_only = a.stats_only != 0;
+
+  if (tid == 0) {
+    for (int i = 0; i < C::NK; ++i) mbar_init(&kfull[i], 1);
+    for (int i = 0; i < C::NV; ++i) mbar_init(&vfull[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const uint64_t pol = policy_evict_first();
+  auto load = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int j) {
+    mbar_arrive_expect_tx(bar, C::TILE);
+    tma_load_3d(dst, map, bar, 0, j * kDecBc, bh, pol);
+    tma_load_3d(dst + C::BOX, map, bar, 64, j * kDecBc, bh, pol);
+  };
+  if (tid == 0) {
+    prefetch_tmap(&a.tk);
+    prefetch_tmap(&a.tv);
+    for (int r = 0; r < nblk && r < C::NK; ++r)
+      load(&a.tk, sK + r * C::TILE, &kfull[r], j0 + r);
+  }
+
+  // A fragments of q (rows = heads; head h = lane / 4, zero for h >= G),
+  // k-step t covers dims 16t .. 16t+15: qa[t][0] dims 16t + 2(lane%4) + {0,1},
+  // qa[t][1] the same + 8.
+  const int hr = lane >> 2;  // this lane's head (fragment row)
+  const int q4 = lane & 3;
+  uint32_t qa[8][2];
+  {
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+        a.q + ((size_t)b * Hq + hkv * G + (hr < G ? hr : 0)) * kDecD);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      qa[t][0] = hr < G ? __ldg(qrow + 8 * t + q4) : 0u;
+      qa[t][1] = hr < G ? __ldg(qrow + 8 * t + 4 + q4) : 0u;
+    }
+  }
+
+  // ldmatrix row addresses: lane l serves row l % 8 of matrix l / 8.
+  //  scores (K, no transpose): matrix m = chunk 2p + m of keys 16w + 8g + l%8
+  //  P.V (V, transposed): matrix m = keys 16w + 8(m&1) + l%8, chunk 2p + m/2
+  const int mi = lane >> 3, mr = lane & 7;
+  const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
+
+  float o[16][2];  // O of head hr, dims 8n + 2 q4 + {0,1}
+#pragma unroll
+  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = 0.f;
+  float m_run[G];  // running max of each head (replicated in every thread)
+#pragma unroll
+  for (int g = 0; g < G; ++g) m_run[g] = -INFINITY;
+  float l_part = 0.f;  // this lane's part of the normaliser of head hr
+  // the kept block waiting for its P.V
+  bool pend = false;
+  uint32_t pp0 = 0, pp1 = 0;  // its P as A fragment (keys 16w + 2q4 (+8))
+  float palpha = 1.f;          // its rescale factor for head hr
+  int kept = 0;                // kept blocks so far (V slot = index % 2)
+
+  const float scale = a.scale, ln_lambda = a.ln_lambda;
+  unsigned long long n_vis = 0, n_skp = 0;
+  bool ok = true;
+
+  auto pv = [&](int kidx) -> bool {
+    const int slot = kidx % C::NV;
+    if (!mbar_wait(&vfull[slot], (uint32_t)(kidx / C::NV) & 1u, kWaitDecodeV,
+                   kidx, slot))
+      return false;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      o[n][0] *= palpha;
+      o[n][1] *= palpha;
+    }
+    const uint32_t vb = aV + slot * C::TILE;
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      uint32_t r0, r1, r2, r3;
+      ldsm_x4_t(vb + swz_off(16 * warp + 8 * (mi & 1) + mr, 2 * p + (mi >> 1)),
+                r0, r1, r2, r3);
+      mma16816_top(o[2 * p][0], o[2 * p][1], pp0, pp1, r0, r1);
+      mma16816_top(o[2 * p + 1][0], o[2 * p + 1][1], pp0, pp1, r2, r3);
+    }
+    return true;
+  };
+
+  for (int r = 0; r < nblk; ++r) {
+    const int j = j0 + r;
+    const int stage = r % C::NK;
+    if (!mbar_wait(&kfull[stage], (uint32_t)(r / C::NK) & 1u, kWaitDecodeK, r,
+                   stage))
+      ok = false;
+    // ---- scores of this warp's 16 keys: sc[g][i] = key 16w + 8g + 2q4 + i
+    float sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    if (ok) {
+      const uint32_t kb = aK + stage * C::TILE;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {  // k-steps 2p, 2p+1 (chunks 4p .. 4p+3)
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4(kb + swz_off(16 * warp + 8 * g + mr, 4 * p + mi), r0, r1, r2,
+                  r3);
+          mma16816_top(sc[g][0], sc[g][1], qa[2 * p][0], qa[2 * p][1], r0, r1);
+          mma16816_top(sc[g][0], sc[g][1], qa[2 * p + 1][0], qa[2 * p + 1][1],
+                       r2, r3);
+        }
+      }
+    }
+    const int kbase = j * kDecBc + 16 * warp + 2 * q4;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int g = 0; g < 2; ++g)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int key = kbase + 8 * g + i;
+        sc[g][i] = (key < a.Lkv && key >= key_lo) ? sc[g][i] * scale : -INFINITY;
+        mx = fmaxf(mx, sc[g][i]);
+      }
+    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
+    float* sMr = sM + (r & 1) * 32;  // [head][warp], double-buffered
+    if (q4 == 0 && hr < G) sMr[hr * 4 + warp] = mx;
+    if (__syncthreads_or(!ok)) { ok = false; break; }
+    // every warp has read K slot `stage`: refill it
+    if (tid == 0 && r + C::NK < nblk)
+      load(&a.tk, sK + stage * C::TILE, &kfull[stage], j + C::NK);
+
+    // ---- decision (the same in every thread)
+    float mt[G];
+    bool skip = ln_lambda > -INFINITY;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float4 w4 = *reinterpret_cast<const float4*>(sMr + g * 4);
+      mt[g] = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
+      if (!(mt[g] - m_run[g] < ln_lambda)) skip = false;
+    }
+    if (tid == 0) {
+      ++n_vis;
+      if (skip) ++n_skp;
+      if (a.mask) a.mask[(size_t)bh * a.nk + j] = skip ? 2 : 1;
+    }
+    if (!skip && !stats_only) {
+      if (tid == 0) load(&a.tv, sV + (kept % C::NV) * C::TILE, &vfull[kept % C::NV], j);
+      // the previous kept block's P.V (its V has had this block to land)
+      if (pend && !pv(kept - 1)) { ok = false; }
+      // new reference, rescale factor and P of head hr
+      float mo = m_run[0], mh = mt[0];  // head hr's (head 0's for padding rows)
+#pragma unroll
+      for (int g = 1; g < G; ++g)
+        if (g == hr) {
+          mo = m_run[g];
+          mh = mt[g];
+        }
+      const float mn = fmaxf(mo, mh);
+      const float al = (mo == -INFINITY) ? 0.f : ex2_approx((mo - mn) * kLog2e);
+      const float mb = mn * kLog2e;
+      float p[2][2];
+#pragma unroll
+      for (int g = 0; g < 2; ++g)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) p[g][i] = ex2_approx(fmaf(sc[g][i], kLog2e, -mb));
+      l_part = al * l_part + ((p[0][0] + p[0][1]) + (p[1][0] + p[1][1]));
+      pp0 = pack_bf16x2(p[0][0], p[0][1]);
+      pp1 = pack_bf16x2(p[1][0], p[1][1]);
+      palpha = al;
+      pend = true;
+      ++kept;
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) m_run[g] = fmaxf(m_run[g], mt[g]);
+    if (__any_sync(FULL, !ok)) { ok = false; }
+  }
+  if (ok && pend && !pv(kept - 1)) ok = false;
+  if (__syncthreads_or(!ok)) ok = false;
+
+  if (!ok) {
+    // outstanding copies get a bounded chance to land before the shared
+    // memory is released
+    if (tid == 0) {
+      for (int i = 0; i < C::NK; ++i)
+        mbar_wait(&kfull[i], 0, kWaitDecodeDrain, i, 0, 1000000);
+      for (int i = 0; i < C::NV; ++i)
+        mbar_wait(&vfull[i], 0, kWaitDecodeDrain, i, 1, 1000000);
+    }
+    return;
+  }
+  if (tid == 0 && a.counters) {
+    atomicAdd(&a.counters[0], n_vis);
+    atomicAdd(&a.counters[1], n_skp);
+  }
+  if (stats_only) return;
+
+  // normaliser: the 4 lanes of a head in this warp, then the 4 warps
+  {
+    float x = l_part;
+    x += __shfl_xor_sync(FULL, x, 1);
+    x += __shfl_xor_sync(FULL, x, 2);
+    if (q4 == 0 && hr < G) sL[warp * 8 + hr] = x;
+  }
+  // per-warp outputs [warp][head][dim] in the (now idle) K ring
+  float* red = reinterpret_cast<float*>(sK);
+  if (hr < G) {
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+      *reinterpret_cast<float2*>(red + ((warp * 8 + hr) * kDecD + 8 * n + 2 * q4)) =
+          make_float2(o[n][0], o[n][1]);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int dd = tid;  // 128 threads = 128 dims
+    const float sum = red[(0 * 8 + g) * kDecD + dd] + red[(1 * 8 + g) * kDecD + dd] +
+                      red[(2 * 8 + g) * kDecD + dd] + red[(3 * 8 + g) * kDecD + dd];
+    const float l = sL[g] + sL[8 + g] + sL[16 + g] + sL[24 + g];
+    const size_t row = (size_t)b * Hq + hkv * G + g;
+    a.o_part[(row * a.S + s) * kDecD + dd] = l > 0.f ? sum / l : 0.f;
+    if (dd == 0)
+      a.lse_part[row * a.S + s] = l > 0.f ? m_run[g] + __logf(l) : -INFINITY;
+  }
+}
+
+}  // namespace blasst

@@ -19,6 +19,13 @@
 //               pending P.V is done), epilogue
 // Tensor memory: Q [0, 64) (bf16 pairs), S [64, 128), O [128, 256): 256
 // columns, two CTAs per SM.
+//
+// Tiles.  With T = G the G heads are one tile (one decision per block).
+// With T = 8 < G the heads form G / 8 tiles of 8 consecutive heads, each
+// voting on its own, exactly as the CUDA-core decode cuts wide groups: the
+// block's V load and P.V run when any tile keeps it, and the rows of a tile
+// that skips it get P = 0 (no exp) and keep their running state, so they
+// come out as if the block had not been touched.
 #pragma once
 
 #include "prefill.cuh"
@@ -35,8 +42,10 @@ struct WideArgs {
   float* o_part;             // [B*Hq, S, 128]
   float* lse_part;           // [B*Hq, S]
   unsigned long long* counters;
-  unsigned char* mask;       // [B*Hkv, nk]
+  unsigned char* mask;       // [B*Hkv*(G/T), nk]
   int Hkv, G, Lkv, nk, S;
+  int T;                     // heads per tile: G, or 8 (G a multiple of 8)
+  int window;                // sliding window: the last `window` keys (0 = all)
   float scale, ln_lambda;
   int stats_only;
 };
@@ -97,9 +106,17 @@ __global__ void __launch_bounds__(kWideThreads, 2)
   const int lane = threadIdx.x & 31;
   const int s = blockIdx.x % a.S;
   const int bh = blockIdx.x / a.S;  // b * Hkv + hkv
-  const int j0 = (int)(((long long)s * a.nk) / a.S);
-  const int j1 = (int)(((long long)(s + 1) * a.nk) / a.S);
+  // first visible key and its block (sliding window); the splits divide
+  // the blocks from there on
+  const int key_lo = (a.window > 0 && a.Lkv > a.window) ? a.Lkv - a.window : 0;
+  const int jlo = key_lo / kWideBc;
+  const int j0 = jlo + (int)(((long long)s * (a.nk - jlo)) / a.S);
+  const int j1 = jlo + (int)(((long long)(s + 1) * (a.nk - jlo)) / a.S);
   const int nb = j1 - j0;
+  const int ntile = a.G / a.T;  // tiles per KV head
+  if (a.mask && s == 0)  // blocks left of the window are not visited
+    for (int e = threadIdx.x; e < ntile * jlo; e += kWideThreads)
+      a.mask[((size_t)bh * ntile + e / jlo) * a.nk + e % jlo] = 0;
 
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint32_t* dec_word = reinterpret_cast<uint32_t*>(smem + C::OFF_DEC);
@@ -245,6 +262,11 @@ __global__ void __launch_bounds__(kWideThreads, 2)
     const bool active = h < a.G;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const bool elected = (quad == 0 && lane == 0);
+    // the first row of each tile keeps the tile's statistics
+    const bool tile_lead = active && (h % a.T) == 0;
+    const size_t mask_row = ((size_t)bh * ntile + h / a.T) * a.nk;
+    const uint32_t tbits = a.T >= 32 ? FULL : ((1u << a.T) - 1u);
+    const int tshift = a.T >= 32 ? 0 : (lane / a.T) * a.T;
     const int b = bh / a.Hkv;
     const int hkv = bh - b * a.Hkv;
     const size_t qrow_i = (size_t)(b * a.Hkv + hkv) * a.G;  // first head row
@@ -289,12 +311,14 @@ __global__ void __launch_bounds__(kWideThreads, 2)
       tmem_ld32(lane_base + C::COL_S + 32, sr[1]);
       tc_wait_ld();
       const int valid = min(kWideBc, a.Lkv - j * kWideBc);
-      if (valid < kWideBc) {
+      const int first = key_lo - j * kWideBc;  // keys below it are hidden
+      if (valid < kWideBc || first > 0) {
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int x = 0; x < 32; ++x)
-            if (c * 32 + x >= valid) sr[c][x] = __float_as_uint(-INFINITY);
+            if (c * 32 + x >= valid || c * 32 + x < first)
+              sr[c][x] = __float_as_uint(-INFINITY);
       }
       float m8[8];
 #pragma unroll
@@ -315,15 +339,22 @@ __global__ void __launch_bounds__(kWideThreads, 2)
       // a failed wait in any thread ends the loop for all, after the vote
       volatile int* abort_w = reinterpret_cast<volatile int*>(smem + C::OFF_TMEM + 4);
       if (!w) *abort_w = 1;
+      // this row's tile: the AND of its T rows' votes (one warp holds a
+      // tile of 8; a tile of all G rows is the whole vote below)
+      const unsigned bal = __ballot_sync(FULL, pred);
       const bool all = named_sync_and(1, 128, pred && w);
       if (*abort_w) { ok = false; break; }
-      const bool skip = all && (ln_lambda > -INFINITY);
-      if (elected) {
+      const bool tile_all = a.T == a.G ? all
+                                       : ((bal >> tshift) & tbits) == tbits;
+      const bool skip = all && (ln_lambda > -INFINITY);        // the block
+      const bool skip_row = tile_all && (ln_lambda > -INFINITY);  // my tile
+      if (elected)
         st_release_shared(&dec_word[jj % C::R],
                           ((uint32_t)(jj + 1) << 1) | (skip ? 1u : 0u));
+      if (tile_lead) {
         ++n_vis;
-        if (skip) ++n_skp;
-        if (a.mask) a.mask[(size_t)bh * a.nk + j] = skip ? 2 : 1;
+        if (skip_row) ++n_skp;
+        if (a.mask) a.mask[mask_row + j] = skip_row ? 2 : 1;
       }
       if (skip || stats_only) {
         if (active) m_crit = fmaxf(m_crit, mt_s);
@@ -331,7 +362,7 @@ __global__ void __launch_bounds__(kWideThreads, 2)
       }
       float alpha = 1.f;
       bool rescale = false;
-      if (active && mt_s != -INFINITY) {
+      if (active && !skip_row && mt_s != -INFINITY) {
         const float m_new = fmaxf(m_crit, mt_s);
         if (m_ref == -INFINITY || m_new > m_ref + kRescaleNats) {
           alpha = (m_ref == -INFINITY) ? 0.f
@@ -340,8 +371,10 @@ __global__ void __launch_bounds__(kWideThreads, 2)
           rescale = true;
         }
       }
-      const float mb = (active && m_ref != -INFINITY) ? m_ref * kPrefLog2e
-                                                      : INFINITY;
+      // a row of a tile that skips the block gets P = 0: exp2(-inf)
+      const float mb = (active && !skip_row && m_ref != -INFINITY)
+                           ? m_ref * kPrefLog2e
+                           : INFINITY;
       // P (bf16, this row's 64 keys = one 128-byte swizzled row) into P
       // slot kp % 2, once the P.V two kept blocks back has read it
       const int psl = kp & 1;
@@ -394,7 +427,7 @@ __global__ void __launch_bounds__(kWideThreads, 2)
       ++kp;
       if (active) m_crit = fmaxf(m_crit, mt_s);
     }
-    if (ok && elected && a.counters && nb > 0) {
+    if (ok && tile_lead && a.counters && nb > 0) {
       atomicAdd(&a.counters[0], n_vis);
       atomicAdd(&a.counters[1], n_skp);
     }

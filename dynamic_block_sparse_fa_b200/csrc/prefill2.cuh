@@ -23,6 +23,12 @@
 // MMA warp issues QK_t(j+1) after P_t.V_j, the arrival of S_t(j+1) also
 // certifies that O_t is no longer being written, so the softmax may rescale
 // O_t without a further wait.
+//
+// SKIP = false builds the dense forward without the skip machinery (no vote
+// barrier, no decision words; V is loaded for every block as soon as its
+// slot is free).  The library runs it for ln lambda = -inf, so the cost of
+// the vote on the dense path can be measured against the SKIP = true kernel
+// run with a threshold that never skips (ln lambda = -FLT_MAX).
 #pragma once
 
 #include "prefill.cuh"
@@ -67,7 +73,7 @@ struct Prefill2Cfg {
   static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
 };
 
-template <int D>
+template <int D, bool SKIP>
 __global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
     prefill2_kernel(const __grid_constant__ PrefillParams p) {
   using C = Prefill2Cfg<D>;
@@ -193,10 +199,10 @@ __global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
     int vcount = 0;
     for (int j = jlo; j < nblk; ++j) {
       if (!stats_only) {
-        bool need = false, ok = true;
+        bool need = !SKIP && (in_range(0, j) || in_range(1, j)), ok = true;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (need || !in_range(t, j)) continue;
+          if (!SKIP || need || !in_range(t, j)) continue;
           const int jt = j - jlo_t[t];
           const bool w = mbar_wait(&bar[C::B_DEC + t * C::R + jt % C::R],
                                    (jt / C::R) & 1, kWaitPrefillLoad, j,
@@ -238,33 +244,43 @@ __global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
     // ------------------------------------------------------------------
     constexpr uint32_t idesc_s = idesc_bf16(128, BN, 0, 0);
     constexpr uint32_t idesc_o = idesc_bf16(128, D, 0, 1);
-    const uint32_t aQ = smem_u32(sQ);
-    const uint32_t aK = smem_u32(sK);
-    const uint32_t aV = smem_u32(sV);
+    // Descriptors of the operand buffers, built once.  Stepping through an
+    // operand only adds (byte offset >> 4) to the start-address field: every
+    // address stays below 256 KB, so the 14-bit field never carries.
+    const uint64_t dQ0 = smem_desc(smem_u32(sQ), 16, 1024, 2);
+    const uint64_t dQ1 = smem_desc(smem_u32(sQ) + C::QBYTES, 16, 1024, 2);
+    const uint64_t dK0 = smem_desc(smem_u32(sK), 16, 1024, 2);
+    const uint64_t dK1 = smem_desc(smem_u32(sK) + C::KBYTES, 16, 1024, 2);
+    const uint64_t dV0 = smem_desc(smem_u32(sV), C::BOX_K, 1024, 2);
+    const uint64_t dV1 = smem_desc(smem_u32(sV) + C::KBYTES, C::BOX_K, 1024, 2);
+    static_assert(C::NKS == 2 && C::NVS == 2, "two K and two V slots");
     auto qk = [&](int t, int j) {
       const int st = (j - jlo) % C::NKS;
       const uint32_t d_s = tmem + C::COL_S + t * 128;
+      const uint64_t da0 = t ? dQ1 : dQ0;
+      const uint64_t db0 = st ? dK1 : dK0;
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
-        const uint32_t off = (uint32_t)(k & 3) * 32;  // 16 columns = 32 B
-        const uint64_t da = smem_desc(
-            aQ + t * C::QBYTES + (k >> 2) * C::BOX_Q + off, 16, 1024, 2);
-        const uint64_t db = smem_desc(
-            aK + st * C::KBYTES + (k >> 2) * C::BOX_K + off, 16, 1024, 2);
-        mma_ss(d_s, da, db, idesc_s, k > 0 ? 1u : 0u);
+        // 16 columns = 32 B within a 64-column box; boxes are BOX_* apart
+        const uint64_t ka = (uint64_t)(((k >> 2) * C::BOX_Q + (k & 3) * 32) >> 4);
+        const uint64_t kb = (uint64_t)(((k >> 2) * C::BOX_K + (k & 3) * 32) >> 4);
+        mma_ss_elect(d_s, da0 + ka, db0 + kb, idesc_s, k > 0 ? 1u : 0u);
       }
-      mma_commit(&bar[C::B_SF + t]);
+      mma_commit_elect(&bar[C::B_SF + t]);
     };
-    // One lane issues.  All waits of a tile's step come before its MMAs, so
-    // the P.V and the next QK^T of a tile go to the tensor core back to back.
-    if (leader) {
+    // The whole warp runs the loop; one elected lane issues each MMA and
+    // commit.  Waits are taken by every lane and made warp-uniform.  All
+    // waits of a tile's step come before its MMAs, so the P.V and the next
+    // QK^T of a tile go to the tensor core back to back.
+    {
       bool ok = mbar_wait(&bar[C::B_Q], 0, kWaitPrefillMma, 0, 0) &&
                 mbar_wait(&bar[C::B_KF], 0, kWaitPrefillMma, 0, 0);
+      ok = __all_sync(FULL, ok);
       tc_fence_after();
       if (ok) {
         for (int t = 0; t < 2; ++t)
           if (in_range(t, jlo)) qk(t, jlo);
-        mma_commit(&bar[C::B_KE]);
+        mma_commit_elect(&bar[C::B_KE]);
       }
       int vcount = 0;
       int npv[2] = {0, 0};  // kept blocks of each tile so far
@@ -277,7 +293,12 @@ __global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
           if (!ok || !(cur || more)) continue;
           const int jt = j - jlo_t[t];
           bool kept = false;
-          if (cur) {
+          if (cur && !SKIP) {
+            kept = true;
+            ok = mbar_wait(&bar[C::B_PF + t], npv[t] & 1, kWaitPrefillMma, j,
+                           300 + t);
+            if (!__all_sync(FULL, ok)) { ok = false; break; }
+          } else if (cur) {
             // The decision word: a skipped block needs nothing more (its
             // scores were read before the vote), a kept one its P (B_PF,
             // one phase per kept block).
@@ -293,13 +314,13 @@ __global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
                   break;
                 }
               }
-              if (!ok) break;
+              if (!__all_sync(FULL, ok)) { ok = false; break; }
             }
             kept = !stats_only && (w & 1u) == 0;
             if (kept) {
               ok = mbar_wait(&bar[C::B_PF + t], npv[t] & 1, kWaitPrefillMma, j,
                              300 + t);
-              if (!ok) break;
+              if (!__all_sync(FULL, ok)) { ok = false; break; }
             }
           }
           if (kept && vslot < 0) {
@@ -307,34 +328,33 @@ __global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
             ok = mbar_wait(&bar[C::B_VF + vslot], (vcount / C::NVS) & 1,
                            kWaitPrefillMma, j, 200 + vslot);
             ++vcount;
-            if (!ok) break;
+            if (!__all_sync(FULL, ok)) { ok = false; break; }
           }
           if (more) {
             const int jr1 = j + 1 - jlo;
             ok = mbar_wait(&bar[C::B_KF + jr1 % C::NKS], (jr1 / C::NKS) & 1,
                            kWaitPrefillMma, j + 1, jr1 % C::NKS);
-            if (!ok) break;
+            if (!__all_sync(FULL, ok)) { ok = false; break; }
           }
           tc_fence_after();
           if (kept) {
             const uint32_t a_p = tmem + C::COL_S + t * 128;
+            const uint64_t dv0 = vslot ? dV1 : dV0;
 #pragma unroll
-            for (int k = 0; k < BN / 16; ++k) {
-              const uint64_t db = smem_desc(aV + vslot * C::KBYTES + k * 2048,
-                                            C::BOX_K, 1024, 2);
-              mma_ts(tmem + C::COL_O + t * 128, a_p + k * 8, db, idesc_o,
+            for (int k = 0; k < BN / 16; ++k)  // 16 keys = 16 rows of 128 B
+              mma_ts_elect(tmem + C::COL_O + t * 128, a_p + k * 8,
+                     dv0 + (uint64_t)((k * 2048) >> 4), idesc_o,
                      (npv[t] > 0 || k > 0) ? 1u : 0u);
-            }
             ++npv[t];
           }
           if (more)
             qk(t, j + 1);
           else
-            mma_commit(&bar[C::B_OD + t]);  // tile t has issued its last MMA
+            mma_commit_elect(&bar[C::B_OD + t]);  // tile t has issued its last MMA
         }
-        if (!ok) break;
-        if (vslot >= 0) mma_commit(&bar[C::B_VE + vslot]);
-        if (j + 1 < nblk) mma_commit(&bar[C::B_KE + (j + 1 - jlo) % C::NKS]);
+        if (!__all_sync(FULL, ok)) { ok = false; break; }
+        if (vslot >= 0) mma_commit_elect(&bar[C::B_VE + vslot]);
+        if (j + 1 < nblk) mma_commit_elect(&bar[C::B_KE + (j + 1 - jlo) % C::NKS]);
       }
     }
     __syncwarp();
@@ -420,16 +440,25 @@ __global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
       const bool pred = !active || mt_s == -INFINITY ||
                         (mt_s - m_crit < ln_lambda);
       tc_fence_before();
-      const bool skip =
-          named_sync_and(bar_id, kBarThreads, pred) && (ln_lambda > -INFINITY);
-      if (abort_t[t]) { ok = false; break; }
+      bool skip = false;
+      if constexpr (SKIP) {
+        skip = named_sync_and(bar_id, kBarThreads, pred) &&
+               (ln_lambda > -INFINITY);
+        if (abort_t[t]) { ok = false; break; }
+      } else {
+        // no vote: every block is kept; a wait that gave up ends the warp
+        __syncwarp();
+        if (__any_sync(FULL, abort_t[t] != 0)) { ok = false; break; }
+      }
       if (elected) {
         ++n_vis;
         if (skip) ++n_skp;
         if (p.mask) p.mask[mask_row + j] = skip ? 2 : 1;
-        st_release_shared(&dec_word[t * C::R + jt % C::R],
-                          ((uint32_t)(jt + 1) << 1) | (skip ? 1u : 0u));
-        mbar_arrive(&bar[C::B_DEC + t * C::R + jt % C::R]);
+        if constexpr (SKIP) {
+          st_release_shared(&dec_word[t * C::R + jt % C::R],
+                            ((uint32_t)(jt + 1) << 1) | (skip ? 1u : 0u));
+          mbar_arrive(&bar[C::B_DEC + t * C::R + jt % C::R]);
+        }
       }
       if (skip || stats_only) {  // the issuer reads the decision word
         if (active) m_crit = fmaxf(m_crit, mt_s);
@@ -541,8 +570,8 @@ __global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
   }
 }
 
-template <int D>
-cudaError_t launch_prefill2(const PrefillProblem& pr, cudaStream_t st) {
+template <int D, bool SKIP>
+cudaError_t launch_prefill2_t(const PrefillProblem& pr, cudaStream_t st) {
   using C = Prefill2Cfg<D>;
   PrefillParams p;
   memset(&p, 0, sizeof p);
@@ -569,12 +598,21 @@ cudaError_t launch_prefill2(const PrefillProblem& pr, cudaStream_t st) {
   p.window = pr.window;
   const long long grid = (long long)((p.nq + 1) / 2) * pr.B * pr.Hq;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(prefill2_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(prefill2_kernel<D, SKIP>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
-  prefill2_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM_ALLOC, st>>>(p);
+  prefill2_kernel<D, SKIP><<<(unsigned)grid, C::THREADS, C::SMEM_ALLOC, st>>>(p);
   return cudaGetLastError();
+}
+
+// The dense forward (ln lambda = -inf, outputs requested) runs the kernel
+// without the vote; every other call runs the skipping kernel.
+template <int D>
+cudaError_t launch_prefill2(const PrefillProblem& pr, cudaStream_t st) {
+  if (pr.ln_lambda == -INFINITY && pr.o != nullptr)
+    return launch_prefill2_t<D, false>(pr, st);
+  return launch_prefill2_t<D, true>(pr, st);
 }
 
 }  // namespace blasst

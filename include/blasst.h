@@ -100,6 +100,13 @@ typedef struct {
  *  d           64 or 128
  *  Br, Bc      (64, 64) or (128, 128)
  *  skip_stats  host pointer to the statistics struct, or NULL
+ *
+ * With 128 x 128 tiles and o given, ln_lambda = -INFINITY runs a dense
+ * kernel built without the skip machinery (no vote, no decision hand-offs,
+ * V loaded for every block without waiting for a decision).  Any finite
+ * ln_lambda runs the skipping kernel; ln_lambda = -FLT_MAX skips nothing
+ * either (no score gap reaches it), so it gives the same result through
+ * the skipping kernel and measures what the vote costs on the dense path.
  */
 blasst_status_t blasst_prefill(const void *q, const void *k, const void *v,
                                void *o, float *lse, int B, int Hq, int Hkv,
@@ -180,8 +187,11 @@ blasst_status_t blasst_prefill_backward(
  * The G = Hq/Hkv query heads sharing a KV head form the rows of one tile, so
  * every K and V byte read serves all G heads.  A tile has at most 8 rows:
  * for G = 16, 32, ... (MQA with many heads) the heads of a KV head are cut
- * into G/8 consecutive tiles of 8 heads, each with its own skip decisions,
- * which read the same KV head (through L2 when they run together).  The Lkv keys are cut into
+ * into G/8 consecutive tiles of 8 heads, each with its own skip decisions.
+ * For 16 <= G <= 128 one tensor-core CTA scores all tiles of a KV head
+ * (the V block is read when any tile keeps it; the rows of a tile that
+ * skips it are left untouched); for G <= 8 and G = 256 the CUDA-core
+ * kernel runs one CTA per tile.  The Lkv keys are cut into
  * nk = ceil(Lkv/Bc) blocks and the blocks into num_splits contiguous splits
  * (split s covers blocks [floor(s*nk/S), floor((s+1)*nk/S))).  Each split
  * runs the blockwise forward independently (its running max starts at

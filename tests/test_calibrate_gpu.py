@@ -48,9 +48,12 @@ def prefill_sample():
 
 @pytest.fixture(scope="module")
 def decode_sample(blasst):
-    x = planted_gap(4, 32, 8, 1, 8192, 128, decode=True, block=64, gap=8.0,
+    # 16 sequences x 8 KV heads x 16K keys in 4 splits of 64 blocks (a
+    # split's first block is never skipped and short splits cap the
+    # reachable sparsity)
+    x = planted_gap(16, 32, 8, 1, 16384, 128, decode=True, block=64, gap=8.0,
                     heavy_frac=0.03, seed=config_seed(1, 77), device="cuda")
-    S = blasst.blasst_decode_splits(4, 8, 8192, 64)
+    S = 4
     delta = C.deltas_decode(x.q, x.k, x.v, 1 / math.sqrt(128), 64, S)
     return x, delta, S
 
@@ -101,11 +104,20 @@ def test_calibrate_decode_matches_oracle(blasst, decode_sample, target, tol):
     x, delta, S = decode_sample
     got = blasst.blasst_calibrate(target, mode="decode", q=x.q, k=x.k, v=x.v,
                                   Bc=64, num_splits=S, tol=tol)
-    _check(got, delta, target, tol, 8192)
-    # the automatic split count resolves to the same S
-    auto = blasst.blasst_calibrate(target, mode="decode", q=x.q, k=x.k,
-                                   v=x.v, Bc=64, num_splits=0, tol=tol)
-    assert auto["ln_lambda"] == got["ln_lambda"]
+    _check(got, delta, target, tol, 16384)
+
+
+def test_calibrate_decode_automatic_splits(blasst, decode_sample):
+    """num_splits = 0 calibrates with the split count blasst_decode_splits
+    gives (the decisions depend on it)."""
+    x, _, _ = decode_sample
+    S = blasst.blasst_decode_splits(16, 8, 16384, 64)
+    a = blasst.blasst_calibrate(0.5, mode="decode", q=x.q, k=x.k, v=x.v,
+                                Bc=64, num_splits=0)
+    b = blasst.blasst_calibrate(0.5, mode="decode", q=x.q, k=x.k, v=x.v,
+                                Bc=64, num_splits=S)
+    for key in ("ln_lambda", "achieved", "iterations", "visited", "skipped"):
+        assert a[key] == b[key], key
 
 
 def test_calibrate_unreachable_and_zero_targets(blasst, decode_sample):
@@ -132,7 +144,7 @@ def test_sharded_search_equals_library_search(blasst, decode_sample, target):
     lib = blasst.blasst_calibrate(target, mode="decode", q=x.q, k=x.k,
                                   v=x.v, Bc=64, num_splits=S, tol=0.002)
     sh = calibrate_sharded(decode_counter(x.q, x.k, x.v, Bc=64, num_splits=S),
-                           target, L=8192, tol=0.002)
+                           target, L=16384, tol=0.002)
     torch.cuda.synchronize()
     for key in ("ln_lambda", "achieved", "iterations", "visited", "skipped",
                 "status"):

@@ -89,6 +89,10 @@ def test_batched_decode_matches_oracle(blasst, case):
 
 
 def test_batch_one_equals_decode(blasst):
+    """batch = 1 is the sequential rule: the same decisions as
+    blasst_decode (which runs it on the warp-MMA kernel; batch 1 runs on the
+    CUDA-core kernel), so masks agree except on near-ties and outputs within
+    the parity tolerance."""
     m = blasst
     x = planted_gap(2, 8, 2, 1, 1500, 128, decode=True, block=64, gap=8.0,
                     heavy_frac=0.05, seed=config_seed(9, 1), device="cuda")
@@ -98,8 +102,13 @@ def test_batch_one_equals_decode(blasst):
     o2, l2 = m.blasst_decode_batched(x.q, x.k, x.v, batch=1, ln_lambda=-3.0,
                                      num_splits=3, stats=s2)
     torch.cuda.synchronize()
-    assert torch.equal(o1, o2) and torch.equal(l1, l2)
-    assert torch.equal(s1.mask, s2.mask)
+    ref = oracle.decode(x.q, x.k, x.v, 1 / math.sqrt(128), -3.0, 64, 3)
+    P.check_mask(s1.mask.cpu().numpy().reshape(2, 2, 24), ref["mask"],
+                 ref["margin"], "decode")
+    P.check_mask(s2.mask.cpu().numpy().reshape(2, 2, 24), ref["mask"],
+                 ref["margin"], "batch 1")
+    P.check_out(P.to_np(o1), P.to_np(o2), "decode vs batch 1")
+    P.check_lse(P.to_np(l1), P.to_np(l2), "decode vs batch 1")
 
 
 def test_batched_skips_superset_of_sequential(blasst):

@@ -3,11 +3,14 @@ many heads, GQA 16:1 and 32:1) against the CPU oracle, through the C ABI.
 
 The decode tile holds at most 8 query heads: for G = Hq/Hkv = 16, 32, 64
 the heads of a KV head are cut into G/8 consecutive tiles with their own
-skip decisions (the oracle's ``tile_heads=8``).  Checks outputs (max 2e-2 /
-mean 2e-3), lse, masks [B, Hkv*G/8, nk] bit-exact except near-ties,
-counters, the statistics-only pass, the sliding window, the batched
-decision rule, the paged cache, a full-size MQA sample, and that a group
-that is not a power of two is refused.
+skip decisions (the oracle's ``tile_heads=8``).  blasst_decode and
+blasst_decode_window run these tiles on the tensor-core kernel (one CTA for
+all tiles of a KV head); the batched rule and the paged cache run them on
+the CUDA-core kernel (one CTA per tile).  Checks outputs (max 2e-2 / mean
+2e-3), lse, masks [B, Hkv*G/8, nk] bit-exact except near-ties, counters,
+the statistics-only pass, the sliding window, the batched decision rule,
+the paged cache against both contiguous kernels, a full-size MQA sample,
+and that a group that is not a power of two is refused.
 """
 import math
 
@@ -120,16 +123,26 @@ def test_mqa_paged_equals_contiguous(blasst):
                     heavy_frac=0.05, seed=config_seed(10, 2), device="cuda")
     nk = -(-L // Bc)
     s1, s2 = m.Stats(mask_numel=B * 4 * nk), m.Stats(mask_numel=B * 4 * nk)
-    o1, l1 = m.blasst_decode(x.q, x.k, x.v, ln_lambda=-3.0, num_splits=3,
-                             stats=s1)
+    # the CUDA-core kernel on the contiguous cache (batch 1 = sequential rule)
+    o1, l1 = m.blasst_decode_batched(x.q, x.k, x.v, batch=1, ln_lambda=-3.0,
+                                     num_splits=3, stats=s1)
     pk = paginate(x.k, x.v, [L] * B, 64, seed=4, spare_pages=3)
     o2, l2 = m.blasst_decode_paged(x.q, pk.k_pages, pk.v_pages,
                                    pk.block_table, pk.seq_lens,
                                    max_seq_len=L, ln_lambda=-3.0,
                                    num_splits=3, stats=s2)
+    # the tensor-core kernel of blasst_decode: same tiles and decisions
+    s3 = m.Stats(mask_numel=B * 4 * nk)
+    o3, l3 = m.blasst_decode(x.q, x.k, x.v, ln_lambda=-3.0, num_splits=3,
+                             stats=s3)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     assert torch.equal(s1.mask, s2.mask)
+    ref = oracle.decode(x.q, x.k, x.v, 1 / math.sqrt(128), -3.0, Bc, 3,
+                        tile_heads=8)
+    P.check_mask(s3.mask.cpu().numpy().reshape(B, 4, nk), ref["mask"],
+                 ref["margin"], "tensor-core tiles of 8")
+    P.check_out(P.to_np(o3), P.to_np(o1), "tensor-core vs CUDA-core tiles")
 
 
 def test_group_not_power_of_two_is_refused(blasst):

@@ -96,6 +96,38 @@ def test_prefill_matches_oracle(blasst, case):
         assert (mask == 2).sum() == 0
 
 
+@pytest.mark.parametrize("d,L,causal", [(128, 2048, True), (64, 1000, True),
+                                         (128, 700, False)])
+def test_dense_kernel_without_vote_equals_voting_kernel(blasst, d, L, causal):
+    """ln lambda = -inf runs the 128x128 kernel built without the vote;
+    -FLT_MAX runs the voting kernel with a threshold nothing reaches.  The
+    arithmetic is the same, so the outputs agree bit for bit, and both
+    match the oracle's dense result."""
+    m = blasst
+    x = planted_gap(1, 4, 2, L, L, d, block=128, gap=8.0, heavy_frac=0.03,
+                    window=256, seed=config_seed(0, 900 + L + d),
+                    device="cuda")
+    nq = nk = -(-L // 128)
+    st = m.Stats(mask_numel=4 * nq * nk)
+    o1, l1 = m.blasst_prefill(x.q, x.k, x.v, causal=causal,
+                              ln_lambda=-math.inf, stats=st)
+    st2 = m.Stats(mask_numel=4 * nq * nk)
+    o2, l2 = m.blasst_prefill(x.q, x.k, x.v, causal=causal,
+                              ln_lambda=-3.4028234663852886e38, stats=st2)
+    torch.cuda.synchronize()
+    assert m.blasst_check_device_error()[0] == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert torch.equal(st.mask, st2.mask) and st.read() == st2.read()
+    assert int((st.mask == 2).sum()) == 0
+    ref = oracle.prefill(x.q, x.k, x.v, 1 / math.sqrt(d), causal, -math.inf,
+                         128, 128)
+    go = np.concatenate([P.to_np(o1)[b, h, i * 128:min((i + 1) * 128, L)]
+                         for (b, h, i) in ref["units"]])
+    ro = np.concatenate([ref["o"][u, :min(128, L - i * 128)]
+                         for u, (b, h, i) in enumerate(ref["units"])])
+    P.check_out(go, ro, "dense kernel without vote")
+
+
 def test_prefill_rejects_bad_arguments(blasst):
     q = torch.zeros(1, 2, 128, 128, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(blasst.BlasstError, match="INVALID_ARG"):
