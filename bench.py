@@ -62,7 +62,8 @@ DEC = dict(B=32, Hq=32, Hkv=8, Lkv=32768, d=128, Bc=64, target=0.70,
 # benchmarked launch.  It holds only for the kernel source it was measured
 # on (sha256 prefix below); a source without a capture reports null.
 DECODE_TRAFFIC = dict(source="dynamic_block_sparse_fa_b200/csrc/decode_mma.cuh",
-                      sha256_16=None, ratio=None)
+                      sha256_16="8e810063372e6f84",
+                      ratio=(950.732288 + 4.634112) / 957.799424)
 PRE = dict(B=1, Hq=32, Hkv=8, L=32768, d=128, Br=128, Bc=128, window=4096)
 
 
@@ -480,6 +481,9 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
     }
 
     # ---------------- 50% calibrated sparsity, same inputs ----------------
+    if args.no_s50:
+        return finish_decode(args, bl, dev, stream, q, k, v, lnl, cal, S, ms_max,
+                             by_call, rank, world, line)
     cal50 = bl.blasst_calibrate(0.50, mode="decode", q=q, k=k, v=v, Bc=Bc,
                                 tol=0.002)
     st50 = bl.Stats(device=dev, mask_numel=B * Hkv * nk)
@@ -509,6 +513,14 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
             f"oracle margins of sequences {DEC_TIE_SEQS} (all heads); a pair "
             f"is a near-tie when |max_r(m~ - m) - ln lambda| < {NEAR_TIE}")
 
+    return finish_decode(args, bl, dev, stream, q, k, v, lnl, cal, S, ms_max,
+                         by_call, rank, world, line)
+
+
+def finish_decode(args, bl, dev, stream, q, k, v, lnl, cal, S, ms_max, by_call,
+                  rank, world, line):
+    """The decode variants on the same cache, and the CPU oracle baseline."""
+    K = args.steps
     if not args.no_paged:
         line["decode_paged"] = run_decode_paged(args, bl, dev, stream, q, k, v,
                                                 lnl, cal["a"], S, ms_max / K,
@@ -516,6 +528,8 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
     if not args.no_window:
         line["decode_window"] = run_decode_window(args, bl, q, k, v, lnl,
                                                   stream)
+        ws = torch.empty(bl.blasst_decode_workspace_size(
+            q.shape[0], q.shape[1], q.shape[2], S), dtype=torch.uint8, device=dev)
         line["decode_batched"] = run_decode_batched(args, bl, q, k, v, lnl, S,
                                                     ws, ms_max / K)
 
@@ -1264,6 +1278,8 @@ def main():
     ap.add_argument("--prefill-L", type=int, default=PRE["L"])
     ap.add_argument("--prefill-lnl", type=float, default=None,
                     help="measure prefill only at this ln(lambda)")
+    ap.add_argument("--no-s50", action="store_true",
+                    help="skip the decode leg at 50%% sparsity (profiling runs)")
     ap.add_argument("--no-sweeps", action="store_true",
                     help="skip the decode length and prefill calibration sweeps")
     ap.add_argument("--sweep-lengths", type=int, nargs="+",
