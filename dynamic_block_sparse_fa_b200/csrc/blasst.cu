@@ -189,34 +189,44 @@ cudaError_t launch_split(const blasst::DecodeArgs& a, long long grid,
 
 // The warp-MMA decode (decode_mma.cuh) for the sequential rule on a
 // contiguous cache with G <= 8, then the merge as for launch_decode.
-template <int G>
+template <int G, int D>
 cudaError_t launch_mma_split(const blasst::DecodeMmaArgs& a, long long grid,
                              cudaStream_t st) {
   using C = blasst::DecodeMmaCfg;
   cudaError_t e = cudaFuncSetAttribute(
-      blasst::decode_mma_kernel<G>,
+      blasst::decode_mma_kernel<G, D>,
       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
-  blasst::decode_mma_kernel<G>
+  blasst::decode_mma_kernel<G, D>
       <<<(unsigned)grid, blasst::kDecThreads, C::SMEM_ALLOC, st>>>(a);
   return cudaGetLastError();
 }
 
 blasst_status_t launch_decode_mma(const blasst::DecodeMmaArgs& a, int G,
-                                  long long grid, bool stats_only, void* o,
-                                  float* lse, int rows, cudaStream_t st) {
+                                  int d, long long grid, bool stats_only,
+                                  void* o, float* lse, int rows,
+                                  cudaStream_t st) {
   cudaError_t e = cudaErrorInvalidValue;
-  switch (G) {
-    case 1: e = launch_mma_split<1>(a, grid, st); break;
-    case 2: e = launch_mma_split<2>(a, grid, st); break;
-    case 4: e = launch_mma_split<4>(a, grid, st); break;
-    case 8: e = launch_mma_split<8>(a, grid, st); break;
+  switch (G * 1000 + d) {
+#define BLASST_LAUNCH_MMA(GG, DD) \
+  case GG * 1000 + DD:            \
+    e = launch_mma_split<GG, DD>(a, grid, st); \
+    break;
+    BLASST_LAUNCH_MMA(1, 128)
+    BLASST_LAUNCH_MMA(2, 128)
+    BLASST_LAUNCH_MMA(4, 128)
+    BLASST_LAUNCH_MMA(8, 128)
+    BLASST_LAUNCH_MMA(1, 64)
+    BLASST_LAUNCH_MMA(2, 64)
+    BLASST_LAUNCH_MMA(4, 64)
+    BLASST_LAUNCH_MMA(8, 64)
+#undef BLASST_LAUNCH_MMA
   }
   if (e != cudaSuccess) return cuda_status(e, "decode split launch");
   if (stats_only) return BLASST_OK;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)rows);
-  cfg.blockDim = dim3(blasst::kDecD);
+  cfg.blockDim = dim3(d);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -412,7 +422,11 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
   if (!std::isfinite(scale) || !valid_ln_lambda(ln_lambda))
     return BLASST_ERR_INVALID_ARG;
   int G = Hq / Hkv;
-  if (d != blasst::kDecD || Bc != blasst::kDecBc || !decode_group_ok(G))
+  if (Bc != blasst::kDecBc || !decode_group_ok(G))
+    return BLASST_ERR_UNSUPPORTED_SHAPE;
+  // d = 128 everywhere; d = 64 on the warp-MMA kernel (the sequential rule
+  // with at most 8 heads per KV head)
+  if (!(d == blasst::kDecD || (d == 64 && batch == 0 && G <= 8)))
     return BLASST_ERR_UNSUPPORTED_SHAPE;
   const int kv_div = G > 8 ? G / 8 : 1;  // tiles of 8 heads above 8
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
@@ -459,7 +473,7 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
     m.ln_lambda = ln_lambda;
     m.stats_only = stats_only ? 1 : 0;
     m.window = window;
-    return launch_decode_mma(m, G, grid_mma, stats_only, o, lse, B * Hq,
+    return launch_decode_mma(m, G, d, grid_mma, stats_only, o, lse, B * Hq,
                              static_cast<cudaStream_t>(stream));
   }
   G /= kv_div;

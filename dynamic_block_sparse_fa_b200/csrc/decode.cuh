@@ -701,7 +701,8 @@ __global__ void __launch_bounds__(kDecThreads, BATCH == 1
 
 // Log-sum-exp merge of the S split partials of one (sequence, query head):
 //   lse = ln sum_s exp(lse_s),  o = sum_s exp(lse_s - lse) o_s.
-// An empty split (lse_s = -inf, o_s = 0) gets weight 0.
+// An empty split (lse_s = -inf, o_s = 0) gets weight 0.  One thread per
+// output column: the block has d (64 or 128) threads.
 __global__ void __launch_bounds__(kDecD)
     decode_combine_kernel(const float* __restrict__ o_part,
                           const float* __restrict__ lse_part,
@@ -710,13 +711,14 @@ __global__ void __launch_bounds__(kDecD)
 #if defined(__CUDA_ARCH__)
   asm volatile("griddepcontrol.wait;" ::: "memory");
 #endif
+  const int D = blockDim.x;
   const size_t row = blockIdx.x;
   const int dd = threadIdx.x;
   const float* lp = lse_part + row * S;
   float mx = -INFINITY;
   for (int s = 0; s < S; ++s) mx = fmaxf(mx, lp[s]);
   if (mx == -INFINITY) {  // no keys at all (a paged sequence of length 0)
-    o[row * kDecD + dd] = __float2bfloat16_rn(0.f);
+    o[row * D + dd] = __float2bfloat16_rn(0.f);
     if (dd == 0 && lse) lse[row] = -INFINITY;
     return;
   }
@@ -724,10 +726,10 @@ __global__ void __launch_bounds__(kDecD)
   for (int s = 0; s < S; ++s) sum += ex2_approx((lp[s] - mx) * kLog2e);
   const float L = mx + __logf(sum);
   float acc = 0.f;
-  const float* op = o_part + row * S * kDecD + dd;
+  const float* op = o_part + row * S * D + dd;
   for (int s = 0; s < S; ++s)
-    acc += ex2_approx((lp[s] - L) * kLog2e) * op[(size_t)s * kDecD];
-  o[row * kDecD + dd] = __float2bfloat16_rn(acc);
+    acc += ex2_approx((lp[s] - L) * kLog2e) * op[(size_t)s * D];
+  o[row * D + dd] = __float2bfloat16_rn(acc);
   if (dd == 0 && lse) lse[row] = L;
 }
 

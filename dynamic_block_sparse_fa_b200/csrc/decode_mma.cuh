@@ -1,6 +1,7 @@
 // decode_mma.cuh -- BLASST decode with the scores and P.V on warp-level
 // tensor-core instructions (mma.sync m16n8k16, bf16 in, f32 accumulate):
-// contiguous bf16 KV cache, G <= 8 query heads per KV head, split-KV.
+// contiguous bf16 KV cache, G <= 8 query heads per KV head, head dimension
+// 64 or 128, split-KV.
 //
 // Method as in decode.cuh ("BLASST: Dynamic BLocked Attention Sparsity via
 // Softmax Thresholding", gist.science summary, section 2 "Criterio de Pulo"
@@ -37,9 +38,9 @@
 namespace blasst {
 
 struct DecodeMmaArgs {
-  CUtensorMap tk, tv;        // [B*Hkv][Lkv][128] bf16, box 64 cols x 64 rows
-  const __nv_bfloat16* q;    // [B, Hq, 128]
-  float* o_part;             // [B*Hq, S, 128]
+  CUtensorMap tk, tv;        // [B*Hkv][Lkv][d] bf16, box 64 cols x 64 rows
+  const __nv_bfloat16* q;    // [B, Hq, d]
+  float* o_part;             // [B*Hq, S, d]
   float* lse_part;           // [B*Hq, S]
   unsigned long long* counters;
   unsigned char* mask;       // [B*Hkv, nk]
@@ -50,8 +51,8 @@ struct DecodeMmaArgs {
 };
 
 struct DecodeMmaCfg {
-  static constexpr int BOX = 64 * 128;      // 64 rows x 128 bytes
-  static constexpr int TILE = 2 * BOX;      // 64 keys x 128 dims, 16 KB
+  static constexpr int BOX = 64 * 128;      // 64 rows x 128 bytes (64 dims)
+  static constexpr int TILE = 2 * BOX;      // slot: 64 keys x up to 128 dims
   static constexpr int NK = 2, NV = 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + NK * TILE;
@@ -105,10 +106,14 @@ __device__ __forceinline__ uint32_t swz_off(int key, int chunk) {
                     (((chunk & 7) ^ (key & 7)) << 4));
 }
 
-template <int G>
+template <int G, int D>
 __global__ void __launch_bounds__(kDecThreads, 3)
     decode_mma_kernel(const __grid_constant__ DecodeMmaArgs a) {
   static_assert(G >= 1 && G <= 8, "at most 8 heads per tile");
+  static_assert(D == 64 || D == 128, "head dimension 64 or 128");
+  constexpr int NBOX = D / 64;     // 64-column boxes per block
+  constexpr int KST = D / 16;      // k-steps of the scores
+  constexpr int NG = D / 8;        // 8-column groups of the output
   using C = DecodeMmaCfg;
   constexpr unsigned FULL = 0xffffffffu;
   extern __shared__ uint8_t smem_raw[];
@@ -148,9 +153,10 @@ __global__ void __launch_bounds__(kDecThreads, 3)
 
   const uint64_t pol = policy_evict_first();
   auto load = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int j) {
-    mbar_arrive_expect_tx(bar, C::TILE);
-    tma_load_3d(dst, map, bar, 0, j * kDecBc, bh, pol);
-    tma_load_3d(dst + C::BOX, map, bar, 64, j * kDecBc, bh, pol);
+    mbar_arrive_expect_tx(bar, NBOX * C::BOX);
+#pragma unroll
+    for (int c = 0; c < NBOX; ++c)
+      tma_load_3d(dst + c * C::BOX, map, bar, c * 64, j * kDecBc, bh, pol);
   };
   if (tid == 0) {
     prefetch_tmap(&a.tk);
@@ -164,12 +170,12 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   // qa[t][1] the same + 8.
   const int hr = lane >> 2;  // this lane's head (fragment row)
   const int q4 = lane & 3;
-  uint32_t qa[8][2];
+  uint32_t qa[KST][2];
   {
     const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-        a.q + ((size_t)b * Hq + hkv * G + (hr < G ? hr : 0)) * kDecD);
+        a.q + ((size_t)b * Hq + hkv * G + (hr < G ? hr : 0)) * D);
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
+    for (int t = 0; t < KST; ++t) {
       qa[t][0] = hr < G ? __ldg(qrow + 8 * t + q4) : 0u;
       qa[t][1] = hr < G ? __ldg(qrow + 8 * t + 4 + q4) : 0u;
     }
@@ -181,9 +187,9 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   const int mi = lane >> 3, mr = lane & 7;
   const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
 
-  float o[16][2];  // O of head hr, dims 8n + 2 q4 + {0,1}
+  float o[NG][2];  // O of head hr, dims 8n + 2 q4 + {0,1}
 #pragma unroll
-  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = 0.f;
+  for (int n = 0; n < NG; ++n) o[n][0] = o[n][1] = 0.f;
   float m_run[G];  // running max of each head (replicated in every thread)
 #pragma unroll
   for (int g = 0; g < G; ++g) m_run[g] = -INFINITY;
@@ -204,13 +210,13 @@ __global__ void __launch_bounds__(kDecThreads, 3)
                    kidx, slot))
       return false;
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {
+    for (int n = 0; n < NG; ++n) {
       o[n][0] *= palpha;
       o[n][1] *= palpha;
     }
     const uint32_t vb = aV + slot * C::TILE;
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {
+    for (int p = 0; p < NG / 2; ++p) {
       uint32_t r0, r1, r2, r3;
       ldsm_x4_t(vb + swz_off(16 * warp + 8 * (mi & 1) + mr, 2 * p + (mi >> 1)),
                 r0, r1, r2, r3);
@@ -231,7 +237,7 @@ __global__ void __launch_bounds__(kDecThreads, 3)
     if (ok) {
       const uint32_t kb = aK + stage * C::TILE;
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {  // k-steps 2p, 2p+1 (chunks 4p .. 4p+3)
+      for (int p = 0; p < KST / 2; ++p) {  // k-steps 2p, 2p+1 (chunks 4p .. 4p+3)
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           uint32_t r0, r1, r2, r3;
@@ -338,21 +344,23 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   float* red = reinterpret_cast<float*>(sK);
   if (hr < G) {
 #pragma unroll
-    for (int n = 0; n < 16; ++n)
-      *reinterpret_cast<float2*>(red + ((warp * 8 + hr) * kDecD + 8 * n + 2 * q4)) =
+    for (int n = 0; n < NG; ++n)
+      *reinterpret_cast<float2*>(red + ((warp * 8 + hr) * D + 8 * n + 2 * q4)) =
           make_float2(o[n][0], o[n][1]);
   }
   __syncthreads();
+  if (tid < D) {
+    const int dd = tid;  // one thread per output column
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const int dd = tid;  // 128 threads = 128 dims
-    const float sum = red[(0 * 8 + g) * kDecD + dd] + red[(1 * 8 + g) * kDecD + dd] +
-                      red[(2 * 8 + g) * kDecD + dd] + red[(3 * 8 + g) * kDecD + dd];
-    const float l = sL[g] + sL[8 + g] + sL[16 + g] + sL[24 + g];
-    const size_t row = (size_t)b * Hq + hkv * G + g;
-    a.o_part[(row * a.S + s) * kDecD + dd] = l > 0.f ? sum / l : 0.f;
-    if (dd == 0)
-      a.lse_part[row * a.S + s] = l > 0.f ? m_run[g] + __logf(l) : -INFINITY;
+    for (int g = 0; g < G; ++g) {
+      const float sum = red[(0 * 8 + g) * D + dd] + red[(1 * 8 + g) * D + dd] +
+                        red[(2 * 8 + g) * D + dd] + red[(3 * 8 + g) * D + dd];
+      const float l = sL[g] + sL[8 + g] + sL[16 + g] + sL[24 + g];
+      const size_t row = (size_t)b * Hq + hkv * G + g;
+      a.o_part[(row * a.S + s) * D + dd] = l > 0.f ? sum / l : 0.f;
+      if (dd == 0)
+        a.lse_part[row * a.S + s] = l > 0.f ? m_run[g] + __logf(l) : -INFINITY;
+    }
   }
 }
 

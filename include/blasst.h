@@ -201,7 +201,8 @@ blasst_status_t blasst_prefill_backward(
  *  o           device bf16 [B,Hq,d], or NULL for a statistics-only pass
  *              (K is read and scored, V is never read)
  *  lse         device float32 [B,Hq] or NULL
- *  d           128;  Hq/Hkv a power of two up to 256;  Bc = 64
+ *  d           128, or 64 with Hq/Hkv <= 8;  Hq/Hkv a power of two up to
+ *              256;  Bc = 64
  *  num_splits  >= 1, or 0 for the automatic choice blasst_decode_splits()
  *  workspace   device buffer of at least blasst_decode_workspace_size()
  *              bytes (16-byte aligned) holding the per-split partials;

@@ -93,7 +93,8 @@ def test_decode_validation(lib):
     assert _decode(lib, k=None) == 1
     assert _decode(lib, lnl=1.0) == 1
     assert _decode(lib, S=5) == 1                      # more splits than blocks
-    assert _decode(lib, d=64) == 2                     # decode built for d=128
+    assert _decode(lib, d=96) == 2                     # d is 64 or 128
+    assert _decode(lib, d=64) == 7                     # d = 64 accepted (no workspace)
     assert _decode(lib, Bc=128) == 2
     assert _decode(lib, Hq=12, Hkv=4) == 2             # G = 3 not built
     assert _decode(lib, v=0x1008) == 3

@@ -85,6 +85,26 @@ def test_decode_matches_oracle(blasst, case):
         assert (mask == 2).sum() == 0
 
 
+D64_CASES = [
+    # B, Hq, Hkv, Lkv, ln_lambda, num_splits: head dimension 64
+    (2, 8, 2, 1000, -3.0, 0),
+    (2, 32, 8, 3000, -2.0, 3),
+    (1, 8, 1, 700, -math.inf, 2),
+    (1, 2, 2, 65, -1.0, 1),
+]
+
+
+@pytest.mark.parametrize("case", D64_CASES)
+def test_decode_head_dim_64_matches_oracle(blasst, case):
+    B, Hq, Hkv, Lkv, ln_lambda, S = case
+    x = planted_gap(B, Hq, Hkv, 1, Lkv, 64, decode=True, block=64, gap=8.0,
+                    heavy_frac=0.05, seed=config_seed(1, 640 + Lkv + Hq),
+                    device="cuda")
+    ref, mask, ties = _run_and_compare(blasst, x, ln_lambda, S)
+    if ln_lambda == -math.inf:
+        assert (mask == 2).sum() == 0
+
+
 def test_decode_rejects_bad_arguments(blasst):
     q = torch.zeros(1, 4, 128, dtype=torch.bfloat16, device="cuda")
     k = torch.zeros(1, 1, 256, 128, dtype=torch.bfloat16, device="cuda")
