@@ -189,28 +189,29 @@ cudaError_t launch_split(const blasst::DecodeArgs& a, long long grid,
 
 // The warp-MMA decode (decode_mma.cuh) for the sequential rule on a
 // contiguous cache with G <= 8, then the merge as for launch_decode.
-template <int G, int D>
+template <int G, int D, bool PAGED>
 cudaError_t launch_mma_split(const blasst::DecodeMmaArgs& a, long long grid,
                              cudaStream_t st) {
   using C = blasst::DecodeMmaCfg;
   cudaError_t e = cudaFuncSetAttribute(
-      blasst::decode_mma_kernel<G, D>,
+      blasst::decode_mma_kernel<G, D, PAGED>,
       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
-  blasst::decode_mma_kernel<G, D>
+  blasst::decode_mma_kernel<G, D, PAGED>
       <<<(unsigned)grid, blasst::kDecThreads, C::SMEM_ALLOC, st>>>(a);
   return cudaGetLastError();
 }
 
 blasst_status_t launch_decode_mma(const blasst::DecodeMmaArgs& a, int G,
-                                  int d, long long grid, bool stats_only,
-                                  void* o, float* lse, int rows,
-                                  cudaStream_t st) {
+                                  int d, bool paged, long long grid,
+                                  bool stats_only, void* o, float* lse,
+                                  int rows, cudaStream_t st) {
   cudaError_t e = cudaErrorInvalidValue;
   switch (G * 1000 + d) {
-#define BLASST_LAUNCH_MMA(GG, DD) \
-  case GG * 1000 + DD:            \
-    e = launch_mma_split<GG, DD>(a, grid, st); \
+#define BLASST_LAUNCH_MMA(GG, DD)                                           \
+  case GG * 1000 + DD:                                                      \
+    e = paged ? launch_mma_split<GG, DD, true>(a, grid, st)                 \
+              : launch_mma_split<GG, DD, false>(a, grid, st);               \
     break;
     BLASST_LAUNCH_MMA(1, 128)
     BLASST_LAUNCH_MMA(2, 128)
@@ -473,8 +474,8 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
     m.ln_lambda = ln_lambda;
     m.stats_only = stats_only ? 1 : 0;
     m.window = window;
-    return launch_decode_mma(m, G, d, grid_mma, stats_only, o, lse, B * Hq,
-                             static_cast<cudaStream_t>(stream));
+    return launch_decode_mma(m, G, d, false, grid_mma, stats_only, o, lse,
+                             B * Hq, static_cast<cudaStream_t>(stream));
   }
   G /= kv_div;
   const long long grid = (long long)B * Hkv * kv_div * S;
@@ -546,7 +547,6 @@ blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
   if (d != blasst::kDecD || !decode_group_ok(G))
     return BLASST_ERR_UNSUPPORTED_SHAPE;
   const int kv_div = G > 8 ? G / 8 : 1;  // tiles of 8 heads above 8
-  G /= kv_div;
   if (page_stride < (long long)Hkv * page_size * d || page_stride % 8 != 0)
     return BLASST_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) ||
@@ -557,6 +557,43 @@ blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
   const int S = num_splits == 0 ? blasst_decode_splits(B, Hkv, max_seq_len, Bc)
                                 : num_splits;
   if (S < 1 || S > nk) return BLASST_ERR_INVALID_ARG;
+  if (G <= 8 && (long long)B * Hkv * S <= 0x7fffffffLL) {
+    // up to 8 heads per KV head: the warp-MMA kernel over the pool
+    const bool stats_only = (o == nullptr);
+    blasst::DecodeMmaArgs m;
+    memset(&m, 0, sizeof m);
+    if (!stats_only) {
+      const blasst_status_t ws = carve_workspace(workspace, workspace_bytes, B,
+                                                 Hq, d, S, &m.o_part,
+                                                 &m.lse_part);
+      if (ws != BLASST_OK) return ws;
+    }
+    const int box_rows = page_size < 64 ? page_size : 64;
+    if (!blasst::encode_pool_map(&m.tk, k_pages, d, page_size, Hkv, num_pages,
+                                 page_stride, box_rows) ||
+        !blasst::encode_pool_map(&m.tv, v_pages, d, page_size, Hkv, num_pages,
+                                 page_stride, box_rows))
+      return cuda_status(cudaErrorInvalidValue, "paged decode tensor maps");
+    m.q = static_cast<const __nv_bfloat16*>(q);
+    m.counters = skip_stats ? skip_stats->counters : nullptr;
+    m.mask = skip_stats ? skip_stats->mask : nullptr;
+    m.Hkv = Hkv;
+    m.Lkv = max_seq_len;
+    m.nk = nk;
+    m.S = S;
+    m.scale = scale;
+    m.ln_lambda = ln_lambda;
+    m.stats_only = stats_only ? 1 : 0;
+    m.block_table = block_table;
+    m.seq_lens = seq_lens;
+    m.max_pages = max_pages;
+    m.num_pages = num_pages;
+    m.log2_page = log2_page;
+    m.per_length = per_length ? 1 : 0;
+    return launch_decode_mma(m, G, d, true, (long long)B * Hkv * S, stats_only,
+                             o, lse, B * Hq, static_cast<cudaStream_t>(stream));
+  }
+  G /= kv_div;
   const long long grid = (long long)B * Hkv * kv_div * S;
   if (grid > 0x7fffffffLL) return BLASST_ERR_UNSUPPORTED_SHAPE;
   const bool stats_only = (o == nullptr);

@@ -1,7 +1,7 @@
 // decode_mma.cuh -- BLASST decode with the scores and P.V on warp-level
 // tensor-core instructions (mma.sync m16n8k16, bf16 in, f32 accumulate):
-// contiguous bf16 KV cache, G <= 8 query heads per KV head, head dimension
-// 64 or 128, split-KV.
+// contiguous or paged bf16 KV cache, G <= 8 query heads per KV head, head
+// dimension 64 or 128, split-KV.
 //
 // Method as in decode.cuh ("BLASST: Dynamic BLocked Attention Sparsity via
 // Softmax Thresholding", gist.science summary, section 2 "Criterio de Pulo"
@@ -30,6 +30,15 @@
 // ring of two blocks and a V ring of two.  The P.V of a kept block runs
 // when the next kept block has been decided (its V load has had a block of
 // scoring to land); its P and rescale factor wait in registers.
+//
+// Paged cache (PAGED): the page pool [num_pages][Hkv][page_size][d] is a
+// 4-D tensor map whose box is min(page_size, 64) rows of one page, so a
+// 64-key block is one to four TMA segments, each from the page the block
+// table names.  Every page id a split will read is range-checked before the
+// first load (a bad id or length sets the error word and the CTA leaves).
+// Rows past the sequence's end that a segment brings in (the rest of its
+// last page) or that no segment covers are masked in the scores and zeroed
+// in V before the P.V, so whatever the pool holds there cannot reach o.
 #pragma once
 
 #include "decode.cuh"
@@ -48,6 +57,11 @@ struct DecodeMmaArgs {
   float scale, ln_lambda;
   int stats_only;
   int window;                // the last `window` keys (0 = all)
+  // paged cache only (tk / tv then map the pools, see above)
+  const int* block_table;    // [B, max_pages]
+  const int* seq_lens;       // [B]; Lkv is then the upper bound on them
+  int max_pages, num_pages, log2_page;
+  int per_length;  // ln_lambda is ln a; sequence b uses min(0, ln a - ln L_b)
 };
 
 struct DecodeMmaCfg {
@@ -101,12 +115,24 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0,
 // Byte offset of the 16-byte chunk `chunk` (0..15: dims 8*chunk ..) of key
 // row `key` in a block stored as two 64-column boxes with the 128-byte
 // swizzle (chunk index XOR key % 8 within each 1024-byte group of rows).
+__device__ __forceinline__ void tma_load_4d(void* dst_smem, const void* tmap,
+                                            uint64_t* bar, int c0, int c1,
+                                            int c2, int c3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_"
+      "tx::bytes.L2::cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(
+          smem_u32(dst_smem)),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)),
+      "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ uint32_t swz_off(int key, int chunk) {
   return (uint32_t)((chunk >> 3) * DecodeMmaCfg::BOX + key * 128 +
                     (((chunk & 7) ^ (key & 7)) << 4));
 }
 
-template <int G, int D>
+template <int G, int D, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, 3)
     decode_mma_kernel(const __grid_constant__ DecodeMmaArgs a) {
   static_assert(G >= 1 && G <= 8, "at most 8 heads per tile");
@@ -128,11 +154,43 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   const int Hq = a.Hkv * G;
   const int b = bh / a.Hkv;
   const int hkv = bh - b * a.Hkv;
-  const int key_lo = (a.window > 0 && a.Lkv > a.window) ? a.Lkv - a.window : 0;
+  int Lb = a.Lkv;  // keys of this sequence
+  float ln_lambda = a.ln_lambda;
+  const int* bt_row = nullptr;
+  if constexpr (PAGED) {
+    Lb = __ldg(a.seq_lens + b);
+    if (Lb < 0 || Lb > a.Lkv) {  // uniform across the CTA
+      if (tid == 0) record_error(kBadSeqLen, (unsigned)b, (unsigned)Lb, 0);
+      return;
+    }
+    // lambda = a / L with L this sequence's own context length
+    if (a.per_length && ln_lambda > -INFINITY && Lb > 0)
+      ln_lambda = fminf(0.f, ln_lambda - logf((float)Lb));
+    bt_row = a.block_table + (size_t)b * a.max_pages;
+  }
+  const int nk_b = (Lb + kDecBc - 1) / kDecBc;
+  const int key_lo = (a.window > 0 && Lb > a.window) ? Lb - a.window : 0;
   const int jlo = key_lo / kDecBc;
-  const int j0 = jlo + (int)(((long long)s * (a.nk - jlo)) / a.S);
-  const int j1 = jlo + (int)(((long long)(s + 1) * (a.nk - jlo)) / a.S);
+  const int j0 = jlo + (int)(((long long)s * (nk_b - jlo)) / a.S);
+  const int j1 = jlo + (int)(((long long)(s + 1) * (nk_b - jlo)) / a.S);
   const int nblk = j1 - j0;
+  const int ps = 1 << a.log2_page;       // paged: rows per page
+  const int seg = ps < 64 ? ps : 64;     // paged: rows per TMA segment
+  if constexpr (PAGED) {
+    // every page id this split reads, before any load
+    bool bad = false;
+    const int t0 = j0 * kDecBc, t1 = min(j1 * kDecBc, Lb);
+    if (t1 > t0)
+      for (int pg = (t0 >> a.log2_page) + tid; pg <= ((t1 - 1) >> a.log2_page);
+           pg += kDecThreads) {
+        const int id = __ldg(bt_row + pg);
+        if (id < 0 || id >= a.num_pages) {
+          bad = true;
+          record_error(kBadPageId, (unsigned)b, (unsigned)pg, (unsigned)id);
+        }
+      }
+    if (__syncthreads_or(bad)) return;
+  }
   if (a.mask && s == 0)  // blocks left of the window are not visited
     for (int j = tid; j < jlo; j += kDecThreads) a.mask[(size_t)bh * a.nk + j] = 0;
 
@@ -153,10 +211,25 @@ __global__ void __launch_bounds__(kDecThreads, 3)
 
   const uint64_t pol = policy_evict_first();
   auto load = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int j) {
-    mbar_arrive_expect_tx(bar, NBOX * C::BOX);
+    if constexpr (!PAGED) {
+      mbar_arrive_expect_tx(bar, NBOX * C::BOX);
 #pragma unroll
-    for (int c = 0; c < NBOX; ++c)
-      tma_load_3d(dst + c * C::BOX, map, bar, c * 64, j * kDecBc, bh, pol);
+      for (int c = 0; c < NBOX; ++c)
+        tma_load_3d(dst + c * C::BOX, map, bar, c * 64, j * kDecBc, bh, pol);
+    } else {
+      // segments of `seg` rows that hold the block's keys (< Lb)
+      const int rows = min(kDecBc, Lb - j * kDecBc);
+      const int nseg = (rows + seg - 1) / seg;
+      mbar_arrive_expect_tx(bar, (uint32_t)(nseg * seg * 128 * NBOX));
+      for (int i = 0; i < nseg; ++i) {
+        const int t = j * kDecBc + i * seg;
+        const int id = __ldg(bt_row + (t >> a.log2_page));
+#pragma unroll
+        for (int c = 0; c < NBOX; ++c)
+          tma_load_4d(dst + c * C::BOX + i * seg * 128, map, bar, c * 64,
+                      t & (ps - 1), hkv, id, pol);
+      }
+    }
   };
   if (tid == 0) {
     prefetch_tmap(&a.tk);
@@ -198,9 +271,10 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   bool pend = false;
   uint32_t pp0 = 0, pp1 = 0;  // its P as A fragment (keys 16w + 2q4 (+8))
   float palpha = 1.f;          // its rescale factor for head hr
+  int prows = kDecBc;          // its keys inside the sequence
   int kept = 0;                // kept blocks so far (V slot = index % 2)
 
-  const float scale = a.scale, ln_lambda = a.ln_lambda;
+  const float scale = a.scale;
   unsigned long long n_vis = 0, n_skp = 0;
   bool ok = true;
 
@@ -215,6 +289,20 @@ __global__ void __launch_bounds__(kDecThreads, 3)
       o[n][1] *= palpha;
     }
     const uint32_t vb = aV + slot * C::TILE;
+    if (PAGED && prows < kDecBc) {
+      // rows past the sequence end: zero this warp's share (16 rows) so
+      // that P = 0 there multiplies zeros, whatever the pool held
+      uint8_t* vs = sV + slot * C::TILE;
+      for (int e = lane; e < 16 * NBOX * 8; e += 32) {
+        const int row = 16 * warp + e / (NBOX * 8);
+        const int c16 = e % (NBOX * 8);  // 16-byte chunk of the row
+        if (row >= prows)
+          *reinterpret_cast<uint4*>(vs + (c16 >> 3) * C::BOX + row * 128 +
+                                    (c16 & 7) * 16) = make_uint4(0, 0, 0, 0);
+      }
+      fence_async_smem();  // before a later TMA load overwrites the slot
+      __syncwarp();
+    }
 #pragma unroll
     for (int p = 0; p < NG / 2; ++p) {
       uint32_t r0, r1, r2, r3;
@@ -256,7 +344,7 @@ __global__ void __launch_bounds__(kDecThreads, 3)
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int key = kbase + 8 * g + i;
-        sc[g][i] = (key < a.Lkv && key >= key_lo) ? sc[g][i] * scale : -INFINITY;
+        sc[g][i] = (key < Lb && key >= key_lo) ? sc[g][i] * scale : -INFINITY;
         mx = fmaxf(mx, sc[g][i]);
       }
     mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
@@ -306,6 +394,7 @@ __global__ void __launch_bounds__(kDecThreads, 3)
       pp0 = pack_bf16x2(p[0][0], p[0][1]);
       pp1 = pack_bf16x2(p[1][0], p[1][1]);
       palpha = al;
+      prows = min(kDecBc, Lb - j * kDecBc);
       pend = true;
       ++kept;
     }

@@ -544,6 +544,27 @@ inline bool encode_map(CUtensorMap* m, const void* base, int D, int rows,
   return r == CUDA_SUCCESS;
 }
 
+// 4-D map over a page pool [pages][heads][page_rows][D] bf16 whose pages
+// are `page_stride` elements apart: box = 64 columns x box_rows rows of one
+// head of one page, 128-byte swizzle.
+inline bool encode_pool_map(CUtensorMap* m, const void* base, int D,
+                            int page_rows, int heads, long long pages,
+                            long long page_stride, int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)page_rows, (cuuint64_t)heads,
+                        (cuuint64_t)pages};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)page_rows * D * 2,
+                           (cuuint64_t)page_stride * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int D, int BN, int BRL>
 cudaError_t launch_prefill_t(const PrefillProblem& pr, cudaStream_t st) {
   using C = PrefillCfg<D, BN, BRL>;

@@ -118,12 +118,31 @@ def test_paged_decode_matches_oracle(blasst, case):
         assert (mask == 2).sum() == 0
 
 
+@pytest.mark.parametrize("ps", [16, 64])
+def test_paged_nan_rows_past_the_sequence_never_reach_the_output(blasst, ps):
+    """Pool rows no sequence owns hold NaN: the kernel may bring the rest of
+    a sequence's last page (or stale rows) into shared memory, but masks
+    those keys and zeroes those V rows, so the outputs stay finite and
+    match the oracle (which reads only the sequences' own rows)."""
+    lens = [1000, 65, 1, 2047]
+    B = len(lens)
+    x = planted_gap(B, 8, 2, 1, max(lens), 128, decode=True, block=64,
+                    gap=8.0, heavy_frac=0.05, seed=config_seed(1, 4242 + ps),
+                    device="cuda")
+    nan = float("nan")
+    pk = paginate(x.k, x.v, lens, ps, seed=ps, spare_pages=3,
+                  poison=(nan, nan))
+    o, lse, _ = _check_paged(blasst, x.q, pk.k_pages, pk.v_pages, pk, lens,
+                             -2.0, 0, False)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
 @pytest.mark.parametrize("ps", [16, 64, 256])
 def test_paged_equals_contiguous_bitwise(blasst, ps):
     """Same tokens, same splits: the paged kernel reads the same bytes in the
-    same order as the CUDA-core contiguous kernel (blasst_decode_batched with
-    batch 1), so the results agree bit for bit; blasst_decode (warp-MMA
-    kernel, same decisions) agrees within the parity tolerance."""
+    same order as the contiguous one (both the warp-MMA kernel), so the
+    results agree bit for bit; the CUDA-core kernel (blasst_decode_batched
+    with batch 1, same decisions) agrees within the parity tolerance."""
     m = blasst
     B, Hq, Hkv, L = 6, 32, 8, 4096 + 64 * 3
     x = planted_gap(B, Hq, Hkv, 1, L, 128, decode=True, block=64, gap=8.0,
@@ -131,17 +150,17 @@ def test_paged_equals_contiguous_bitwise(blasst, ps):
     pk = paginate(x.k, x.v, [L] * B, ps, seed=3, spare_pages=2,
                   poison=POISON)
     for lnl in (-math.inf, -3.0):
-        o1, l1 = m.blasst_decode_batched(x.q, x.k, x.v, batch=1,
-                                         ln_lambda=lnl, num_splits=3)
+        o1, l1 = m.blasst_decode(x.q, x.k, x.v, ln_lambda=lnl, num_splits=3)
         o2, l2 = m.blasst_decode_paged(x.q, pk.k_pages, pk.v_pages,
                                        pk.block_table, pk.seq_lens,
                                        max_seq_len=L, ln_lambda=lnl,
                                        num_splits=3)
-        o3, l3 = m.blasst_decode(x.q, x.k, x.v, ln_lambda=lnl, num_splits=3)
+        o3, l3 = m.blasst_decode_batched(x.q, x.k, x.v, batch=1,
+                                         ln_lambda=lnl, num_splits=3)
         torch.cuda.synchronize()
         assert torch.equal(o1, o2) and torch.equal(l1, l2)
-        P.check_out(P.to_np(o3), P.to_np(o2), "decode vs paged")
-        P.check_lse(P.to_np(l3), P.to_np(l2), "decode vs paged")
+        P.check_out(P.to_np(o3), P.to_np(o2), "CUDA-core vs paged")
+        P.check_lse(P.to_np(l3), P.to_np(l2), "CUDA-core vs paged")
 
 
 def test_paged_bad_table_and_length_are_reported(blasst):
@@ -231,8 +250,7 @@ def test_paged_full_size_shuffled_pool(blasst):
     pk = paginate(k, v, [L] * B, 64, seed=11, spare_pages=64)
     s1 = m.Stats(mask_numel=B * Hkv * nk)
     s2 = m.Stats(mask_numel=B * Hkv * nk)
-    o1, l1 = m.blasst_decode_batched(q, k, v, batch=1, ln_lambda=lnl,
-                                     stats=s1)
+    o1, l1 = m.blasst_decode(q, k, v, ln_lambda=lnl, stats=s1)
     o2, l2 = m.blasst_decode_paged(q, pk.k_pages, pk.v_pages, pk.block_table,
                                    pk.seq_lens, max_seq_len=L, ln_lambda=lnl,
                                    stats=s2)
