@@ -45,7 +45,8 @@ class BlasstError(RuntimeError):
 
 class SkipStats(ctypes.Structure):
     """Host struct of device pointers (blasst_skip_stats_t)."""
-    _fields_ = [("counters", ctypes.c_void_p), ("mask", ctypes.c_void_p)]
+    _fields_ = [("counters", ctypes.c_void_p), ("mask", ctypes.c_void_p),
+                ("margin", ctypes.c_void_p)]
 
 
 class CalibSample(ctypes.Structure):
@@ -181,12 +182,18 @@ class Stats:
     """Device skip counters (uint64[2]: visited, skipped) and an optional
     per-(tile, block) decision mask, allocated with torch."""
 
-    def __init__(self, device="cuda", mask_numel: int = 0):
+    def __init__(self, device="cuda", mask_numel: int = 0,
+                 margin: bool = False):
         self.counters = torch.zeros(2, dtype=torch.int64, device=device)
         self.mask = (torch.zeros(mask_numel, dtype=torch.uint8, device=device)
                      if mask_numel else None)
-        self._c = SkipStats(self.counters.data_ptr(),
-                            self.mask.data_ptr() if self.mask is not None else None)
+        self.margin = (torch.full((mask_numel,), float("nan"),
+                                  dtype=torch.float32, device=device)
+                       if margin and mask_numel else None)
+        self._c = SkipStats(
+            self.counters.data_ptr(),
+            self.mask.data_ptr() if self.mask is not None else None,
+            self.margin.data_ptr() if self.margin is not None else None)
 
     @property
     def c_struct(self):
@@ -196,6 +203,16 @@ class Stats:
         blasst_skip_stats_reset(self.counters, stream)
         if self.mask is not None:
             self.mask.zero_()
+        if self.margin is not None:
+            self.margin.fill_(float("nan"))
+
+    def near_ties(self, width: float = 1e-3) -> int:
+        """Visited pairs whose decision margin is within `width` of 0 (the
+        margin buffer must have been requested and filled)."""
+        if self.margin is None:
+            raise ValueError("Stats(margin=True) was not requested")
+        m = self.margin
+        return int(((self.mask > 0) & (m.abs() < width)).sum().item())
 
     def read(self):
         v, s = (int(x) for x in self.counters.tolist())

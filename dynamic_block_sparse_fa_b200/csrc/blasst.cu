@@ -466,6 +466,7 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
     m.q = static_cast<const __nv_bfloat16*>(q);
     m.counters = skip_stats ? skip_stats->counters : nullptr;
     m.mask = skip_stats ? skip_stats->mask : nullptr;
+    m.margin = skip_stats ? skip_stats->margin : nullptr;
     m.Hkv = Hkv;
     m.Lkv = Lkv;
     m.nk = nk;
@@ -577,6 +578,7 @@ blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
     m.q = static_cast<const __nv_bfloat16*>(q);
     m.counters = skip_stats ? skip_stats->counters : nullptr;
     m.mask = skip_stats ? skip_stats->mask : nullptr;
+    m.margin = skip_stats ? skip_stats->margin : nullptr;
     m.Hkv = Hkv;
     m.Lkv = max_seq_len;
     m.nk = nk;
@@ -787,6 +789,7 @@ blasst_status_t blasst_prefill_window(const void* q, const void* k,
   p.Bc = Bc;
   p.counters = skip_stats ? skip_stats->counters : nullptr;
   p.mask = skip_stats ? skip_stats->mask : nullptr;
+  p.margin = skip_stats ? skip_stats->margin : nullptr;
   p.window = window;
   cudaError_t e = blasst::launch_prefill(p, static_cast<cudaStream_t>(stream));
   return cuda_status(e, "prefill launch");
@@ -971,7 +974,7 @@ blasst_status_t sparsity_at(const blasst_calib_sample_t* s, double ln_lambda,
                             unsigned long long* vis, unsigned long long* skp) {
   blasst_status_t rc = blasst_skip_stats_reset(counters, st);
   if (rc != BLASST_OK) return rc;
-  blasst_skip_stats_t stats = {counters, nullptr};
+  blasst_skip_stats_t stats = {counters, nullptr, nullptr};
   const float lnl = (float)ln_lambda;
   if (s->mode == 0) {
     rc = blasst_prefill(s->q, s->k, s->v, nullptr, nullptr, s->B, s->Hq,

@@ -53,6 +53,7 @@ struct DecodeMmaArgs {
   float* lse_part;           // [B*Hq, S]
   unsigned long long* counters;
   unsigned char* mask;       // [B*Hkv, nk]
+  float* margin;             // [B*Hkv, nk] decision margins (may be null)
   int Hkv, Lkv, nk, S;
   float scale, ln_lambda;
   int stats_only;
@@ -369,6 +370,12 @@ __global__ void __launch_bounds__(kDecThreads, 3)
       ++n_vis;
       if (skip) ++n_skp;
       if (a.mask) a.mask[(size_t)bh * a.nk + j] = skip ? 2 : 1;
+      if (a.margin) {  // max over the heads of m~ - m (+inf while m = -inf)
+        float dl = -INFINITY;
+#pragma unroll
+        for (int g = 0; g < G; ++g) dl = fmaxf(dl, mt[g] - m_run[g]);
+        a.margin[(size_t)bh * a.nk + j] = dl - ln_lambda;
+      }
     }
     if (!skip && !stats_only) {
       if (tid == 0) load(&a.tv, sV + (kept % C::NV) * C::TILE, &vfull[kept % C::NV], j);

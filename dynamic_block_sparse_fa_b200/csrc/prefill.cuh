@@ -47,6 +47,7 @@ struct PrefillProblem {
   int Br, Bc;
   unsigned long long* counters;
   unsigned char* mask;
+  float* margin;  // decision margins, layout of mask (may be null)
   int window;  // 0 = none
 };
 
@@ -56,6 +57,7 @@ struct __align__(64) PrefillParams {
   float* lse;
   unsigned long long* counters;
   unsigned char* mask;
+  float* margin;
   int B, Hq, Hkv, Lq, Lkv, nq, nk, G;
   float scale, ln_lambda;
   int causal, stats_only;
@@ -92,7 +94,8 @@ struct PrefillCfg {
   static constexpr int NBAR = B_OD + 1;
   static constexpr int OFF_DEC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_TMEM = OFF_DEC + R * 4;
-  static constexpr int SMEM = OFF_TMEM + 16;
+  static constexpr int OFF_XM = OFF_TMEM + 16;  // f32 [2][4]: warp margin maxima
+  static constexpr int SMEM = OFF_XM + 32;
   static constexpr int SMEM_ALLOC = SMEM + 1024;  // slack for 1024 alignment
   static constexpr int TMEM_COLS = (2 * BN + D <= 256) ? 256 : 512;
   static constexpr int COL_S = 0;  // buffer b at COL_S + b * BN
@@ -362,6 +365,14 @@ __global__ void __launch_bounds__(192, 1)
       const float mt_s = mt * scale;  // -inf stays -inf (scale > 0)
       const bool pred = !active || mt_s == -INFINITY ||
                         (mt_s - m_crit < ln_lambda);
+      float* xm = reinterpret_cast<float*>(smem + C::OFF_XM) + (j & 1) * 4;
+      if (p.margin) {  // max over the rows of m~ - m, per warp
+        float dl = (active && mt_s != -INFINITY) ? mt_s - m_crit : -INFINITY;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1)
+          dl = fmaxf(dl, __shfl_xor_sync(0xffffffffu, dl, o));
+        if (lane == 0) xm[warp & 3] = dl;
+      }
       tc_fence_before();
       const bool skip =
           named_sync_and(1, 128, pred) && (ln_lambda > -INFINITY);
@@ -369,6 +380,9 @@ __global__ void __launch_bounds__(192, 1)
         ++n_vis;
         if (skip) ++n_skp;
         if (p.mask) p.mask[mask_row + j] = skip ? 2 : 1;
+        if (p.margin)
+          p.margin[mask_row + j] =
+              fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3])) - ln_lambda;
         dec_flag[j % C::R] = skip ? 0 : 1;
         mbar_arrive(&bar[C::B_DEC + j % C::R]);
       }
@@ -578,6 +592,7 @@ cudaError_t launch_prefill_t(const PrefillProblem& pr, cudaStream_t st) {
   p.lse = pr.lse;
   p.counters = pr.counters;
   p.mask = pr.mask;
+  p.margin = pr.margin;
   p.B = pr.B;
   p.Hq = pr.Hq;
   p.Hkv = pr.Hkv;

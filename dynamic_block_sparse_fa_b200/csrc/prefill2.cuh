@@ -64,7 +64,8 @@ struct Prefill2Cfg {
   static constexpr int OFF_TMEM = OFF_DEC + 2 * R * 4;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;      // int [2]
   static constexpr int WPT = 4;  // softmax warps per tile (thread = row)
-  static constexpr int SMEM = OFF_ABORT + 8;
+  static constexpr int OFF_XM = OFF_ABORT + 8;  // f32 [2][2 tiles][4]: margins
+  static constexpr int SMEM = OFF_XM + 64;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
   static constexpr int TMEM_COLS = 512;
   static constexpr int COL_S = 0;    // tile t at COL_S + t * 128
@@ -73,7 +74,9 @@ struct Prefill2Cfg {
   static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
 };
 
-template <int D, bool SKIP>
+// MARGIN: also write each visited pair's decision margin (p.margin); a
+// separate instance, so that the timed kernel carries no code for it.
+template <int D, bool SKIP, bool MARGIN>
 __global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
     prefill2_kernel(const __grid_constant__ PrefillParams p) {
   using C = Prefill2Cfg<D>;
@@ -439,6 +442,14 @@ __global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
       const float mt_s = mt * scale;  // the row's block max
       const bool pred = !active || mt_s == -INFINITY ||
                         (mt_s - m_crit < ln_lambda);
+      float* xm = reinterpret_cast<float*>(smem + C::OFF_XM) + ((jt & 1) * 2 + t) * 4;
+      if constexpr (MARGIN) {  // max over the rows of m~ - m, per warp
+        float dl = (active && mt_s != -INFINITY) ? mt_s - m_crit : -INFINITY;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1)
+          dl = fmaxf(dl, __shfl_xor_sync(FULL, dl, o));
+        if (lane == 0) xm[wi] = dl;
+      }
       tc_fence_before();
       bool skip = false;
       if constexpr (SKIP) {
@@ -454,6 +465,9 @@ __global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
         ++n_vis;
         if (skip) ++n_skp;
         if (p.mask) p.mask[mask_row + j] = skip ? 2 : 1;
+        if (MARGIN)
+          p.margin[mask_row + j] =
+              fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3])) - ln_lambda;
         if constexpr (SKIP) {
           st_release_shared(&dec_word[t * C::R + jt % C::R],
                             ((uint32_t)(jt + 1) << 1) | (skip ? 1u : 0u));
@@ -570,7 +584,7 @@ __global__ void __launch_bounds__(64 + 2 * 4 * 32, 1)
   }
 }
 
-template <int D, bool SKIP>
+template <int D, bool SKIP, bool MARGIN>
 cudaError_t launch_prefill2_t(const PrefillProblem& pr, cudaStream_t st) {
   using C = Prefill2Cfg<D>;
   PrefillParams p;
@@ -583,6 +597,7 @@ cudaError_t launch_prefill2_t(const PrefillProblem& pr, cudaStream_t st) {
   p.lse = pr.lse;
   p.counters = pr.counters;
   p.mask = pr.mask;
+  p.margin = pr.margin;
   p.B = pr.B;
   p.Hq = pr.Hq;
   p.Hkv = pr.Hkv;
@@ -598,11 +613,12 @@ cudaError_t launch_prefill2_t(const PrefillProblem& pr, cudaStream_t st) {
   p.window = pr.window;
   const long long grid = (long long)((p.nq + 1) / 2) * pr.B * pr.Hq;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(prefill2_kernel<D, SKIP>,
+  cudaError_t e = cudaFuncSetAttribute(prefill2_kernel<D, SKIP, MARGIN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
-  prefill2_kernel<D, SKIP><<<(unsigned)grid, C::THREADS, C::SMEM_ALLOC, st>>>(p);
+  prefill2_kernel<D, SKIP, MARGIN>
+      <<<(unsigned)grid, C::THREADS, C::SMEM_ALLOC, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -610,9 +626,10 @@ cudaError_t launch_prefill2_t(const PrefillProblem& pr, cudaStream_t st) {
 // without the vote; every other call runs the skipping kernel.
 template <int D>
 cudaError_t launch_prefill2(const PrefillProblem& pr, cudaStream_t st) {
+  if (pr.margin != nullptr) return launch_prefill2_t<D, true, true>(pr, st);
   if (pr.ln_lambda == -INFINITY && pr.o != nullptr)
-    return launch_prefill2_t<D, false>(pr, st);
-  return launch_prefill2_t<D, true>(pr, st);
+    return launch_prefill2_t<D, false, false>(pr, st);
+  return launch_prefill2_t<D, true, false>(pr, st);
 }
 
 }  // namespace blasst

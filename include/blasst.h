@@ -62,6 +62,7 @@ typedef enum {
 /*
  * Skip statistics ("sparsity" = skipped / visited (tile, block) pairs).
  * The struct itself lives in HOST memory; its fields are DEVICE pointers.
+ * Every field may be NULL (not written).
  *
  *  counters  device uint64[2]: [0] += visited pairs, [1] += skipped pairs.
  *            Kernels ADD to them (atomics), so one pair of counters can sum
@@ -75,11 +76,25 @@ typedef enum {
  *            layout: the library cannot check a device buffer's size.  Entries of pairs that are not visited are
  *            written as 0 by prefill only for tiles it runs; callers that
  *            need them zeroed clear the buffer first.
- * A NULL blasst_skip_stats_t* disables both.
+ *  margin    optional device float32 buffer, same layout as mask, receiving
+ *            for every visited pair the margin of its decision
+ *              max_r (m~_r - m_r) - ln_lambda
+ *            (rows r of the tile with a visible key in the block; m_r the
+ *            running max before the block, so the tile's first visited
+ *            block gives +inf).  The pair is skipped exactly when the
+ *            margin is < 0; a pair with |margin| < 1e-3 is a near-tie, whose
+ *            decision a float32 rounding difference may flip.  Written by
+ *            blasst_prefill / blasst_prefill_window, blasst_decode,
+ *            blasst_decode_window, blasst_decode_noalloc and
+ *            blasst_decode_paged with Hq/Hkv <= 8; other calls leave it
+ *            untouched.  Computing it costs a max-reduction per pair, so
+ *            pass NULL in timed calls.
+ * A NULL blasst_skip_stats_t* disables all three.
  */
 typedef struct {
     unsigned long long *counters;
     unsigned char *mask;
+    float *margin;
 } blasst_skip_stats_t;
 
 /*
