@@ -505,6 +505,18 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
         "speedup_vs_dense": _r(ms_dense / ms50, 4)}
     line["decode"]["hbm_frac_dense"] = _r(
         by_dense / (ms_dense / K / 1e3) / 1e9 / hbm_peak, 4)
+    # near-ties over the whole batch, from the library's own margins
+    lib_ties = {}
+    for key, l in (("s70", lnl), ("s50", cal50["ln_lambda"])):
+        stm = bl.Stats(device=dev, mask_numel=B * Hkv * nk, margin=True)
+        bl.blasst_decode(q, k, v, ln_lambda=l, o=o, lse=lse, workspace=ws,
+                         stats=stm)
+        torch.cuda.synchronize()
+        lib_ties[key] = stm.near_ties()
+        del stm
+    line["decode"]["near_ties_library"] = dict(
+        lib_ties, what=f"all {B * Hkv * nk} pairs of the call, from the "
+                       f"library's decision margins (|margin| < {NEAR_TIE})")
     if rank == 0 and not args.no_cpu:
         line["decode"]["near_ties"] = {
             key: decode_near_ties(q, k, v, l, S, DEC_TIE_SEQS)
@@ -684,6 +696,14 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
         r["a"] = cal["a"]
         r["speedup_vs_dense"] = round(dense["us"] / r["us"], 4)
         out[key] = r
+    nq_, nk_ = -(-L // Br), -(-L // Bc)
+    for key in ("s50", "s70"):
+        stm = bl.Stats(device=dev, mask_numel=B * Hq * nq_ * nk_, margin=True)
+        bl.blasst_prefill(q, k, v, ln_lambda=out[key]["ln_lambda"], Br=Br,
+                          Bc=Bc, o=o, lse=lse, stats=stm)
+        torch.cuda.synchronize()
+        out[key]["near_ties_library"] = stm.near_ties()
+        del stm
     if not args.no_cpu:
         tiles = [(0, h, i) for h in (0, 17) for i in range(0, 256, 4)]
         for key in ("s50", "s70"):
@@ -879,15 +899,17 @@ def run_prefill_sweep(args, bl, dev, stream, tf_peak):
     from synth import config_seed, planted_gap
     lengths, targets = args.prefill_sweep_lengths, (0.0, 0.3, 0.5, 0.7, 0.9)
     flush = l2_flush_buffer(dev)
-    reps = 3
+    # repetitions per length: short calls are timed more often
+    reps_of = {L: max(3, min(20, (20 * 65536) // (L * 4))) for L in lengths}
     xs = {L: planted_gap(1, 32, 8, L, L, 128, block=128, gap_range=(4.0, 12.0),
                          heavy_frac=0.02, window=512, seed=config_seed(4, L),
                          device=dev) for L in lengths}
     dense_ms = {}
     for L, x in xs.items():
         o = torch.empty_like(x.q)
+        reps = reps_of[L]
         dense_ms[L] = time_calls_flushed(lambda: bl.blasst_prefill(
-            x.q, x.k, x.v, o=o, want_lse=False), reps, 1, stream, flush) / reps
+            x.q, x.k, x.v, o=o, want_lse=False), reps, 2, stream, flush) / reps
     out = {"workload": "prefill B1 Hq32 Hkv8 d128 causal 128x128, gap per head "
                        "U[4,12] nats, lambda = a/L with a fitted per target "
                        "over the lengths (log space)",
@@ -911,9 +933,10 @@ def run_prefill_sweep(args, bl, dev, stream, tf_peak):
             torch.cuda.synchronize()
             sp = st.sparsity()
             o = torch.empty_like(x.q)
+            reps = reps_of[L]
             ms = time_calls_flushed(lambda: bl.blasst_prefill(
                 x.q, x.k, x.v, ln_lambda=lnl, o=o, want_lse=False),
-                reps, 1, stream, flush) / reps
+                reps, 2, stream, flush) / reps
             rec = {"L": L, "target": tgt, "a": a, "ln_lambda": lnl,
                    "sparsity": round(sp, 5), "deviation": round(abs(sp - tgt), 5),
                    "calibration_reached_target_at_L": cals[L]["status"] == 0,
