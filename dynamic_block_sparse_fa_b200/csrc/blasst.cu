@@ -189,29 +189,31 @@ cudaError_t launch_split(const blasst::DecodeArgs& a, long long grid,
 
 // The warp-MMA decode (decode_mma.cuh) for the sequential rule on a
 // contiguous cache with G <= 8, then the merge as for launch_decode.
-template <int G, int D, bool PAGED>
+template <int G, int D, bool PAGED, int BATCH = 1>
 cudaError_t launch_mma_split(const blasst::DecodeMmaArgs& a, long long grid,
                              cudaStream_t st) {
   using C = blasst::DecodeMmaCfg;
   cudaError_t e = cudaFuncSetAttribute(
-      blasst::decode_mma_kernel<G, D, PAGED>,
+      blasst::decode_mma_kernel<G, D, PAGED, BATCH>,
       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
-  blasst::decode_mma_kernel<G, D, PAGED>
+  blasst::decode_mma_kernel<G, D, PAGED, BATCH>
       <<<(unsigned)grid, blasst::kDecThreads, C::SMEM_ALLOC, st>>>(a);
   return cudaGetLastError();
 }
 
+// paged: the pool form; batch 2: the batched decision rule (contiguous)
 blasst_status_t launch_decode_mma(const blasst::DecodeMmaArgs& a, int G,
                                   int d, bool paged, long long grid,
                                   bool stats_only, void* o, float* lse,
-                                  int rows, cudaStream_t st) {
+                                  int rows, cudaStream_t st, int batch = 1) {
   cudaError_t e = cudaErrorInvalidValue;
   switch (G * 1000 + d) {
 #define BLASST_LAUNCH_MMA(GG, DD)                                           \
   case GG * 1000 + DD:                                                      \
     e = paged ? launch_mma_split<GG, DD, true>(a, grid, st)                 \
-              : launch_mma_split<GG, DD, false>(a, grid, st);               \
+              : (batch == 2 ? launch_mma_split<GG, DD, false, 2>(a, grid, st) \
+                            : launch_mma_split<GG, DD, false>(a, grid, st)); \
     break;
     BLASST_LAUNCH_MMA(1, 128)
     BLASST_LAUNCH_MMA(2, 128)
@@ -407,8 +409,9 @@ blasst_status_t wide_launch(const void* q, const void* k_cache,
 // Contiguous-cache decode.  batch = 0: blasst_decode / blasst_decode_window
 // (the sequential rule on the fastest kernel for the group: the warp-MMA
 // kernel for G <= 8, the tensor-core tiles for 16 <= G <= 128, the
-// CUDA-core kernel above); batch = 1 or 2: blasst_decode_batched, always on
-// the CUDA-core split kernel (batch 1 = the sequential rule).
+// CUDA-core kernel above); batch = 2: the batched rule (warp-MMA kernel for
+// G <= 8, else the CUDA-core kernel); batch = 1: the sequential rule on the
+// CUDA-core split kernel (a second, independent implementation).
 blasst_status_t decode_contiguous(const void* q, const void* k_cache,
                                   const void* v_cache, void* o, float* lse,
                                   int B, int Hq, int Hkv, int Lkv, int d,
@@ -425,9 +428,9 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
   int G = Hq / Hkv;
   if (Bc != blasst::kDecBc || !decode_group_ok(G))
     return BLASST_ERR_UNSUPPORTED_SHAPE;
-  // d = 128 everywhere; d = 64 on the warp-MMA kernel (the sequential rule
-  // with at most 8 heads per KV head)
-  if (!(d == blasst::kDecD || (d == 64 && batch == 0 && G <= 8)))
+  // d = 128 everywhere; d = 64 on the warp-MMA kernel (the sequential or
+  // the batched rule with at most 8 heads per KV head)
+  if (!(d == blasst::kDecD || (d == 64 && batch != 1 && G <= 8)))
     return BLASST_ERR_UNSUPPORTED_SHAPE;
   const int kv_div = G > 8 ? G / 8 : 1;  // tiles of 8 heads above 8
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
@@ -449,8 +452,9 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
                        window, 8, ln_lambda, S, workspace, workspace_bytes,
                        skip_stats, stream);
   const long long grid_mma = (long long)B * Hkv * S;
-  if (batch == 0 && G <= 8 && grid_mma <= 0x7fffffffLL) {
-    // the sequential rule on the warp-MMA kernel
+  if (batch != 1 && G <= 8 && grid_mma <= 0x7fffffffLL) {
+    // the sequential rule (batch 0) or the batched rule (batch 2) on the
+    // warp-MMA kernel
     const bool stats_only = (o == nullptr);
     blasst::DecodeMmaArgs m;
     memset(&m, 0, sizeof m);
@@ -476,7 +480,8 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
     m.stats_only = stats_only ? 1 : 0;
     m.window = window;
     return launch_decode_mma(m, G, d, false, grid_mma, stats_only, o, lse,
-                             B * Hq, static_cast<cudaStream_t>(stream));
+                             B * Hq, static_cast<cudaStream_t>(stream),
+                             batch == 2 ? 2 : 1);
   }
   G /= kv_div;
   const long long grid = (long long)B * Hkv * kv_div * S;

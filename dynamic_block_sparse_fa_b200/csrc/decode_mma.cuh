@@ -71,8 +71,8 @@ struct DecodeMmaCfg {
   static constexpr int NK = 2, NV = 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + NK * TILE;
-  static constexpr int OFF_M = OFF_V + NV * TILE;   // f32 [2][8 heads][4 warps]
-  static constexpr int OFF_L = OFF_M + 2 * 8 * 4 * 4;  // f32 [4 warps][8]
+  static constexpr int OFF_M = OFF_V + NV * TILE;  // f32 [2][2][8 heads][4 warps]
+  static constexpr int OFF_L = OFF_M + 2 * 2 * 8 * 4 * 4;  // f32 [4 warps][8]
   static constexpr int OFF_BAR = OFF_L + 4 * 8 * 4;    // u64 [NK + NV]
   static constexpr int SMEM = OFF_BAR + (NK + NV) * 8;
   static constexpr int SMEM_ALLOC = SMEM + 1024;  // 1024-byte alignment
@@ -133,10 +133,16 @@ __device__ __forceinline__ uint32_t swz_off(int key, int chunk) {
                     (((chunk & 7) ^ (key & 7)) << 4));
 }
 
-template <int G, int D, bool PAGED>
+// BATCH = 2: the batched decision rule (contiguous cache): blocks r and
+// r+1 are scored before either is decided, and each is judged against
+// Mb = max(running max before r, maxima of both blocks); kept blocks use Mb
+// as the reference of P.  (A skip never moves the running max, so the
+// running max is always the reference of O and l, in both rules.)
+template <int G, int D, bool PAGED, int BATCH = 1>
 __global__ void __launch_bounds__(kDecThreads, 3)
     decode_mma_kernel(const __grid_constant__ DecodeMmaArgs a) {
   static_assert(G >= 1 && G <= 8, "at most 8 heads per tile");
+  static_assert(BATCH == 1 || (BATCH == 2 && !PAGED), "pairs: contiguous");
   static_assert(D == 64 || D == 128, "head dimension 64 or 128");
   constexpr int NBOX = D / 64;     // 64-column boxes per block
   constexpr int KST = D / 16;      // k-steps of the scores
@@ -315,14 +321,16 @@ __global__ void __launch_bounds__(kDecThreads, 3)
     return true;
   };
 
-  for (int r = 0; r < nblk; ++r) {
+  // Scores of this warp's 16 keys of block r of the split (sc[g][i] = key
+  // 16w + 8g + 2q4 + i, scaled, -inf where hidden); returns the block max of
+  // head hr over the warp's keys.
+  auto score = [&](int r, float (&sc)[2][2]) -> float {
     const int j = j0 + r;
     const int stage = r % C::NK;
     if (!mbar_wait(&kfull[stage], (uint32_t)(r / C::NK) & 1u, kWaitDecodeK, r,
                    stage))
       ok = false;
-    // ---- scores of this warp's 16 keys: sc[g][i] = key 16w + 8g + 2q4 + i
-    float sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    sc[0][0] = sc[0][1] = sc[1][0] = sc[1][1] = 0.f;
     if (ok) {
       const uint32_t kb = aK + stage * C::TILE;
 #pragma unroll
@@ -349,7 +357,58 @@ __global__ void __launch_bounds__(kDecThreads, 3)
         mx = fmaxf(mx, sc[g][i]);
       }
     mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
+    return fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
+  };
+  // Statistics, mask and margin of block j (thread 0).
+  auto record = [&](int j, bool skip, const float (&mt)[G], const float (&mref)[G]) {
+    if (tid == 0) {
+      ++n_vis;
+      if (skip) ++n_skp;
+      if (a.mask) a.mask[(size_t)bh * a.nk + j] = skip ? 2 : 1;
+      if (a.margin) {  // max over the heads of m~ - m (+inf while m = -inf)
+        float dl = -INFINITY;
+#pragma unroll
+        for (int g = 0; g < G; ++g) dl = fmaxf(dl, mt[g] - mref[g]);
+        a.margin[(size_t)bh * a.nk + j] = dl - ln_lambda;
+      }
+    }
+  };
+  // A kept block: its V load, the previous kept block's P.V (its V has had
+  // at least this block's scoring to land), then this block's P against
+  // the new reference mn of head hr (mo the old one).
+  auto keep = [&](int j, const float (&sc)[2][2], float mo, float mn) {
+    if (tid == 0) load(&a.tv, sV + (kept % C::NV) * C::TILE, &vfull[kept % C::NV], j);
+    if (pend && !pv(kept - 1)) ok = false;
+    const float al = (mo == -INFINITY) ? 0.f : ex2_approx((mo - mn) * kLog2e);
+    const float mb = mn * kLog2e;
+    float p[2][2];
+#pragma unroll
+    for (int g = 0; g < 2; ++g)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) p[g][i] = ex2_approx(fmaf(sc[g][i], kLog2e, -mb));
+    l_part = al * l_part + ((p[0][0] + p[0][1]) + (p[1][0] + p[1][1]));
+    pp0 = pack_bf16x2(p[0][0], p[0][1]);
+    pp1 = pack_bf16x2(p[1][0], p[1][1]);
+    palpha = al;
+    prows = min(kDecBc, Lb - j * kDecBc);
+    pend = true;
+    ++kept;
+  };
+  // head hr's entry of a per-head array (head 0's for padding rows)
+  auto mine = [&](const float (&x)[G]) {
+    float v = x[0];
+#pragma unroll
+    for (int g = 1; g < G; ++g)
+      if (g == hr) v = x[g];
+    return v;
+  };
+
+  if constexpr (BATCH == 1) {
+  for (int r = 0; r < nblk; ++r) {
+    const int j = j0 + r;
+    const int stage = r % C::NK;
+    float sc[2][2];
+    const float mx = score(r, sc);
     float* sMr = sM + (r & 1) * 32;  // [head][warp], double-buffered
     if (q4 == 0 && hr < G) sMr[hr * 4 + warp] = mx;
     if (__syncthreads_or(!ok)) { ok = false; break; }
@@ -366,48 +425,65 @@ __global__ void __launch_bounds__(kDecThreads, 3)
       mt[g] = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
       if (!(mt[g] - m_run[g] < ln_lambda)) skip = false;
     }
-    if (tid == 0) {
-      ++n_vis;
-      if (skip) ++n_skp;
-      if (a.mask) a.mask[(size_t)bh * a.nk + j] = skip ? 2 : 1;
-      if (a.margin) {  // max over the heads of m~ - m (+inf while m = -inf)
-        float dl = -INFINITY;
-#pragma unroll
-        for (int g = 0; g < G; ++g) dl = fmaxf(dl, mt[g] - m_run[g]);
-        a.margin[(size_t)bh * a.nk + j] = dl - ln_lambda;
-      }
-    }
+    record(j, skip, mt, m_run);
     if (!skip && !stats_only) {
-      if (tid == 0) load(&a.tv, sV + (kept % C::NV) * C::TILE, &vfull[kept % C::NV], j);
-      // the previous kept block's P.V (its V has had this block to land)
-      if (pend && !pv(kept - 1)) { ok = false; }
-      // new reference, rescale factor and P of head hr
-      float mo = m_run[0], mh = mt[0];  // head hr's (head 0's for padding rows)
-#pragma unroll
-      for (int g = 1; g < G; ++g)
-        if (g == hr) {
-          mo = m_run[g];
-          mh = mt[g];
-        }
-      const float mn = fmaxf(mo, mh);
-      const float al = (mo == -INFINITY) ? 0.f : ex2_approx((mo - mn) * kLog2e);
-      const float mb = mn * kLog2e;
-      float p[2][2];
-#pragma unroll
-      for (int g = 0; g < 2; ++g)
-#pragma unroll
-        for (int i = 0; i < 2; ++i) p[g][i] = ex2_approx(fmaf(sc[g][i], kLog2e, -mb));
-      l_part = al * l_part + ((p[0][0] + p[0][1]) + (p[1][0] + p[1][1]));
-      pp0 = pack_bf16x2(p[0][0], p[0][1]);
-      pp1 = pack_bf16x2(p[1][0], p[1][1]);
-      palpha = al;
-      prows = min(kDecBc, Lb - j * kDecBc);
-      pend = true;
-      ++kept;
+      const float mo = mine(m_run);
+      keep(j, sc, mo, fmaxf(mo, mine(mt)));
     }
 #pragma unroll
     for (int g = 0; g < G; ++g) m_run[g] = fmaxf(m_run[g], mt[g]);
     if (__any_sync(FULL, !ok)) { ok = false; }
+  }
+  } else {
+  for (int r = 0; r < nblk; r += 2) {
+    const bool two = r + 1 < nblk;
+    float sc0[2][2], sc1[2][2];
+    float* sMp = sM + ((r >> 1) & 1) * 64;  // [block of the pair][head][warp]
+    const float mx0 = score(r, sc0);
+    if (q4 == 0 && hr < G) sMp[hr * 4 + warp] = mx0;
+    if (two) {
+      const float mx1 = score(r + 1, sc1);
+      if (q4 == 0 && hr < G) sMp[32 + hr * 4 + warp] = mx1;
+    }
+    if (__syncthreads_or(!ok)) { ok = false; break; }
+    // both K slots have been read: refill them
+    if (tid == 0) {
+      if (r + 2 < nblk) load(&a.tk, sK + (r % C::NK) * C::TILE, &kfull[r % C::NK], j0 + r + 2);
+      if (r + 3 < nblk)
+        load(&a.tk, sK + ((r + 1) % C::NK) * C::TILE, &kfull[(r + 1) % C::NK], j0 + r + 3);
+    }
+    float mt0[G], mt1[G], Mb[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float4 w0 = *reinterpret_cast<const float4*>(sMp + g * 4);
+      mt0[g] = fmaxf(fmaxf(w0.x, w0.y), fmaxf(w0.z, w0.w));
+      if (two) {
+        const float4 w1 = *reinterpret_cast<const float4*>(sMp + 32 + g * 4);
+        mt1[g] = fmaxf(fmaxf(w1.x, w1.y), fmaxf(w1.z, w1.w));
+      } else {
+        mt1[g] = -INFINITY;
+      }
+      Mb[g] = fmaxf(m_run[g], fmaxf(mt0[g], mt1[g]));
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (u == 1 && !two) break;
+      const int j = j0 + r + u;
+      bool skip = ln_lambda > -INFINITY;
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+        if (!((u ? mt1[g] : mt0[g]) - Mb[g] < ln_lambda)) skip = false;
+      record(j, skip, u ? mt1 : mt0, Mb);
+      if (!skip && !stats_only) {
+        keep(j, u ? sc1 : sc0, mine(m_run), mine(Mb));
+#pragma unroll
+        for (int g = 0; g < G; ++g) m_run[g] = Mb[g];  // the new reference
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) m_run[g] = Mb[g];
+    if (__any_sync(FULL, !ok)) { ok = false; }
+  }
   }
   if (ok && pend && !pv(kept - 1)) ok = false;
   if (__syncthreads_or(!ok)) ok = false;

@@ -131,6 +131,22 @@ def test_batched_skips_superset_of_sequential(blasst):
     assert bat.sum() > seq.sum()
 
 
+def test_batched_head_dim_64_matches_oracle(blasst):
+    m = blasst
+    x = planted_gap(2, 8, 2, 1, 1999, 64, decode=True, block=64, gap=8.0,
+                    heavy_frac=0.05, seed=config_seed(9, 64), device="cuda")
+    nk = -(-1999 // 64)
+    st = m.Stats(mask_numel=2 * 2 * nk)
+    o, lse = m.blasst_decode_batched(x.q, x.k, x.v, batch=2, ln_lambda=-3.0,
+                                     num_splits=3, stats=st)
+    torch.cuda.synchronize()
+    ref = oracle.decode_batched(x.q, x.k, x.v, 1 / 8.0, -3.0, 64, 3, 2)
+    P.check_out(P.to_np(o), ref["o"], "batched d64 o")
+    P.check_lse(P.to_np(lse), ref["lse"], "batched d64 lse")
+    P.check_mask(st.mask.cpu().numpy().reshape(2, 2, nk), ref["mask"],
+                 ref["margin"], "batched d64 mask")
+
+
 def test_batched_rejects_bad_batch(blasst):
     m = blasst
     x = planted_gap(1, 8, 2, 1, 512, 128, decode=True, block=64,
