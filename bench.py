@@ -413,7 +413,7 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
     o_h = torch.empty(B, Hq, d, dtype=torch.bfloat16).pin_memory()
     l_h = torch.empty(B, Hq, dtype=torch.float32).pin_memory()
 
-    def e2e_step():
+    def e2e_ops():
         q.copy_(q_h, non_blocking=True)
         kv_new_d.copy_(kv_new_h, non_blocking=True)
         k[:, :, Lkv - 1].copy_(kv_new_d[0])
@@ -421,6 +421,33 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
         bl.blasst_decode(q, k, v, ln_lambda=lnl, o=o, lse=lse, workspace=ws)
         o_h.copy_(o, non_blocking=True)
         l_h.copy_(lse, non_blocking=True)
+
+    # The step's copies and launches as one CUDA graph (captured once,
+    # replayed every step): the host pays one launch instead of ~10.
+    graph = None
+    if not args.no_e2e and not args.no_graph:
+        try:
+            side = torch.cuda.Stream(device=dev)
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                for _ in range(2):
+                    e2e_ops()
+            stream.wait_stream(side)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                e2e_ops()
+            torch.cuda.synchronize()
+        except Exception as exc:  # report and time the launches one by one
+            graph = None
+            print(f"e2e graph capture failed ({exc}); timing eager steps",
+                  file=sys.stderr)
+
+    def e2e_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            e2e_ops()
         stream.synchronize()  # the host reads the step's result
 
     ms_e2e = (time_calls(e2e_step, K, W, stream, barrier)
@@ -475,7 +502,8 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": _r(e2e_max / K, 4),
                 "what": "h2d of q and the new token's K/V rows, decode, "
-                        "d2h of o and lse, host sync, per step"},
+                        "d2h of o and lse, host sync, per step",
+                "cuda_graph": graph is not None},
         "gpu_launches": 2 * K,
         "clocks": clk.summary(),
     }
@@ -1301,6 +1329,8 @@ def main():
     ap.add_argument("--prefill-L", type=int, default=PRE["L"])
     ap.add_argument("--prefill-lnl", type=float, default=None,
                     help="measure prefill only at this ln(lambda)")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the end-to-end step as separate launches")
     ap.add_argument("--no-s50", action="store_true",
                     help="skip the decode leg at 50%% sparsity (profiling runs)")
     ap.add_argument("--no-sweeps", action="store_true",
