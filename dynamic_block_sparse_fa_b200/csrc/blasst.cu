@@ -159,7 +159,8 @@ size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits) {
   const size_t rows = (size_t)B * Hq * num_splits;
   const size_t o_bytes = (rows * d * sizeof(float) + 255) & ~(size_t)255;
   const size_t l_bytes = (rows * sizeof(float) + 255) & ~(size_t)255;
-  return o_bytes + l_bytes;
+  const size_t w_bytes = ((size_t)B * sizeof(int) + 255) & ~(size_t)255;
+  return o_bytes + l_bytes + w_bytes;
 }
 
 }  // extern "C"
@@ -292,17 +293,38 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
 // blasst_decode_workspace_size).
 blasst_status_t carve_workspace(void* workspace, size_t workspace_bytes,
                                 int B, int Hq, int d, int S, float** o_part,
-                                float** lse_part) {
+                                float** lse_part, int** order = nullptr) {
   const size_t need = blasst_decode_workspace_size(B, Hq, d, S);
   if (!workspace || workspace_bytes < need) return BLASST_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return BLASST_ERR_MISALIGNED;
   const size_t rows = (size_t)B * Hq * S;
+  const size_t o_bytes = (rows * d * sizeof(float) + 255) & ~(size_t)255;
+  const size_t l_bytes = (rows * sizeof(float) + 255) & ~(size_t)255;
   *o_part = static_cast<float*>(workspace);
-  *lse_part = reinterpret_cast<float*>(
-      static_cast<char*>(workspace) +
-      ((rows * d * sizeof(float) + 255) & ~(size_t)255));
+  *lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + o_bytes);
+  if (order)
+    *order = reinterpret_cast<int*>(static_cast<char*>(workspace) + o_bytes +
+                                    l_bytes);
   return BLASST_OK;
+}
+
+// Paged calls whose grid is more than one wave decode the longest sequences
+// first: the order (a permutation of the B sequences, see
+// decode_order_kernel) goes to the workspace's last region.  NULL when the
+// order cannot matter (one sequence, or every CTA resident at once).
+int* paged_work_order(const int* seq_lens, int B, long long ctas, int* region,
+                      cudaStream_t st, blasst_status_t* rc) {
+  *rc = BLASST_OK;
+  if (B < 2 || ctas <= (long long)kNumSmB200 * 3) return nullptr;
+  blasst::decode_order_kernel<<<(unsigned)((B + 255) / 256), 256, 0, st>>>(
+      seq_lens, B, region);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    *rc = cuda_status(e, "paged decode work order");
+    return nullptr;
+  }
+  return region;
 }
 }  // namespace
 
@@ -568,10 +590,11 @@ blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
     const bool stats_only = (o == nullptr);
     blasst::DecodeMmaArgs m;
     memset(&m, 0, sizeof m);
+    int* region = nullptr;
     if (!stats_only) {
       const blasst_status_t ws = carve_workspace(workspace, workspace_bytes, B,
                                                  Hq, d, S, &m.o_part,
-                                                 &m.lse_part);
+                                                 &m.lse_part, &region);
       if (ws != BLASST_OK) return ws;
     }
     const int box_rows = page_size < 64 ? page_size : 64;
@@ -597,6 +620,12 @@ blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
     m.num_pages = num_pages;
     m.log2_page = log2_page;
     m.per_length = per_length ? 1 : 0;
+    if (region) {
+      blasst_status_t rc;
+      m.order = paged_work_order(seq_lens, B, (long long)B * Hkv * S, region,
+                                 static_cast<cudaStream_t>(stream), &rc);
+      if (rc != BLASST_OK) return rc;
+    }
     return launch_decode_mma(m, G, d, true, (long long)B * Hkv * S, stats_only,
                              o, lse, B * Hq, static_cast<cudaStream_t>(stream));
   }
@@ -606,12 +635,20 @@ blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
   const bool stats_only = (o == nullptr);
   float* o_part = nullptr;
   float* lse_part = nullptr;
+  int* region = nullptr;
   if (!stats_only) {
     const blasst_status_t ws = carve_workspace(workspace, workspace_bytes, B,
-                                               Hq, d, S, &o_part, &lse_part);
+                                               Hq, d, S, &o_part, &lse_part,
+                                               &region);
     if (ws != BLASST_OK) return ws;
   }
   blasst::DecodeArgs a = {};
+  if (region) {
+    blasst_status_t rc;
+    a.order = paged_work_order(seq_lens, B, grid, region,
+                               static_cast<cudaStream_t>(stream), &rc);
+    if (rc != BLASST_OK) return rc;
+  }
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k = static_cast<const __nv_bfloat16*>(k_pages);
   a.v = static_cast<const __nv_bfloat16*>(v_pages);

@@ -48,6 +48,9 @@ struct DecodeArgs {
   long long page_stride;   // elements
   int log2_page, max_pages, num_pages;
   int per_length;  // ln_lambda is ln a; sequence b uses min(0, ln a - ln L_b)
+  // paged: the sequence decoded by each slot of the grid (NULL: slot b is
+  // sequence b), from decode_order_kernel
+  const int* order;
   // sliding window: the token sees only the last `window` keys (0 = all);
   // the splits divide the blocks that hold them
   int window;
@@ -156,10 +159,14 @@ __global__ void __launch_bounds__(kDecThreads, BATCH == 1
   const int warp = tid >> 5;
 
   const int s = blockIdx.x % a.S;
-  const int bh = blockIdx.x / a.S;  // b * Hkv + hkv (tiles)
+  const int slot = blockIdx.x / a.S;  // sequence slot * Hkv + hkv (tiles)
   const int Hq = a.Hkv * G;
-  const int b = bh / a.Hkv;
-  const int hkv = bh - b * a.Hkv;
+  const int hkv = slot % a.Hkv;
+  int b = slot / a.Hkv;
+  if constexpr (PAGED) {
+    if (a.order) b = __ldg(a.order + b);
+  }
+  const int bh = b * a.Hkv + hkv;
   const int hkv_c = hkv / a.kv_div;  // the cache head of this tile
   int Lb = a.Lkv;  // keys of this sequence
   float ln_lambda = a.ln_lambda;
@@ -701,6 +708,33 @@ __global__ void __launch_bounds__(kDecThreads, BATCH == 1
 
 // Log-sum-exp merge of the S split partials of one (sequence, query head):
 //   lse = ln sum_s exp(lse_s),  o = sum_s exp(lse_s - lse) o_s.
+// Work order of a paged call: order[r] is the sequence with the r-th
+// longest length (ties by index), so that the CTAs of the longest sequences
+// start first and the last wave holds the shortest splits.  Which CTA runs a
+// split changes nothing in what the split computes.  rank(i) counts the
+// sequences before i in the strict order (length descending, index
+// ascending); distinct sequences get distinct ranks in [0, B), so `order`
+// is a permutation.  Grid ceil(B / 256) x 256 threads.
+__global__ void __launch_bounds__(256)
+    decode_order_kernel(const int* __restrict__ seq_lens, int B,
+                        int* __restrict__ order) {
+  __shared__ int len[256];
+  const int i = blockIdx.x * 256 + threadIdx.x;
+  const int li = i < B ? __ldg(seq_lens + i) : 0;
+  int rank = 0;
+  for (int j0 = 0; j0 < B; j0 += 256) {
+    __syncthreads();
+    if (j0 + (int)threadIdx.x < B) len[threadIdx.x] = __ldg(seq_lens + j0 + threadIdx.x);
+    __syncthreads();
+    const int n = min(256, B - j0);
+    for (int jj = 0; jj < n; ++jj) {
+      const int lj = len[jj];
+      rank += (lj > li || (lj == li && j0 + jj < i)) ? 1 : 0;
+    }
+  }
+  if (i < B) order[rank] = i;
+}
+
 // An empty split (lse_s = -inf, o_s = 0) gets weight 0.  One thread per
 // output column: the block has d (64 or 128) threads.
 __global__ void __launch_bounds__(kDecD)

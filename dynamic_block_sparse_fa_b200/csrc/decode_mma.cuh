@@ -63,6 +63,7 @@ struct DecodeMmaArgs {
   const int* seq_lens;       // [B]; Lkv is then the upper bound on them
   int max_pages, num_pages, log2_page;
   int per_length;  // ln_lambda is ln a; sequence b uses min(0, ln a - ln L_b)
+  const int* order;  // paged: sequence of each grid slot (NULL: slot b is b)
 };
 
 struct DecodeMmaCfg {
@@ -157,10 +158,14 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   const int warp = tid >> 5;
 
   const int s = blockIdx.x % a.S;
-  const int bh = blockIdx.x / a.S;  // b * Hkv + hkv
+  const int slot = blockIdx.x / a.S;  // sequence slot * Hkv + hkv
   const int Hq = a.Hkv * G;
-  const int b = bh / a.Hkv;
-  const int hkv = bh - b * a.Hkv;
+  const int hkv = slot % a.Hkv;
+  int b = slot / a.Hkv;
+  if constexpr (PAGED) {
+    if (a.order) b = __ldg(a.order + b);
+  }
+  const int bh = b * a.Hkv + hkv;
   int Lb = a.Lkv;  // keys of this sequence
   float ln_lambda = a.ln_lambda;
   const int* bt_row = nullptr;

@@ -363,6 +363,12 @@ blasst_status_t blasst_decode_noalloc(const void *q, const void *k_cache,
  *  skip_stats      as blasst_decode; the mask layout is
  *                  [B, Hkv * T, ceil(max_seq_len / 64)] and blocks past a
  *                  sequence's end are not written
+ * When the call has more (sequence, KV head, split) work items than the
+ * GPU holds at once, a small kernel first sorts the sequences by length
+ * into the workspace and the CTAs take the longest sequences' splits
+ * first, so that the last wave holds the shortest splits.  Which CTA runs a
+ * split changes nothing in what it computes: outputs, decisions and
+ * counters are the same bits in any order.
  * The block table and the lengths live on the device, so they are checked
  * there: before any copy of a split is issued, its kernel checks its
  * sequence's length and every page id it will read.  A bad value is not
@@ -384,8 +390,9 @@ blasst_status_t blasst_decode_paged(const void *q, const void *k_pages,
                                     const blasst_skip_stats_t *skip_stats,
                                     void *stream);
 
-/* Bytes of decode workspace: B*Hq*S*(d+1) float32 values, rounded up to 256.
- * num_splits must be the resolved value (>= 1). */
+/* Bytes of decode workspace: B*Hq*S*(d+1) float32 values (the split
+ * partials) and B int32 values (blasst_decode_paged's work order), each
+ * region rounded up to 256.  num_splits must be the resolved value (>= 1). */
 size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits);
 
 /* The automatic split count used when num_splits == 0.  Pure function of

@@ -234,7 +234,9 @@ def test_split_policy_and_workspace(lib):
         assert 1 <= s <= max(1, nk // 8)
     ws = m.blasst_decode_workspace_size(32, 32, 128, 5)
     rows = 32 * 32 * 5
-    assert ws >= rows * 129 * 4 and ws % 256 == 0
+    assert ws >= rows * 129 * 4 + 32 * 4 and ws % 256 == 0
+    # partials, lse and the paged work order, each region 256-byte aligned
+    assert m.blasst_decode_workspace_size(1, 1, 128, 1) == 512 + 256 + 256
 
 
 def test_mla_split_policy(lib):

@@ -316,3 +316,57 @@ def test_paged_varlen_per_length_sampled(blasst):
         P.check_mask(mask[b:b + 1, :, :nk], ref["mask"], ref["margin"],
                      f"seq {b}")
         assert np.all(mask[b, :, nk:] == 0)
+
+
+def test_paged_varlen_work_order_is_invisible(blasst):
+    """Batch 32 of lengths 1K..64K (one tie) in 16-token pages, 5 splits:
+    1280 work items, more than the GPU holds at once, so the call sorts the
+    sequences by length and decodes the longest first.  Every sequence's
+    output, lse and decisions equal, bit for bit, a contiguous decode of that
+    sequence alone (40 work items, natural order), and the counters add up;
+    o and lse are poisoned with NaN first, so a sequence that no CTA decoded
+    would show."""
+    m = blasst
+    B, Hq, Hkv, d, S, lnl = 32, 32, 8, 128, 5, -5.5
+    g = torch.Generator().manual_seed(config_seed(6, 7))
+    lens = torch.randint(1024, 65536 + 1, (B,), generator=g).tolist()
+    lens[3] = lens[9]  # equal lengths: the index orders them
+    Lmax = max(lens)
+    assert B * Hkv * S > 148 * 3
+    q = torch.empty(B, Hq, d, dtype=torch.bfloat16, device="cuda")
+    k = torch.empty(B, Hkv, Lmax, d, dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    planted_gap_kv_inplace(k, v, q, block=64, gap=8.0, heavy_frac=0.03,
+                           seed=config_seed(6, 8))
+    pk = paginate(k, v, lens, 16, seed=14, spare_pages=8, poison=POISON)
+    del k, v
+    nk_max = -(-Lmax // 64)
+    st = m.Stats(mask_numel=B * Hkv * nk_max)
+    o = torch.full((B, Hq, d), float("nan"), dtype=torch.bfloat16,
+                   device="cuda")
+    lse = torch.full((B, Hq), float("nan"), dtype=torch.float32,
+                     device="cuda")
+    m.blasst_decode_paged(q, pk.k_pages, pk.v_pages, pk.block_table,
+                          pk.seq_lens, max_seq_len=Lmax, ln_lambda=lnl,
+                          num_splits=S, o=o, lse=lse, stats=st)
+    torch.cuda.synchronize()
+    assert m.blasst_check_device_error()[0] == 0
+    mask = st.mask.view(B, Hkv, nk_max)
+    vis = skp = 0
+    for b in range(B):
+        L = lens[b]
+        npg, nk = -(-L // 16), -(-L // 64)
+        ids = pk.block_table[b, :npg].long()
+        kb = pk.k_pages[ids].transpose(0, 1).reshape(Hkv, npg * 16, d)[:, :L]
+        vb = pk.v_pages[ids].transpose(0, 1).reshape(Hkv, npg * 16, d)[:, :L]
+        sb = m.Stats(mask_numel=Hkv * nk)
+        ob, lb = m.blasst_decode(q[b:b + 1], kb[None].contiguous(),
+                                 vb[None].contiguous(), ln_lambda=lnl,
+                                 num_splits=S, stats=sb)
+        torch.cuda.synchronize()
+        assert torch.equal(ob, o[b:b + 1]) and torch.equal(lb, lse[b:b + 1]), b
+        assert torch.equal(sb.mask.view(Hkv, nk), mask[b, :, :nk]), b
+        assert not mask[b, :, nk:].any(), b
+        v1, s1 = sb.read()
+        vis, skp = vis + v1, skp + s1
+    assert st.read() == (vis, skp)
