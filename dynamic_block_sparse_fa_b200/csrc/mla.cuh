@@ -21,13 +21,17 @@
 // add the other CTA's partial to their own.  IEEE addition commutes, so
 // both CTAs hold the same scores bit for bit and take the same decisions
 // without exchanging them.
-//   warp 0      TMA producer: this rank's boxes of each cache block, ring of 3
-//   warp 1      MMA issuer (one lane): partial S = Q_r c_r^T (TS, 16 or 20
-//               products, N = 64), issued as soon as the previous S has been
-//               read; for a kept block O_r += P V_r (TS, 4 products, N = 256)
+//   warp 0      TMA producer: this rank's boxes of each cache block, ring of 4
+//   warp 1      MMA issuer (whole warp, one elected lane issues): partial
+//               S = Q_r c_r^T (TS, 16 or 20 products, N = 64), issued as soon
+//               as the previous S has been read; for a kept block
+//               O_r += P V_r (TS, 4 products, N = 256).  Order S(1), S(2),
+//               PV(0), S(3), PV(1), ...: the scores run one block ahead
 //   warps 2..5  one thread per head (TMEM lane): Q_r into TMEM, partial
-//               score exchange, row max, vote, exp, P, lazy O rescale,
-//               epilogue
+//               score exchange one block ahead (block j+1's partial is read
+//               and sent before block j is decided, so the exchange overlaps
+//               the vote and the exps), row max, vote, exp, P, lazy O
+//               rescale, epilogue
 // Tensor memory: Q_r [0, 160) (bf16 pairs), P [160, 192), S [192, 256),
 // O_r [256, 512).
 #pragma once
@@ -59,7 +63,7 @@ struct MlaPairCfg {
   static constexpr int BOX = 64 * 128;        // 64 keys x 64 columns (bf16)
   static constexpr int NBX = 5;               // boxes per ring slot (rank 1)
   static constexpr int SLOT = NBX * BOX;      // 40960 bytes
-  static constexpr int NK = 3;                // ring slots
+  static constexpr int NK = 4;                // ring slots
   static constexpr int XBYTES = 64 * 128 * 4; // a partial score block, f32
   static constexpr int OFF_K = 0;
   static constexpr int OFF_X = OFF_K + NK * SLOT;  // [2] partials from the peer
@@ -160,7 +164,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaPairThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA
-    if (lane == 0 && nb > 0) {
+    if (nb > 0) {
       constexpr uint32_t id_s = idesc_bf16(128, kMlaBc, 0, 0);
       constexpr uint32_t id_o = idesc_bf16(128, 256, 0, 1);
       const uint32_t aK = smem_u32(smem + C::OFF_K);
@@ -169,58 +173,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaPairThreads, 1)
         const uint32_t kb = aK + (jj % C::NK) * C::SLOT;
 #pragma unroll 4
         for (int k = 0; k < nmma; ++k)
-          mma_ts(tmem + C::COL_S, tmem + C::COL_Q + k * 8,
+          mma_ts_elect(tmem + C::COL_S, tmem + C::COL_Q + k * 8,
                  smem_desc(kb + (k >> 2) * C::BOX + (k & 3) * 32, 16, 1024, 2),
                  id_s, k > 0 ? 1u : 0u);
-        mma_commit(&bar[C::B_SF]);
+        mma_commit_elect(&bar[C::B_SF]);
       };
-      bool ok = mbar_wait(&bar[C::B_QR], 0, kWaitMlaPair, 0, 10) &&
-                mbar_wait(&bar[C::B_KF], 0, kWaitMlaPair, 0, 11);
-      tc_fence_after();
-      if (ok) score(0);
+      // P.V of block jj once its decision is known (kept: after its P),
+      // then the block's ring slot is released
       int npv = 0;
-      for (int jj = 0; jj < nb && ok; ++jj) {
+      auto value = [&](int jj) -> bool {
         const int sl = jj % C::NK;
-        if (jj + 1 < nb) {
-          // my partial S(jj) has been read: S(jj+1) overwrites it
-          const int sn = (jj + 1) % C::NK;
-          ok = mbar_wait(&bar[C::B_SR], jj & 1, kWaitMlaPair, jj, 16) &&
-               mbar_wait(&bar[C::B_KF + sn], ((jj + 1) / C::NK) & 1,
-                         kWaitMlaPair, jj + 1, 11 + sn);
-          if (!ok) break;
-          tc_fence_after();
-          score(jj + 1);
-        }
         const uint32_t want = (uint32_t)(jj + 1) << 1;
         uint32_t w = ld_acquire_shared(&dec_word[jj % C::R]);
         if ((w & ~1u) != want) {
           const long long t0 = clock64();
+          bool tout = false;
           while (((w = ld_acquire_shared(&dec_word[jj % C::R])) & ~1u) != want) {
             if (clock64() - t0 > kWaitLimitCycles) {
               record_error(kWaitMlaPair, jj, 0, 13);
-              ok = false;
+              tout = true;
               break;
             }
           }
-          if (!ok) break;
+          if (__any_sync(FULL, tout)) return false;
         }
         if (!stats_only && (w & 1u) == 0) {
-          ok = mbar_wait(&bar[C::B_PF], npv & 1, kWaitMlaPair, jj, 14);
-          if (!ok) break;
+          if (!__all_sync(FULL, mbar_wait(&bar[C::B_PF], npv & 1, kWaitMlaPair, jj, 14)))
+            return false;
           tc_fence_after();
           // my 256 value columns: the slot's first 4 boxes, MN-major
           const uint32_t kb = aK + sl * C::SLOT;
 #pragma unroll
           for (int k = 0; k < kMlaBc / 16; ++k)
-            mma_ts(tmem + C::COL_O, tmem + C::COL_P + k * 8,
+            mma_ts_elect(tmem + C::COL_O, tmem + C::COL_P + k * 8,
                    smem_desc(kb + k * 2048, C::BOX, 1024, 2), id_o,
                    (npv > 0 || k > 0) ? 1u : 0u);
           ++npv;
-          mma_commit(&bar[C::B_PVD]);
+          mma_commit_elect(&bar[C::B_PVD]);
         }
-        mma_commit(&bar[C::B_KE + sl]);
+        mma_commit_elect(&bar[C::B_KE + sl]);
+        return true;
+      };
+      bool ok = __all_sync(FULL, mbar_wait(&bar[C::B_QR], 0, kWaitMlaPair, 0, 10) &&
+                                 mbar_wait(&bar[C::B_KF], 0, kWaitMlaPair, 0, 11));
+      tc_fence_after();
+      if (ok) score(0);
+      // The head threads read S(jj+1) before they decide block jj, so the
+      // scores of block jj+1 go to the tensor core ahead of P.V(jj-1):
+      // order S(1), S(2), PV(0), S(3), PV(1), ...
+      for (int jj = 0; jj < nb && ok; ++jj) {
+        if (jj + 1 < nb) {
+          // my partial S(jj) has been read: S(jj+1) overwrites it
+          const int sn = (jj + 1) % C::NK;
+          ok = __all_sync(FULL, mbar_wait(&bar[C::B_SR], jj & 1, kWaitMlaPair, jj, 16) &&
+                                mbar_wait(&bar[C::B_KF + sn], ((jj + 1) / C::NK) & 1,
+                                          kWaitMlaPair, jj + 1, 11 + sn));
+          if (!ok) break;
+          tc_fence_after();
+          score(jj + 1);
+        }
+        if (jj >= 1) ok = value(jj - 1);
       }
-      mma_commit(&bar[C::B_OD]);
+      if (ok) value(nb - 1);
+      mma_commit_elect(&bar[C::B_OD]);
     }
     __syncwarp();
   } else {
@@ -270,29 +285,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaPairThreads, 1)
     unsigned long long n_vis = 0, n_skp = 0;
     bool ok = true;
     int npv = 0;         // kept blocks so far (one P.V each)
-    bool wfail = false;  // a wait after the vote gave up: leave at the next one
-    for (int jj = 0; jj < nb; ++jj) {
-      const int j = j0 + jj;
-      const int xb = jj & 1;
-      bool w = mbar_wait(&bar[C::B_SF], jj & 1, kWaitMlaPair, jj, 20) && !wfail;
+    // Block jj's partial goes to the peer one step ahead: the head threads
+    // read S(jj+1) and send it before they decide block jj, so that the
+    // exchange of block jj+1 runs while block jj is voted on and
+    // exponentiated.  cur: block jj's scores; nxt: block jj+1's partial.
+    bool w = true;  // this thread's waits so far
+    uint32_t cur[2][32], nxt[2][32];
+    auto read_send = [&](int jj, uint32_t (&sr)[2][32]) {
+      if (!mbar_wait(&bar[C::B_SF], jj & 1, kWaitMlaPair, jj, 20)) w = false;
       tc_fence_after();
-      uint32_t sr[2][32];
       tmem_ld32(lane_base + C::COL_S, sr[0]);
       tmem_ld32(lane_base + C::COL_S + 32, sr[1]);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[C::B_SR]);  // S(jj+1) may overwrite S
-      // my partial into the peer's X[xb] as [4-key group][head] float4s,
-      // counted on the peer's X[xb] barrier
-      const uint32_t xp = x_peer + xb * C::XBYTES + h * 16;
+      // my partial into the peer's X[jj & 1] as [4-key group][head]
+      // float4s, counted on the peer's X[jj & 1] barrier
+      const uint32_t xp = x_peer + (jj & 1) * C::XBYTES + h * 16;
 #pragma unroll
       for (int q4 = 0; q4 < 16; ++q4) {
         const uint32_t* v = &sr[q4 >> 3][(q4 & 7) * 4];
-        st_async_v4(xp + q4 * 2048, v[0], v[1], v[2], v[3], xf_peer + xb * 8);
+        st_async_v4(xp + q4 * 2048, v[0], v[1], v[2], v[3],
+                    xf_peer + (jj & 1) * 8);
       }
-      // the peer's partial, added to mine (the peer adds in the other
-      // order: the same sums)
+    };
+    if (nb > 0) read_send(0, cur);
+    for (int jj = 0; jj < nb; ++jj) {
+      const int j = j0 + jj;
+      const int xb = jj & 1;
+      if (jj > 0) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int x = 0; x < 32; ++x) cur[c][x] = nxt[c][x];
+      }
+      uint32_t (&sr)[2][32] = cur;
+      // the peer's partial of block jj (sent one step ago), added to mine
+      // (the peer adds in the other order: the same sums)
       if (!mbar_wait_cluster(&bar[C::B_XF + xb], (jj >> 1) & 1, kWaitMlaPair,
                              jj, 32 + xb))
         w = false;
@@ -311,6 +341,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaPairThreads, 1)
         v[2] = __float_as_uint(__uint_as_float(v[2]) + o4.z);
         v[3] = __float_as_uint(__uint_as_float(v[3]) + o4.w);
       }
+      // X[xb] has been read: the peer may now refill it (block jj+2), which
+      // it does only after it has received my partial of block jj+1
+      if (jj + 1 < nb) read_send(jj + 1, nxt);
       const int valid = min(kMlaBc, a.L - j * kMlaBc);  // keys of the block
       if (valid < kMlaBc) {
 #pragma unroll
@@ -355,7 +388,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaPairThreads, 1)
       // P and O are free once the previous P.V is done
       if (npv > 0 &&
           !mbar_wait(&bar[C::B_PVD], (npv - 1) & 1, kWaitMlaPair, jj, 22))
-        wfail = true;
+        w = false;
       tc_fence_after();
       float alpha = 1.f;
       bool rescale = false;
