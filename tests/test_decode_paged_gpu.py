@@ -370,3 +370,43 @@ def test_paged_varlen_work_order_is_invisible(blasst):
         v1, s1 = sb.read()
         vis, skp = vis + v1, skp + s1
     assert st.read() == (vis, skp)
+
+
+def test_paged_varlen_work_order_cuda_core_kernel(blasst):
+    """The same work order on the CUDA-core paged kernel (16 query heads per
+    KV head, two tiles of 8): batch 32 of lengths 1K..16K, 5 splits, 640
+    work items.  Every sequence equals, bit for bit, the contiguous CUDA-core
+    kernel (blasst_decode_batched with batch 1) on that sequence alone."""
+    m = blasst
+    B, Hq, Hkv, d, S, lnl = 32, 32, 2, 128, 5, -4.0
+    g = torch.Generator().manual_seed(config_seed(6, 9))
+    lens = torch.randint(1024, 16384 + 1, (B,), generator=g).tolist()
+    Lmax = max(lens)
+    assert B * Hkv * 2 * S > 148 * 3
+    q = torch.empty(B, Hq, d, dtype=torch.bfloat16, device="cuda")
+    k = torch.empty(B, Hkv, Lmax, d, dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    planted_gap_kv_inplace(k, v, q, block=64, gap=8.0, heavy_frac=0.03,
+                           seed=config_seed(6, 10))
+    pk = paginate(k, v, lens, 16, seed=15, spare_pages=8, poison=POISON)
+    del k, v
+    o = torch.full((B, Hq, d), float("nan"), dtype=torch.bfloat16,
+                   device="cuda")
+    lse = torch.full((B, Hq), float("nan"), dtype=torch.float32,
+                     device="cuda")
+    m.blasst_decode_paged(q, pk.k_pages, pk.v_pages, pk.block_table,
+                          pk.seq_lens, max_seq_len=Lmax, ln_lambda=lnl,
+                          num_splits=S, o=o, lse=lse)
+    torch.cuda.synchronize()
+    assert m.blasst_check_device_error()[0] == 0
+    for b in range(B):
+        L = lens[b]
+        npg = -(-L // 16)
+        ids = pk.block_table[b, :npg].long()
+        kb = pk.k_pages[ids].transpose(0, 1).reshape(Hkv, npg * 16, d)[:, :L]
+        vb = pk.v_pages[ids].transpose(0, 1).reshape(Hkv, npg * 16, d)[:, :L]
+        ob, lb = m.blasst_decode_batched(q[b:b + 1], kb[None].contiguous(),
+                                         vb[None].contiguous(), batch=1,
+                                         ln_lambda=lnl, num_splits=S)
+        torch.cuda.synchronize()
+        assert torch.equal(ob, o[b:b + 1]) and torch.equal(lb, lse[b:b + 1]), b
