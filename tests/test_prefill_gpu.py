@@ -143,7 +143,7 @@ def test_prefill_rejects_bad_arguments(blasst):
 
 
 @pytest.mark.parametrize("which", ["s70", "dense"])
-def test_prefill_full_size_sampled(blasst, which):
+def test_prefill_full_size_sampled(blasst, which, capsys):
     """B 1, Hq 32, Hkv 8, L 32768, d 128, causal, 128x128 tiles, planted gap
     8 with sink + 2% heavy blocks + 512-token window boost, at the lambda
     calibrated to 70% sparsity and at the dense path; compared with the
@@ -168,8 +168,9 @@ def test_prefill_full_size_sampled(blasst, which):
                int(rng.integers(256))) for _ in range(64)]
     ref, mask, ties = _compare(m, x, True, 128, lnl, units=units,
                                check_stats_only=False)
-    print(f"full-size prefill ({which}, ln lambda {lnl}): {len(units)} tiles, "
-          f"oracle sparsity {ref['skipped'] / ref['visited']:.4f}, "
-          f"near-ties {ties}")
+    with capsys.disabled():  # shown in a quiet run too
+        print(f"\nfull-size prefill ({which}, ln lambda {lnl}): {len(units)} "
+              f"tiles, oracle sparsity {ref['skipped'] / ref['visited']:.4f}, "
+              f"near-ties {ties}")
     if which == "dense":
         assert (mask == 2).sum() == 0
