@@ -8,8 +8,9 @@ from .blasst import (BlasstError, Stats, blasst_calibrate,
                      blasst_check_device_error, blasst_decode,
                      blasst_decode_batched, blasst_decode_noalloc,
                      blasst_decode_paged,
+                     blasst_decode_group_splits,
                      blasst_decode_splits, blasst_decode_wide,
-                     blasst_decode_window,
+                     blasst_decode_wide_splits, blasst_decode_window,
                      blasst_decode_workspace_size,
                      blasst_fit_a, blasst_last_error, blasst_mla_decode,
                      blasst_mla_decode_splits,
@@ -24,8 +25,9 @@ __all__ = ["BlasstError", "Stats", "blasst_calibrate",
            "blasst_check_device_error", "blasst_decode",
            "blasst_decode_batched", "blasst_decode_noalloc",
            "blasst_decode_paged",
+           "blasst_decode_group_splits",
            "blasst_decode_splits", "blasst_decode_wide",
-           "blasst_decode_window",
+           "blasst_decode_wide_splits", "blasst_decode_window",
            "blasst_decode_workspace_size", "blasst_fit_a", "blasst_last_error",
            "blasst_mla_decode", "blasst_mla_decode_splits",
            "blasst_mla_decode_workspace_size",

@@ -119,6 +119,10 @@ _lib.blasst_decode_workspace_size.restype = _sz
 _lib.blasst_decode_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.blasst_decode_splits.restype = _i
 _lib.blasst_decode_splits.argtypes = [_i, _i, _i, _i]
+_lib.blasst_decode_wide_splits.restype = _i
+_lib.blasst_decode_wide_splits.argtypes = [_i, _i, _i, _i]
+_lib.blasst_decode_group_splits.restype = _i
+_lib.blasst_decode_group_splits.argtypes = [_i, _i, _i, _i, _i]
 _lib.blasst_calibrate.restype = _i
 _lib.blasst_calibrate.argtypes = [_d, ctypes.POINTER(CalibSample), _d, _vp,
                                   ctypes.POINTER(CalibResult), _vp]
@@ -140,7 +144,8 @@ _lib.blasst_version.argtypes = []
 EXPORTED = ["blasst_prefill", "blasst_decode", "blasst_decode_noalloc",
             "blasst_decode_paged",
             "blasst_decode_workspace_size",
-            "blasst_decode_splits", "blasst_calibrate", "blasst_fit_a",
+            "blasst_decode_splits", "blasst_decode_wide_splits",
+            "blasst_decode_group_splits", "blasst_calibrate", "blasst_fit_a",
             "blasst_skip_stats_reset", "blasst_check_device_error",
             "blasst_selftest_wait_timeout",
             "blasst_strerror", "blasst_last_error", "blasst_version"]
@@ -421,6 +426,14 @@ def blasst_decode_splits(B, Hkv, Lkv, Bc=64) -> int:
     return int(_lib.blasst_decode_splits(B, Hkv, Lkv, Bc))
 
 
+def blasst_decode_wide_splits(B, Hkv, Lkv, Bc=64) -> int:
+    return int(_lib.blasst_decode_wide_splits(B, Hkv, Lkv, Bc))
+
+
+def blasst_decode_group_splits(B, Hq, Hkv, Lkv, Bc=64) -> int:
+    return int(_lib.blasst_decode_group_splits(B, Hq, Hkv, Lkv, Bc))
+
+
 def blasst_decode(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
                   num_splits=0, o=None, lse=None, want_lse=True,
                   workspace=None, stats: Stats | None = None,
@@ -435,7 +448,7 @@ def blasst_decode(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
         scale = 1.0 / math.sqrt(d)
     jlo = (Lkv - window) // Bc if 0 < window < Lkv else 0
     S = (num_splits if num_splits > 0
-         else blasst_decode_splits(B, Hkv, Lkv - jlo * Bc, Bc))
+         else blasst_decode_group_splits(B, Hq, Hkv, Lkv - jlo * Bc, Bc))
     ws_bytes = 0
     if not stats_only:
         if o is None:
@@ -470,7 +483,8 @@ def blasst_decode_wide(q, k, v, *, scale=None, ln_lambda=-math.inf, Bc=64,
     _, Hkv, Lkv, _ = k.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    S = num_splits if num_splits > 0 else blasst_decode_splits(B, Hkv, Lkv, Bc)
+    S = (num_splits if num_splits > 0
+         else blasst_decode_wide_splits(B, Hkv, Lkv, Bc))
     ws_bytes = 0
     if not stats_only:
         if o is None:

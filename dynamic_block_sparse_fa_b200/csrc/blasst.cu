@@ -154,6 +154,39 @@ int blasst_decode_splits(int B, int Hkv, int Lkv, int Bc) {
   return (int)best;
 }
 
+int blasst_decode_wide_splits(int B, int Hkv, int Lkv, int Bc) {
+  if (B < 1 || Hkv < 1 || Lkv < 1 || Bc < 1) return 1;
+  const long long nk = (Lkv + (long long)Bc - 1) / Bc;
+  const long long units = (long long)B * Hkv;
+  // The tensor-core kernel of wide groups keeps 2 CTAs per SM.  Modelled
+  // time of S splits: the waves of (sequence, KV head, split) items times
+  // one item's time, nk / S blocks plus the fixed cost of an item (its q,
+  // its partial write and merge row: about two blocks).  The S with at least
+  // 8 blocks per split that minimises it, fewer splits on ties.
+  const long long slots = (long long)kNumSmB200 * 2;
+  const long long s_max = nk / 8 > 1 ? nk / 8 : 1;
+  long long best = 1;
+  double best_t = 0.0;
+  for (long long s = 1; s <= s_max; ++s) {
+    const double waves = std::ceil((double)(units * s) / (double)slots);
+    const double t = waves * ((double)nk / (double)s + 2.0);
+    if (s == 1 || t < best_t - 1e-9) {
+      best_t = t;
+      best = s;
+    }
+  }
+  return (int)best;
+}
+
+int blasst_decode_group_splits(int B, int Hq, int Hkv, int Lkv, int Bc) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lkv < 1 || Bc < 1 || Hq % Hkv != 0)
+    return 1;
+  const int G = Hq / Hkv;
+  if (G > 8 && G <= 128 && Bc == blasst::kWideBc)
+    return blasst_decode_wide_splits(B, Hkv, Lkv, Bc);
+  return blasst_decode_splits(B, Hkv, Lkv, Bc);
+}
+
 size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits) {
   if (B < 1 || Hq < 1 || d < 1 || num_splits < 1) return 0;
   const size_t rows = (size_t)B * Hq * num_splits;
@@ -461,9 +494,12 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
   const int nk = (Lkv + Bc - 1) / Bc;
   // blocks that hold the visible keys (all of them without a window)
   const int jlo = (window > 0 && Lkv > window) ? (Lkv - window) / Bc : 0;
-  const int S = num_splits == 0
-                    ? blasst_decode_splits(B, Hkv, Lkv - jlo * Bc, Bc)
-                    : num_splits;
+  // the automatic count: the group's own policy for the sequential rule
+  // (its kernel follows from G), the GQA one for the CUDA-core kernel
+  const int S = num_splits != 0 ? num_splits
+                : batch == 0 ? blasst_decode_group_splits(B, Hq, Hkv,
+                                                          Lkv - jlo * Bc, Bc)
+                             : blasst_decode_splits(B, Hkv, Lkv - jlo * Bc, Bc);
   if (S < 1 || S > nk - jlo) return BLASST_ERR_INVALID_ARG;
   // Wide groups (16 to 128 heads per KV head): the tiles of 8 run on the
   // tensor core, one CTA per (sequence, KV head, split) for all of them;
@@ -756,7 +792,7 @@ blasst_status_t blasst_decode_noalloc(const void* q, const void* k_cache,
                                       void* stream) {
   if (B < 1 || Hq < 1 || Hkv < 1 || Lkv < 1 || Bc < 1 || num_splits < 0)
     return BLASST_ERR_INVALID_ARG;
-  const int S = num_splits == 0 ? blasst_decode_splits(B, Hkv, Lkv, Bc)
+  const int S = num_splits == 0 ? blasst_decode_group_splits(B, Hq, Hkv, Lkv, Bc)
                                 : num_splits;
   const size_t need = blasst_decode_workspace_size(B, Hq, d, S);
   if (o && need > kNoAllocScratchBytes) {
@@ -858,7 +894,7 @@ blasst_status_t blasst_decode_wide(const void* q, const void* k_cache,
       (o && !aligned16(o)))
     return BLASST_ERR_MISALIGNED;
   const int nk = (Lkv + Bc - 1) / Bc;
-  const int S = num_splits == 0 ? blasst_decode_splits(B, Hkv, Lkv, Bc)
+  const int S = num_splits == 0 ? blasst_decode_wide_splits(B, Hkv, Lkv, Bc)
                                 : num_splits;
   if (S < 1 || S > nk) return BLASST_ERR_INVALID_ARG;
   return wide_launch(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Lkv, scale, 0,

@@ -218,7 +218,8 @@ blasst_status_t blasst_prefill_backward(
  *  lse         device float32 [B,Hq] or NULL
  *  d           128, or 64 with Hq/Hkv <= 8;  Hq/Hkv a power of two up to
  *              256;  Bc = 64
- *  num_splits  >= 1, or 0 for the automatic choice blasst_decode_splits()
+ *  num_splits  >= 1, or 0 for the automatic choice
+ *              blasst_decode_group_splits(B, Hq, Hkv, Lkv, 64)
  *  workspace   device buffer of at least blasst_decode_workspace_size()
  *              bytes (16-byte aligned) holding the per-split partials;
  *              caller-owned, contents need not be initialised.  May be NULL
@@ -245,8 +246,8 @@ blasst_status_t blasst_decode(const void *q, const void *k_cache,
  * read nor counted, and their mask bytes are written 0 (not visited).
  *
  *  window       >= 0; 0 (or >= Lkv) is blasst_decode exactly
- *  num_splits   1 .. nk - jlo, or 0 = blasst_decode_splits(B, Hkv,
- *               Lkv - 64 jlo, 64)
+ *  num_splits   1 .. nk - jlo, or 0 = blasst_decode_group_splits(B, Hq,
+ *               Hkv, Lkv - 64 jlo, 64)
  *  other arguments, layouts, ownership and errors as blasst_decode.
  */
 blasst_status_t blasst_decode_window(const void *q, const void *k_cache,
@@ -291,7 +292,8 @@ blasst_status_t blasst_decode_batched(const void *q, const void *k_cache,
  * device-wide synchronisation.  (No counterpart in the BLASST papers: this
  * is a deployment convenience of this library.)
  *
- * Same arguments and results as blasst_decode minus the workspace.  The
+ * Same arguments and results as blasst_decode minus the workspace (the
+ * automatic split count is blasst_decode's).  The
  * split partials go to an 8 MiB array that the library holds in device
  * memory on every GPU that loads it, until the process exits.
  *  - The first call on a device looks up that array's device address for
@@ -395,13 +397,32 @@ blasst_status_t blasst_decode_paged(const void *q, const void *k_pages,
  * region rounded up to 256.  num_splits must be the resolved value (>= 1). */
 size_t blasst_decode_workspace_size(int B, int Hq, int d, int num_splits);
 
-/* The automatic split count used when num_splits == 0.  Pure function of
- * its arguments (so a reference can reproduce the masks): at least two waves
- * of (sequence, KV head, split) work items on a 148-SM B200 with 3 resident
- * CTAs per SM, at least 8 blocks per split, and among the counts up to twice
- * that minimum the one that fills the last wave best (fewest splits on
- * ties).  Batch 32 x 8 KV heads at 32K keys gives 5; batch 148 gives 1. */
+/* The automatic split count of the kernels that keep 3 CTAs per SM: every
+ * blasst_decode_paged and blasst_decode_batched call, and blasst_decode
+ * (window, no-alloc) for Hq/Hkv <= 8 or 256.  Pure function of its arguments
+ * (so a reference can reproduce the masks, which depend on the splits): at
+ * least two waves of (sequence, KV head, split) work items on a 148-SM B200
+ * with 3 resident CTAs per SM, at least 8 blocks per split, and among the
+ * counts up to twice that minimum the one that fills the last wave best
+ * (fewest splits on ties).  Batch 32 x 8 KV heads at 32K keys gives 5;
+ * batch 148 gives 1. */
 int blasst_decode_splits(int B, int Hkv, int Lkv, int Bc);
+
+/* The automatic split count of the tensor-core kernel for wide head groups
+ * (2 CTAs per SM): blasst_decode_wide, and blasst_decode (window, no-alloc)
+ * for 16 <= Hq/Hkv <= 128.  Pure function of its arguments: among the counts
+ * with at least 8 blocks per split, the one that minimises
+ * ceil(B*Hkv*S / 296) * (nk/S + 2) -- the waves of work items times one
+ * item's blocks plus its fixed cost of about two blocks (q, partial write,
+ * merge row) -- fewest splits on ties.  Batch 32 x 1 KV head at 32K keys
+ * gives 9 (one wave). */
+int blasst_decode_wide_splits(int B, int Hkv, int Lkv, int Bc);
+
+/* The automatic split count of blasst_decode, blasst_decode_window and
+ * blasst_decode_noalloc for Hq/Hkv query heads per KV head:
+ * blasst_decode_wide_splits for 16 <= Hq/Hkv <= 128 with Bc = 64, else
+ * blasst_decode_splits.  Returns 1 for invalid arguments. */
+int blasst_decode_group_splits(int B, int Hq, int Hkv, int Lkv, int Bc);
 
 /*
  * blasst_decode_wide -- blasst_decode on the tensor core for wide head
@@ -413,7 +434,8 @@ int blasst_decode_splits(int B, int Hkv, int Lkv, int Bc);
  * with G > 8 (tiles of 8 heads), the whole group votes together; the mask
  * layout is [B, Hkv, ceil(Lkv/64)].
  *
- *  d = 128, Bc = 64, 1 <= Hq/Hkv <= 128 (else UNSUPPORTED_SHAPE); other
+ *  d = 128, Bc = 64, 1 <= Hq/Hkv <= 128 (else UNSUPPORTED_SHAPE);
+ *  num_splits 0 = blasst_decode_wide_splits(B, Hkv, Lkv, 64); other
  *  arguments, workspace (blasst_decode_workspace_size), ownership and
  *  errors as blasst_decode.
  */

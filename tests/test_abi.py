@@ -239,6 +239,41 @@ def test_split_policy_and_workspace(lib):
     assert m.blasst_decode_workspace_size(1, 1, 128, 1) == 512 + 256 + 256
 
 
+def _wide_policy(B, Hkv, L, Bc=64):
+    """The wide-group split policy as include/blasst.h states it: among
+    the counts with at least 8 blocks per split, the one minimising
+    ceil(B*Hkv*S / 296) * (nk/S + 2), fewest splits on ties."""
+    nk = -(-L // Bc)
+    best, best_t = 1, None
+    for s in range(1, max(1, nk // 8) + 1):
+        t = math.ceil(B * Hkv * s / 296) * (nk / s + 2.0)
+        if best_t is None or t < best_t - 1e-9:
+            best, best_t = s, t
+    return best
+
+
+def test_wide_and_group_split_policies(lib):
+    import dynamic_block_sparse_fa_b200 as m
+    # MQA batch 32 at 32K: one wave of 288 of the 296 slots
+    assert m.blasst_decode_wide_splits(32, 1, 32768, 64) == 9
+    assert m.blasst_decode_wide_splits(148, 1, 32768, 64) == 2
+    for B in (1, 3, 16, 32, 100, 148, 512):
+        for Hkv in (1, 2, 8):
+            for L in (64, 500, 4096, 32768, 131072):
+                assert (m.blasst_decode_wide_splits(B, Hkv, L, 64)
+                        == _wide_policy(B, Hkv, L)), (B, Hkv, L)
+    # blasst_decode's choice follows the kernel the group runs on
+    for B, Hq, Hkv, L in [(32, 32, 8, 32768), (4, 8, 8, 1000),
+                          (2, 256, 1, 4096), (32, 32, 1, 32768),
+                          (8, 128, 1, 8192), (8, 64, 4, 5000)]:
+        G = Hq // Hkv
+        want = (m.blasst_decode_wide_splits(B, Hkv, L, 64) if 8 < G <= 128
+                else m.blasst_decode_splits(B, Hkv, L, 64))
+        assert m.blasst_decode_group_splits(B, Hq, Hkv, L, 64) == want
+    assert m.blasst_decode_group_splits(1, 3, 2, 100, 64) == 1  # Hq % Hkv
+    assert m.blasst_decode_group_splits(0, 8, 8, 100, 64) == 1
+
+
 def test_mla_split_policy(lib):
     """One CTA pair per (sequence, split), one CTA per SM: the count with the
     fewest SM waves per split, at most two waves, 8 blocks per split or

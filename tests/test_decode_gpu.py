@@ -32,7 +32,7 @@ def _run_and_compare(m, x, ln_lambda, S_req, Bc=64):
     B, Hq, d = q.shape
     Hkv, Lkv = k.shape[1], k.shape[2]
     nk = -(-Lkv // Bc)
-    S = S_req if S_req > 0 else m.blasst_decode_splits(B, Hkv, Lkv, Bc)
+    S = S_req if S_req > 0 else m.blasst_decode_group_splits(B, Hq, Hkv, Lkv, Bc)
     stats = m.Stats(mask_numel=B * Hkv * nk)
     scale = 1.0 / math.sqrt(d)
     o, lse = m.blasst_decode(q, k, v, scale=scale, ln_lambda=ln_lambda, Bc=Bc,

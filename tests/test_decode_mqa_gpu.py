@@ -44,7 +44,12 @@ def _compare(m, x, ln_lambda, S_req, window=0, batch=1, bs=None):
     T = _tiles(Hq, Hkv)
     nk = -(-Lkv // Bc)
     jlo = (Lkv - window) // Bc if 0 < window < Lkv else 0
-    S = S_req if S_req > 0 else m.blasst_decode_splits(B, Hkv, Lkv - jlo * Bc)
+    if S_req > 0:
+        S = S_req
+    elif batch == 2:  # the batched rule keeps the GQA policy
+        S = m.blasst_decode_splits(B, Hkv, Lkv - jlo * Bc)
+    else:
+        S = m.blasst_decode_group_splits(B, Hq, Hkv, Lkv - jlo * Bc)
     scale = 1.0 / math.sqrt(d)
     stats = m.Stats(mask_numel=B * Hkv * T * nk)
 

@@ -32,7 +32,7 @@ def _compare(m, q, k, v, lnl, S_req, bs=None):
     B, Hq, d = q.shape
     Hkv, L = k.shape[1], k.shape[2]
     nk = -(-L // BC)
-    S = S_req if S_req > 0 else m.blasst_decode_splits(B, Hkv, L)
+    S = S_req if S_req > 0 else m.blasst_decode_wide_splits(B, Hkv, L)
     scale = 1.0 / math.sqrt(d)
     st = m.Stats(mask_numel=B * Hkv * nk)
     o, lse = m.blasst_decode_wide(q, k, v, scale=scale, ln_lambda=lnl,

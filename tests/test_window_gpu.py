@@ -141,7 +141,8 @@ def _decode_compare(m, x, W, ln_lambda, S_req):
     Bc = 64
     nk = -(-Lkv // Bc)
     jlo = (Lkv - W) // Bc if 0 < W < Lkv else 0
-    S = S_req if S_req > 0 else m.blasst_decode_splits(B, Hkv, Lkv - jlo * Bc)
+    S = (S_req if S_req > 0
+         else m.blasst_decode_group_splits(B, Hq, Hkv, Lkv - jlo * Bc))
     stats = m.Stats(mask_numel=B * Hkv * nk)
     stats.mask.fill_(7)  # blocks left of the window must be written 0
     scale = 1.0 / math.sqrt(d)

@@ -54,7 +54,7 @@ def _run_case(m, b, i):
     x = planted_gap(B, Hq, Hkv, 1, Lkv, 128, decode=True, block=64,
                     gap=8.0, heavy_frac=0.03,
                     seed=config_seed(1, 7000 + i), device="cuda")
-    S_res = S if S else m.blasst_decode_splits(B, Hkv, Lkv, 64)
+    S_res = S if S else m.blasst_decode_group_splits(B, Hq, Hkv, Lkv, 64)
     o_ref, lse_ref = m.blasst_decode(x.q, x.k, x.v, ln_lambda=lnl,
                                      num_splits=S)
     o = torch.full_like(o_ref, float("nan"))
