@@ -410,3 +410,50 @@ def test_paged_varlen_work_order_cuda_core_kernel(blasst):
                                          ln_lambda=lnl, num_splits=S)
         torch.cuda.synchronize()
         assert torch.equal(ob, o[b:b + 1]) and torch.equal(lb, lse[b:b + 1]), b
+
+
+def test_paged_work_order_many_sequences(blasst):
+    """600 sequences of 64..4096 keys (ties included), 4 query heads on one
+    KV head, one split: 600 work items, so the work order is computed by
+    three blocks of the ordering kernel (ranks counted across 256-length
+    tiles).  No output row is left unwritten (o and lse start as NaN, so a
+    sequence missing from the permutation would show), and sampled
+    sequences equal a contiguous decode of each alone bit for bit."""
+    m = blasst
+    B, Hq, Hkv, d, S, lnl = 600, 4, 1, 128, 1, -4.0
+    g = torch.Generator().manual_seed(config_seed(6, 11))
+    lens = torch.randint(64, 4096 + 1, (B,), generator=g).tolist()
+    for i in range(0, B, 50):  # runs of equal lengths
+        lens[i + 1] = lens[i]
+    Lmax = max(lens)
+    q = torch.empty(B, Hq, d, dtype=torch.bfloat16, device="cuda")
+    k = torch.empty(B, Hkv, Lmax, d, dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    planted_gap_kv_inplace(k, v, q, block=64, gap=8.0, heavy_frac=0.03,
+                           seed=config_seed(6, 12))
+    pk = paginate(k, v, lens, 16, seed=16, spare_pages=8, poison=POISON)
+    del k, v
+    o = torch.full((B, Hq, d), float("nan"), dtype=torch.bfloat16,
+                   device="cuda")
+    lse = torch.full((B, Hq), float("nan"), dtype=torch.float32,
+                     device="cuda")
+    m.blasst_decode_paged(q, pk.k_pages, pk.v_pages, pk.block_table,
+                          pk.seq_lens, max_seq_len=Lmax, ln_lambda=lnl,
+                          num_splits=S, o=o, lse=lse)
+    torch.cuda.synchronize()
+    assert m.blasst_check_device_error()[0] == 0
+    assert not torch.isnan(o.float()).any() and not torch.isnan(lse).any()
+    order = sorted(range(B), key=lambda i: (-lens[i], i))
+    picks = sorted({order[0], order[1], order[255], order[256], order[511],
+                    order[512], order[-1], 0})
+    for b in picks:
+        L = lens[b]
+        npg = -(-L // 16)
+        ids = pk.block_table[b, :npg].long()
+        kb = pk.k_pages[ids].transpose(0, 1).reshape(Hkv, npg * 16, d)[:, :L]
+        vb = pk.v_pages[ids].transpose(0, 1).reshape(Hkv, npg * 16, d)[:, :L]
+        ob, lb = m.blasst_decode(q[b:b + 1], kb[None].contiguous(),
+                                 vb[None].contiguous(), ln_lambda=lnl,
+                                 num_splits=S)
+        torch.cuda.synchronize()
+        assert torch.equal(ob, o[b:b + 1]) and torch.equal(lb, lse[b:b + 1]), b
