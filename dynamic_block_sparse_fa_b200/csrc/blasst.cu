@@ -279,7 +279,7 @@ blasst_status_t launch_decode_mma(const blasst::DecodeMmaArgs& a, int G,
 
 blasst_status_t launch_decode(const blasst::DecodeArgs& a, int G, bool paged,
                               long long grid, bool stats_only, void* o,
-                              float* lse, int rows, int S, cudaStream_t st,
+                              float* lse, int rows, cudaStream_t st,
                               int batch = 1) {
   cudaError_t e = cudaErrorInvalidValue;
   switch (G) {
@@ -570,7 +570,7 @@ blasst_status_t decode_contiguous(const void* q, const void* k_cache,
   a.stats_only = stats_only ? 1 : 0;
   a.window = window;
 
-  return launch_decode(a, G, false, grid, stats_only, o, lse, B * Hq, S,
+  return launch_decode(a, G, false, grid, stats_only, o, lse, B * Hq,
                        static_cast<cudaStream_t>(stream), batch);
 }
 }  // namespace
@@ -707,7 +707,7 @@ blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
   a.max_pages = max_pages;
   a.num_pages = num_pages;
   a.per_length = per_length ? 1 : 0;
-  return launch_decode(a, G, true, grid, stats_only, o, lse, B * Hq, S,
+  return launch_decode(a, G, true, grid, stats_only, o, lse, B * Hq,
                        static_cast<cudaStream_t>(stream));
 }
 
