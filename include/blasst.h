@@ -203,10 +203,11 @@ blasst_status_t blasst_prefill_backward(
  * every K and V byte read serves all G heads.  A tile has at most 8 rows:
  * for G = 16, 32, ... (MQA with many heads) the heads of a KV head are cut
  * into G/8 consecutive tiles of 8 heads, each with its own skip decisions.
- * For 16 <= G <= 128 one tensor-core CTA scores all tiles of a KV head
- * (the V block is read when any tile keeps it; the rows of a tile that
- * skips it are left untouched); for G <= 8 and G = 256 the CUDA-core
- * kernel runs one CTA per tile.  The Lkv keys are cut into
+ * For 16 <= G <= 128 one tensor-core CTA (tcgen05) scores all tiles of a
+ * KV head (the V block is read when any tile keeps it; the rows of a tile
+ * that skips it are left untouched); for G <= 8 a warp-level tensor-core
+ * kernel (mma.sync, K and V by TMA) runs one CTA per (sequence, KV head,
+ * split); for G = 256 the CUDA-core kernel runs one CTA per tile.  The Lkv keys are cut into
  * nk = ceil(Lkv/Bc) blocks and the blocks into num_splits contiguous splits
  * (split s covers blocks [floor(s*nk/S), floor((s+1)*nk/S))).  Each split
  * runs the blockwise forward independently (its running max starts at
