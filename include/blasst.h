@@ -208,8 +208,9 @@ blasst_status_t blasst_prefill_backward(
  * that skips it are left untouched); for G <= 8 a warp-level tensor-core
  * kernel (mma.sync, K and V by TMA) runs one CTA per (sequence, KV head,
  * split); for G = 256 the CUDA-core kernel runs one CTA per tile.  The
- * Lkv keys are cut into nk = ceil(Lkv/Bc) blocks and the blocks into num_splits contiguous splits
- * (split s covers blocks [floor(s*nk/S), floor((s+1)*nk/S))).  Each split
+ * Lkv keys are cut into nk = ceil(Lkv/Bc) blocks and the blocks into
+ * num_splits contiguous splits (split s covers blocks
+ * [floor(s*nk/S), floor((s+1)*nk/S))).  Each split
  * runs the blockwise forward independently (its running max starts at
  * -inf), reading V only for kept blocks; a second kernel merges the splits:
  * lse = ln sum_s exp(lse_s), o = sum_s exp(lse_s - lse) o_s.
