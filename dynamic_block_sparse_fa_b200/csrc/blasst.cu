@@ -608,7 +608,8 @@ blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
   if ((long long)max_seq_len > (long long)max_pages * page_size)
     return BLASST_ERR_INVALID_ARG;
   int G = Hq / Hkv;
-  if (d != blasst::kDecD || !decode_group_ok(G))
+  // d 128, or 64 on the warp-MMA kernel (up to 8 heads per KV head)
+  if (!(d == blasst::kDecD || (d == 64 && G <= 8)) || !decode_group_ok(G))
     return BLASST_ERR_UNSUPPORTED_SHAPE;
   const int kv_div = G > 8 ? G / 8 : 1;  // tiles of 8 heads above 8
   if (page_stride < (long long)Hkv * page_size * d || page_stride % 8 != 0)

@@ -360,7 +360,8 @@ blasst_status_t blasst_decode_noalloc(const void *q, const void *k_cache,
  *                  (finite or -INFINITY), and sequence b uses
  *                  ln lambda_b = min(0, ln a - ln L_b), L_b its own length
  *                  (gist.science summary, section 2 "Calibracao Automatica")
- *  d = 128, Hq/Hkv a power of two up to 256 (tiles as blasst_decode)
+ *  d = 128, or 64 with Hq/Hkv <= 8; Hq/Hkv a power of two up to 256
+ *                  (tiles as blasst_decode)
  *  num_splits      >= 1 (at most ceil(max_seq_len / 64)), or 0 = automatic
  *  workspace       as blasst_decode: blasst_decode_workspace_size(B, Hq, d,
  *                  resolved num_splits) bytes

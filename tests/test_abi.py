@@ -369,6 +369,8 @@ def test_paged_decode_validation(lib):
     assert _paged(lib, lnl=-math.inf, per_length=1) == 7
     assert _paged(lib, S=5) == 1                       # more splits than blocks
     assert _paged(lib, Hq=24, Hkv=2) == 2              # G = 12 not built
-    assert _paged(lib, d=64) == 2
+    assert _paged(lib, d=64) == 7                      # d 64 with G <= 8 ...
+    assert _paged(lib, d=64, Hq=32, Hkv=2) == 2        # ... not with G = 16
+    assert _paged(lib, d=96) == 2
     assert _paged(lib, kp=0x1008) == 3                 # misaligned pool
     assert _paged(lib, P=0) == 1

@@ -118,6 +118,54 @@ def test_paged_decode_matches_oracle(blasst, case):
         assert (mask == 2).sum() == 0
 
 
+PAGED_D64_CASES = [
+    # head dimension 64 (the warp-MMA kernel, up to 8 heads per KV head)
+    (8, 2, [1000, 64, 65, 3000], 16, -3.0, 0, False, "separate"),
+    (4, 4, [2048, 129], 64, -2.0, 3, False, "interleaved"),
+    (8, 1, [700, 5000], 32, math.log(40.0), 2, True, "separate"),
+]
+
+
+@pytest.mark.parametrize("case", PAGED_D64_CASES)
+def test_paged_decode_d64_matches_oracle(blasst, case):
+    Hq, Hkv, lens, ps, ln_lambda, S, per_length, layout = case
+    B = len(lens)
+    Lmax = max(lens)
+    x = planted_gap(B, Hq, Hkv, 1, Lmax, 64, decode=True, block=64, gap=8.0,
+                    heavy_frac=0.03, seed=config_seed(1, 3 * Lmax + Hq + ps),
+                    device="cuda")
+    pk = paginate(x.k, x.v, lens, ps, seed=Lmax + ps + 1, spare_pages=5,
+                  poison=POISON)
+    kp, vp = _pool(pk, layout)
+    _check_paged(blasst, x.q, kp, vp, pk, lens, ln_lambda, S, per_length)
+
+
+def test_paged_d64_equals_contiguous_bitwise(blasst):
+    """Head dimension 64, same tokens, same splits: the paged and the
+    contiguous warp-MMA kernels give the same bits; 16 query heads per KV
+    head at d 64 (the CUDA-core kernel, d 128 only) is refused."""
+    m = blasst
+    B, Hq, Hkv, L = 3, 16, 4, 2000
+    x = planted_gap(B, Hq, Hkv, 1, L, 64, decode=True, block=64, gap=8.0,
+                    heavy_frac=0.03, seed=config_seed(1, 98), device="cuda")
+    pk = paginate(x.k, x.v, [L] * B, 16, seed=4, spare_pages=2,
+                  poison=POISON)
+    for lnl in (-math.inf, -3.0):
+        o1, l1 = m.blasst_decode(x.q, x.k, x.v, ln_lambda=lnl, num_splits=3)
+        o2, l2 = m.blasst_decode_paged(x.q, pk.k_pages, pk.v_pages,
+                                       pk.block_table, pk.seq_lens,
+                                       max_seq_len=L, ln_lambda=lnl,
+                                       num_splits=3)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    q16 = torch.zeros(1, 16, 64, dtype=torch.bfloat16, device="cuda")
+    kp = torch.zeros(4, 1, 64, 64, dtype=torch.bfloat16, device="cuda")
+    bt = torch.zeros(1, 4, dtype=torch.int32, device="cuda")
+    sl = torch.tensor([100], dtype=torch.int32, device="cuda")
+    with pytest.raises(m.BlasstError, match="UNSUPPORTED"):
+        m.blasst_decode_paged(q16, kp, kp, bt, sl)
+
+
 @pytest.mark.parametrize("ps", [16, 64])
 def test_paged_nan_rows_past_the_sequence_never_reach_the_output(blasst, ps):
     """Pool rows no sequence owns hold NaN: the kernel may bring the rest of
