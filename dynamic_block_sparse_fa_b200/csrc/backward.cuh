@@ -19,8 +19,9 @@
 //                       V_j stay in shared memory while the kept query tiles
 //                       of the G query heads stream through; dK_j, dV_j
 //                       accumulate in tensor memory, each pair's dQ tile is
-//                       staged in shared memory and added to the f32
-//                       accumulator by TMA bulk reductions
+//                       staged in shared memory (four 32-column boxes through
+//                       two 16 KB halves) and added to the f32 accumulator
+//                       by TMA bulk reductions
 //   bwd_dq_kernel       dQ = bf16(scale * accumulator)
 // bwd_dkdv_kernel: warp 0 TMA producer (Q_i, dO_i ring of 2), warp 1 MMA
 // issuer (one lane), warps 2..5 one thread per tensor-memory lane.  Per kept
@@ -105,6 +106,10 @@ __device__ __forceinline__ void bulk_commit_group() {
 // the shared-memory sources of every committed bulk group have been read
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// all but the most recently committed bulk group have been read
+__device__ __forceinline__ void bulk_wait_read_but_one() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -399,6 +404,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool w2 =
             ok && mbar_wait(&bar[C::B_DPF], n & 1, kWaitBackward, n, 31);
         ok = __all_sync(FULL, w2);
+        // the buffer holds the previous pair's last dQ staging until the
+        // reduction has read it (its wait is taken here, after P)
+        if (n > 0) {
+          if (warp == 2 && lane == 0) bulk_wait_read_all();
+          named_sync(1, 128);
+        }
         tc_fence_after();
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
@@ -442,20 +453,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (ok) {
           tc_fence_after();
 #pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              uint32_t a[32];
-              tmem_ld32(lane_base + 128 + h * 64 + u * 32, a);
-              tc_wait_ld();
-              uint8_t* row = sDS + u * (C::TILE / 2) + rr * 128;
-#pragma unroll
-              for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4*>(row + ((c ^ (rr & 7)) * 16)) =
-                    make_uint4(a[4 * c], a[4 * c + 1], a[4 * c + 2],
-                               a[4 * c + 3]);
+          for (int h = 0; h < 4; ++h) {
+            // four 32-column boxes through the buffer's two 16 KB halves:
+            // a half is written again once the reduction of the box two
+            // rounds back has read it
+            const int half = h & 1;
+            if (h >= 2) {
+              if (warp == 2 && lane == 0) bulk_wait_read_but_one();
+              named_sync(1, 128);
             }
-            if (h == 1) {  // TMEM [128, 256) is free for the next dP^T
+            uint32_t a[32];
+            tmem_ld32(lane_base + 128 + h * 32, a);
+            tc_wait_ld();
+            uint8_t* row = sDS + half * (C::TILE / 2) + rr * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(row + ((c ^ (rr & 7)) * 16)) =
+                  make_uint4(a[4 * c], a[4 * c + 1], a[4 * c + 2],
+                             a[4 * c + 3]);
+            if (h == 3) {  // TMEM [128, 256) is free for the next dP^T
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&bar[C::B_DQR]);
@@ -463,14 +479,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             fence_async_smem();
             named_sync(1, 128);
             if (warp == 2 && lane == 0) {
-#pragma unroll
-              for (int u = 0; u < 2; ++u)
-                tma_reduce_add_3d(&p.tdq, sDS + u * (C::TILE / 2),
-                                  h * 64 + u * 32, i * 128, b * p.Hq + hq);
+              tma_reduce_add_3d(&p.tdq, sDS + half * (C::TILE / 2), h * 32,
+                                i * 128, b * p.Hq + hq);
               bulk_commit_group();
-              bulk_wait_read_all();
             }
-            named_sync(1, 128);
           }
         }
         ++n;
