@@ -370,12 +370,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool w1 = mbar_wait(&bar[C::B_SF], n & 1, kWaitBackward, n, 30);
         ok = __all_sync(FULL, w1);
         tc_fence_after();
+        // rows that see every query column of the tile need no mask; a warp
+        // whose 32 rows all do takes the unmasked loop
+        const bool row_full = key_ok && i * 128 + 127 < p.Lq &&
+                              (!p.causal || key <= i * 128 + off);
+        const bool warp_full = __all_sync(FULL, row_full);
+        const float4* lse4 = reinterpret_cast<const float4*>(lse_s);
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           if (!ok) break;
           uint32_t sv[32];
           tmem_ld32(lane_base + 0 + cc * 32, sv);
           tc_wait_ld();
+          if (warp_full) {
+#pragma unroll
+            for (int x = 0; x < 32; x += 4) {
+              const float4 l4 = lse4[(cc * 32 + x) >> 2];
+              const float p0 = ex2_approx(fmaf(__uint_as_float(sv[x]), sl2, -l4.x));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(sv[x + 1]), sl2, -l4.y));
+              const float p2 = ex2_approx(fmaf(__uint_as_float(sv[x + 2]), sl2, -l4.z));
+              const float p3 = ex2_approx(fmaf(__uint_as_float(sv[x + 3]), sl2, -l4.w));
+              pk[cc * 16 + (x >> 1)] = pack_bf16x2(p0, p1);
+              pk[cc * 16 + (x >> 1) + 1] = pack_bf16x2(p2, p3);
+            }
+          } else {
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
             float pv[2];
@@ -390,6 +408,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                             : 0.f;
             }
             pk[cc * 16 + (x >> 1)] = pack_bf16x2(pv[0], pv[1]);
+          }
           }
           uint32_t st16[16];
 #pragma unroll
@@ -419,12 +438,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_wait_ld();
           uint32_t dk16[16];
 #pragma unroll
-          for (int x = 0; x < 32; x += 2) {
-            const uint32_t pw = pk[cc * 16 + (x >> 1)];
-            const int c = cc * 32 + x;
+          for (int x = 0; x < 32; x += 4) {
+            const float4 d4 =
+                reinterpret_cast<const float4*>(del_s)[(cc * 32 + x) >> 2];
+            const uint32_t pw0 = pk[cc * 16 + (x >> 1)];
+            const uint32_t pw1 = pk[cc * 16 + (x >> 1) + 1];
             dk16[x >> 1] = pack_bf16x2(
-                bf16lo(pw) * (__uint_as_float(dp[x]) - del_s[c]),
-                bf16hi(pw) * (__uint_as_float(dp[x + 1]) - del_s[c + 1]));
+                bf16lo(pw0) * (__uint_as_float(dp[x]) - d4.x),
+                bf16hi(pw0) * (__uint_as_float(dp[x + 1]) - d4.y));
+            dk16[(x >> 1) + 1] = pack_bf16x2(
+                bf16lo(pw1) * (__uint_as_float(dp[x + 2]) - d4.z),
+                bf16hi(pw1) * (__uint_as_float(dp[x + 3]) - d4.w));
           }
           tmem_st16(lane_base + 128 + cc * 16, dk16);
           // dS^T row rr, query columns 32cc..32cc+31: box cc/2, 16-byte
