@@ -13,7 +13,8 @@
 // nothing.
 //
 // Three kernels:
-//   bwd_prep_kernel     D per query row (from O and dO), zeroes the f32 dQ
+//   bwd_prep_kernel     D and lse * log2 e per query row (rows padded to 16
+//                       bytes, for the producer's TMA), zeroes the f32 dQ
 //                       accumulator
 //   bwd_dkdv_kernel     one CTA per (sequence, KV head, key block j): K_j and
 //                       V_j stay in shared memory while the kept query tiles
@@ -52,7 +53,10 @@ struct BwdParams {
   const float* lse;           // [B, Hq, Lq] natural log
   const unsigned char* mask;  // [B, Hq, nq, nk]; 1 = kept (null: all kept)
   float* dq_acc;              // [B, Hq, Lq, D]
-  float* delta;               // [B, Hq, Lq]
+  float* delta;               // [B*Hq][Lqp]: D per query row
+  float* lse2;                // [B*Hq][Lqp]: lse * log2 e per query row
+  CUtensorMap tdel, tlse2;    // those two, 128-column boxes
+  int Lqp;                    // Lq rounded up to 4 (16-byte row stride)
   __nv_bfloat16* dq;          // [B, Hq, Lq, D]
   __nv_bfloat16* dk;          // [B, Hkv, Lkv, D]
   __nv_bfloat16* dv;          // [B, Hkv, Lkv, D]
@@ -83,7 +87,8 @@ struct BwdCfg {
   static constexpr int B_DSR = 8;   // dS^T written (one arrival per warp)
   static constexpr int B_DQF = 9;   // dQ tile in TMEM
   static constexpr int B_DQR = 10;  // dQ tile read out (one arrival per warp)
-  static constexpr int NBAR = 11;
+  static constexpr int B_LF = 11;   // the pair's lse and D in shared memory
+  static constexpr int NBAR = 12;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_TMEM + 8;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
@@ -128,7 +133,16 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
             bf16lo(a.y) * bf16lo(g.y) + bf16hi(a.y) * bf16hi(g.y);
 #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
-  if (lane == 0) p.delta[row] = s;
+  if (lane == 0) {
+    const long long r = row / p.Lq, q = row - r * p.Lq;
+    p.delta[r * p.Lqp + q] = s;
+    p.lse2[r * p.Lqp + q] = p.lse[row] * kPrefLog2e;
+    if (q == p.Lq - 1)  // the row's padding columns: finite, never used
+      for (int c = p.Lq; c < p.Lqp; ++c) {
+        p.delta[r * p.Lqp + c] = 0.f;
+        p.lse2[r * p.Lqp + c] = 0.f;
+      }
+  }
   reinterpret_cast<float4*>(p.dq_acc + row * kBwdD)[lane] =
       make_float4(0.f, 0.f, 0.f, 0.f);
 }
@@ -190,6 +204,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&bar[C::B_DSR], 4);
     mbar_init(&bar[C::B_DQF], 1);
     mbar_init(&bar[C::B_DQR], 4);
+    mbar_init(&bar[C::B_LF], 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -240,6 +255,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tma_load_3d(smem + C::OFF_DO + s * C::TILE + c * C::BOX, &p.tdo,
                         &bar[C::B_QF + s], c * 64, i * 128, zq, pol_q);
           }
+          // this pair's lse and D, once the previous pair's dS phase (the
+          // last reader of the one shared slot) is over
+          if (n >= 1 && !mbar_wait(&bar[C::B_DSR], (n - 1) & 1,
+                                   kWaitBackward, n, 40)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar[C::B_LF], 2 * 512);
+          tma_load_3d(smem + C::OFF_LSE, &p.tlse2, &bar[C::B_LF], i * 128, zq,
+                      0, pol_q);
+          tma_load_3d(smem + C::OFF_DEL, &p.tdel, &bar[C::B_LF], i * 128, zq,
+                      0, pol_q);
           ++n;
         }
       }
@@ -350,20 +377,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true, stop = false;
     for (int g = 0; g < p.G && !stop; ++g) {
       const int hq = hkv * p.G + g;
-      const size_t rowbase = (size_t)(b * p.Hq + hq) * p.Lq;
       for (int i = 0; i < p.nq; ++i) {
         if (!kept(g, i)) continue;
         // All four warps leave together: a wait that gave up in any of them
         // ends the loop for all at this barrier (never between barriers).
         if (!named_sync_and(1, 128, ok)) { ok = false; stop = true; break; }
-        // this pair's lse (log2 units) and D per query column
+        // this pair's lse (log2 units) and D per query column, loaded by
+        // the producer
         {
-          const int qr = i * 128 + rr;
-          lse_s[rr] = qr < p.Lq ? __ldg(p.lse + rowbase + qr) * kPrefLog2e
-                                : INFINITY;
-          del_s[rr] = qr < p.Lq ? p.delta[rowbase + qr] : 0.f;
+          const bool wl = mbar_wait(&bar[C::B_LF], n & 1, kWaitBackward, n, 33);
+          ok = __all_sync(FULL, wl);
         }
-        named_sync(1, 128);
         // P^T (thread = key row, 128 query columns) into TMEM [0, 64) as
         // bf16; the packed values stay in registers for dS.
         uint32_t pk[64];
@@ -589,7 +613,26 @@ struct BwdProblem {
 
 inline size_t bwd_workspace_bytes(int B, int Hq, int Lq) {
   const size_t rows = (size_t)B * Hq * Lq;
-  return rows * kBwdD * 4 + ((rows * 4 + 255) & ~(size_t)255);
+  const size_t prow = (size_t)B * Hq * ((Lq + 3) & ~3);
+  // dQ accumulator, then D and lse * log2 e with 16-byte row strides
+  return rows * kBwdD * 4 + 2 * (((prow + 63) & ~(size_t)63) * 4);
+}
+
+// [planes][cols] f32 with a 16-byte row stride, 128-column boxes of one row
+inline bool encode_rows_f32(CUtensorMap* m, void* base, int cols,
+                            long long planes) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)planes, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 4,
+                           (cuuint64_t)planes * cols * 4};
+  cuuint32_t box[3] = {128, 1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 inline cudaError_t launch_backward(const BwdProblem& pr, cudaStream_t st) {
@@ -605,9 +648,14 @@ inline cudaError_t launch_backward(const BwdProblem& pr, cudaStream_t st) {
   p.lse = pr.lse;
   p.mask = pr.mask;
   const size_t rows = (size_t)pr.B * pr.Hq * pr.Lq;
+  p.Lqp = (pr.Lq + 3) & ~3;
+  const size_t prow = (size_t)pr.B * pr.Hq * p.Lqp;
   p.dq_acc = pr.workspace;
   p.delta = pr.workspace + rows * kBwdD;
-  if (!encode_map_f32(&p.tdq, p.dq_acc, pr.Lq, (long long)pr.B * pr.Hq))
+  p.lse2 = p.delta + ((prow + 63) & ~(size_t)63);
+  if (!encode_map_f32(&p.tdq, p.dq_acc, pr.Lq, (long long)pr.B * pr.Hq) ||
+      !encode_rows_f32(&p.tdel, p.delta, p.Lqp, (long long)pr.B * pr.Hq) ||
+      !encode_rows_f32(&p.tlse2, p.lse2, p.Lqp, (long long)pr.B * pr.Hq))
     return cudaErrorInvalidValue;
   p.dq = static_cast<__nv_bfloat16*>(pr.dq);
   p.dk = static_cast<__nv_bfloat16*>(pr.dk);

@@ -181,8 +181,9 @@ blasst_status_t blasst_prefill_window(const void *q, const void *k,
  *  d = 128, Br = Bc = 128 (else BLASST_ERR_UNSUPPORTED_SHAPE); causal with
  *              Lq > Lkv is rejected
  *  workspace   device buffer of blasst_prefill_backward_workspace_size()
- *              bytes, 256-byte aligned, caller-owned (f32 dQ accumulator and
- *              the per-row D); contents need not be initialised
+ *              bytes, 256-byte aligned, caller-owned (f32 dQ accumulator,
+ *              the per-row D and lse * log2 e); contents need not be
+ *              initialised
  * Asynchronous on `stream`; three kernel launches; allocates nothing.
  * Errors as blasst_prefill (BLASST_ERR_WORKSPACE for a missing or small
  * workspace).
