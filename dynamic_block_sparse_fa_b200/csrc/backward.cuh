@@ -35,10 +35,13 @@
 //                          B = Q_i MN-major)           -> [384, 512)
 //   dQ_i = dS K_j         (SS, A = dS MN-major from shared memory,
 //                          B = K_j MN-major)           -> [128, 256)
-// and the threads signal P^T and dS^T separately, so the dV product runs
-// while dS is computed, and the next pair's S^T product runs while the dQ
-// tile is read out (it lands in the dP^T columns, which the next dP^T waits
-// for).  Tensor memory is the whole 512 columns: one CTA per SM.
+// Pairs are pipelined one deep.  The threads take pair n's dS, then pair
+// n+1's P while the tensor core runs dK_n and dQ_n, then read pair n's dQ
+// tile out (it lands in the dP^T columns, which dP^T_{n+1} waits for).  The
+// issuer's order per pair: dK_n, dQ_n | dV_{n+1} | dP^T_{n+1}, S^T_{n+2};
+// S^T_{n+2} comes last because its Q slot is the one dK_n releases.  The
+// producer brings each pair's lse (ring of 2) and D (one slot) by TMA.
+// Tensor memory is the whole 512 columns: one CTA per SM.
 #pragma once
 
 #include "prefill.cuh"
@@ -75,8 +78,8 @@ struct BwdCfg {
   static constexpr int OFF_Q = OFF_V + TILE;     // [2]
   static constexpr int OFF_DO = OFF_Q + 2 * TILE;  // [2]
   static constexpr int OFF_DS = OFF_DO + 2 * TILE;  // dS^T [keys][queries]
-  static constexpr int OFF_LSE = OFF_DS + TILE;     // f32 [128] lse * log2 e
-  static constexpr int OFF_DEL = OFF_LSE + 512;     // f32 [128] D
+  static constexpr int OFF_LSE = OFF_DS + TILE;      // f32 [2][128] lse * log2 e
+  static constexpr int OFF_DEL = OFF_LSE + 2 * 512;  // f32 [128] D
   static constexpr int OFF_BAR = OFF_DEL + 512;
   static constexpr int B_KV = 0;
   static constexpr int B_QF = 1;    // [2]
@@ -87,8 +90,10 @@ struct BwdCfg {
   static constexpr int B_DSR = 8;   // dS^T written (one arrival per warp)
   static constexpr int B_DQF = 9;   // dQ tile in TMEM
   static constexpr int B_DQR = 10;  // dQ tile read out (one arrival per warp)
-  static constexpr int B_LF = 11;   // the pair's lse and D in shared memory
-  static constexpr int NBAR = 12;
+  static constexpr int B_LF = 11;   // [2] a pair's lse in its ring slot
+  static constexpr int B_LE = 13;   // [2] that slot read (one arrival per warp)
+  static constexpr int B_DF = 15;   // the pair's D in shared memory
+  static constexpr int NBAR = 16;
   static constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_TMEM + 8;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
@@ -189,6 +194,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int hq = hkv * p.G + g;
     return __ldg(p.mask + ((size_t)(b * p.Hq + hq) * p.nq + i) * p.nk + jb) == 1;
   };
+  // the next kept pair after (g, i) in (head, tile) order; false at the end
+  auto next_kept = [&](int& g, int& i) -> bool {
+    ++i;
+    while (g < p.G) {
+      if (i >= p.nq) {
+        ++g;
+        i = 0;
+        continue;
+      }
+      if (kept(g, i)) return true;
+      ++i;
+    }
+    return false;
+  };
 
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
@@ -204,7 +223,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&bar[C::B_DSR], 4);
     mbar_init(&bar[C::B_DQF], 1);
     mbar_init(&bar[C::B_DQR], 4);
-    mbar_init(&bar[C::B_LF], 1);
+    for (int r = 0; r < 2; ++r) {
+      mbar_init(&bar[C::B_LF + r], 1);
+      mbar_init(&bar[C::B_LE + r], 4);
+    }
+    mbar_init(&bar[C::B_DF], 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -255,17 +278,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tma_load_3d(smem + C::OFF_DO + s * C::TILE + c * C::BOX, &p.tdo,
                         &bar[C::B_QF + s], c * 64, i * 128, zq, pol_q);
           }
-          // this pair's lse and D, once the previous pair's dS phase (the
-          // last reader of the one shared slot) is over
+          // lse of pair n into slot s once pair n-2's P phase has read it
+          if (n >= 2 &&
+              !mbar_wait(&bar[C::B_LE + s], ((n >> 1) - 1) & 1, kWaitBackward,
+                         n, 41)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar[C::B_LF + s], 512);
+          tma_load_3d(smem + C::OFF_LSE + s * 512, &p.tlse2, &bar[C::B_LF + s],
+                      i * 128, zq, 0, pol_q);
+          // D of pair n once pair n-1's dS phase (its one reader) is over;
+          // that phase needs this D's predecessor, so DSR cannot run ahead
           if (n >= 1 && !mbar_wait(&bar[C::B_DSR], (n - 1) & 1,
                                    kWaitBackward, n, 40)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&bar[C::B_LF], 2 * 512);
-          tma_load_3d(smem + C::OFF_LSE, &p.tlse2, &bar[C::B_LF], i * 128, zq,
-                      0, pol_q);
-          tma_load_3d(smem + C::OFF_DEL, &p.tdel, &bar[C::B_LF], i * 128, zq,
+          mbar_arrive_expect_tx(&bar[C::B_DF], 512);
+          tma_load_3d(smem + C::OFF_DEL, &p.tdel, &bar[C::B_DF], i * 128, zq,
                       0, pol_q);
           ++n;
         }
@@ -294,7 +325,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         return smem_desc(base + k * 2048, C::BOX, 1024, 2);
       };
       bool ok = mbar_wait(&bar[C::B_KV], 0, kWaitBackward, 0, 20);
-      // S^T of pair n is issued at the end of pair n-1's step (or here).
+      // S^T of pair n: K Q_n^T into [0, 128)
       auto issue_s = [&](int n) {
         const int s = n & 1;
         ok = ok && mbar_wait(&bar[C::B_QF + s], (n >> 1) & 1, kWaitBackward,
@@ -307,58 +338,74 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_ss(tmem + 0, kmaj(aK, k), kmaj(q_s, k), id_kk, k > 0 ? 1u : 0u);
         mma_commit(&bar[C::B_SF]);
       };
+      // dP^T of pair n: V dO_n^T into [128, 256) (its dO arrived with Q)
+      auto issue_dp = [&](int n) {
+        const uint32_t do_s = aDO + (n & 1) * C::TILE;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ss(tmem + 128, kmaj(aV, k), kmaj(do_s, k), id_kk,
+                 k > 0 ? 1u : 0u);
+        mma_commit(&bar[C::B_DPF]);
+      };
+      // dV += P^T dO_n once the threads have written P^T of pair n
+      auto issue_dv = [&](int n) {
+        ok = ok && mbar_wait(&bar[C::B_PR], n & 1, kWaitBackward, n, 24);
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t do_s = aDO + (n & 1) * C::TILE;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ts(tmem + 256, tmem + 0 + k * 8, mnmaj(do_s, k), id_km,
+                 (n > 0 || k > 0) ? 1u : 0u);
+      };
+      // Pairs are pipelined one deep: while the threads compute P of pair
+      // n+1, the tensor core runs dK and dQ of pair n.  Per pair n:
+      //   [dS_n written]  dK_n, dQ_n
+      //   [P_{n+1}]       dV_{n+1}
+      //   [dQ_n read]     dP^T_{n+1}, then S^T_{n+2}
+      // S^T_{n+2} comes last: its Q slot is the one dK_n has just released.
+      int g = 0, i = -1;
+      bool have = next_kept(g, i);
       int n = 0;
-      bool pending = false;  // S^T of pair n issued
-      for (int g = 0; g < p.G && ok; ++g) {
-        for (int i = 0; i < p.nq && ok; ++i) {
-          if (!kept(g, i)) continue;
-          const int s = n & 1;
-          if (!pending) issue_s(n);
-          pending = false;
-          // dP^T overwrites the columns the previous dQ tile was read from
-          if (ok && n > 0)
-            ok = mbar_wait(&bar[C::B_DQR], (n - 1) & 1, kWaitBackward, n, 23);
+      if (have && ok) {
+        issue_s(0);
+        if (ok) issue_dp(0);
+        issue_dv(0);
+        int g1 = g, i1 = i;
+        if (next_kept(g1, i1)) issue_s(1);
+      }
+      while (have && ok) {
+        const int s = n & 1;
+        ok = mbar_wait(&bar[C::B_DSR], n & 1, kWaitBackward, n, 25);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t q_s = aQ + s * C::TILE;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ts(tmem + 384, tmem + 128 + k * 8, mnmaj(q_s, k), id_km,
+                 (n > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ss(tmem + 128, mnmaj(aDS, k), mnmaj(aK, k), id_mm,
+                 k > 0 ? 1u : 0u);
+        mma_commit(&bar[C::B_DQF]);
+        mma_commit(&bar[C::B_QE + s]);
+        int g2 = g, i2 = i;
+        const bool h2 = next_kept(g2, i2);
+        if (h2) {
+          issue_dv(n + 1);
+          // dP^T overwrites the columns dQ_n is read from
+          ok = ok && mbar_wait(&bar[C::B_DQR], n & 1, kWaitBackward, n, 23);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t q_s = aQ + s * C::TILE, do_s = aDO + s * C::TILE;
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mma_ss(tmem + 128, kmaj(aV, k), kmaj(do_s, k), id_kk,
-                   k > 0 ? 1u : 0u);
-          mma_commit(&bar[C::B_DPF]);
-          ok = mbar_wait(&bar[C::B_PR], n & 1, kWaitBackward, n, 24);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mma_ts(tmem + 256, tmem + 0 + k * 8, mnmaj(do_s, k), id_km,
-                   (n > 0 || k > 0) ? 1u : 0u);
-          ok = mbar_wait(&bar[C::B_DSR], n & 1, kWaitBackward, n, 25);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mma_ts(tmem + 384, tmem + 128 + k * 8, mnmaj(q_s, k), id_km,
-                   (n > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mma_ss(tmem + 128, mnmaj(aDS, k), mnmaj(aK, k), id_mm,
-                   k > 0 ? 1u : 0u);
-          mma_commit(&bar[C::B_DQF]);
-          mma_commit(&bar[C::B_QE + s]);
-          ++n;
-          // the next kept pair's S^T now, behind this pair's dQ product
-          int g2 = g, i2 = i + 1;
-          while (g2 < p.G) {
-            if (i2 >= p.nq) { ++g2; i2 = 0; continue; }
-            if (kept(g2, i2)) break;
-            ++i2;
-          }
-          if (g2 < p.G) {
-            issue_s(n);
-            pending = ok;
-          }
+          issue_dp(n + 1);
+          int g3 = g2, i3 = i2;
+          if (next_kept(g3, i3)) issue_s(n + 2);
         }
+        ++n;
+        g = g2;
+        i = i2;
+        have = h2;
       }
     }
     __syncwarp();
@@ -374,24 +421,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool key_ok = key < p.Lkv;
     const float sl2 = p.scale * kPrefLog2e;
     int n = 0;
-    bool ok = true, stop = false;
-    for (int g = 0; g < p.G && !stop; ++g) {
-      const int hq = hkv * p.G + g;
-      for (int i = 0; i < p.nq; ++i) {
-        if (!kept(g, i)) continue;
-        // All four warps leave together: a wait that gave up in any of them
-        // ends the loop for all at this barrier (never between barriers).
-        if (!named_sync_and(1, 128, ok)) { ok = false; stop = true; break; }
-        // this pair's lse (log2 units) and D per query column, loaded by
-        // the producer
-        {
-          const bool wl = mbar_wait(&bar[C::B_LF], n & 1, kWaitBackward, n, 33);
-          ok = __all_sync(FULL, wl);
-        }
+    bool ok = true;
+    uint32_t pk[64];  // P^T of a pair, from its P phase to its dS phase
+    // P^T of pair m (query tile i) into TMEM [0, 64); its lse in slot m & 1
+    auto p_phase = [&](int m, int i) {
+      const float* lse_m = lse_s + (m & 1) * 128;
+      {
+        const bool wl = ok && mbar_wait(&bar[C::B_LF + (m & 1)], (m >> 1) & 1,
+                                        kWaitBackward, m, 33);
+        ok = __all_sync(FULL, wl);
+      }
         // P^T (thread = key row, 128 query columns) into TMEM [0, 64) as
         // bf16; the packed values stay in registers for dS.
-        uint32_t pk[64];
-        const bool w1 = mbar_wait(&bar[C::B_SF], n & 1, kWaitBackward, n, 30);
+        const bool w1 = ok && mbar_wait(&bar[C::B_SF], m & 1, kWaitBackward, m, 30);
         ok = __all_sync(FULL, w1);
         tc_fence_after();
         // rows that see every query column of the tile need no mask; a warp
@@ -399,13 +441,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool row_full = key_ok && i * 128 + 127 < p.Lq &&
                               (!p.causal || key <= i * 128 + off);
         const bool warp_full = __all_sync(FULL, row_full);
-        const float4* lse4 = reinterpret_cast<const float4*>(lse_s);
+        const float4* lse4 = reinterpret_cast<const float4*>(lse_m);
+        // chunk cc + 1 is read while chunk cc is exponentiated; P of chunk
+        // cc goes to columns [16 cc, 16 cc + 16), all read already
+        uint32_t svb[2][32];
+        if (ok) {
+          tmem_ld32(lane_base + 0, svb[0]);
+          tc_wait_ld();
+        }
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           if (!ok) break;
-          uint32_t sv[32];
-          tmem_ld32(lane_base + 0 + cc * 32, sv);
-          tc_wait_ld();
+          if (cc < 3) tmem_ld32(lane_base + (cc + 1) * 32, svb[(cc + 1) & 1]);
+          const uint32_t (&sv)[32] = svb[cc & 1];
           if (warp_full) {
 #pragma unroll
             for (int x = 0; x < 32; x += 4) {
@@ -428,7 +476,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               const bool valid = key_ok && qr < p.Lq &&
                                  (!p.causal || key <= qr + off);
               pv[e] = valid ? ex2_approx(fmaf(__uint_as_float(sv[x + e]), sl2,
-                                              -lse_s[c]))
+                                              -lse_m[c]))
                             : 0.f;
             }
             pk[cc * 16 + (x >> 1)] = pack_bf16x2(pv[0], pv[1]);
@@ -438,28 +486,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int u = 0; u < 16; ++u) st16[u] = pk[cc * 16 + u];
           tmem_st16(lane_base + 0 + cc * 16, st16);
+          if (cc < 3) tc_wait_ld();
         }
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (ok && lane == 0) mbar_arrive(&bar[C::B_PR]);
+        if (ok && lane == 0) {
+          mbar_arrive(&bar[C::B_PR]);
+          mbar_arrive(&bar[C::B_LE + (m & 1)]);  // the lse slot is free
+        }
+    };
+    // dS^T of pair m, once its D and its dP^T have arrived
+    auto d_phase = [&](int m) {
+      {
+        const bool wd = ok && mbar_wait(&bar[C::B_DF], m & 1, kWaitBackward, m, 34);
+        ok = __all_sync(FULL, wd);
+      }
         // dS^T = P^T o (dP^T - D) into TMEM [128, 192) and shared memory
         const bool w2 =
-            ok && mbar_wait(&bar[C::B_DPF], n & 1, kWaitBackward, n, 31);
+            ok && mbar_wait(&bar[C::B_DPF], m & 1, kWaitBackward, m, 31);
         ok = __all_sync(FULL, w2);
         // the buffer holds the previous pair's last dQ staging until the
         // reduction has read it (its wait is taken here, after P)
-        if (n > 0) {
+        if (m > 0) {
           if (warp == 2 && lane == 0) bulk_wait_read_all();
           named_sync(1, 128);
         }
         tc_fence_after();
+        // the same overlap: dS^T of chunk cc goes to [128 + 16 cc, +16),
+        // below the dP^T columns still to be read
+        uint32_t dpb[2][32];
+        if (ok) {
+          tmem_ld32(lane_base + 128, dpb[0]);
+          tc_wait_ld();
+        }
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           if (!ok) break;
-          uint32_t dp[32];
-          tmem_ld32(lane_base + 128 + cc * 32, dp);
-          tc_wait_ld();
+          if (cc < 3) tmem_ld32(lane_base + 128 + (cc + 1) * 32, dpb[(cc + 1) & 1]);
+          const uint32_t (&dp)[32] = dpb[cc & 1];
           uint32_t dk16[16];
 #pragma unroll
           for (int x = 0; x < 32; x += 4) {
@@ -485,18 +550,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 make_uint4(dk16[4 * u], dk16[4 * u + 1], dk16[4 * u + 2],
                            dk16[4 * u + 3]);
           }
+          if (cc < 3) tc_wait_ld();
         }
         tc_wait_st();
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
         if (ok && lane == 0) mbar_arrive(&bar[C::B_DSR]);
+    };
+    // the dQ tile of pair m (query tile i of head hq) out to the accumulator
+    auto e_phase = [&](int m, int i, int hq) {
         // dQ tile (TMEM lane = query row) from [128, 256): staged in the dS
         // buffer (free once the dQ product is done) as two rounds of two
         // 32-column boxes (128-byte swizzle), each added to the f32
         // accumulator by TMA reductions issued by one thread.
         const bool w3 =
-            ok && mbar_wait(&bar[C::B_DQF], n & 1, kWaitBackward, n, 32);
+            ok && mbar_wait(&bar[C::B_DQF], m & 1, kWaitBackward, m, 32);
         ok = named_sync_and(1, 128, __all_sync(FULL, w3));
         if (ok) {
           tc_fence_after();
@@ -533,8 +602,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
           }
         }
-        ++n;
+    };
+    // One pair deep: P of pair n+1 runs while the tensor core does dK and
+    // dQ of pair n, then pair n's dQ tile is read out.
+    int g = 0, i = -1;
+    bool have = next_kept(g, i);
+    if (have) {
+      ok = named_sync_and(1, 128, ok);
+      p_phase(0, i);
+    }
+    while (have && ok) {
+      d_phase(n);
+      int g2 = g, i2 = i;
+      const bool h2 = next_kept(g2, i2);
+      if (h2) {
+        // All four warps leave together: a wait that gave up in any of them
+        // ends the loop for all at this barrier (never between barriers).
+        if (!named_sync_and(1, 128, ok)) {
+          ok = false;
+          break;
+        }
+        p_phase(n + 1, i2);
       }
+      e_phase(n, i, hkv * p.G + g);
+      ++n;
+      g = g2;
+      i = i2;
+      have = h2;
     }
     // dK_j, dV_j (TMEM lane = key row); zero when no pair was kept.  The
     // tensor-memory loads are warp-collective, so every lane takes part and
