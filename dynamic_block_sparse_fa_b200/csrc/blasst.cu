@@ -635,10 +635,18 @@ blasst_status_t blasst_decode_paged(const void* q, const void* k_pages,
       if (ws != BLASST_OK) return ws;
     }
     const int box_rows = page_size < 64 ? page_size : 64;
-    if (!blasst::encode_pool_map(&m.tk, k_pages, d, page_size, Hkv, num_pages,
-                                 page_stride, box_rows) ||
-        !blasst::encode_pool_map(&m.tv, v_pages, d, page_size, Hkv, num_pages,
-                                 page_stride, box_rows))
+    // d 128: whole rows per copy (5-D map); d 64: one 64-column box
+    const bool maps_ok =
+        d == 128
+            ? blasst::encode_pool_map_rows(&m.tk, k_pages, page_size, Hkv,
+                                           num_pages, page_stride, box_rows) &&
+                  blasst::encode_pool_map_rows(&m.tv, v_pages, page_size, Hkv,
+                                               num_pages, page_stride, box_rows)
+            : blasst::encode_pool_map(&m.tk, k_pages, d, page_size, Hkv,
+                                      num_pages, page_stride, box_rows) &&
+                  blasst::encode_pool_map(&m.tv, v_pages, d, page_size, Hkv,
+                                          num_pages, page_stride, box_rows);
+    if (!maps_ok)
       return cuda_status(cudaErrorInvalidValue, "paged decode tensor maps");
     m.q = static_cast<const __nv_bfloat16*>(q);
     m.counters = skip_stats ? skip_stats->counters : nullptr;

@@ -32,9 +32,11 @@
 // scoring to land); its P and rescale factor wait in registers.
 //
 // Paged cache (PAGED): the page pool [num_pages][Hkv][page_size][d] is a
-// 4-D tensor map whose box is min(page_size, 64) rows of one page, so a
-// 64-key block is one to four TMA segments, each from the page the block
-// table names.  Every page id a split will read is range-checked before the
+// tensor map whose box is min(page_size, 64) rows of one page, so a 64-key
+// block is one to four TMA segments, each from the page the block table
+// names.  At d = 128 the map is 5-D (64 columns, 2 halves, rows, heads,
+// pages) and one copy brings a segment's whole 256-byte rows, stored row by
+// row in shared memory; at d = 64 it is 4-D with one 64-column box.  Every page id a split will read is range-checked before the
 // first load (a bad id or length sets the error word and the CTA leaves).
 // Rows past the sequence's end that a segment brings in (the rest of its
 // last page) or that no segment covers are masked in the scores and zeroed
@@ -114,9 +116,6 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0,
       : "memory");
 }
 
-// Byte offset of the 16-byte chunk `chunk` (0..15: dims 8*chunk ..) of key
-// row `key` in a block stored as two 64-column boxes with the 128-byte
-// swizzle (chunk index XOR key % 8 within each 1024-byte group of rows).
 __device__ __forceinline__ void tma_load_4d(void* dst_smem, const void* tmap,
                                             uint64_t* bar, int c0, int c1,
                                             int c2, int c3, uint64_t policy) {
@@ -129,9 +128,33 @@ __device__ __forceinline__ void tma_load_4d(void* dst_smem, const void* tmap,
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_5d(void* dst_smem, const void* tmap,
+                                            uint64_t* bar, int c0, int c1,
+                                            int c2, int c3, int c4,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_"
+      "tx::bytes.L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(
+          smem_u32(dst_smem)),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(smem_u32(bar)),
+      "l"(policy)
+      : "memory");
+}
+
+// Byte offset of the 16-byte chunk `chunk` (0..15: dims 8*chunk ..) of key
+// row `key` in a block stored as two 64-column boxes with the 128-byte
+// swizzle (chunk index XOR key % 8 within each 1024-byte group of rows).
 __device__ __forceinline__ uint32_t swz_off(int key, int chunk) {
   return (uint32_t)((chunk >> 3) * DecodeMmaCfg::BOX + key * 128 +
                     (((chunk & 7) ^ (key & 7)) << 4));
+}
+
+// The same for a block stored row by row (paged cache, d = 128): key row
+// `key` is 256 bytes, its two 64-column halves two consecutive 128-byte
+// lines, and the 128-byte swizzle XORs the chunk with the line index % 8.
+__device__ __forceinline__ uint32_t swz_off_rows(int key, int chunk) {
+  const int line = 2 * key + (chunk >> 3);
+  return (uint32_t)(line * 128 + (((chunk & 7) ^ (line & 7)) << 4));
 }
 
 // BATCH = 2: the batched decision rule (contiguous cache): blocks r and
@@ -146,6 +169,12 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   static_assert(BATCH == 1 || (BATCH == 2 && !PAGED), "pairs: contiguous");
   static_assert(D == 64 || D == 128, "head dimension 64 or 128");
   constexpr int NBOX = D / 64;     // 64-column boxes per block
+  // paged d = 128: a segment's rows arrive whole (both halves) in one copy
+  constexpr bool ROWS = PAGED && NBOX == 2;
+  auto kv_off = [](int key, int chunk) {
+    if constexpr (ROWS) return swz_off_rows(key, chunk);
+    else return swz_off(key, chunk);
+  };
   constexpr int KST = D / 16;      // k-steps of the scores
   constexpr int NG = D / 8;        // 8-column groups of the output
   using C = DecodeMmaCfg;
@@ -236,10 +265,15 @@ __global__ void __launch_bounds__(kDecThreads, 3)
       for (int i = 0; i < nseg; ++i) {
         const int t = j * kDecBc + i * seg;
         const int id = __ldg(bt_row + (t >> a.log2_page));
+        if constexpr (ROWS) {
+          tma_load_5d(dst + i * seg * 256, map, bar, 0, 0, t & (ps - 1), hkv,
+                      id, pol);
+        } else {
 #pragma unroll
-        for (int c = 0; c < NBOX; ++c)
-          tma_load_4d(dst + c * C::BOX + i * seg * 128, map, bar, c * 64,
-                      t & (ps - 1), hkv, id, pol);
+          for (int c = 0; c < NBOX; ++c)
+            tma_load_4d(dst + c * C::BOX + i * seg * 128, map, bar, c * 64,
+                        t & (ps - 1), hkv, id, pol);
+        }
       }
     }
   };
@@ -308,9 +342,11 @@ __global__ void __launch_bounds__(kDecThreads, 3)
       for (int e = lane; e < 16 * NBOX * 8; e += 32) {
         const int row = 16 * warp + e / (NBOX * 8);
         const int c16 = e % (NBOX * 8);  // 16-byte chunk of the row
+        // (every chunk of the row, so the swizzle order does not matter)
+        const int off = ROWS ? row * 256 + c16 * 16
+                             : (c16 >> 3) * C::BOX + row * 128 + (c16 & 7) * 16;
         if (row >= prows)
-          *reinterpret_cast<uint4*>(vs + (c16 >> 3) * C::BOX + row * 128 +
-                                    (c16 & 7) * 16) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(vs + off) = make_uint4(0, 0, 0, 0);
       }
       fence_async_smem();  // before a later TMA load overwrites the slot
       __syncwarp();
@@ -318,7 +354,7 @@ __global__ void __launch_bounds__(kDecThreads, 3)
 #pragma unroll
     for (int p = 0; p < NG / 2; ++p) {
       uint32_t r0, r1, r2, r3;
-      ldsm_x4_t(vb + swz_off(16 * warp + 8 * (mi & 1) + mr, 2 * p + (mi >> 1)),
+      ldsm_x4_t(vb + kv_off(16 * warp + 8 * (mi & 1) + mr, 2 * p + (mi >> 1)),
                 r0, r1, r2, r3);
       mma16816_top(o[2 * p][0], o[2 * p][1], pp0, pp1, r0, r1);
       mma16816_top(o[2 * p + 1][0], o[2 * p + 1][1], pp0, pp1, r2, r3);
@@ -343,7 +379,7 @@ __global__ void __launch_bounds__(kDecThreads, 3)
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           uint32_t r0, r1, r2, r3;
-          ldsm_x4(kb + swz_off(16 * warp + 8 * g + mr, 4 * p + mi), r0, r1, r2,
+          ldsm_x4(kb + kv_off(16 * warp + 8 * g + mr, 4 * p + mi), r0, r1, r2,
                   r3);
           mma16816_top(sc[g][0], sc[g][1], qa[2 * p][0], qa[2 * p][1], r0, r1);
           mma16816_top(sc[g][0], sc[g][1], qa[2 * p + 1][0], qa[2 * p + 1][1],

@@ -579,6 +579,29 @@ inline bool encode_pool_map(CUtensorMap* m, const void* base, int D,
   return r == CUDA_SUCCESS;
 }
 
+// The page pool at D = 128 as 5-D (64 columns, 2 column halves, page rows,
+// heads, pages): one copy brings box_rows whole rows of a page (both halves,
+// 256 bytes a row), each half a 128-byte line under the 128-byte swizzle.
+inline bool encode_pool_map_rows(CUtensorMap* m, const void* base,
+                                 int page_rows, int heads, long long pages,
+                                 long long page_stride, int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  constexpr int D = 128;
+  cuuint64_t dims[5] = {64, 2, (cuuint64_t)page_rows, (cuuint64_t)heads,
+                        (cuuint64_t)pages};
+  cuuint64_t strides[4] = {128, (cuuint64_t)D * 2,
+                           (cuuint64_t)page_rows * D * 2,
+                           (cuuint64_t)page_stride * 2};
+  cuuint32_t box[5] = {64, 2, (cuuint32_t)box_rows, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base),
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int D, int BN, int BRL>
 cudaError_t launch_prefill_t(const PrefillProblem& pr, cudaStream_t st) {
   using C = PrefillCfg<D, BN, BRL>;
