@@ -12,10 +12,12 @@
 // A pair the forward skipped (or did not visit) does no MMA and loads
 // nothing.
 //
-// Three kernels:
+// Three kernels (five with a mask):
 //   bwd_prep_kernel     D and lse * log2 e per query row (rows padded to 16
 //                       bytes, for the producer's TMA), zeroes the f32 dQ
 //                       accumulator
+//   bwd_count_kernel,   with a mask: kept pairs per CTA, and the CTAs in
+//   bwd_order_kernel    order of those counts, most first
 //   bwd_dkdv_kernel     one CTA per (sequence, KV head, key block j): K_j and
 //                       V_j stay in shared memory while the kept query tiles
 //                       of the G query heads stream through; dK_j, dV_j
@@ -63,11 +65,16 @@ struct BwdParams {
   __nv_bfloat16* dq;          // [B, Hq, Lq, D]
   __nv_bfloat16* dk;          // [B, Hkv, Lkv, D]
   __nv_bfloat16* dv;          // [B, Hkv, Lkv, D]
+  int* counts;                // masked: kept pairs per grid slot (scratch)
+  const int* order;           // masked: grid slot of each CTA (null: own)
   int B, Hq, Hkv, Lq, Lkv, nq, nk, G, causal;
   float scale;
 };
 
 constexpr int kBwdD = 128;
+// the work order's rank kernel is quadratic in the CTA count: above this
+// many CTAs the grid keeps its own order
+constexpr long long kBwdOrderMaxSlots = 32768;
 constexpr int kBwdThreads = 192;
 
 struct BwdCfg {
@@ -153,6 +160,59 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
 }
 
 // dQ = bf16(scale * accumulator), 8 elements per thread.
+// Work order of a masked backward.  A CTA's work is its kept (head, tile)
+// pairs, which a sparse mask spreads very unevenly over the key blocks, so
+// the CTAs go out by kept pairs, most first (ties in grid order).  Grid slot
+// s = jb * (B*Hkv) + b*Hkv + hkv is the CTA of key block jb; one warp counts
+// a slot's pairs.
+__global__ void __launch_bounds__(256) bwd_count_kernel(const BwdParams p) {
+  const int nbk = p.B * p.Hkv;
+  const long long n = (long long)nbk * p.nk;
+  const long long s = ((long long)blockIdx.x * 256 + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (s >= n) return;
+  const int jb = (int)(s / nbk);
+  const int bk = (int)(s - (long long)jb * nbk);
+  const int b = bk / p.Hkv;
+  const int hkv = bk - b * p.Hkv;
+  const int off = p.Lkv - p.Lq;
+  int c = 0;
+  const int cand = p.G * p.nq;
+  for (int x = lane; x < cand; x += 32) {
+    const int g = x / p.nq;
+    const int i = x - g * p.nq;
+    if (p.causal && min((i + 1) * 128, p.Lq) - 1 + off < jb * 128) continue;
+    const int hq = hkv * p.G + g;
+    c += __ldg(p.mask + ((size_t)(b * p.Hq + hq) * p.nq + i) * p.nk + jb) == 1;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if (lane == 0) p.counts[s] = c;
+}
+
+// order[rank of slot s] = s, rank = slots with more kept pairs, or as many
+// and a lower index.  The ranks are a permutation of 0 .. n-1.
+__global__ void __launch_bounds__(256) bwd_order_kernel(const BwdParams p,
+                                                         int* order) {
+  __shared__ int tile[2048];
+  const int n = p.B * p.Hkv * p.nk;
+  const int s = blockIdx.x * 256 + threadIdx.x;
+  const int cs = s < n ? p.counts[s] : 0;
+  int rank = 0;
+  for (int t0 = 0; t0 < n; t0 += 2048) {
+    const int m = min(2048, n - t0);
+    __syncthreads();
+    for (int u = threadIdx.x; u < m; u += 256) tile[u] = p.counts[t0 + u];
+    __syncthreads();
+    if (s < n)
+      for (int u = 0; u < m; ++u) {
+        const int cu = tile[u];
+        rank += (cu > cs) || (cu == cs && t0 + u < s);
+      }
+  }
+  if (s < n) order[rank] = s;
+}
+
 __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p) {
   const long long n8 = (long long)p.B * p.Hq * p.Lq * (kBwdD / 8);
   const long long i = (long long)blockIdx.x * 256 + threadIdx.x;
@@ -181,8 +241,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // Causal key block j has the most query tiles for j = 0: CTAs go out in
   // ascending j over all (sequence, KV head), longest first.
   const int nbk = p.B * p.Hkv;
-  const int jb = blockIdx.x / nbk;   // key block
-  const int bk = blockIdx.x - jb * nbk;  // b * Hkv + hkv
+  const int slot = p.order ? __ldg(p.order + blockIdx.x) : (int)blockIdx.x;
+  const int jb = slot / nbk;         // key block
+  const int bk = slot - jb * nbk;    // b * Hkv + hkv
   const int b = bk / p.Hkv;
   const int hkv = bk - b * p.Hkv;
   const int off = p.Lkv - p.Lq;      // bottom-right causal alignment
@@ -773,6 +834,22 @@ inline cudaError_t launch_backward(const BwdProblem& pr, cudaStream_t st) {
   bwd_prep_kernel<<<(unsigned)prep_blocks, 256, 0, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  // With a mask, the CTAs go out by kept pairs.  The counts and the order
+  // (2 ints per slot) live in dq, which only the last kernel writes; the
+  // order is skipped when dq is too small for them or the slots are many.
+  const size_t dq_bytes = rows * kBwdD * 2;
+  if (p.mask && grid <= kBwdOrderMaxSlots &&
+      (size_t)grid * 2 * sizeof(int) <= dq_bytes) {
+    p.counts = static_cast<int*>(pr.dq);
+    int* order = p.counts + grid;
+    bwd_count_kernel<<<(unsigned)((grid * 32 + 255) / 256), 256, 0, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    bwd_order_kernel<<<(unsigned)((grid + 255) / 256), 256, 0, st>>>(p, order);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    p.order = order;
+  }
   e = cudaFuncSetAttribute(bwd_dkdv_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            BwdCfg::SMEM_ALLOC);

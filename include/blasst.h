@@ -176,7 +176,9 @@ blasst_status_t blasst_prefill_window(const void *q, const void *k,
  *  mask        the forward's decision bytes (skip_stats.mask layout
  *              [B,Hq,ceil(Lq/128),ceil(Lkv/128)], 1 = kept), or NULL for
  *              the dense backward (every visible pair kept)
- *  dq          device bf16 [B,Hq,Lq,d] (written)
+ *  dq          device bf16 [B,Hq,Lq,d] (written; with a mask it first
+ *              holds, as scratch, each key block's count of kept pairs and
+ *              the order the key blocks run in: most kept pairs first)
  *  dk, dv      device bf16 [B,Hkv,Lkv,d] (written)
  *  d = 128, Br = Bc = 128 (else BLASST_ERR_UNSUPPORTED_SHAPE); causal with
  *              Lq > Lkv is rejected
@@ -184,7 +186,9 @@ blasst_status_t blasst_prefill_window(const void *q, const void *k,
  *              bytes, 256-byte aligned, caller-owned (f32 dQ accumulator,
  *              the per-row D and lse * log2 e); contents need not be
  *              initialised
- * Asynchronous on `stream`; three kernel launches; allocates nothing.
+ * Asynchronous on `stream`; three kernel launches (five with a mask, for
+ * the work order, unless B*Hkv*ceil(Lkv/128) exceeds 32768 or dq is too
+ * small to hold 8 bytes per key block); allocates nothing.
  * Errors as blasst_prefill (BLASST_ERR_WORKSPACE for a missing or small
  * workspace).
  */
