@@ -178,7 +178,8 @@ blasst_status_t blasst_prefill_window(const void *q, const void *k,
  *              the dense backward (every visible pair kept)
  *  dq          device bf16 [B,Hq,Lq,d] (written; with a mask it first
  *              holds, as scratch, each key block's count of kept pairs and
- *              the order the key blocks run in: most kept pairs first)
+ *              the order the key blocks run in: most kept pairs first; so
+ *              dq must not overlap any input)
  *  dk, dv      device bf16 [B,Hkv,Lkv,d] (written)
  *  d = 128, Br = Bc = 128 (else BLASST_ERR_UNSUPPORTED_SHAPE); causal with
  *              Lq > Lkv is rejected
