@@ -177,6 +177,17 @@ def _arg(t, name, dtype=torch.bfloat16, contiguous=True):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _overlaps(a, b):
+    """Whether the storage spans of two tensors intersect (None: never)."""
+    if a is None or b is None or a.device != b.device:
+        return False
+    a0 = a.data_ptr()
+    b0 = b.data_ptr()
+    a1 = a0 + a.numel() * a.element_size()
+    b1 = b0 + b.numel() * b.element_size()
+    return a0 < b1 and b0 < a1
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -360,6 +371,11 @@ def blasst_prefill_backward(q, k, v, o, lse, dout, *, mask=None, scale=None,
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    # dq also holds the work order of a masked call before it is written
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse),
+                    ("dout", dout), ("mask", mask)):
+        if _overlaps(dq, t):
+            raise ValueError(f"dq overlaps {name}")
     need = blasst_prefill_backward_workspace_size(B, Hq, Lq, d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8,

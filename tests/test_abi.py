@@ -222,6 +222,27 @@ def test_binding_rejects_host_and_mistyped_tensors(lib):
         b._arg(torch.zeros(4, dtype=torch.float16), "x")
 
 
+def test_backward_binding_rejects_dq_overlapping_an_input(lib):
+    """dq holds the masked backward's work order before it is written, so
+    the binding refuses a dq that shares storage with an input (checked on
+    the host, before any pointer reaches the library)."""
+    import torch
+    import dynamic_block_sparse_fa_b200 as m
+    from dynamic_block_sparse_fa_b200 import blasst as b
+    q = torch.zeros(1, 2, 128, 128, dtype=torch.bfloat16)
+    k = torch.zeros(1, 1, 128, 128, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 2, 128)
+    dout = torch.zeros_like(q)
+    with pytest.raises(ValueError, match="dq overlaps dout"):
+        m.blasst_prefill_backward(q, k, k, q.clone(), lse, dout, dq=dout[:, 1:])
+    with pytest.raises(ValueError, match="dq overlaps q"):
+        m.blasst_prefill_backward(q, k, k, q.clone(), lse, dout, dq=q)
+    flat = torch.zeros(100)
+    assert b._overlaps(flat[10:20], flat[19:30])
+    assert not b._overlaps(flat[10:20], flat[20:30])
+    assert not b._overlaps(flat, None)
+
+
 def test_split_policy_and_workspace(lib):
     import dynamic_block_sparse_fa_b200 as m
     # batch 32 x 8 KV heads at 32K: 5 splits; batch 148: 1 split
