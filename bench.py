@@ -65,6 +65,9 @@ DECODE_TRAFFIC = dict(source="dynamic_block_sparse_fa_b200/csrc/decode_mma.cuh",
                       sha256_16="e08531a69c43a4a1",
                       ratio=(950.654720 + 4.106496) / 957.799424)
 PRE = dict(B=1, Hq=32, Hkv=8, L=32768, d=128, Br=128, Bc=128, window=4096)
+# B200 data-sheet figures, reported beside the measured denominators: HBM3e
+# ~8 TB/s, dense bf16 tensor ~2.25 PFLOP/s
+NOMINAL = dict(hbm_gbs=8000.0, bf16_tflops=2250.0)
 
 
 def _measured_traffic(spec, algorithmic_bytes):
@@ -504,6 +507,8 @@ def run_decode(args, bl, dev, stream, world, rank, local, dist, barrier,
             "achieved": round(achieved, 1), "peak": hbm_peak,
             "peak_kind": peak_kind + " copy bandwidth", "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4),
+            "nominal_peak": NOMINAL["hbm_gbs"],
+            "frac_of_nominal": round(achieved / NOMINAL["hbm_gbs"], 4),
             "traffic": _measured_traffic(DECODE_TRAFFIC, by_call),
             "traffic_unit": "bytes per launch",
         },
@@ -718,7 +723,11 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
         return out, {"bound": "tensor", "kernel": "prefill2_kernel<128>",
                      "achieved": r["executed_tflops"], "peak": tf_peak,
                      "peak_kind": peak_kind + " bf16 burst", "unit": "TFLOP/s",
-                     "frac": r["tensor_frac"], "traffic": None}
+                     "frac": r["tensor_frac"],
+                     "nominal_peak": NOMINAL["bf16_tflops"],
+                     "frac_of_nominal": round(r["executed_tflops"]
+                                              / NOMINAL["bf16_tflops"], 4),
+                     "traffic": None}
     dense = measure(-math.inf)
     out["dense"] = dense
     # the skipping kernel at a threshold that never skips: the dense path
@@ -772,7 +781,11 @@ def run_prefill(args, bl, dev, stream, tf_peak, peak_kind):
     roof = {"bound": "tensor", "kernel": "prefill2_kernel<128> at 70%",
             "achieved": best["executed_tflops"], "peak": tf_peak,
             "peak_kind": peak_kind + " bf16 burst", "unit": "TFLOP/s",
-            "frac": best["tensor_frac"], "traffic": None}
+            "frac": best["tensor_frac"],
+            "nominal_peak": NOMINAL["bf16_tflops"],
+            "frac_of_nominal": round(best["executed_tflops"]
+                                     / NOMINAL["bf16_tflops"], 4),
+            "traffic": None}
     return out, roof
 
 
